@@ -1,0 +1,147 @@
+"""The SVDQuant W4A4 linear layer, step by step, on the CPU in float64.
+
+TEST INFRASTRUCTURE ONLY: see the package docstring.
+
+The layer (blog "Bringing Nunchaku 4-bit Diffusion Inference to Diffusers",
+section "Background: SVDQuant and Nunchaku"): outliers are first moved into
+the weights, the hardest part of each weight matrix is kept in a small
+16-bit low-rank branch, and the remaining residual is quantised to 4 bits;
+activations are quantised to 4 bits on the fly (section "Introducing Nunchaku
+Lite": 4-bit weights and activations). Written as one formula:
+
+    Y = (X . L1) . L2  +  Q4(X) . Q4(R)^T  +  b,    R = W - (L1 . L2)^T
+
+with L1: K x r and L2: r x N in bfloat16 (the figure caption in that section:
+the down projection X.L1 is fused with the activation quantiser, the up
+projection (X.L1).L2 with the 4-bit GEMM). Smoothing is the identity here
+(lambda = 1), which is exactly the formula above.
+
+Functions, in the order the method applies them:
+  lowrank_factors   truncated SVD of W^T             (load time)
+  residual          R = W - (L1 L2)^T                 (load time)
+  pack_weight       NVFP4 of R, its global scale      (load time)
+  quantize_act      NVFP4 of X                        (every call)
+  down_proj         XL1 = bf16(X . L1)                (every call)
+  forward           Y                                  (every call)
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+import numpy as np
+import torch
+
+from . import nvfp4
+
+
+def to_f64(t) -> np.ndarray:
+    """A CPU tensor (any float dtype, bf16 included) or array -> float64 array, exactly."""
+    if isinstance(t, torch.Tensor):
+        return t.detach().to(torch.float64).cpu().numpy()
+    return np.asarray(t, dtype=np.float64)
+
+
+# ------------------------------------------------------------------ load time
+def lowrank_factors(W, r: int):
+    """Rank-r factors of W^T (K x N) from a float64 SVD.
+
+    W^T = U diag(s) V^T; L1 = bf16(U_r diag(s_r)) (K x r), L2 = bf16(V_r^T)
+    (r x N). The pages do not say how the singular values are split between
+    the factors; any split is valid because everything downstream uses these
+    exact bf16 factors. Returns (L1, L2, s) with s all singular values (float64).
+    """
+    Wt = to_f64(W).T
+    U, s, Vt = np.linalg.svd(Wt, full_matrices=False)
+    L1 = nvfp4.bf16_round(U[:, :r] * s[:r])
+    L2 = nvfp4.bf16_round(Vt[:r, :])
+    return L1, L2, s
+
+
+def residual(W, L1, L2) -> np.ndarray:
+    """R[n,k] = W[n,k] - sum_j L1[k,j] L2[j,n], float64, j ascending, then fp32 RN.
+
+    Each product of two bf16 numbers is exact in float64; the running sum is
+    rounded after each addition in the stated order, so the result is fully
+    determined.
+    """
+    W = to_f64(W)
+    L1 = to_f64(L1)
+    L2 = to_f64(L2)
+    s = np.zeros_like(W)
+    for j in range(L1.shape[1]):
+        s += np.outer(L2[j, :], L1[:, j])
+    return (W - s).astype(np.float32)
+
+
+@dataclass
+class PackedWeight:
+    codes: np.ndarray    # uint8 [N, K] one E2M1 code per element
+    scales: np.ndarray   # uint8 [N, K/16] E4M3 block scales
+    g_w: np.float32      # global decode scale of R
+    L1: np.ndarray       # float64 [K, r] (bf16 values)
+    L2: np.ndarray       # float64 [r, N] (bf16 values)
+
+
+def pack_weight(W, L1, L2) -> PackedWeight:
+    R = residual(W, L1, L2)
+    g_w = nvfp4.global_scale(R)
+    codes, scales = nvfp4.quantize_rows(R, g_w)
+    return PackedWeight(codes, scales, g_w, to_f64(L1), to_f64(L2))
+
+
+# ------------------------------------------------------------------ per call
+def act_global_scale(X) -> np.float32:
+    """Static (calibrated) activation decode scale, g_X = fp32(amax|X| / 2688)."""
+    return nvfp4.global_scale(to_f64(X).astype(np.float32))
+
+
+def quantize_act(X, g_x):
+    """NVFP4 of the activation rows: (codes [M, K], scales [M, K/16])."""
+    return nvfp4.quantize_rows(to_f64(X).astype(np.float32), g_x)
+
+
+def down_proj(X, L1) -> np.ndarray:
+    """XL1 = bf16(X . L1), accumulated in float64 (the 16-bit branch's input)."""
+    return nvfp4.bf16_round(to_f64(X) @ to_f64(L1))
+
+
+@dataclass
+class Forward:
+    codes: np.ndarray    # activation codes [M, K]
+    scales: np.ndarray   # activation scales [M, K/16]
+    xl1: np.ndarray      # float64 [M, r] (bf16 values)
+    y64: np.ndarray      # float64 [M, N] exact-precision output
+    y_ref: np.ndarray    # float64 [M, N] y64 rounded to bf16
+
+
+def gemm_4bit(codes_x, scales_x, codes_w, scales_w) -> np.ndarray:
+    """acc[m,n] = sum_k dec(cX)dec(SX) * dec(cR)dec(SR), in float64 (no global scales)."""
+    xq = nvfp4.dequantize_rows(codes_x, scales_x)
+    wq = nvfp4.dequantize_rows(codes_w, scales_w)
+    return xq @ wq.T
+
+
+def forward(X, pw: PackedWeight, bias, g_x) -> Forward:
+    """Y = acc * g_X * g_W + XL1 . L2 + b, float64; y_ref = bf16(Y)."""
+    codes, scales = quantize_act(X, g_x)
+    xl1 = down_proj(X, pw.L1)
+    acc = gemm_4bit(codes, scales, pw.codes, pw.scales)
+    y = acc * float(g_x) * float(pw.g_w) + xl1 @ pw.L2
+    if bias is not None:
+        y = y + to_f64(bias)[None, :]
+    return Forward(codes, scales, xl1, y, nvfp4.bf16_round(y))
+
+
+# ------------------------------------------------------------------ metrics
+def rel_fro(a, b) -> float:
+    a = np.asarray(a, dtype=np.float64)
+    b = np.asarray(b, dtype=np.float64)
+    return float(np.linalg.norm(a - b) / np.linalg.norm(b))
+
+
+def max_abs_over_row_rms(a, ref) -> float:
+    """max_{m,n} |a - ref| / rms(ref[m, :])."""
+    a = np.asarray(a, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    rms = np.sqrt(np.mean(ref * ref, axis=1, keepdims=True))
+    return float(np.max(np.abs(a - ref) / rms))
