@@ -1,0 +1,157 @@
+/*
+ * svdq.h — C ABI of the B200 (sm_100a) SVDQuant W4A4 NVFP4 linear layer.
+ *
+ * The layer (blog "Bringing Nunchaku 4-bit Diffusion Inference to Diffusers",
+ * sections "Background: SVDQuant and Nunchaku" and "Introducing Nunchaku Lite"):
+ *
+ *     Y = (X . L1) . L2  +  Q4(X) . Q4(R)^T  +  b,        R = W - (L1 . L2)^T
+ *
+ * X: M x K activations (bf16), W: N x K weight (bf16), L1: K x r and L2: r x N
+ * the 16-bit low-rank factors (bf16), b: N bias (bf16), Y: M x N (bf16).
+ * Q4 is NVFP4: one E2M1 code per element, one E4M3 scale per 16 contiguous
+ * K-elements ("group_size": 16 in the blog's quantization_config), and one
+ * FP32 decode scale per tensor (g_x for X, g_w for R).
+ *
+ * Conventions for every entry point
+ * ---------------------------------
+ *  - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *    never allocates or frees device memory. Buffers must be 16-byte aligned.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *    Work is enqueued asynchronously; no call synchronises the host, except
+ *    svdq_read_device_error.
+ *  - Every function returns an svdq_status. Arguments are validated on the
+ *    host before any launch; an invalid call launches nothing and returns
+ *    SVDQ_ERR_INVALID_ARG / _UNSUPPORTED_SHAPE / _MISALIGNED. A device that is
+ *    not compute capability 10.0 (B200, sm_100a) gives
+ *    SVDQ_ERR_UNSUPPORTED_DEVICE (the blog's hardware section: the quantizer
+ *    checks the GPU's capability and raises a clear error rather than produce
+ *    wrong outputs). A failed launch gives SVDQ_ERR_CUDA.
+ *  - Kernels never spin without bound. A wait that exceeds its limit records
+ *    SVDQ_ERR_TIMEOUT in a per-device error word and the kernel returns;
+ *    svdq_read_device_error reports it after the caller synchronises.
+ *  - Shape rules: K % 256 == 0, N % 128 == 0, r in {16, 32, 64, 128},
+ *    M >= 0 (M == 0 is a no-op). Leading dimensions are in elements, multiples
+ *    of 8 and at least the row length.
+ *
+ * Data layouts (all row-major)
+ * ----------------------------
+ *  codes   uint8 [rows][K/2]; byte j holds element 2j in bits 0..3 and element
+ *          2j+1 in bits 4..7. E2M1 code: sign bit 3, exponent bits 2..1 (bias
+ *          1), mantissa bit 0.
+ *  scales  uint8 E4M3 codes (bias 7, max 448), one per 16 K-elements, in a
+ *          tiled order the tensor cores read directly: rows are padded to a
+ *          multiple of 128; the byte of (row, kb) with kb = k/16 sits at
+ *              ((row/128) * (K/64) + kb/4) * 512 + (row%32) * 16
+ *                  + ((row%128)/32) * 4 + kb%4
+ *          (svdq_scale_offset computes it on the host).
+ *  l1t     bf16 [r][K]   = L1 transposed (packed by svdq_pack_weight)
+ *  l2t     bf16 [N][r]   = L2 transposed (packed by svdq_pack_weight)
+ *  xl1     bf16 [M][r]   = bf16(X . L1), fp32 accumulation
+ */
+#ifndef SVDQ_H_
+#define SVDQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum svdq_status {
+  SVDQ_OK = 0,
+  SVDQ_ERR_INVALID_ARG = 1,        /* null pointer, negative size, bad rank */
+  SVDQ_ERR_UNSUPPORTED_SHAPE = 2,  /* K % 256, N % 128, leading dimension  */
+  SVDQ_ERR_MISALIGNED = 3,         /* a pointer not 16-byte aligned          */
+  SVDQ_ERR_UNSUPPORTED_DEVICE = 4, /* current device is not sm_100 / no GPU  */
+  SVDQ_ERR_CUDA = 5,               /* a CUDA runtime call or launch failed   */
+  SVDQ_ERR_TIMEOUT = 6,            /* a kernel wait ran out (device error)   */
+  SVDQ_ERR_WORKSPACE = 7           /* workspace too small                    */
+} svdq_status;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* svdq_status_string(int status);
+
+/* Library version, major*10000 + minor*100 + patch. */
+int svdq_version(void);
+
+/* Byte offset of the E4M3 scale of (row, kblock) in the tiled scale layout
+ * described above, for a tensor with K columns. Host-only, pure function.
+ * Errors: INVALID_ARG if row < 0, kblock outside [0, K/16) or out == NULL;
+ * UNSUPPORTED_SHAPE if K % 64 != 0. */
+svdq_status svdq_scale_offset(int K, int row, int kblock, size_t* out);
+
+/* ------------------------------------------------------------ sizes (host) */
+/* Bytes of each packed-weight buffer for an N x K weight with rank r. */
+svdq_status svdq_weight_sizes(int N, int K, int r, size_t* codes_bytes, size_t* scales_bytes,
+                              size_t* l1t_bytes, size_t* l2t_bytes);
+/* Bytes of the quantised-activation buffers for M rows (scales padded to 128 rows). */
+svdq_status svdq_act_sizes(int M, int K, int r, size_t* codes_bytes, size_t* scales_bytes,
+                           size_t* xl1_bytes);
+/* Workspace bytes svdq_linear_forward needs (activation codes, scales and XL1). */
+svdq_status svdq_forward_workspace_size(int M, int K, int r, size_t* bytes);
+
+/* ------------------------------------------------------------ load time */
+/* Pack one layer (untimed, load time). Blog section "Background: SVDQuant and
+ * Nunchaku": the low-rank branch holds the hardest part of the weight, the
+ * remaining residual is quantised to 4 bits.
+ *   W   bf16 [N][K], L1 bf16 [K][r], L2 bf16 [r][N]   (inputs; L1.L2 is the
+ *       rank-r factorisation of W^T)
+ *   Writes: w_codes [N][K/2], w_scales (tiled), *g_w (device float),
+ *           l1t [r][K], l2t [N][r].
+ * R[n,k] = W[n,k] - sum_j L1[k,j] L2[j,n] is formed in float64 (j ascending,
+ * products exact) and rounded once to float32; g_w = fp32(amax|R| / 2688)
+ * (1 if R == 0); then R is quantised with the NVFP4 rule of svdq_quantize_act.
+ * The output buffers must not overlap the inputs. */
+svdq_status svdq_pack_weight(int N, int K, int r, const void* W, const void* L1, const void* L2,
+                             void* w_codes, void* w_scales, float* g_w, void* l1t, void* l2t,
+                             void* stream);
+
+/* Calibrated (static) activation scale: *g_out = fp32(amax|X| / 2688), or 1
+ * for an all-zero X. X bf16 [M][ldx]; g_out is a device float. */
+svdq_status svdq_act_global_scale(int M, int K, const void* X, int64_t ldx, float* g_out,
+                                  void* stream);
+
+/* ------------------------------------------------------------ per call */
+/* Activation quantisation fused with the low-rank down projection (blog
+ * figure caption in "Background: SVDQuant and Nunchaku": the down projection
+ * is fused with the quantisation kernel). One pass over X [M][ldx] (bf16):
+ *   per 16-element block: S = e4m3_rn_sat(amax / fp32(6 g_x)),
+ *   sd = fp32(dec(S) g_x), code = e2m1_rn_sat(fp32(x * fp32(1/sd))) (0 if sd == 0);
+ *   xl1 = bf16(X . L1) with fp32 accumulation (L1 given as l1t [r][K]).
+ * Writes codes [M][K/2], scales (tiled, rows padded to 128; padding rows are
+ * written as zero scales), xl1 [M][r]. Deterministic. */
+svdq_status svdq_quantize_act(int M, int K, int r, const void* X, int64_t ldx, float g_x,
+                              const void* l1t, void* codes, void* scales, void* xl1, void* stream);
+
+/* The block-scaled FP4 GEMM with the low-rank up projection and bias fused in
+ * its epilogue (blog figure caption: the up projection is fused with the 4-bit
+ * compute kernel):
+ *   Y[m,n] = bf16( g_x * g_w * sum_k dec(Xc)dec(SX) dec(Rc)dec(SR)
+ *                  + sum_j xl1[m,j] L2[j,n] + b[n] )
+ * a_codes/a_scales/xl1 as written by svdq_quantize_act; w_* as written by
+ * svdq_pack_weight; bias may be NULL; Y bf16 [M][ldy]. */
+svdq_status svdq_w4a4_gemm(int M, int N, int K, int r, const void* a_codes, const void* a_scales,
+                           const void* xl1, float g_x, const void* w_codes, const void* w_scales,
+                           const float* g_w, const void* l2t, const void* bias, void* Y,
+                           int64_t ldy, void* stream);
+
+/* The whole layer: svdq_quantize_act into `workspace`, then svdq_w4a4_gemm.
+ * workspace_bytes must be >= svdq_forward_workspace_size(M, K, r). */
+svdq_status svdq_linear_forward(int M, int N, int K, int r, const void* X, int64_t ldx, float g_x,
+                                const void* w_codes, const void* w_scales, const float* g_w,
+                                const void* l1t, const void* l2t, const void* bias, void* Y,
+                                int64_t ldy, void* workspace, size_t workspace_bytes,
+                                void* stream);
+
+/* ------------------------------------------------------------ errors */
+/* Reads (and, if clear != 0, resets) the device error word of the current
+ * device: 0 or an svdq_status recorded by a kernel (e.g. SVDQ_ERR_TIMEOUT).
+ * Synchronises the device first. */
+svdq_status svdq_read_device_error(int* code, int clear);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SVDQ_H_ */

@@ -1,0 +1,108 @@
+"""Host-side checks of the C ABI: the library loads without a GPU, exports every
+symbol include/svdq.h declares, validates arguments before touching a device,
+and reports a missing/unsupported device as SVDQ_ERR_UNSUPPORTED_DEVICE."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+import torch
+
+from tests import layouts
+from w4a4_rank_corrected_svdq_b200 import _lib
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "svdq.h")
+
+
+def _declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(svdq_[a-z0-9_]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    from w4a4_rank_corrected_svdq_b200 import build
+    build.build()
+    return _lib.lib()
+
+
+def test_every_declared_symbol_is_exported_and_bound(L):
+    names = _declared_functions()
+    assert "svdq_linear_forward" in names and "svdq_pack_weight" in names and "svdq_quantize_act" in names
+    for n in names:
+        assert hasattr(L, n), n
+        assert n in _lib.SIGNATURES, n
+
+
+def test_status_strings_and_version(L):
+    assert L.svdq_status_string(0) == b"SVDQ_OK"
+    assert L.svdq_status_string(6) == b"SVDQ_ERR_TIMEOUT"
+    assert L.svdq_status_string(99) == b"SVDQ_ERR_UNKNOWN"
+    assert L.svdq_version() >= 100
+
+
+def test_scale_offset_matches_documented_layout(L):
+    K = 512
+    offs = layouts.scale_offsets(300, K)
+    for row in (0, 1, 31, 32, 100, 127, 128, 255, 299):
+        for kb in (0, 1, 3, 4, 17, K // 16 - 1):
+            assert _lib.svdq_scale_offset(K, row, kb) == offs[row, kb]
+    # a 128-row block of a K-column tensor is a permutation of its K/16*128 bytes
+    blk = layouts.scale_offsets(128, K).ravel()
+    assert np.array_equal(np.sort(blk), np.arange(128 * K // 16))
+
+
+def test_scale_offset_errors(L):
+    out = ctypes.c_size_t()
+    assert L.svdq_scale_offset(100, 0, 0, ctypes.byref(out)) == 2
+    assert L.svdq_scale_offset(256, -1, 0, ctypes.byref(out)) == 1
+    assert L.svdq_scale_offset(256, 0, 16, ctypes.byref(out)) == 1
+    assert L.svdq_scale_offset(256, 0, 0, None) == 1
+
+
+def test_sizes(L):
+    assert _lib.svdq_weight_sizes(256, 512, 32) == (256 * 256, 256 * 32, 32 * 512 * 2, 256 * 32 * 2)
+    assert _lib.svdq_act_sizes(129, 512, 16) == (129 * 256, 256 * 32, 129 * 16 * 2)
+    ws = _lib.svdq_forward_workspace_size(129, 512, 16)
+    assert ws >= sum(_lib.svdq_act_sizes(129, 512, 16))
+    with pytest.raises(_lib.SvdqError):
+        _lib.svdq_weight_sizes(100, 512, 32)      # N % 128
+    with pytest.raises(_lib.SvdqError):
+        _lib.svdq_weight_sizes(128, 500, 32)      # K % 256
+    with pytest.raises(_lib.SvdqError):
+        _lib.svdq_weight_sizes(128, 512, 24)      # rank
+
+
+def test_validation_happens_before_device_checks(L):
+    p = ctypes.c_void_p(0x10000)          # never dereferenced: validation fails first
+    odd = ctypes.c_void_p(0x10008)
+    # bad K
+    assert L.svdq_quantize_act(4, 100, 32, p, 100, 1.0, p, p, p, p, None) == 2
+    # null pointer
+    assert L.svdq_quantize_act(4, 256, 32, None, 256, 1.0, p, p, p, p, None) == 1
+    # misaligned pointer
+    assert L.svdq_quantize_act(4, 256, 32, odd, 256, 1.0, p, p, p, p, None) == 3
+    # bad leading dimension
+    assert L.svdq_w4a4_gemm(4, 128, 256, 32, p, p, p, 1.0, p, p, p, p, None, p, 100, None) == 2
+    # workspace too small
+    assert L.svdq_linear_forward(4, 128, 256, 32, p, 256, 1.0, p, p, p, p, p, None, p, 128, p, 16, None) == 7
+    # M == 0 is a valid no-op
+    assert L.svdq_w4a4_gemm(0, 128, 256, 32, None, None, None, 1.0, None, None, None, None, None, None, 128,
+                            None) == 0
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU path")
+def test_no_gpu_is_unsupported_device(L):
+    p = ctypes.c_void_p(0x10000)
+    assert L.svdq_quantize_act(4, 256, 32, p, 256, 1.0, p, p, p, p, None) == 4
+    assert L.svdq_pack_weight(128, 256, 32, p, p, p, p, p, p, p, p, None) == 4
+    code = ctypes.c_int()
+    assert L.svdq_read_device_error(ctypes.byref(code), 0) == 4
+
+
+def test_ulp_helper():
+    a = np.array([1.0, 1.0, -1.0, 0.0])
+    b = np.array([1.0 + 2 ** -7, 1.0, -1.0 - 2 ** -7, -0.0])
+    assert layouts.bf16_ulp_distance(a, b).tolist() == [1, 0, 1, 0]

@@ -1,0 +1,162 @@
+"""GPU parity: the CUDA path through the C ABI against the float64 CPU oracle.
+
+Bars (from the layer's acceptance criteria):
+  * activation codes and scales, packed weight codes / scales / g_w: bit-exact;
+  * XL1: within 1 bf16 ulp (fp32 tensor-core accumulation vs float64);
+  * Y: relative Frobenius error <= 1e-3 against the oracle output rounded to
+    bf16, and max |Y - y64| <= 2e-2 * RMS of the y64 row.
+Inputs come from the seeded generators in workloads.py; the oracle computes
+the expected values; nothing flows from the GPU into the oracle.
+"""
+import numpy as np
+import pytest
+import torch
+
+import workloads
+from oracle import nvfp4, svdq as osv
+from tests import layouts
+
+pytestmark = pytest.mark.gpu
+
+REL_FRO = 1e-3
+MAX_ROWRMS = 2e-2
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from w4a4_rank_corrected_svdq_b200 import _lib, build
+    build.build()
+    return _lib
+
+
+def _bf16_np(t):
+    return t.detach().to(torch.float64).cpu().numpy()
+
+
+def _to_dev(a64):
+    return torch.from_numpy(np.ascontiguousarray(a64)).to(torch.bfloat16).cuda()
+
+
+def _layer(M, K, N, r, seed=7, bias=True):
+    spec, (X, W, b) = workloads.small_layer(M, K, N, r, seed=seed, bias_std=0.01 if bias else 0.0)
+    L1, L2, _ = osv.lowrank_factors(W, r)
+    return X, W, b, L1, L2
+
+
+def _check_act(lib, X, L1, r, g_x, qa, M, K):
+    ref = osv.quantize_act(X, g_x)
+    codes = layouts.unpack_codes(qa.codes.cpu().numpy(), M, K)
+    scales_buf = qa.scales.cpu().numpy()
+    scales = layouts.untile_scales(scales_buf, M, K)
+    assert np.array_equal(codes, ref[0]), f"codes differ at {np.argwhere(codes != ref[0])[:5]}"
+    assert np.array_equal(scales, ref[1]), f"scales differ at {np.argwhere(scales != ref[1])[:5]}"
+    mpad = (M + 127) // 128 * 128
+    if mpad > M:   # padding rows must hold zero scales
+        pad = layouts.untile_scales(scales_buf, mpad, K)[M:]
+        assert not pad.any()
+    xl1_ref = osv.down_proj(X, L1)
+    ulps = layouts.bf16_ulp_distance(_bf16_np(qa.xl1), xl1_ref)
+    assert ulps.max() <= 1, f"XL1 max ulp {ulps.max()}"
+
+
+def _check_y(Y, fwd, rows=None):
+    y = _bf16_np(Y)
+    if rows is not None:
+        y = y[rows]
+    rel = osv.rel_fro(y, fwd.y_ref)
+    mx = osv.max_abs_over_row_rms(y, fwd.y64)
+    assert rel <= REL_FRO, f"rel Frobenius {rel:.3e}"
+    assert mx <= MAX_ROWRMS, f"max |err| / row-RMS {mx:.3e}"
+    return rel, mx
+
+
+# ------------------------------------------------------------------ calibration
+def test_act_global_scale_bitexact(lib):
+    X, *_ = _layer(300, 512, 128, 16)
+    g = lib.svdq_act_global_scale(X.cuda()).item()
+    assert np.float32(g) == osv.act_global_scale(X)
+
+
+# ------------------------------------------------------------------ activation kernel
+@pytest.mark.parametrize("M,K,r", [(256, 1024, 32), (1, 256, 16), (127, 512, 32), (129, 512, 64),
+                                   (300, 768, 128), (64, 4096, 32), (1000, 256, 16)])
+def test_quantize_act_bitexact(lib, M, K, r):
+    X, W, b, L1, L2 = _layer(M, K, 128, r)
+    g_x = osv.act_global_scale(X)
+    pw = lib.PackedWeight(128, K, r, "cuda")
+    pw.l1t.copy_(_to_dev(L1.T))
+    qa = lib.svdq_quantize_act(X.cuda(), float(g_x), pw)
+    torch.cuda.synchronize()
+    _check_act(lib, X, L1, r, g_x, qa, M, K)
+
+
+def test_quantize_act_zero_rows_and_strided_input(lib):
+    M, K, r = 130, 512, 32
+    X, W, b, L1, L2 = _layer(M, K, 128, r)
+    X = X.clone()
+    X[3] = 0
+    X[7, 16:48] = 0
+    big = torch.zeros((M, K + 64), dtype=torch.bfloat16)
+    big[:, :K] = X
+    g_x = osv.act_global_scale(X)
+    pw = lib.PackedWeight(128, K, r, "cuda")
+    pw.l1t.copy_(_to_dev(L1.T))
+    qa = lib.svdq_quantize_act(big.cuda()[:, :K], float(g_x), pw)
+    torch.cuda.synchronize()
+    _check_act(lib, X, L1, r, g_x, qa, M, K)
+
+
+# ------------------------------------------------------------------ weight packing
+@pytest.mark.parametrize("N,K,r", [(128, 256, 16), (256, 512, 32), (384, 1024, 64), (256, 512, 128)])
+def test_pack_weight_bitexact(lib, N, K, r):
+    X, W, b, L1, L2 = _layer(8, K, N, r)
+    pw = lib.svdq_pack_weight(W.cuda(), _to_dev(L1), _to_dev(L2))
+    torch.cuda.synchronize()
+    ref = osv.pack_weight(W, L1, L2)
+    codes = layouts.unpack_codes(pw.codes.cpu().numpy(), N, K)
+    scales = layouts.untile_scales(pw.scales.cpu().numpy(), N, K)
+    assert np.float32(pw.g_w.item()) == ref.g_w
+    assert np.array_equal(scales, ref.scales)
+    assert np.array_equal(codes, ref.codes)
+    assert np.array_equal(_bf16_np(pw.l1t), L1.T)
+    assert np.array_equal(_bf16_np(pw.l2t), L2.T)
+
+
+# ------------------------------------------------------------------ full layer
+@pytest.mark.parametrize("M,K,N,r,bias", [(256, 1024, 1024, 32, True), (1, 256, 128, 16, True),
+                                          (129, 512, 384, 64, False), (300, 768, 256, 128, True),
+                                          (517, 1280, 640, 32, True)])
+def test_linear_forward_parity(lib, M, K, N, r, bias):
+    X, W, b, L1, L2 = _layer(M, K, N, r, bias=bias)
+    g_x = osv.act_global_scale(X)
+    pw = lib.svdq_pack_weight(W.cuda(), _to_dev(L1), _to_dev(L2))
+    Y = lib.svdq_linear_forward(X.cuda(), float(g_x), pw, b.cuda() if bias else None)
+    torch.cuda.synchronize()
+    assert lib.svdq_read_device_error() == 0
+    fwd = osv.forward(X, osv.pack_weight(W, L1, L2), b if bias else None, g_x)
+    _check_y(Y, fwd)
+
+
+def test_linear_forward_config1(lib):
+    spec = workloads.WORKLOADS[1].layers[0]
+    X, W, b = workloads.make_layer(spec)
+    L1, L2, _ = osv.lowrank_factors(W, spec.r)
+    g_x = osv.act_global_scale(X)
+    pw = lib.svdq_pack_weight(W.cuda(), _to_dev(L1), _to_dev(L2))
+    qa = lib.svdq_quantize_act(X.cuda(), float(g_x), pw)
+    Y = lib.svdq_w4a4_gemm(qa, float(g_x), pw, b.cuda())
+    torch.cuda.synchronize()
+    _check_act(lib, X, L1, spec.r, g_x, qa, spec.M, spec.K)
+    fwd = osv.forward(X, osv.pack_weight(W, L1, L2), b, g_x)
+    _check_y(Y, fwd)
+    # deterministic: a second call gives identical bits
+    Y2 = lib.svdq_linear_forward(X.cuda(), float(g_x), pw, b.cuda())
+    torch.cuda.synchronize()
+    assert torch.equal(Y, Y2)
+
+
+def test_m_zero_is_noop(lib):
+    pw = lib.PackedWeight(128, 256, 16, "cuda")
+    X = torch.empty((0, 256), dtype=torch.bfloat16, device="cuda")
+    Y = lib.svdq_linear_forward(X, 1.0, pw)
+    assert Y.shape == (0, 128)

@@ -1,0 +1,23 @@
+"""B200 (sm_100a) SVDQuant W4A4 NVFP4 linear layer.
+
+Y = (X . L1) . L2 + Q4(X) . Q4(R)^T + b with a rank-r bf16 low-rank branch and
+an NVFP4 residual R = W - (L1 . L2)^T (blog "Bringing Nunchaku 4-bit Diffusion
+Inference to Diffusers"). The work runs in hand-written CUDA kernels behind
+the C ABI of include/svdq.h; this package is its ctypes binding.
+"""
+from ._lib import (  # noqa: F401
+    PackedWeight,
+    QuantAct,
+    SvdqError,
+    lib,
+    svdq_act_global_scale,
+    svdq_act_sizes,
+    svdq_forward_workspace_size,
+    svdq_linear_forward,
+    svdq_pack_weight,
+    svdq_quantize_act,
+    svdq_read_device_error,
+    svdq_scale_offset,
+    svdq_w4a4_gemm,
+    svdq_weight_sizes,
+)

@@ -1,0 +1,219 @@
+"""ctypes binding of libsvdq.so (the C ABI in include/svdq.h).
+
+Argument marshalling only: every function here checks tensor dtypes, shapes,
+devices and contiguity, passes raw device pointers and the current CUDA
+stream to the C function of the same name, and raises SvdqError on a non-OK
+status. No arithmetic of the layer happens in Python, and there is no
+fallback: if the library cannot be loaded, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libsvdq.so")
+
+STATUS = {
+    0: "SVDQ_OK", 1: "SVDQ_ERR_INVALID_ARG", 2: "SVDQ_ERR_UNSUPPORTED_SHAPE", 3: "SVDQ_ERR_MISALIGNED",
+    4: "SVDQ_ERR_UNSUPPORTED_DEVICE", 5: "SVDQ_ERR_CUDA", 6: "SVDQ_ERR_TIMEOUT", 7: "SVDQ_ERR_WORKSPACE",
+}
+
+# (name, restype, argtypes) for every symbol declared in include/svdq.h
+_i, _i64, _f, _p, _sz = ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_void_p, ctypes.c_size_t
+_psz, _pi = ctypes.POINTER(ctypes.c_size_t), ctypes.POINTER(ctypes.c_int)
+SIGNATURES = {
+    "svdq_status_string": (ctypes.c_char_p, [_i]),
+    "svdq_version": (_i, []),
+    "svdq_scale_offset": (_i, [_i, _i, _i, _psz]),
+    "svdq_weight_sizes": (_i, [_i, _i, _i, _psz, _psz, _psz, _psz]),
+    "svdq_act_sizes": (_i, [_i, _i, _i, _psz, _psz, _psz]),
+    "svdq_forward_workspace_size": (_i, [_i, _i, _i, _psz]),
+    "svdq_pack_weight": (_i, [_i, _i, _i, _p, _p, _p, _p, _p, _p, _p, _p, _p]),
+    "svdq_act_global_scale": (_i, [_i, _i, _p, _i64, _p, _p]),
+    "svdq_quantize_act": (_i, [_i, _i, _i, _p, _i64, _f, _p, _p, _p, _p, _p]),
+    "svdq_w4a4_gemm": (_i, [_i, _i, _i, _i, _p, _p, _p, _f, _p, _p, _p, _p, _p, _p, _i64, _p]),
+    "svdq_linear_forward": (_i, [_i, _i, _i, _i, _p, _i64, _f, _p, _p, _p, _p, _p, _p, _p, _i64, _p, _sz, _p]),
+    "svdq_read_device_error": (_i, [_pi, _i]),
+}
+
+
+class SvdqError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn} failed: {STATUS.get(status, status)}")
+        self.status = status
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libsvdq.so (built in-tree by build.py); raises if it is missing."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libsvdq.so not built ({LIB_PATH}); run python -m w4a4_rank_corrected_svdq_b200.build")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _check(name: str, status: int) -> None:
+    if status != 0:
+        raise SvdqError(name, status)
+
+
+def _stream(t: torch.Tensor | None = None):
+    dev = t.device if t is not None else torch.device("cuda")
+    return ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+
+
+def _ptr(t: torch.Tensor | None):
+    return ctypes.c_void_p(0 if t is None else t.data_ptr())
+
+
+def _dev(t: torch.Tensor, name: str, dtype=None, shape=None):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    return t
+
+
+def _rows(t: torch.Tensor, name: str, cols: int) -> int:
+    """Leading dimension (elements) of a 2-D tensor with unit column stride."""
+    if t.dim() != 2 or t.shape[1] != cols or t.stride(1) != 1:
+        raise ValueError(f"{name} must be 2-D [rows, {cols}] with unit column stride")
+    return t.stride(0)
+
+
+# ------------------------------------------------------------------ sizes
+def svdq_scale_offset(K: int, row: int, kblock: int) -> int:
+    out = ctypes.c_size_t()
+    _check("svdq_scale_offset", lib().svdq_scale_offset(K, row, kblock, ctypes.byref(out)))
+    return out.value
+
+
+def svdq_weight_sizes(N: int, K: int, r: int):
+    a, b, c, d = (ctypes.c_size_t() for _ in range(4))
+    _check("svdq_weight_sizes", lib().svdq_weight_sizes(N, K, r, *(ctypes.byref(x) for x in (a, b, c, d))))
+    return a.value, b.value, c.value, d.value
+
+
+def svdq_act_sizes(M: int, K: int, r: int):
+    a, b, c = (ctypes.c_size_t() for _ in range(3))
+    _check("svdq_act_sizes", lib().svdq_act_sizes(M, K, r, *(ctypes.byref(x) for x in (a, b, c))))
+    return a.value, b.value, c.value
+
+
+def svdq_forward_workspace_size(M: int, K: int, r: int) -> int:
+    out = ctypes.c_size_t()
+    _check("svdq_forward_workspace_size", lib().svdq_forward_workspace_size(M, K, r, ctypes.byref(out)))
+    return out.value
+
+
+# ------------------------------------------------------------------ packed weight
+class PackedWeight:
+    """Device buffers of one packed layer (allocated by torch, filled by svdq_pack_weight)."""
+
+    def __init__(self, N: int, K: int, r: int, device):
+        cb, sb, lb1, lb2 = svdq_weight_sizes(N, K, r)
+        self.N, self.K, self.r = N, K, r
+        self.codes = torch.empty(cb, dtype=torch.uint8, device=device)
+        self.scales = torch.empty(sb, dtype=torch.uint8, device=device)
+        self.g_w = torch.empty(1, dtype=torch.float32, device=device)
+        self.l1t = torch.empty((r, K), dtype=torch.bfloat16, device=device)
+        self.l2t = torch.empty((N, r), dtype=torch.bfloat16, device=device)
+
+
+def svdq_pack_weight(W: torch.Tensor, L1: torch.Tensor, L2: torch.Tensor, out: PackedWeight | None = None):
+    N, K = W.shape
+    r = L1.shape[1]
+    _dev(W, "W", torch.bfloat16)
+    _dev(L1, "L1", torch.bfloat16, (K, r))
+    _dev(L2, "L2", torch.bfloat16, (r, N))
+    for t, n in ((W, "W"), (L1, "L1"), (L2, "L2")):
+        if not t.is_contiguous():
+            raise ValueError(f"{n} must be contiguous")
+    pw = out if out is not None else PackedWeight(N, K, r, W.device)
+    _check("svdq_pack_weight", lib().svdq_pack_weight(
+        N, K, r, _ptr(W), _ptr(L1), _ptr(L2), _ptr(pw.codes), _ptr(pw.scales), _ptr(pw.g_w), _ptr(pw.l1t),
+        _ptr(pw.l2t), _stream(W)))
+    return pw
+
+
+def svdq_act_global_scale(X: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
+    _dev(X, "X", torch.bfloat16)
+    M, K = X.shape
+    ldx = _rows(X, "X", K)
+    g = out if out is not None else torch.empty(1, dtype=torch.float32, device=X.device)
+    _check("svdq_act_global_scale", lib().svdq_act_global_scale(M, K, _ptr(X), ldx, _ptr(g), _stream(X)))
+    return g
+
+
+# ------------------------------------------------------------------ per call
+class QuantAct:
+    def __init__(self, M: int, K: int, r: int, device):
+        cb, sb, xb = svdq_act_sizes(M, K, r)
+        self.M, self.K, self.r = M, K, r
+        self.codes = torch.empty(cb, dtype=torch.uint8, device=device)
+        self.scales = torch.empty(sb, dtype=torch.uint8, device=device)
+        self.xl1 = torch.empty((M, r), dtype=torch.bfloat16, device=device)
+
+
+def svdq_quantize_act(X: torch.Tensor, g_x: float, pw: PackedWeight, out: QuantAct | None = None) -> QuantAct:
+    _dev(X, "X", torch.bfloat16)
+    M, K = X.shape
+    ldx = _rows(X, "X", K)
+    qa = out if out is not None else QuantAct(M, K, pw.r, X.device)
+    _check("svdq_quantize_act", lib().svdq_quantize_act(
+        M, K, pw.r, _ptr(X), ldx, float(g_x), _ptr(pw.l1t), _ptr(qa.codes), _ptr(qa.scales), _ptr(qa.xl1),
+        _stream(X)))
+    return qa
+
+
+def svdq_w4a4_gemm(qa: QuantAct, g_x: float, pw: PackedWeight, bias: torch.Tensor | None = None,
+                   out: torch.Tensor | None = None) -> torch.Tensor:
+    M, N, K, r = qa.M, pw.N, pw.K, pw.r
+    if bias is not None:
+        _dev(bias, "bias", torch.bfloat16, (N,))
+    Y = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=qa.codes.device)
+    _dev(Y, "Y", torch.bfloat16)
+    ldy = _rows(Y, "Y", N)
+    _check("svdq_w4a4_gemm", lib().svdq_w4a4_gemm(
+        M, N, K, r, _ptr(qa.codes), _ptr(qa.scales), _ptr(qa.xl1), float(g_x), _ptr(pw.codes), _ptr(pw.scales),
+        _ptr(pw.g_w), _ptr(pw.l2t), _ptr(bias), _ptr(Y), ldy, _stream(Y)))
+    return Y
+
+
+def svdq_linear_forward(X: torch.Tensor, g_x: float, pw: PackedWeight, bias: torch.Tensor | None = None,
+                        out: torch.Tensor | None = None, workspace: torch.Tensor | None = None) -> torch.Tensor:
+    _dev(X, "X", torch.bfloat16)
+    M, K = X.shape
+    N, r = pw.N, pw.r
+    ldx = _rows(X, "X", K)
+    if bias is not None:
+        _dev(bias, "bias", torch.bfloat16, (N,))
+    Y = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=X.device)
+    _dev(Y, "Y", torch.bfloat16)
+    ldy = _rows(Y, "Y", N)
+    need = svdq_forward_workspace_size(M, K, r)
+    ws = workspace if workspace is not None else torch.empty(max(need, 16), dtype=torch.uint8, device=X.device)
+    _check("svdq_linear_forward", lib().svdq_linear_forward(
+        M, N, K, r, _ptr(X), ldx, float(g_x), _ptr(pw.codes), _ptr(pw.scales), _ptr(pw.g_w), _ptr(pw.l1t),
+        _ptr(pw.l2t), _ptr(bias), _ptr(Y), ldy, _ptr(ws), ws.numel(), _stream(X)))
+    return Y
+
+
+def svdq_read_device_error(clear: bool = True) -> int:
+    code = ctypes.c_int()
+    _check("svdq_read_device_error", lib().svdq_read_device_error(ctypes.byref(code), int(clear)))
+    return code.value

@@ -1,0 +1,426 @@
+// svdq_api.cu — the C ABI (include/svdq.h): argument validation, device
+// checks, tensor-map encoding and kernel launches. One translation unit holds
+// every kernel so the per-device error word is a single symbol.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/svdq.h"
+#include "gemm_w4a4.cuh"
+#include "pack_weight.cuh"
+#include "quantize_act.cuh"
+
+namespace svdq {
+namespace {
+
+constexpr int kVersion = 100;  // 0.1.0
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool valid_rank(int r) { return r == 16 || r == 32 || r == 64 || r == 128; }
+size_t round_up(size_t x, size_t m) { return (x + m - 1) / m * m; }
+
+// ------------------------------------------------------------------ device checks
+struct DeviceInfo {
+  int sm_count = 0;
+  int ok = -1;  // -1 unknown, 0 unsupported, 1 supported
+};
+constexpr int kMaxDevices = 64;
+DeviceInfo g_devices[kMaxDevices];
+std::mutex g_dev_mutex;
+
+svdq_status current_device(int* dev_out, DeviceInfo* info_out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return SVDQ_ERR_UNSUPPORTED_DEVICE;
+  }
+  if (dev < 0 || dev >= kMaxDevices) return SVDQ_ERR_UNSUPPORTED_DEVICE;
+  std::lock_guard<std::mutex> lock(g_dev_mutex);
+  DeviceInfo& di = g_devices[dev];
+  if (di.ok < 0) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+      cudaGetLastError();
+      return SVDQ_ERR_UNSUPPORTED_DEVICE;
+    }
+    di.sm_count = sms;
+    di.ok = (major == 10 && minor == 0) ? 1 : 0;
+  }
+  if (di.ok != 1) return SVDQ_ERR_UNSUPPORTED_DEVICE;
+  if (dev_out) *dev_out = dev;
+  if (info_out) *info_out = di;
+  return SVDQ_OK;
+}
+
+// cudaFuncSetAttribute for the dynamic shared memory size, once per (kernel, device).
+template <typename Kernel>
+void ensure_smem_attr(Kernel kern, int bytes, std::atomic<uint64_t>& done) {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const uint64_t bit = 1ull << (dev & 63);
+  if (done.load(std::memory_order_acquire) & bit) return;
+  cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  done.fetch_or(bit, std::memory_order_acq_rel);
+}
+
+svdq_status launch_status() {
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    std::fprintf(stderr, "svdq: CUDA error: %s\n", cudaGetErrorString(e));
+    return SVDQ_ERR_CUDA;
+  }
+  return SVDQ_OK;
+}
+
+// ------------------------------------------------------------------ tensor maps
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+    else
+      cudaGetLastError();
+  });
+  return fn;
+}
+
+// 2-D row-major tensor [rows][cols] of `elem_bytes` elements, row pitch `pitch_bytes`.
+bool make_tmap_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int elem_bytes, uint64_t cols,
+                  uint64_t rows, uint64_t pitch_bytes, uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle sw) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  (void)elem_bytes;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {pitch_bytes};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+CUtensorMapSwizzle lr_swizzle(int r) {
+  const int row_bytes = (r < 64 ? r : 64) * 2;
+  return row_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                          : (row_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
+}
+
+// ------------------------------------------------------------------ launches
+template <int R>
+svdq_status launch_quantize(int M, int K, const void* X, int64_t ldx, float g_x, const void* l1t, void* codes,
+                            void* scales, void* xl1, cudaStream_t stream, int sm_count) {
+  const int row_tiles = (M + kQuantRows - 1) / kQuantRows;
+  int ks = 1;
+  while (ks < 8 && row_tiles * ks < 2 * sm_count && (K / (2 * ks)) % 32 == 0 && K / (2 * ks) >= 128) ks *= 2;
+  const int kchunk = K / ks;
+  const size_t smem = static_cast<size_t>(kQuantRows) * R * sizeof(float);
+  auto kern = quantize_act_kernel<R>;
+  static std::atomic<uint64_t> attr_done{0};
+  ensure_smem_attr(kern, static_cast<int>(smem), attr_done);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(ks, row_tiles, 1);
+  cfg.blockDim = dim3(kQuantThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = ks;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaLaunchKernelEx(&cfg, kern, static_cast<const __nv_bfloat16*>(X), ldx, M, K, g_x,
+                     static_cast<const __nv_bfloat16*>(l1t), static_cast<uint8_t*>(codes),
+                     static_cast<uint8_t*>(scales), static_cast<__nv_bfloat16*>(xl1), kchunk);
+  return launch_status();
+}
+
+svdq_status quantize_dispatch(int M, int K, int r, const void* X, int64_t ldx, float g_x, const void* l1t,
+                              void* codes, void* scales, void* xl1, cudaStream_t st, int sms) {
+  switch (r) {
+    case 16: return launch_quantize<16>(M, K, X, ldx, g_x, l1t, codes, scales, xl1, st, sms);
+    case 32: return launch_quantize<32>(M, K, X, ldx, g_x, l1t, codes, scales, xl1, st, sms);
+    case 64: return launch_quantize<64>(M, K, X, ldx, g_x, l1t, codes, scales, xl1, st, sms);
+    default: return launch_quantize<128>(M, K, X, ldx, g_x, l1t, codes, scales, xl1, st, sms);
+  }
+}
+
+template <int R>
+svdq_status launch_gemm(int M, int N, int K, const void* a_codes, const void* a_scales, const void* xl1, float g_x,
+                        const void* w_codes, const void* w_scales, const float* g_w, const void* l2t,
+                        const void* bias, void* Y, int64_t ldy, cudaStream_t stream, int sm_count) {
+  using C = GemmCfg<R>;
+  CUtensorMap tm_a, tm_b, tm_x, tm_l;
+  const uint64_t kb = static_cast<uint64_t>(K / 2);
+  if (!make_tmap_2d(&tm_a, a_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, kb, M, kb, kBKBytes, kBM,
+                    CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_tmap_2d(&tm_b, w_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, kb, N, kb, kBKBytes, kBN,
+                    CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_tmap_2d(&tm_x, xl1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, R, M, R * 2, C::kLrAtomCols, kBM,
+                    lr_swizzle(R)) ||
+      !make_tmap_2d(&tm_l, l2t, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, R, N, R * 2, C::kLrAtomCols, kBN,
+                    lr_swizzle(R)))
+    return SVDQ_ERR_CUDA;
+  auto kern = w4a4_gemm_kernel<R>;
+  static std::atomic<uint64_t> attr_done{0};
+  ensure_smem_attr(kern, C::kSmemBytes, attr_done);
+  const int tiles = ((M + kBM - 1) / kBM) * (N / kBN);
+  const int grid = tiles < sm_count ? tiles : sm_count;
+  kern<<<grid, kGemmThreads, C::kSmemBytes, stream>>>(
+      tm_a, tm_b, tm_x, tm_l, static_cast<const uint8_t*>(a_scales), static_cast<const uint8_t*>(w_scales), g_x, g_w,
+      static_cast<const __nv_bfloat16*>(bias), static_cast<__nv_bfloat16*>(Y), ldy, M, N, K);
+  return launch_status();
+}
+
+svdq_status gemm_dispatch(int M, int N, int K, int r, const void* a_codes, const void* a_scales, const void* xl1,
+                          float g_x, const void* w_codes, const void* w_scales, const float* g_w, const void* l2t,
+                          const void* bias, void* Y, int64_t ldy, cudaStream_t st, int sms) {
+  switch (r) {
+    case 16:
+      return launch_gemm<16>(M, N, K, a_codes, a_scales, xl1, g_x, w_codes, w_scales, g_w, l2t, bias, Y, ldy, st, sms);
+    case 32:
+      return launch_gemm<32>(M, N, K, a_codes, a_scales, xl1, g_x, w_codes, w_scales, g_w, l2t, bias, Y, ldy, st, sms);
+    case 64:
+      return launch_gemm<64>(M, N, K, a_codes, a_scales, xl1, g_x, w_codes, w_scales, g_w, l2t, bias, Y, ldy, st, sms);
+    default:
+      return launch_gemm<128>(M, N, K, a_codes, a_scales, xl1, g_x, w_codes, w_scales, g_w, l2t, bias, Y, ldy, st,
+                              sms);
+  }
+}
+
+// amax|X| over an M x K bf16 matrix with row pitch ldx -> *g as fp32 bits.
+__global__ void act_amax_kernel(const __nv_bfloat16* __restrict__ X, int64_t ldx, int M, int K, unsigned* bits) {
+  float am = 0.0f;
+  const int vec_per_row = K / 8;
+  const int64_t total = static_cast<int64_t>(M) * vec_per_row;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t row = i / vec_per_row;
+    const int col = static_cast<int>(i % vec_per_row) * 8;
+    float f[8];
+    bf16x8_to_f32(ldg_nc_v4(X + row * ldx + col), f);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) am = fmaxf(am, fabsf(f[j]));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
+  if ((threadIdx.x & 31) == 0) atomicMax(bits, __float_as_uint(am));
+}
+
+template <int R>
+svdq_status launch_pack(int N, int K, const void* W, const void* L1, const void* l2t, void* codes, void* scales,
+                        float* g_w, cudaStream_t st) {
+  const int warps = (K / 32) * ((N + kPackRowsPerWarp - 1) / kPackRowsPerWarp);
+  const int blocks = (warps + kPackThreads / 32 - 1) / (kPackThreads / 32);
+  if (cudaMemsetAsync(g_w, 0, sizeof(float), st) != cudaSuccess) return launch_status();
+  residual_amax_kernel<R><<<blocks, kPackThreads, 0, st>>>(static_cast<const __nv_bfloat16*>(W),
+                                                           static_cast<const __nv_bfloat16*>(L1),
+                                                           static_cast<const __nv_bfloat16*>(l2t), N, K,
+                                                           reinterpret_cast<unsigned*>(g_w));
+  finalize_global_scale_kernel<<<1, 1, 0, st>>>(g_w);
+  residual_quant_kernel<R><<<blocks, kPackThreads, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(W), static_cast<const __nv_bfloat16*>(L1),
+      static_cast<const __nv_bfloat16*>(l2t), N, K, g_w, static_cast<uint8_t*>(codes), static_cast<uint8_t*>(scales));
+  return launch_status();
+}
+
+svdq_status check_layer_shape(int N, int K, int r) {
+  if (N <= 0 || K <= 0 || !valid_rank(r)) return SVDQ_ERR_INVALID_ARG;
+  if (K % 256 != 0 || N % 128 != 0) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+  return SVDQ_OK;
+}
+
+}  // namespace
+}  // namespace svdq
+
+using namespace svdq;
+
+extern "C" {
+
+const char* svdq_status_string(int status) {
+  switch (status) {
+    case SVDQ_OK: return "SVDQ_OK";
+    case SVDQ_ERR_INVALID_ARG: return "SVDQ_ERR_INVALID_ARG";
+    case SVDQ_ERR_UNSUPPORTED_SHAPE: return "SVDQ_ERR_UNSUPPORTED_SHAPE";
+    case SVDQ_ERR_MISALIGNED: return "SVDQ_ERR_MISALIGNED";
+    case SVDQ_ERR_UNSUPPORTED_DEVICE: return "SVDQ_ERR_UNSUPPORTED_DEVICE";
+    case SVDQ_ERR_CUDA: return "SVDQ_ERR_CUDA";
+    case SVDQ_ERR_TIMEOUT: return "SVDQ_ERR_TIMEOUT";
+    case SVDQ_ERR_WORKSPACE: return "SVDQ_ERR_WORKSPACE";
+    default: return "SVDQ_ERR_UNKNOWN";
+  }
+}
+
+int svdq_version(void) { return kVersion; }
+
+svdq_status svdq_scale_offset(int K, int row, int kblock, size_t* out) {
+  if (out == nullptr || row < 0 || K <= 0 || kblock < 0) return SVDQ_ERR_INVALID_ARG;
+  if (K % 64 != 0) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+  if (kblock >= K / 16) return SVDQ_ERR_INVALID_ARG;
+  *out = scale_offset(K, row, kblock);
+  return SVDQ_OK;
+}
+
+svdq_status svdq_weight_sizes(int N, int K, int r, size_t* codes_bytes, size_t* scales_bytes, size_t* l1t_bytes,
+                              size_t* l2t_bytes) {
+  const svdq_status s = check_layer_shape(N, K, r);
+  if (s != SVDQ_OK) return s;
+  if (!codes_bytes || !scales_bytes || !l1t_bytes || !l2t_bytes) return SVDQ_ERR_INVALID_ARG;
+  *codes_bytes = static_cast<size_t>(N) * (K / 2);
+  *scales_bytes = static_cast<size_t>(N) * (K / 16);
+  *l1t_bytes = static_cast<size_t>(r) * K * 2;
+  *l2t_bytes = static_cast<size_t>(N) * r * 2;
+  return SVDQ_OK;
+}
+
+svdq_status svdq_act_sizes(int M, int K, int r, size_t* codes_bytes, size_t* scales_bytes, size_t* xl1_bytes) {
+  if (M < 0 || K <= 0 || !valid_rank(r) || !codes_bytes || !scales_bytes || !xl1_bytes) return SVDQ_ERR_INVALID_ARG;
+  if (K % 256 != 0) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+  *codes_bytes = static_cast<size_t>(M) * (K / 2);
+  *scales_bytes = round_up(static_cast<size_t>(M), 128) * (K / 16);
+  *xl1_bytes = static_cast<size_t>(M) * r * 2;
+  return SVDQ_OK;
+}
+
+svdq_status svdq_forward_workspace_size(int M, int K, int r, size_t* bytes) {
+  size_t c, s, x;
+  const svdq_status st = svdq_act_sizes(M, K, r, &c, &s, &x);
+  if (st != SVDQ_OK) return st;
+  if (!bytes) return SVDQ_ERR_INVALID_ARG;
+  *bytes = round_up(c, 256) + round_up(s, 256) + round_up(x, 256);
+  return SVDQ_OK;
+}
+
+svdq_status svdq_pack_weight(int N, int K, int r, const void* W, const void* L1, const void* L2, void* w_codes,
+                             void* w_scales, float* g_w, void* l1t, void* l2t, void* stream) {
+  svdq_status s = check_layer_shape(N, K, r);
+  if (s != SVDQ_OK) return s;
+  if (!W || !L1 || !L2 || !w_codes || !w_scales || !g_w || !l1t || !l2t) return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(W) || !aligned16(L1) || !aligned16(L2) || !aligned16(w_codes) || !aligned16(w_scales) ||
+      !aligned16(l1t) || !aligned16(l2t) || (reinterpret_cast<uintptr_t>(g_w) & 3u))
+    return SVDQ_ERR_MISALIGNED;
+  DeviceInfo di;
+  if ((s = current_device(nullptr, &di)) != SVDQ_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // l2t = L2^T (N x r), l1t = L1^T (r x K)
+  transpose_bf16_kernel<<<dim3((N + 31) / 32, (r + 31) / 32), 256, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(L2), static_cast<__nv_bfloat16*>(l2t), r, N);
+  transpose_bf16_kernel<<<dim3((r + 31) / 32, (K + 31) / 32), 256, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(L1), static_cast<__nv_bfloat16*>(l1t), K, r);
+  if ((s = launch_status()) != SVDQ_OK) return s;
+  switch (r) {
+    case 16: return launch_pack<16>(N, K, W, L1, l2t, w_codes, w_scales, g_w, st);
+    case 32: return launch_pack<32>(N, K, W, L1, l2t, w_codes, w_scales, g_w, st);
+    case 64: return launch_pack<64>(N, K, W, L1, l2t, w_codes, w_scales, g_w, st);
+    default: return launch_pack<128>(N, K, W, L1, l2t, w_codes, w_scales, g_w, st);
+  }
+}
+
+svdq_status svdq_act_global_scale(int M, int K, const void* X, int64_t ldx, float* g_out, void* stream) {
+  if (M < 0 || K <= 0 || !X || !g_out) return SVDQ_ERR_INVALID_ARG;
+  if (K % 8 != 0 || ldx < K || ldx % 8 != 0) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(X) || (reinterpret_cast<uintptr_t>(g_out) & 3u)) return SVDQ_ERR_MISALIGNED;
+  svdq_status s;
+  DeviceInfo di;
+  if ((s = current_device(nullptr, &di)) != SVDQ_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(g_out, 0, sizeof(float), st) != cudaSuccess) return launch_status();
+  if (M > 0) {
+    const int64_t vecs = static_cast<int64_t>(M) * (K / 8);
+    int64_t blocks = (vecs + 255) / 256;
+    if (blocks > 8 * di.sm_count) blocks = 8 * di.sm_count;
+    act_amax_kernel<<<static_cast<int>(blocks), 256, 0, st>>>(static_cast<const __nv_bfloat16*>(X), ldx, M, K,
+                                                                reinterpret_cast<unsigned*>(g_out));
+  }
+  finalize_global_scale_kernel<<<1, 1, 0, st>>>(g_out);
+  return launch_status();
+}
+
+svdq_status svdq_quantize_act(int M, int K, int r, const void* X, int64_t ldx, float g_x, const void* l1t,
+                              void* codes, void* scales, void* xl1, void* stream) {
+  if (M < 0 || K <= 0 || !valid_rank(r)) return SVDQ_ERR_INVALID_ARG;
+  if (K % 256 != 0 || ldx < K || ldx % 8 != 0) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+  if (M == 0) return SVDQ_OK;
+  if (!X || !l1t || !codes || !scales || !xl1) return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(l1t) || !aligned16(codes) || !aligned16(scales) || !aligned16(xl1))
+    return SVDQ_ERR_MISALIGNED;
+  svdq_status s;
+  DeviceInfo di;
+  if ((s = current_device(nullptr, &di)) != SVDQ_OK) return s;
+  return quantize_dispatch(M, K, r, X, ldx, g_x, l1t, codes, scales, xl1, static_cast<cudaStream_t>(stream),
+                           di.sm_count);
+}
+
+svdq_status svdq_w4a4_gemm(int M, int N, int K, int r, const void* a_codes, const void* a_scales, const void* xl1,
+                           float g_x, const void* w_codes, const void* w_scales, const float* g_w, const void* l2t,
+                           const void* bias, void* Y, int64_t ldy, void* stream) {
+  if (M < 0) return SVDQ_ERR_INVALID_ARG;
+  svdq_status s = check_layer_shape(N, K, r);
+  if (s != SVDQ_OK) return s;
+  if (ldy < N || ldy % 8 != 0) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+  if (M == 0) return SVDQ_OK;
+  if (!a_codes || !a_scales || !xl1 || !w_codes || !w_scales || !g_w || !l2t || !Y) return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(a_codes) || !aligned16(a_scales) || !aligned16(xl1) || !aligned16(w_codes) ||
+      !aligned16(w_scales) || !aligned16(l2t) || !aligned16(Y) || (bias && !aligned16(bias)) ||
+      (reinterpret_cast<uintptr_t>(g_w) & 3u))
+    return SVDQ_ERR_MISALIGNED;
+  DeviceInfo di;
+  if ((s = current_device(nullptr, &di)) != SVDQ_OK) return s;
+  return gemm_dispatch(M, N, K, r, a_codes, a_scales, xl1, g_x, w_codes, w_scales, g_w, l2t, bias, Y, ldy,
+                       static_cast<cudaStream_t>(stream), di.sm_count);
+}
+
+svdq_status svdq_linear_forward(int M, int N, int K, int r, const void* X, int64_t ldx, float g_x,
+                                const void* w_codes, const void* w_scales, const float* g_w, const void* l1t,
+                                const void* l2t, const void* bias, void* Y, int64_t ldy, void* workspace,
+                                size_t workspace_bytes, void* stream) {
+  if (M < 0) return SVDQ_ERR_INVALID_ARG;
+  svdq_status s = check_layer_shape(N, K, r);
+  if (s != SVDQ_OK) return s;
+  if (ldx < K || ldx % 8 != 0 || ldy < N || ldy % 8 != 0) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+  if (M == 0) return SVDQ_OK;
+  size_t need = 0, c = 0, sc = 0, x = 0;
+  svdq_forward_workspace_size(M, K, r, &need);
+  svdq_act_sizes(M, K, r, &c, &sc, &x);
+  if (!workspace) return SVDQ_ERR_INVALID_ARG;
+  if (workspace_bytes < need) return SVDQ_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return SVDQ_ERR_MISALIGNED;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint8_t* a_codes = ws;
+  uint8_t* a_scales = ws + round_up(c, 256);
+  uint8_t* xl1 = a_scales + round_up(sc, 256);
+  s = svdq_quantize_act(M, K, r, X, ldx, g_x, l1t, a_codes, a_scales, xl1, stream);
+  if (s != SVDQ_OK) return s;
+  return svdq_w4a4_gemm(M, N, K, r, a_codes, a_scales, xl1, g_x, w_codes, w_scales, g_w, l2t, bias, Y, ldy, stream);
+}
+
+svdq_status svdq_read_device_error(int* code, int clear) {
+  if (!code) return SVDQ_ERR_INVALID_ARG;
+  svdq_status s;
+  if ((s = current_device(nullptr, nullptr)) != SVDQ_OK) return s;
+  if (cudaDeviceSynchronize() != cudaSuccess) return launch_status();
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_device_error, sizeof(int)) != cudaSuccess) return launch_status();
+  *code = v;
+  if (clear) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int)) != cudaSuccess) return launch_status();
+  }
+  return SVDQ_OK;
+}
+
+}  // extern "C"
