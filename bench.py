@@ -1,0 +1,325 @@
+"""Throughput of the SVDQuant W4A4 NVFP4 linear layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Workload: the FLUX-like DiT fused QKV projection (M=4608 tokens, K=3072,
+N=9216, rank 32), seeded synthetic inputs from workloads.py. One step = one
+forward of the layer over the batch: activation quantisation + down
+projection, then the block-scaled FP4 GEMM with the fused low-rank up
+projection and bias. Inputs are resident in HBM; L2 is flushed (256 MiB write)
+before every timed step; each step is timed with CUDA events on the launching
+stream. Multi-GPU: independent replicas (the layer shards by tokens with no
+exchange), max time over ranks. Rank 0 prints one JSON line.
+
+--impl reference times the CPU oracle (float64 restatement of the layer) on
+the host cores on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "W4A4 linear TFLOP/s and tokens/s on 1 B200; % of NVFP4 tensor peak / HBM roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FP4_PER_BF16 = 4.0   # nominal dense fp4 / bf16 tensor throughput ratio (9 / 2.25 PFLOP/s)
+FLUSH_BYTES = 256 << 20
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def _flops(M, N, K, r):
+    return 2.0 * M * N * K + 2.0 * M * r * (K + N)
+
+
+def _quant_bytes(M, K, r):
+    return 2 * M * K + M * K / 2 + M * K / 16 + 2 * M * r + 2 * K * r
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms while running."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200",
+                 "-i", str(self.index)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        self.out = ""
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+
+    def summary(self):
+        rows = [l.split(",") for l in (self.out or "").strip().splitlines() if l.count(",") >= 6]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        sm = [float(r[0]) for r in rows if r[0].strip().replace(".", "").isdigit()]
+        mx = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if "Active" == r[3 + i].strip()})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def _dist_init():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def _max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def _barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ------------------------------------------------------------------ CPU oracle timing
+def _oracle_setup(spec, X, W, b, budget_s: float):
+    """Load-time work of the CPU oracle (untimed) and the size of a bounded
+    sample: the first S rows of X against the first Ns output features (rows
+    and output features are independent in the layer, so the sample is an
+    exact slice of the workload) sized to take about `budget_s` per forward."""
+    from oracle import svdq as osv
+    L1, L2, _ = osv.lowrank_factors(W, spec.r)
+    g_x = osv.act_global_scale(X)
+    full = osv.pack_weight(W, L1, L2)
+    S = 64
+
+    def sliced(ns):
+        return osv.PackedWeight(full.codes[:ns], full.scales[:ns], full.g_w, full.L1, full.L2[:, :ns])
+
+    t0 = time.perf_counter()
+    osv.forward(X[:S], sliced(128), b[:128], g_x)
+    t_unit = max(time.perf_counter() - t0, 1e-3)
+    ns = int(max(1, min(spec.N // 128, budget_s / t_unit))) * 128
+    return sliced(ns), g_x, S, ns
+
+
+def _oracle_time(X, pw, b, g_x, S, ns) -> float:
+    from oracle import svdq as osv
+    t0 = time.perf_counter()
+    osv.forward(X[:S], pw, b[:ns], g_x)
+    return time.perf_counter() - t0
+
+
+def _cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count()
+
+
+def run_reference(args, spec):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    X, W, b = workloads.make_layer(spec)
+    budget = max(0.05, min(5.0, 120.0 / max(1, args.steps + args.warmup)))
+    pw, g_x, S, ns = _oracle_setup(spec, X, W, b, budget)
+    times = []
+    for i in range(args.warmup + args.steps):
+        dt = _oracle_time(X, pw, b, g_x, S, ns)
+        if i >= args.warmup:
+            times.append(dt)
+    t = statistics.mean(times)
+    value = _flops(S, ns, spec.K, spec.r) / t / 1e12
+    sample = f"first {S} rows x first {ns} of {spec.N} output features per step (float64 numpy oracle)"
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": spec.name, "M": spec.M, "K": spec.K, "N": spec.N, "r": spec.r},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": _cores(), "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }))
+    return 0
+
+
+# ------------------------------------------------------------------ GPU arm
+def run_ours(args, spec):
+    world, rank, local = _dist_init()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    import w4a4_rank_corrected_svdq_b200 as svdq
+
+    M, K, N, r = spec.M, spec.K, spec.N, spec.r
+    X, W, b = workloads.make_layer(spec)
+    L1, L2 = workloads.factor_stand_ins(spec)
+    Xd, Wd, bd = X.to(dev), W.to(dev), b.to(dev)
+    pw = svdq.svdq_pack_weight(Wd, L1.to(dev), L2.to(dev))
+    g_x = float(svdq.svdq_act_global_scale(Xd).item())
+    qa = svdq.QuantAct(M, K, r, dev)
+    Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        svdq.svdq_quantize_act(Xd, g_x, pw, out=qa)
+        svdq.svdq_w4a4_gemm(qa, g_x, pw, bd, out=Y)
+
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        step()
+    torch.cuda.synchronize()
+    if svdq.svdq_read_device_error() != 0:
+        raise RuntimeError("device error during warm-up")
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    _barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        for i in range(args.steps):
+            flush.fill_(i & 0xFF)
+            ev[i][0].record(stream)
+            svdq.svdq_quantize_act(Xd, g_x, pw, out=qa)
+            ev[i][1].record(stream)
+            svdq.svdq_w4a4_gemm(qa, g_x, pw, bd, out=Y)
+            ev[i][2].record(stream)
+        torch.cuda.synchronize()
+    _barrier(world)
+    t_q = [e[0].elapsed_time(e[1]) for e in ev]
+    t_g = [e[1].elapsed_time(e[2]) for e in ev]
+    t_step = [a + g for a, g in zip(t_q, t_g)]
+    total_ms = _max_over_ranks(sum(t_step), world)
+    ms_per_step = total_ms / args.steps
+    gemm_ms = statistics.mean(t_g)
+    quant_ms = statistics.mean(t_q)
+
+    # ---- end to end through the public forward, host buffers, copies timed
+    e2e_steps = min(args.steps, 50)
+    Xh = X.pin_memory()
+    Yh = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
+    ws = torch.empty(svdq.svdq_forward_workspace_size(M, K, r), dtype=torch.uint8, device=dev)
+    Xe = torch.empty_like(Xd)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for _ in range(2):
+        Xe.copy_(Xh, non_blocking=True)
+        svdq.svdq_linear_forward(Xe, g_x, pw, bd, out=Y, workspace=ws)
+        Yh.copy_(Y, non_blocking=True)
+    torch.cuda.synchronize()
+    _barrier(world)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        Xe.copy_(Xh, non_blocking=True)
+        svdq.svdq_linear_forward(Xe, g_x, pw, bd, out=Y, workspace=ws)
+        Yh.copy_(Y, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = _max_over_ranks(e0.elapsed_time(e1), world) / e2e_steps
+    if svdq.svdq_read_device_error() != 0:
+        raise RuntimeError("device error during timing")
+
+    peaks, kind = _peaks()
+    fp4_peak = peaks["bf16_tflops"] * FP4_PER_BF16
+    gemm_tflops = 2.0 * M * N * K / (gemm_ms * 1e-3) / 1e12
+    quant_gbs = _quant_bytes(M, K, r) / (quant_ms * 1e-3) / 1e9
+    flops = _flops(M, N, K, r)
+    value = world * flops / (ms_per_step * 1e-3) / 1e12
+    tokens = world * M / (ms_per_step * 1e-3)
+    out = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "nvfp4", "data": "synthetic",
+        "config": {"workload": spec.name, "M": M, "K": K, "N": N, "r": r, "global_batch_tokens": world * M,
+                   "parallelism": f"replicas x{world}" if world > 1 else "single",
+                   "l2": "flushed before every timed step (256 MiB write)",
+                   "factors": "seeded stand-in low-rank factors (timing does not depend on their values)"},
+        "tokens_per_s": tokens,
+        "roofline": {"bound": "tensor", "achieved": gemm_tflops, "peak": fp4_peak, "unit": "TFLOP/s",
+                     "frac": gemm_tflops / fp4_peak, "traffic": None,
+                     "kernel": "w4a4_gemm_kernel", "peak_source": f"{kind} bf16 burst x {FP4_PER_BF16:g} (fp4/bf16)"},
+        "kernels": {
+            "w4a4_gemm_kernel": {"ms": gemm_ms, "tflops": gemm_tflops, "frac_of_fp4_peak": gemm_tflops / fp4_peak},
+            "quantize_act_kernel": {"ms": quant_ms, "gbs": quant_gbs, "frac_of_hbm": quant_gbs / peaks["hbm_gbs"]},
+        },
+        "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2, "ms_per_step": e2e_ms},
+        "gpu_launches": 2 * args.steps,
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        opw, og, S, ns = _oracle_setup(spec, X, W, b, budget_s=10.0)
+        dt = _oracle_time(X, opw, b, og, S, ns)
+        out["cpu_baseline"] = {"value": _flops(S, ns, K, r) / dt / 1e12, "unit": "TFLOP/s", "cores": _cores(),
+                               "kind": "oracle",
+                               "sample": f"first {S} rows x first {ns} of {N} output features, one forward"}
+    if rank == 0:
+        print(json.dumps(out))
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    spec = workloads.WORKLOADS[2].layers[0]
+    if args.impl == "reference":
+        return run_reference(args, spec)
+    return run_ours(args, spec)
+
+
+if __name__ == "__main__":
+    sys.exit(main())
