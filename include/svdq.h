@@ -144,6 +144,29 @@ svdq_status svdq_linear_forward(int M, int N, int K, int r, const void* X, int64
                                 int64_t ldy, void* workspace, size_t workspace_bytes,
                                 void* stream);
 
+/* Same computation as svdq_linear_forward, for callers that cannot supply a
+ * workspace: plugin interfaces of inference runtimes that pass only a layer's
+ * inputs and outputs, and code running after the process has fixed its device
+ * memory budget, where calling an allocator is not allowed. (The blog has no
+ * counterpart; this is an interface convenience.)
+ *   - Allocates nothing. The intermediates go to one fixed scratch array of
+ *     16 MiB (16777216 bytes) inside the library, which every GPU that loads
+ *     the library keeps until the process exits.
+ *   - Shapes whose svdq_forward_workspace_size exceeds that limit are rejected
+ *     with SVDQ_ERR_WORKSPACE (and a message on stderr) before any launch;
+ *     e.g. M=4608, K=3072, r=32 (8.3 MB) fits, M=18432, K=3072 does not.
+ *   - The first call on a device looks up the scratch array's device address
+ *     (cudaGetSymbolAddress, with that device current); make that first call
+ *     before any stream capture on that device.
+ *   - All calls on a device share the scratch: calls that may overlap on the
+ *     GPU (different streams, or several host threads) race and must be
+ *     serialised by the caller. No part of the scratch needs to start at zero.
+ * Arguments, layouts and errors otherwise as svdq_linear_forward. */
+svdq_status svdq_linear_forward_noalloc(int M, int N, int K, int r, const void* X, int64_t ldx, float g_x,
+                                        const void* w_codes, const void* w_scales, const float* g_w,
+                                        const void* l1t, const void* l2t, const void* bias, void* Y,
+                                        int64_t ldy, void* stream);
+
 /* ------------------------------------------------------------ errors */
 /* Reads (and, if clear != 0, resets) the device error word of the current
  * device: 0 or an svdq_status recorded by a kernel (e.g. SVDQ_ERR_TIMEOUT).

@@ -37,6 +37,7 @@ SIGNATURES = {
     "svdq_w4a4_gemm": (_i, [_i, _i, _i, _i, _p, _p, _p, _f, _p, _p, _p, _p, _p, _p, _i64, _p]),
     "svdq_linear_forward": (_i, [_i, _i, _i, _i, _p, _i64, _f, _p, _p, _p, _p, _p, _p, _p, _i64, _p, _sz, _p]),
     "svdq_read_device_error": (_i, [_pi, _i]),
+    "svdq_linear_forward_noalloc": (_i, [_i, _i, _i, _i, _p, _i64, _f, _p, _p, _p, _p, _p, _p, _p, _i64, _p]),
 }
 
 

@@ -424,3 +424,77 @@ svdq_status svdq_read_device_error(int* code, int clear) {
 }
 
 }  // extern "C"
+
+// ----------------------------------------------------------------------------
+// Forward without caller-provided workspace.
+//
+// Some callers cannot hand the library a workspace buffer: plugin interfaces
+// of inference runtimes that pass only the layer's inputs and outputs, and
+// code that runs after the process has fixed its device-memory budget, where
+// calling the allocator (and its implicit synchronisation) is not allowed.
+// For them the intermediates of svdq_linear_forward (activation codes, block
+// scales, XL1) live in one fixed scratch array inside the library.
+//
+// The array is a file-scope __device__ object of kNoAllocScratchBytes bytes;
+// every GPU that loads the library holds it until the process exits. Host code
+// must not pass the array's name to a kernel (on the host it names a shadow
+// variable, not device memory): the device address is fetched with
+// cudaGetSymbolAddress once per device, with that device current, on the
+// first call made on that device.
+// ----------------------------------------------------------------------------
+namespace svdq {
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;  // 16 MiB per device
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+void* g_noalloc_ptr[kMaxDevices] = {};
+std::mutex g_noalloc_mutex;
+
+// Device address of the scratch array on the current device (set up once per device).
+svdq_status noalloc_scratch(int dev, void** out) {
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || p == nullptr) {
+      std::fprintf(stderr, "svdq: cudaGetSymbolAddress(scratch) failed: %s\n", cudaGetErrorString(e));
+      cudaGetLastError();
+      return SVDQ_ERR_CUDA;
+    }
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return SVDQ_OK;
+}
+
+}  // namespace
+}  // namespace svdq
+
+extern "C" svdq_status svdq_linear_forward_noalloc(int M, int N, int K, int r, const void* X, int64_t ldx,
+                                                   float g_x, const void* w_codes, const void* w_scales,
+                                                   const float* g_w, const void* l1t, const void* l2t,
+                                                   const void* bias, void* Y, int64_t ldy, void* stream) {
+  if (M < 0) return SVDQ_ERR_INVALID_ARG;
+  svdq_status s = check_layer_shape(N, K, r);
+  if (s != SVDQ_OK) return s;
+  if (ldx < K || ldx % 8 != 0 || ldy < N || ldy % 8 != 0) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+  if (M == 0) return SVDQ_OK;
+  size_t need = 0;
+  if ((s = svdq_forward_workspace_size(M, K, r, &need)) != SVDQ_OK) return s;
+  if (need > kNoAllocScratchBytes) {
+    std::fprintf(stderr,
+                 "svdq_linear_forward_noalloc: M=%d K=%d r=%d needs %zu bytes of scratch, the built-in limit is "
+                 "%zu bytes; use svdq_linear_forward with a workspace\n",
+                 M, K, r, need, kNoAllocScratchBytes);
+    return SVDQ_ERR_WORKSPACE;
+  }
+  int dev = 0;
+  if ((s = current_device(&dev, nullptr)) != SVDQ_OK) return s;
+  void* scratch = nullptr;
+  if ((s = noalloc_scratch(dev, &scratch)) != SVDQ_OK) return s;
+  // Nothing in the scratch has to start at zero: the quantize kernel of this
+  // call writes every byte the GEMM of this call reads.
+  return svdq_linear_forward(M, N, K, r, X, ldx, g_x, w_codes, w_scales, g_w, l1t, l2t, bias, Y, ldy, scratch,
+                             kNoAllocScratchBytes, stream);
+}
