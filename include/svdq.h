@@ -44,8 +44,14 @@
  *              ((row/128) * (K/64) + kb/4) * 512 + (row%32) * 16
  *                  + ((row%128)/32) * 4 + kb%4
  *          (svdq_scale_offset computes it on the host).
+ *  gscale  fp32 [4] (device): {g_x, g_w, alpha = fp32(g_x * g_w), 0}
  *  l1t     bf16 [r][K]   = L1 transposed (packed by svdq_pack_weight)
- *  l2t     bf16 [N][r]   = L2 transposed (packed by svdq_pack_weight)
+ *  l2s     bf16 [2][N][r]: the up-projection pre-divided by alpha, split in
+ *          two bf16 parts so that hi + lo = L2^T / alpha to ~2^-17:
+ *          v = fp32(L2[j][n] / alpha), hi = bf16(v), lo = bf16(v - hi);
+ *          plane 0 holds hi, plane 1 holds lo. (The 4-bit product and the
+ *          low-rank product then share one fp32 accumulator, which the
+ *          epilogue multiplies by alpha once.)
  *  xl1     bf16 [M][r]   = bf16(X . L1), fp32 accumulation
  */
 #ifndef SVDQ_H_
@@ -84,7 +90,7 @@ svdq_status svdq_scale_offset(int K, int row, int kblock, size_t* out);
 /* ------------------------------------------------------------ sizes (host) */
 /* Bytes of each packed-weight buffer for an N x K weight with rank r. */
 svdq_status svdq_weight_sizes(int N, int K, int r, size_t* codes_bytes, size_t* scales_bytes,
-                              size_t* l1t_bytes, size_t* l2t_bytes);
+                              size_t* l1t_bytes, size_t* l2s_bytes);
 /* Bytes of the quantised-activation buffers for M rows (scales padded to 128 rows). */
 svdq_status svdq_act_sizes(int M, int K, int r, size_t* codes_bytes, size_t* scales_bytes,
                            size_t* xl1_bytes);
@@ -95,17 +101,20 @@ svdq_status svdq_forward_workspace_size(int M, int K, int r, size_t* bytes);
 /* Pack one layer (untimed, load time). Blog section "Background: SVDQuant and
  * Nunchaku": the low-rank branch holds the hardest part of the weight, the
  * remaining residual is quantised to 4 bits.
- *   W   bf16 [N][K], L1 bf16 [K][r], L2 bf16 [r][N]   (inputs; L1.L2 is the
- *       rank-r factorisation of W^T)
- *   Writes: w_codes [N][K/2], w_scales (tiled), *g_w (device float),
- *           l1t [r][K], l2t [N][r].
+ *   W   bf16 [N][K], L1 bf16 [K][r], L2 bf16 [r][N]   (L1.L2 is the rank-r
+ *       factorisation of W^T)
+ *   g_x device float: the layer's calibrated (static) activation decode scale,
+ *       e.g. from svdq_act_global_scale on calibration activations.
+ *   Writes: w_codes [N][K/2], w_scales (tiled), gscale[4], l1t [r][K],
+ *           l2s [2][N][r] (layouts above).
  * R[n,k] = W[n,k] - sum_j L1[k,j] L2[j,n] is formed in float64 (j ascending,
  * products exact) and rounded once to float32; g_w = fp32(amax|R| / 2688)
  * (1 if R == 0); then R is quantised with the NVFP4 rule of svdq_quantize_act.
+ * Requires alpha = g_x g_w >= 2^-100 (so L2 / alpha stays finite in bf16).
  * The output buffers must not overlap the inputs. */
 svdq_status svdq_pack_weight(int N, int K, int r, const void* W, const void* L1, const void* L2,
-                             void* w_codes, void* w_scales, float* g_w, void* l1t, void* l2t,
-                             void* stream);
+                             const float* g_x, void* w_codes, void* w_scales, float* gscale, void* l1t,
+                             void* l2s, void* stream);
 
 /* Calibrated (static) activation scale: *g_out = fp32(amax|X| / 2688), or 1
  * for an all-zero X. X bf16 [M][ldx]; g_out is a device float. */
@@ -119,28 +128,30 @@ svdq_status svdq_act_global_scale(int M, int K, const void* X, int64_t ldx, floa
  *   per 16-element block: S = e4m3_rn_sat(amax / fp32(6 g_x)),
  *   sd = fp32(dec(S) g_x), code = e2m1_rn_sat(fp32(x * fp32(1/sd))) (0 if sd == 0);
  *   xl1 = bf16(X . L1) with fp32 accumulation (L1 given as l1t [r][K]).
+ * g_x is a device float (gscale[0] of a packed layer).
  * Writes codes [M][K/2], scales (tiled, rows padded to 128; padding rows are
  * written as zero scales), xl1 [M][r]. Deterministic. */
-svdq_status svdq_quantize_act(int M, int K, int r, const void* X, int64_t ldx, float g_x,
+svdq_status svdq_quantize_act(int M, int K, int r, const void* X, int64_t ldx, const float* g_x,
                               const void* l1t, void* codes, void* scales, void* xl1, void* stream);
 
 /* The block-scaled FP4 GEMM with the low-rank up projection and bias fused in
  * its epilogue (blog figure caption: the up projection is fused with the 4-bit
  * compute kernel):
- *   Y[m,n] = bf16( g_x * g_w * sum_k dec(Xc)dec(SX) dec(Rc)dec(SR)
- *                  + sum_j xl1[m,j] L2[j,n] + b[n] )
- * a_codes/a_scales/xl1 as written by svdq_quantize_act; w_* as written by
- * svdq_pack_weight; bias may be NULL; Y bf16 [M][ldy]. */
+ *   Y[m,n] = bf16( alpha * ( sum_k dec(Xc)dec(SX) dec(Rc)dec(SR)
+ *                            + sum_j xl1[m,j] (hi + lo)[n,j] ) + b[n] )
+ *          = bf16( g_x g_w * Q4(X).Q4(R)^T + xl1 . L2 + b )   (to fp32 accuracy)
+ * a_codes/a_scales/xl1 as written by svdq_quantize_act; w_codes, w_scales,
+ * gscale, l2s as written by svdq_pack_weight; bias may be NULL; Y bf16 [M][ldy]. */
 svdq_status svdq_w4a4_gemm(int M, int N, int K, int r, const void* a_codes, const void* a_scales,
-                           const void* xl1, float g_x, const void* w_codes, const void* w_scales,
-                           const float* g_w, const void* l2t, const void* bias, void* Y,
-                           int64_t ldy, void* stream);
+                           const void* xl1, const void* w_codes, const void* w_scales, const float* gscale,
+                           const void* l2s, const void* bias, void* Y, int64_t ldy, void* stream);
 
-/* The whole layer: svdq_quantize_act into `workspace`, then svdq_w4a4_gemm.
+/* The whole layer: svdq_quantize_act (with g_x = gscale[0]) into `workspace`,
+ * then svdq_w4a4_gemm.
  * workspace_bytes must be >= svdq_forward_workspace_size(M, K, r). */
-svdq_status svdq_linear_forward(int M, int N, int K, int r, const void* X, int64_t ldx, float g_x,
-                                const void* w_codes, const void* w_scales, const float* g_w,
-                                const void* l1t, const void* l2t, const void* bias, void* Y,
+svdq_status svdq_linear_forward(int M, int N, int K, int r, const void* X, int64_t ldx,
+                                const void* w_codes, const void* w_scales, const float* gscale,
+                                const void* l1t, const void* l2s, const void* bias, void* Y,
                                 int64_t ldy, void* workspace, size_t workspace_bytes,
                                 void* stream);
 
@@ -162,9 +173,9 @@ svdq_status svdq_linear_forward(int M, int N, int K, int r, const void* X, int64
  *     GPU (different streams, or several host threads) race and must be
  *     serialised by the caller. No part of the scratch needs to start at zero.
  * Arguments, layouts and errors otherwise as svdq_linear_forward. */
-svdq_status svdq_linear_forward_noalloc(int M, int N, int K, int r, const void* X, int64_t ldx, float g_x,
-                                        const void* w_codes, const void* w_scales, const float* g_w,
-                                        const void* l1t, const void* l2t, const void* bias, void* Y,
+svdq_status svdq_linear_forward_noalloc(int M, int N, int K, int r, const void* X, int64_t ldx,
+                                        const void* w_codes, const void* w_scales, const float* gscale,
+                                        const void* l1t, const void* l2s, const void* bias, void* Y,
                                         int64_t ldy, void* stream);
 
 /* ------------------------------------------------------------ errors */

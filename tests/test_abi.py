@@ -63,7 +63,7 @@ def test_scale_offset_errors(L):
 
 
 def test_sizes(L):
-    assert _lib.svdq_weight_sizes(256, 512, 32) == (256 * 256, 256 * 32, 32 * 512 * 2, 256 * 32 * 2)
+    assert _lib.svdq_weight_sizes(256, 512, 32) == (256 * 256, 256 * 32, 32 * 512 * 2, 2 * 256 * 32 * 2)
     assert _lib.svdq_act_sizes(129, 512, 16) == (129 * 256, 256 * 32, 129 * 16 * 2)
     ws = _lib.svdq_forward_workspace_size(129, 512, 16)
     assert ws >= sum(_lib.svdq_act_sizes(129, 512, 16))
@@ -79,25 +79,25 @@ def test_validation_happens_before_device_checks(L):
     p = ctypes.c_void_p(0x10000)          # never dereferenced: validation fails first
     odd = ctypes.c_void_p(0x10008)
     # bad K
-    assert L.svdq_quantize_act(4, 100, 32, p, 100, 1.0, p, p, p, p, None) == 2
+    assert L.svdq_quantize_act(4, 100, 32, p, 100, p, p, p, p, p, None) == 2
     # null pointer
-    assert L.svdq_quantize_act(4, 256, 32, None, 256, 1.0, p, p, p, p, None) == 1
+    assert L.svdq_quantize_act(4, 256, 32, None, 256, p, p, p, p, p, None) == 1
     # misaligned pointer
-    assert L.svdq_quantize_act(4, 256, 32, odd, 256, 1.0, p, p, p, p, None) == 3
+    assert L.svdq_quantize_act(4, 256, 32, odd, 256, p, p, p, p, p, None) == 3
     # bad leading dimension
-    assert L.svdq_w4a4_gemm(4, 128, 256, 32, p, p, p, 1.0, p, p, p, p, None, p, 100, None) == 2
+    assert L.svdq_w4a4_gemm(4, 128, 256, 32, p, p, p, p, p, p, p, None, p, 100, None) == 2
     # workspace too small
-    assert L.svdq_linear_forward(4, 128, 256, 32, p, 256, 1.0, p, p, p, p, p, None, p, 128, p, 16, None) == 7
+    assert L.svdq_linear_forward(4, 128, 256, 32, p, 256, p, p, p, p, p, None, p, 128, p, 16, None) == 7
     # M == 0 is a valid no-op
-    assert L.svdq_w4a4_gemm(0, 128, 256, 32, None, None, None, 1.0, None, None, None, None, None, None, 128,
+    assert L.svdq_w4a4_gemm(0, 128, 256, 32, None, None, None, None, None, None, None, None, None, 128,
                             None) == 0
 
 
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU path")
 def test_no_gpu_is_unsupported_device(L):
     p = ctypes.c_void_p(0x10000)
-    assert L.svdq_quantize_act(4, 256, 32, p, 256, 1.0, p, p, p, p, None) == 4
-    assert L.svdq_pack_weight(128, 256, 32, p, p, p, p, p, p, p, p, None) == 4
+    assert L.svdq_quantize_act(4, 256, 32, p, 256, p, p, p, p, p, None) == 4
+    assert L.svdq_pack_weight(128, 256, 32, p, p, p, p, p, p, p, p, p, None) == 4
     code = ctypes.c_int()
     assert L.svdq_read_device_error(ctypes.byref(code), 0) == 4
 

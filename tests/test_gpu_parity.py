@@ -43,6 +43,14 @@ def _layer(M, K, N, r, seed=7, bias=True):
     return X, W, b, L1, L2
 
 
+def _act_only_weight(lib, K, r, L1, g_x):
+    """A packed-weight holder carrying only what svdq_quantize_act reads (g_x, l1t)."""
+    pw = lib.PackedWeight(128, K, r, "cuda")
+    pw.gscale.copy_(torch.tensor([float(g_x), 1.0, float(g_x), 0.0]))
+    pw.l1t.copy_(_to_dev(L1.T))
+    return pw
+
+
 def _check_act(lib, X, L1, r, g_x, qa, M, K):
     ref = osv.quantize_act(X, g_x)
     codes = layouts.unpack_codes(qa.codes.cpu().numpy(), M, K)
@@ -75,6 +83,8 @@ def test_act_global_scale_bitexact(lib):
     X, *_ = _layer(300, 512, 128, 16)
     g = lib.svdq_act_global_scale(X.cuda()).item()
     assert np.float32(g) == osv.act_global_scale(X)
+    z = lib.svdq_act_global_scale(torch.zeros((5, 256), dtype=torch.bfloat16, device="cuda")).item()
+    assert z == 1.0
 
 
 # ------------------------------------------------------------------ activation kernel
@@ -83,9 +93,8 @@ def test_act_global_scale_bitexact(lib):
 def test_quantize_act_bitexact(lib, M, K, r):
     X, W, b, L1, L2 = _layer(M, K, 128, r)
     g_x = osv.act_global_scale(X)
-    pw = lib.PackedWeight(128, K, r, "cuda")
-    pw.l1t.copy_(_to_dev(L1.T))
-    qa = lib.svdq_quantize_act(X.cuda(), float(g_x), pw)
+    pw = _act_only_weight(lib, K, r, L1, g_x)
+    qa = lib.svdq_quantize_act(X.cuda(), pw)
     torch.cuda.synchronize()
     _check_act(lib, X, L1, r, g_x, qa, M, K)
 
@@ -99,9 +108,8 @@ def test_quantize_act_zero_rows_and_strided_input(lib):
     big = torch.zeros((M, K + 64), dtype=torch.bfloat16)
     big[:, :K] = X
     g_x = osv.act_global_scale(X)
-    pw = lib.PackedWeight(128, K, r, "cuda")
-    pw.l1t.copy_(_to_dev(L1.T))
-    qa = lib.svdq_quantize_act(big.cuda()[:, :K], float(g_x), pw)
+    pw = _act_only_weight(lib, K, r, L1, g_x)
+    qa = lib.svdq_quantize_act(big.cuda()[:, :K], pw)
     torch.cuda.synchronize()
     _check_act(lib, X, L1, r, g_x, qa, M, K)
 
@@ -110,16 +118,24 @@ def test_quantize_act_zero_rows_and_strided_input(lib):
 @pytest.mark.parametrize("N,K,r", [(128, 256, 16), (256, 512, 32), (384, 1024, 64), (256, 512, 128)])
 def test_pack_weight_bitexact(lib, N, K, r):
     X, W, b, L1, L2 = _layer(8, K, N, r)
-    pw = lib.svdq_pack_weight(W.cuda(), _to_dev(L1), _to_dev(L2))
+    g_x = osv.act_global_scale(X)
+    pw = lib.svdq_pack_weight(W.cuda(), _to_dev(L1), _to_dev(L2), float(g_x))
     torch.cuda.synchronize()
     ref = osv.pack_weight(W, L1, L2)
     codes = layouts.unpack_codes(pw.codes.cpu().numpy(), N, K)
     scales = layouts.untile_scales(pw.scales.cpu().numpy(), N, K)
-    assert np.float32(pw.g_w.item()) == ref.g_w
+    gs = pw.gscale.cpu().numpy()
+    assert gs[0] == g_x and gs[1] == ref.g_w and gs[2] == np.float32(g_x * ref.g_w) and gs[3] == 0
     assert np.array_equal(scales, ref.scales)
     assert np.array_equal(codes, ref.codes)
     assert np.array_equal(_bf16_np(pw.l1t), L1.T)
-    assert np.array_equal(_bf16_np(pw.l2t), L2.T)
+    # l2s: documented encoding of L2^T / alpha as bf16 hi + lo (include/svdq.h)
+    v = (L2.T.astype(np.float32) / np.float32(gs[2])).astype(np.float32)
+    hi = nvfp4.bf16_round(v)
+    lo = nvfp4.bf16_round((v - hi.astype(np.float32)).astype(np.float32))
+    l2s = _bf16_np(pw.l2s)
+    assert np.array_equal(l2s[0], hi) and np.array_equal(l2s[1], lo)
+    assert np.max(np.abs((l2s[0] + l2s[1]) * float(gs[2]) - L2.T)) <= 2 ** -15 * np.max(np.abs(L2))
 
 
 # ------------------------------------------------------------------ full layer
@@ -129,8 +145,8 @@ def test_pack_weight_bitexact(lib, N, K, r):
 def test_linear_forward_parity(lib, M, K, N, r, bias):
     X, W, b, L1, L2 = _layer(M, K, N, r, bias=bias)
     g_x = osv.act_global_scale(X)
-    pw = lib.svdq_pack_weight(W.cuda(), _to_dev(L1), _to_dev(L2))
-    Y = lib.svdq_linear_forward(X.cuda(), float(g_x), pw, b.cuda() if bias else None)
+    pw = lib.svdq_pack_weight(W.cuda(), _to_dev(L1), _to_dev(L2), float(g_x))
+    Y = lib.svdq_linear_forward(X.cuda(), pw, b.cuda() if bias else None)
     torch.cuda.synchronize()
     assert lib.svdq_read_device_error() == 0
     fwd = osv.forward(X, osv.pack_weight(W, L1, L2), b if bias else None, g_x)
@@ -141,16 +157,18 @@ def test_linear_forward_config1(lib):
     spec = workloads.WORKLOADS[1].layers[0]
     X, W, b = workloads.make_layer(spec)
     L1, L2, _ = osv.lowrank_factors(W, spec.r)
+    g_x = lib.svdq_act_global_scale(X.cuda())      # calibration on the GPU, then pack
+    assert np.float32(g_x.item()) == osv.act_global_scale(X)
+    pw = lib.svdq_pack_weight(W.cuda(), _to_dev(L1), _to_dev(L2), g_x)
     g_x = osv.act_global_scale(X)
-    pw = lib.svdq_pack_weight(W.cuda(), _to_dev(L1), _to_dev(L2))
-    qa = lib.svdq_quantize_act(X.cuda(), float(g_x), pw)
-    Y = lib.svdq_w4a4_gemm(qa, float(g_x), pw, b.cuda())
+    qa = lib.svdq_quantize_act(X.cuda(), pw)
+    Y = lib.svdq_w4a4_gemm(qa, pw, b.cuda())
     torch.cuda.synchronize()
     _check_act(lib, X, L1, spec.r, g_x, qa, spec.M, spec.K)
     fwd = osv.forward(X, osv.pack_weight(W, L1, L2), b, g_x)
     _check_y(Y, fwd)
     # deterministic: a second call gives identical bits
-    Y2 = lib.svdq_linear_forward(X.cuda(), float(g_x), pw, b.cuda())
+    Y2 = lib.svdq_linear_forward(X.cuda(), pw, b.cuda())
     torch.cuda.synchronize()
     assert torch.equal(Y, Y2)
 
@@ -158,5 +176,5 @@ def test_linear_forward_config1(lib):
 def test_m_zero_is_noop(lib):
     pw = lib.PackedWeight(128, 256, 16, "cuda")
     X = torch.empty((0, 256), dtype=torch.bfloat16, device="cuda")
-    Y = lib.svdq_linear_forward(X, 1.0, pw)
+    Y = lib.svdq_linear_forward(X, pw)
     assert Y.shape == (0, 128)

@@ -31,12 +31,12 @@ def _p(t):
     return ctypes.c_void_p(0 if t is None else t.data_ptr())
 
 
-def _noalloc(L, X, g_x, pw, bias, Y):
+def _noalloc(L, X, pw, bias, Y):
     M, K = X.shape
     stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
-    return L.svdq_linear_forward_noalloc(M, pw.N, K, pw.r, _p(X), X.stride(0), float(g_x), _p(pw.codes),
-                                         _p(pw.scales), _p(pw.g_w), _p(pw.l1t), _p(pw.l2t), _p(bias), _p(Y),
-                                         Y.stride(0), stream)
+    return L.svdq_linear_forward_noalloc(M, pw.N, K, pw.r, _p(X), X.stride(0), _p(pw.codes), _p(pw.scales),
+                                         _p(pw.gscale), _p(pw.l1t), _p(pw.l2s), _p(bias), _p(Y), Y.stride(0),
+                                         stream)
 
 
 @pytest.mark.parametrize("M,K,N,r", [(256, 1024, 1024, 32), (333, 768, 384, 64)])
@@ -45,14 +45,14 @@ def test_noalloc_forward_matches_workspace_forward(lib, M, K, N, r):
     _, (X, W, b) = workloads.small_layer(M, K, N, r, seed=21)
     L1, L2, _ = osv.lowrank_factors(W, r)
     to_dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(torch.bfloat16).cuda()  # noqa: E731
-    pw = lib.svdq_pack_weight(W.cuda(), to_dev(L1), to_dev(L2))
     g_x = float(osv.act_global_scale(X))
+    pw = lib.svdq_pack_weight(W.cuda(), to_dev(L1), to_dev(L2), g_x)
     Xd, bd = X.cuda(), b.cuda()
-    ref = lib.svdq_linear_forward(Xd, g_x, pw, bd).double().cpu().numpy()
+    ref = lib.svdq_linear_forward(Xd, pw, bd).double().cpu().numpy()
     outs = []
     for _ in range(2):                       # two calls in a row share the scratch
         Y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
-        assert _noalloc(L, Xd, g_x, pw, bd, Y) == 0
+        assert _noalloc(L, Xd, pw, bd, Y) == 0
         torch.cuda.synchronize()
         outs.append(Y.double().cpu().numpy())
     assert lib.svdq_read_device_error() == 0
@@ -67,4 +67,4 @@ def test_noalloc_rejects_shapes_beyond_the_scratch_limit(lib):
     p = ctypes.c_void_p(0x10000)             # never dereferenced: the size check fails first
     M, K, N, r = 18432, 3072, 128, 32        # workspace about 33 MB > 16 MiB
     assert lib.svdq_forward_workspace_size(M, K, r) > (16 << 20)
-    assert L.svdq_linear_forward_noalloc(M, N, K, r, p, K, 1.0, p, p, p, p, p, None, p, N, None) == 7
+    assert L.svdq_linear_forward_noalloc(M, N, K, r, p, K, p, p, p, p, p, None, p, N, None) == 7

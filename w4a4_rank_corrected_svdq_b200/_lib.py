@@ -31,13 +31,13 @@ SIGNATURES = {
     "svdq_weight_sizes": (_i, [_i, _i, _i, _psz, _psz, _psz, _psz]),
     "svdq_act_sizes": (_i, [_i, _i, _i, _psz, _psz, _psz]),
     "svdq_forward_workspace_size": (_i, [_i, _i, _i, _psz]),
-    "svdq_pack_weight": (_i, [_i, _i, _i, _p, _p, _p, _p, _p, _p, _p, _p, _p]),
+    "svdq_pack_weight": (_i, [_i, _i, _i, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p]),
     "svdq_act_global_scale": (_i, [_i, _i, _p, _i64, _p, _p]),
-    "svdq_quantize_act": (_i, [_i, _i, _i, _p, _i64, _f, _p, _p, _p, _p, _p]),
-    "svdq_w4a4_gemm": (_i, [_i, _i, _i, _i, _p, _p, _p, _f, _p, _p, _p, _p, _p, _p, _i64, _p]),
-    "svdq_linear_forward": (_i, [_i, _i, _i, _i, _p, _i64, _f, _p, _p, _p, _p, _p, _p, _p, _i64, _p, _sz, _p]),
+    "svdq_quantize_act": (_i, [_i, _i, _i, _p, _i64, _p, _p, _p, _p, _p, _p]),
+    "svdq_w4a4_gemm": (_i, [_i, _i, _i, _i, _p, _p, _p, _p, _p, _p, _p, _p, _p, _i64, _p]),
+    "svdq_linear_forward": (_i, [_i, _i, _i, _i, _p, _i64, _p, _p, _p, _p, _p, _p, _p, _i64, _p, _sz, _p]),
     "svdq_read_device_error": (_i, [_pi, _i]),
-    "svdq_linear_forward_noalloc": (_i, [_i, _i, _i, _i, _p, _i64, _f, _p, _p, _p, _p, _p, _p, _p, _i64, _p]),
+    "svdq_linear_forward_noalloc": (_i, [_i, _i, _i, _i, _p, _i64, _p, _p, _p, _p, _p, _p, _p, _i64, _p]),
 }
 
 
@@ -123,19 +123,31 @@ def svdq_forward_workspace_size(M: int, K: int, r: int) -> int:
 
 # ------------------------------------------------------------------ packed weight
 class PackedWeight:
-    """Device buffers of one packed layer (allocated by torch, filled by svdq_pack_weight)."""
+    """Device buffers of one packed layer (allocated by torch, filled by svdq_pack_weight).
+
+    gscale = [g_x, g_w, g_x*g_w, 0]; l2s = [2, N, r] bf16 hi / lo parts of L2^T / (g_x g_w)."""
 
     def __init__(self, N: int, K: int, r: int, device):
         cb, sb, lb1, lb2 = svdq_weight_sizes(N, K, r)
         self.N, self.K, self.r = N, K, r
         self.codes = torch.empty(cb, dtype=torch.uint8, device=device)
         self.scales = torch.empty(sb, dtype=torch.uint8, device=device)
-        self.g_w = torch.empty(1, dtype=torch.float32, device=device)
+        self.gscale = torch.empty(4, dtype=torch.float32, device=device)
         self.l1t = torch.empty((r, K), dtype=torch.bfloat16, device=device)
-        self.l2t = torch.empty((N, r), dtype=torch.bfloat16, device=device)
+        self.l2s = torch.empty((2, N, r), dtype=torch.bfloat16, device=device)
+
+    @property
+    def g_x(self) -> torch.Tensor:
+        return self.gscale[0:1]
+
+    @property
+    def g_w(self) -> torch.Tensor:
+        return self.gscale[1:2]
 
 
-def svdq_pack_weight(W: torch.Tensor, L1: torch.Tensor, L2: torch.Tensor, out: PackedWeight | None = None):
+def svdq_pack_weight(W: torch.Tensor, L1: torch.Tensor, L2: torch.Tensor, g_x, out: PackedWeight | None = None):
+    """Pack one layer. g_x: the calibrated activation scale, a CUDA float32 tensor of
+    one element (e.g. from svdq_act_global_scale) or a Python float."""
     N, K = W.shape
     r = L1.shape[1]
     _dev(W, "W", torch.bfloat16)
@@ -144,10 +156,13 @@ def svdq_pack_weight(W: torch.Tensor, L1: torch.Tensor, L2: torch.Tensor, out: P
     for t, n in ((W, "W"), (L1, "L1"), (L2, "L2")):
         if not t.is_contiguous():
             raise ValueError(f"{n} must be contiguous")
+    if not isinstance(g_x, torch.Tensor):
+        g_x = torch.tensor([float(g_x)], dtype=torch.float32, device=W.device)
+    _dev(g_x, "g_x", torch.float32)
     pw = out if out is not None else PackedWeight(N, K, r, W.device)
     _check("svdq_pack_weight", lib().svdq_pack_weight(
-        N, K, r, _ptr(W), _ptr(L1), _ptr(L2), _ptr(pw.codes), _ptr(pw.scales), _ptr(pw.g_w), _ptr(pw.l1t),
-        _ptr(pw.l2t), _stream(W)))
+        N, K, r, _ptr(W), _ptr(L1), _ptr(L2), _ptr(g_x), _ptr(pw.codes), _ptr(pw.scales), _ptr(pw.gscale),
+        _ptr(pw.l1t), _ptr(pw.l2s), _stream(W)))
     return pw
 
 
@@ -170,18 +185,19 @@ class QuantAct:
         self.xl1 = torch.empty((M, r), dtype=torch.bfloat16, device=device)
 
 
-def svdq_quantize_act(X: torch.Tensor, g_x: float, pw: PackedWeight, out: QuantAct | None = None) -> QuantAct:
+def svdq_quantize_act(X: torch.Tensor, pw: PackedWeight, out: QuantAct | None = None) -> QuantAct:
+    """Quantise X with the layer's calibrated g_x (pw.gscale[0]) and project it onto L1."""
     _dev(X, "X", torch.bfloat16)
     M, K = X.shape
     ldx = _rows(X, "X", K)
     qa = out if out is not None else QuantAct(M, K, pw.r, X.device)
     _check("svdq_quantize_act", lib().svdq_quantize_act(
-        M, K, pw.r, _ptr(X), ldx, float(g_x), _ptr(pw.l1t), _ptr(qa.codes), _ptr(qa.scales), _ptr(qa.xl1),
+        M, K, pw.r, _ptr(X), ldx, _ptr(pw.gscale), _ptr(pw.l1t), _ptr(qa.codes), _ptr(qa.scales), _ptr(qa.xl1),
         _stream(X)))
     return qa
 
 
-def svdq_w4a4_gemm(qa: QuantAct, g_x: float, pw: PackedWeight, bias: torch.Tensor | None = None,
+def svdq_w4a4_gemm(qa: QuantAct, pw: PackedWeight, bias: torch.Tensor | None = None,
                    out: torch.Tensor | None = None) -> torch.Tensor:
     M, N, K, r = qa.M, pw.N, pw.K, pw.r
     if bias is not None:
@@ -190,12 +206,12 @@ def svdq_w4a4_gemm(qa: QuantAct, g_x: float, pw: PackedWeight, bias: torch.Tenso
     _dev(Y, "Y", torch.bfloat16)
     ldy = _rows(Y, "Y", N)
     _check("svdq_w4a4_gemm", lib().svdq_w4a4_gemm(
-        M, N, K, r, _ptr(qa.codes), _ptr(qa.scales), _ptr(qa.xl1), float(g_x), _ptr(pw.codes), _ptr(pw.scales),
-        _ptr(pw.g_w), _ptr(pw.l2t), _ptr(bias), _ptr(Y), ldy, _stream(Y)))
+        M, N, K, r, _ptr(qa.codes), _ptr(qa.scales), _ptr(qa.xl1), _ptr(pw.codes), _ptr(pw.scales),
+        _ptr(pw.gscale), _ptr(pw.l2s), _ptr(bias), _ptr(Y), ldy, _stream(Y)))
     return Y
 
 
-def svdq_linear_forward(X: torch.Tensor, g_x: float, pw: PackedWeight, bias: torch.Tensor | None = None,
+def svdq_linear_forward(X: torch.Tensor, pw: PackedWeight, bias: torch.Tensor | None = None,
                         out: torch.Tensor | None = None, workspace: torch.Tensor | None = None) -> torch.Tensor:
     _dev(X, "X", torch.bfloat16)
     M, K = X.shape
@@ -209,8 +225,8 @@ def svdq_linear_forward(X: torch.Tensor, g_x: float, pw: PackedWeight, bias: tor
     need = svdq_forward_workspace_size(M, K, r)
     ws = workspace if workspace is not None else torch.empty(max(need, 16), dtype=torch.uint8, device=X.device)
     _check("svdq_linear_forward", lib().svdq_linear_forward(
-        M, N, K, r, _ptr(X), ldx, float(g_x), _ptr(pw.codes), _ptr(pw.scales), _ptr(pw.g_w), _ptr(pw.l1t),
-        _ptr(pw.l2t), _ptr(bias), _ptr(Y), ldy, _ptr(ws), ws.numel(), _stream(X)))
+        M, N, K, r, _ptr(X), ldx, _ptr(pw.codes), _ptr(pw.scales), _ptr(pw.gscale), _ptr(pw.l1t),
+        _ptr(pw.l2s), _ptr(bias), _ptr(Y), ldy, _ptr(ws), ws.numel(), _stream(X)))
     return Y
 
 

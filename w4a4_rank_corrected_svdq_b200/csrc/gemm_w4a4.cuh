@@ -2,7 +2,10 @@
 // cores (tcgen05, kind::mxf4nvf4, UE4M3 scales per 16 K-elements) with the
 // low-rank up projection, the global scales and the bias fused in the epilogue:
 //
-//   Y[m,n] = bf16( g_x g_w * sum_k (cX SX)(cR SR)  +  sum_j XL1[m,j] L2[j,n]  +  b[n] )
+//   Y[m,n] = bf16( alpha * ( sum_k (cX SX)(cR SR) + sum_j XL1[m,j] (hi + lo)[n,j] ) + b[n] )
+//
+// where alpha = g_x g_w and hi + lo = L2^T / alpha (two bf16 parts, packed at
+// load time), so the low-rank term carries the up projection to ~2^-17.
 //
 // Blog "Bringing Nunchaku 4-bit Diffusion Inference to Diffusers", figure
 // caption in "Background: SVDQuant and Nunchaku": the low-rank up projection
@@ -13,13 +16,13 @@
 //  * warp 0     TMA producer: E2M1 code tiles (128 rows x 128 bytes, 128-byte
 //               swizzle) for A and B, their scale atoms (2 KB each, one bulk
 //               copy: the tiled scale layout is exactly what the MMA wants), and
-//               per tile the XL1 and L2^T tiles for the low-rank MMA.
+//               per tile the XL1, hi and lo tiles for the low-rank MMA.
 //  * warp 1     TMEM owner and MMA issuer (one thread): per 256-wide K block it
 //               moves the scales smem -> TMEM (tcgen05.cp) and issues four
-//               128x128x64 block-scaled MMAs; per tile it then issues r/16
-//               128x128x16 bf16 MMAs for XL1 . L2 into a separate accumulator
-//               (the global scales multiply only the 4-bit product).
-//  * warps 2-5  epilogue: TMEM -> registers, y = acc * (g_x g_w) + lr + b,
+//               128x128x64 block-scaled MMAs; per tile it then issues 2r/16
+//               128x128x16 bf16 MMAs for XL1 . (hi + lo) into a separate
+//               accumulator.
+//  * warps 2-5  epilogue: TMEM -> registers, y = alpha * (acc + lr) + b,
 //               bf16, global stores.
 // TMEM (512 columns): two 4-bit accumulators [0,128) and [128,256) so the
 // epilogue of one tile overlaps the main loop of the next, the low-rank
@@ -44,14 +47,14 @@ struct GemmCfg {
   static constexpr int kBBytes = kBN * kBKBytes;
   static constexpr int kSFBytes = 2048;  // 4 scale atoms of 512 bytes
   static constexpr int kStageBytes = kABytes + kBBytes + 2 * kSFBytes;
-  static constexpr int kStages = (R == 128) ? 4 : 5;
+  static constexpr int kStages = (R == 128) ? 3 : (R == 64 ? 4 : 5);
   static constexpr int kLrAtomCols = R < 64 ? R : 64;  // bf16 columns per swizzle atom row
   static constexpr int kLrAtoms = R / kLrAtomCols;
   static constexpr int kLrRowBytes = kLrAtomCols * 2;
   static constexpr int kLrAtomBytes = 128 * kLrRowBytes;
   static constexpr int kLrTileBytes = kLrAtoms * kLrAtomBytes;  // 128 x R bf16
   static constexpr int kLrOff = kStages * kStageBytes;
-  static constexpr int kBarOff = kLrOff + 2 * kLrTileBytes;
+  static constexpr int kBarOff = kLrOff + 3 * kLrTileBytes;  // XL1, hi, lo tiles
   static constexpr int kBarBytes = 256;
   static constexpr int kSmemBytes = kBarOff + kBarBytes + 1024;  // + alignment slack
   static constexpr SwizzleMode kLrSwizzle =
@@ -73,9 +76,9 @@ struct GemmBarriers {
 template <int R>
 __global__ void __launch_bounds__(kGemmThreads, 1) w4a4_gemm_kernel(
     const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
-    const __grid_constant__ CUtensorMap tm_xl1, const __grid_constant__ CUtensorMap tm_l2t,
-    const uint8_t* __restrict__ a_scales, const uint8_t* __restrict__ w_scales, float g_x,
-    const float* __restrict__ g_w, const __nv_bfloat16* __restrict__ bias, __nv_bfloat16* __restrict__ Y,
+    const __grid_constant__ CUtensorMap tm_xl1, const __grid_constant__ CUtensorMap tm_l2s,
+    const uint8_t* __restrict__ a_scales, const uint8_t* __restrict__ w_scales,
+    const float* __restrict__ gscale, const __nv_bfloat16* __restrict__ bias, __nv_bfloat16* __restrict__ Y,
     int64_t ldy, int M, int N, int K) {
   using C = GemmCfg<R>;
   constexpr int S = C::kStages;
@@ -83,7 +86,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) w4a4_gemm_kernel(
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   GemmBarriers* bars = reinterpret_cast<GemmBarriers*>(smem + C::kBarOff);
   uint8_t* lr_x = smem + C::kLrOff;
-  uint8_t* lr_w = lr_x + C::kLrTileBytes;
+  uint8_t* lr_hi = lr_x + C::kLrTileBytes;
+  uint8_t* lr_lo = lr_hi + C::kLrTileBytes;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -112,7 +116,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) w4a4_gemm_kernel(
     prefetch_tmap(&tm_a);
     prefetch_tmap(&tm_b);
     prefetch_tmap(&tm_xl1);
-    prefetch_tmap(&tm_l2t);
+    prefetch_tmap(&tm_l2s);
   }
   if (warp == 1) {
     tmem_alloc(&bars->tmem_base, 512);
@@ -152,10 +156,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1) w4a4_gemm_kernel(
         }
         if (!ok) break;
         if (!mbar_wait(&bars->lr_empty, (it & 1) ^ 1, abort)) { ok = false; break; }
-        mbar_arrive_expect_tx(&bars->lr_full, 2 * C::kLrTileBytes);
+        mbar_arrive_expect_tx(&bars->lr_full, 3 * C::kLrTileBytes);
         for (int a = 0; a < C::kLrAtoms; ++a) {
           tma_load_2d(lr_x + a * C::kLrAtomBytes, &tm_xl1, a * 64, mb * kBM, &bars->lr_full);
-          tma_load_2d(lr_w + a * C::kLrAtomBytes, &tm_l2t, a * 64, nb * kBN, &bars->lr_full);
+          tma_load_2d(lr_hi + a * C::kLrAtomBytes, &tm_l2s, a * 64, nb * kBN, &bars->lr_full);
+          tma_load_2d(lr_lo + a * C::kLrAtomBytes, &tm_l2s, a * 64, N + nb * kBN, &bars->lr_full);
         }
         ++lr_filled;
       }
@@ -210,13 +215,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1) w4a4_gemm_kernel(
         if (!mbar_wait(&bars->lr_full, it & 1, abort)) { ok = false; break; }
         if (it > 0 && !mbar_wait(&bars->acc_empty[b ^ 1], ((it - 1) >> 1) & 1, abort)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t sx = smem_u32(lr_x), sw = smem_u32(lr_w);
+        const uint32_t sx = smem_u32(lr_x), shi = smem_u32(lr_hi), slo = smem_u32(lr_lo);
         constexpr int kStepsPerAtom = C::kLrAtomCols / 16;
 #pragma unroll
         for (int j = 0; j < R / 16; ++j) {
           const uint32_t off = (j / kStepsPerAtom) * C::kLrAtomBytes + (j % kStepsPerAtom) * 32;
-          mma_bf16(t_lr, smem_desc(sx + off, 16, 8 * C::kLrRowBytes, C::kLrSwizzle),
-                   smem_desc(sw + off, 16, 8 * C::kLrRowBytes, C::kLrSwizzle), idesc_bf16, j != 0 ? 1u : 0u);
+          const uint64_t xdesc = smem_desc(sx + off, 16, 8 * C::kLrRowBytes, C::kLrSwizzle);
+          mma_bf16(t_lr, xdesc, smem_desc(shi + off, 16, 8 * C::kLrRowBytes, C::kLrSwizzle), idesc_bf16,
+                   j != 0 ? 1u : 0u);
+          mma_bf16(t_lr, xdesc, smem_desc(slo + off, 16, 8 * C::kLrRowBytes, C::kLrSwizzle), idesc_bf16, 1u);
         }
         tc_commit(&bars->lr_empty);
         tc_commit(&bars->acc_full[b]);
@@ -229,7 +236,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) w4a4_gemm_kernel(
   } else {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;  // TMEM lane quadrant this warp may access
-    const float alpha = __fmul_rn(g_x, *g_w);
+    const float alpha = gscale[2];
     int it = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
       const int mb = tile % num_mb, nb = tile / num_mb;
@@ -264,9 +271,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) w4a4_gemm_kernel(
         uint32_t packed[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const float y0 = __fadd_rn(__fmaf_rn(__uint_as_float(va[2 * i]), alpha, __uint_as_float(vl[2 * i])), bf[2 * i]);
-          const float y1 =
-              __fadd_rn(__fmaf_rn(__uint_as_float(va[2 * i + 1]), alpha, __uint_as_float(vl[2 * i + 1])), bf[2 * i + 1]);
+          const float s0 = __fadd_rn(__uint_as_float(va[2 * i]), __uint_as_float(vl[2 * i]));
+          const float s1 = __fadd_rn(__uint_as_float(va[2 * i + 1]), __uint_as_float(vl[2 * i + 1]));
+          const float y0 = __fmaf_rn(s0, alpha, bf[2 * i]);
+          const float y1 = __fmaf_rn(s1, alpha, bf[2 * i + 1]);
           const __nv_bfloat162 h = __floats2bfloat162_rn(y0, y1);
           packed[i] = *reinterpret_cast<const uint32_t*>(&h);
         }

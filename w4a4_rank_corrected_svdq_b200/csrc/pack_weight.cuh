@@ -99,11 +99,39 @@ __global__ void finalize_global_scale_kernel(float* g) {
   *g = (am == 0.0f) ? 1.0f : __fdiv_rn(am, kGlobalDivisor);
 }
 
+// gscale = {g_x, g_w, alpha = fp32(g_x g_w), 0}; gscale[1] holds the amax bits of R on entry.
+__global__ void finalize_gscale_kernel(float* gscale, const float* g_x) {
+  const float am = __uint_as_float(*reinterpret_cast<unsigned*>(gscale + 1));
+  const float gw = (am == 0.0f) ? 1.0f : __fdiv_rn(am, kGlobalDivisor);
+  const float gx = *g_x;
+  gscale[0] = gx;
+  gscale[1] = gw;
+  gscale[2] = __fmul_rn(gx, gw);
+  gscale[3] = 0.0f;
+}
+
+// l2s[0][n][j] = hi, l2s[1][n][j] = lo with v = fp32(L2[j][n] / alpha), hi = bf16(v), lo = bf16(v - hi).
+__global__ void make_l2s_kernel(const __nv_bfloat16* __restrict__ L2, const float* __restrict__ gscale,
+                                __nv_bfloat16* __restrict__ l2s, int N, int r) {
+  const float alpha = gscale[2];
+  const int64_t total = static_cast<int64_t>(N) * r;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t n = i / r;
+    const int j = static_cast<int>(i % r);
+    const float v = __fdiv_rn(__bfloat162float(L2[static_cast<int64_t>(j) * N + n]), alpha);
+    const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+    const __nv_bfloat16 lo = __float2bfloat16_rn(__fsub_rn(v, __bfloat162float(hi)));
+    l2s[i] = hi;
+    l2s[total + i] = lo;
+  }
+}
+
 // Pass 2: quantise R with g_w. Lanes 0-15 hold one 16-element block, 16-31 the next.
 template <int R>
 __global__ void __launch_bounds__(kPackThreads) residual_quant_kernel(
     const __nv_bfloat16* __restrict__ W, const __nv_bfloat16* __restrict__ L1,
-    const __nv_bfloat16* __restrict__ l2t, int N, int K, const float* __restrict__ g_w,
+    const __nv_bfloat16* __restrict__ l2t, int N, int K, const float* __restrict__ gscale,
     uint8_t* __restrict__ codes, uint8_t* __restrict__ scales) {
   const int lane = threadIdx.x & 31;
   const int gw = blockIdx.x * (kPackThreads / 32) + (threadIdx.x >> 5);
@@ -114,7 +142,7 @@ __global__ void __launch_bounds__(kPackThreads) residual_quant_kernel(
   const int k = slab * 32 + lane;
   float l1row[R];
   load_l1_row<R>(L1, k, l1row);
-  const float g = *g_w;
+  const float g = gscale[1];
   const float d = __fmul_rn(6.0f, g);
   const int n_end = min(N, n_begin + kPackRowsPerWarp);
   for (int n = n_begin; n < n_end; ++n) {

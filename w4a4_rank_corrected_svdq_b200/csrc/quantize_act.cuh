@@ -30,7 +30,7 @@ constexpr int kQuantRows = 128;
 
 template <int R>
 __global__ void __launch_bounds__(kQuantThreads) quantize_act_kernel(
-    const __nv_bfloat16* __restrict__ X, int64_t ldx, int M, int K, float g,
+    const __nv_bfloat16* __restrict__ X, int64_t ldx, int M, int K, const float* __restrict__ g_x,
     const __nv_bfloat16* __restrict__ l1t, uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
     __nv_bfloat16* __restrict__ xl1, int kchunk) {
   namespace cg = cooperative_groups;
@@ -52,6 +52,7 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_act_kernel(
   const bool v1 = row1 < M;
   const int k_begin = ks * kchunk;
   const int k_end = min(K, k_begin + kchunk);
+  const float g = *g_x;
   const float d = __fmul_rn(6.0f, g);
 
   const __nv_bfloat16* x0 = X + static_cast<int64_t>(v0 ? row0 : 0) * ldx;

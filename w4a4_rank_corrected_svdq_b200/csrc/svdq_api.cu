@@ -121,7 +121,7 @@ CUtensorMapSwizzle lr_swizzle(int r) {
 
 // ------------------------------------------------------------------ launches
 template <int R>
-svdq_status launch_quantize(int M, int K, const void* X, int64_t ldx, float g_x, const void* l1t, void* codes,
+svdq_status launch_quantize(int M, int K, const void* X, int64_t ldx, const float* g_x, const void* l1t, void* codes,
                             void* scales, void* xl1, cudaStream_t stream, int sm_count) {
   const int row_tiles = (M + kQuantRows - 1) / kQuantRows;
   int ks = 1;
@@ -149,7 +149,7 @@ svdq_status launch_quantize(int M, int K, const void* X, int64_t ldx, float g_x,
   return launch_status();
 }
 
-svdq_status quantize_dispatch(int M, int K, int r, const void* X, int64_t ldx, float g_x, const void* l1t,
+svdq_status quantize_dispatch(int M, int K, int r, const void* X, int64_t ldx, const float* g_x, const void* l1t,
                               void* codes, void* scales, void* xl1, cudaStream_t st, int sms) {
   switch (r) {
     case 16: return launch_quantize<16>(M, K, X, ldx, g_x, l1t, codes, scales, xl1, st, sms);
@@ -160,8 +160,8 @@ svdq_status quantize_dispatch(int M, int K, int r, const void* X, int64_t ldx, f
 }
 
 template <int R>
-svdq_status launch_gemm(int M, int N, int K, const void* a_codes, const void* a_scales, const void* xl1, float g_x,
-                        const void* w_codes, const void* w_scales, const float* g_w, const void* l2t,
+svdq_status launch_gemm(int M, int N, int K, const void* a_codes, const void* a_scales, const void* xl1,
+                        const void* w_codes, const void* w_scales, const float* gscale, const void* l2s,
                         const void* bias, void* Y, int64_t ldy, cudaStream_t stream, int sm_count) {
   using C = GemmCfg<R>;
   CUtensorMap tm_a, tm_b, tm_x, tm_l;
@@ -172,8 +172,8 @@ svdq_status launch_gemm(int M, int N, int K, const void* a_codes, const void* a_
                     CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_tmap_2d(&tm_x, xl1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, R, M, R * 2, C::kLrAtomCols, kBM,
                     lr_swizzle(R)) ||
-      !make_tmap_2d(&tm_l, l2t, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, R, N, R * 2, C::kLrAtomCols, kBN,
-                    lr_swizzle(R)))
+      !make_tmap_2d(&tm_l, l2s, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, R, 2 * static_cast<uint64_t>(N), R * 2,
+                    C::kLrAtomCols, kBN, lr_swizzle(R)))
     return SVDQ_ERR_CUDA;
   auto kern = w4a4_gemm_kernel<R>;
   static std::atomic<uint64_t> attr_done{0};
@@ -181,24 +181,20 @@ svdq_status launch_gemm(int M, int N, int K, const void* a_codes, const void* a_
   const int tiles = ((M + kBM - 1) / kBM) * (N / kBN);
   const int grid = tiles < sm_count ? tiles : sm_count;
   kern<<<grid, kGemmThreads, C::kSmemBytes, stream>>>(
-      tm_a, tm_b, tm_x, tm_l, static_cast<const uint8_t*>(a_scales), static_cast<const uint8_t*>(w_scales), g_x, g_w,
+      tm_a, tm_b, tm_x, tm_l, static_cast<const uint8_t*>(a_scales), static_cast<const uint8_t*>(w_scales), gscale,
       static_cast<const __nv_bfloat16*>(bias), static_cast<__nv_bfloat16*>(Y), ldy, M, N, K);
   return launch_status();
 }
 
 svdq_status gemm_dispatch(int M, int N, int K, int r, const void* a_codes, const void* a_scales, const void* xl1,
-                          float g_x, const void* w_codes, const void* w_scales, const float* g_w, const void* l2t,
+                          const void* w_codes, const void* w_scales, const float* gscale, const void* l2s,
                           const void* bias, void* Y, int64_t ldy, cudaStream_t st, int sms) {
   switch (r) {
-    case 16:
-      return launch_gemm<16>(M, N, K, a_codes, a_scales, xl1, g_x, w_codes, w_scales, g_w, l2t, bias, Y, ldy, st, sms);
-    case 32:
-      return launch_gemm<32>(M, N, K, a_codes, a_scales, xl1, g_x, w_codes, w_scales, g_w, l2t, bias, Y, ldy, st, sms);
-    case 64:
-      return launch_gemm<64>(M, N, K, a_codes, a_scales, xl1, g_x, w_codes, w_scales, g_w, l2t, bias, Y, ldy, st, sms);
+    case 16: return launch_gemm<16>(M, N, K, a_codes, a_scales, xl1, w_codes, w_scales, gscale, l2s, bias, Y, ldy, st, sms);
+    case 32: return launch_gemm<32>(M, N, K, a_codes, a_scales, xl1, w_codes, w_scales, gscale, l2s, bias, Y, ldy, st, sms);
+    case 64: return launch_gemm<64>(M, N, K, a_codes, a_scales, xl1, w_codes, w_scales, gscale, l2s, bias, Y, ldy, st, sms);
     default:
-      return launch_gemm<128>(M, N, K, a_codes, a_scales, xl1, g_x, w_codes, w_scales, g_w, l2t, bias, Y, ldy, st,
-                              sms);
+      return launch_gemm<128>(M, N, K, a_codes, a_scales, xl1, w_codes, w_scales, gscale, l2s, bias, Y, ldy, st, sms);
   }
 }
 
@@ -222,19 +218,26 @@ __global__ void act_amax_kernel(const __nv_bfloat16* __restrict__ X, int64_t ldx
 }
 
 template <int R>
-svdq_status launch_pack(int N, int K, const void* W, const void* L1, const void* l2t, void* codes, void* scales,
-                        float* g_w, cudaStream_t st) {
+svdq_status launch_pack(int N, int K, const void* W, const void* L1, const void* L2, const float* g_x, void* codes,
+                        void* scales, float* gscale, void* l2s, cudaStream_t st) {
+  // The residual kernels read L2 transposed (N x r); plane 1 of l2s serves as
+  // that scratch until make_l2s_kernel overwrites both planes at the end.
+  __nv_bfloat16* l2t_scratch = static_cast<__nv_bfloat16*>(l2s) + static_cast<size_t>(N) * R;
+  transpose_bf16_kernel<<<dim3((N + 31) / 32, (R + 31) / 32), 256, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(L2), l2t_scratch, R, N);
   const int warps = (K / 32) * ((N + kPackRowsPerWarp - 1) / kPackRowsPerWarp);
   const int blocks = (warps + kPackThreads / 32 - 1) / (kPackThreads / 32);
-  if (cudaMemsetAsync(g_w, 0, sizeof(float), st) != cudaSuccess) return launch_status();
+  if (cudaMemsetAsync(gscale, 0, 4 * sizeof(float), st) != cudaSuccess) return launch_status();
   residual_amax_kernel<R><<<blocks, kPackThreads, 0, st>>>(static_cast<const __nv_bfloat16*>(W),
-                                                           static_cast<const __nv_bfloat16*>(L1),
-                                                           static_cast<const __nv_bfloat16*>(l2t), N, K,
-                                                           reinterpret_cast<unsigned*>(g_w));
-  finalize_global_scale_kernel<<<1, 1, 0, st>>>(g_w);
+                                                           static_cast<const __nv_bfloat16*>(L1), l2t_scratch, N, K,
+                                                           reinterpret_cast<unsigned*>(gscale + 1));
+  finalize_gscale_kernel<<<1, 1, 0, st>>>(gscale, g_x);
   residual_quant_kernel<R><<<blocks, kPackThreads, 0, st>>>(
-      static_cast<const __nv_bfloat16*>(W), static_cast<const __nv_bfloat16*>(L1),
-      static_cast<const __nv_bfloat16*>(l2t), N, K, g_w, static_cast<uint8_t*>(codes), static_cast<uint8_t*>(scales));
+      static_cast<const __nv_bfloat16*>(W), static_cast<const __nv_bfloat16*>(L1), l2t_scratch, N, K, gscale,
+      static_cast<uint8_t*>(codes), static_cast<uint8_t*>(scales));
+  const int64_t total = static_cast<int64_t>(N) * R;
+  make_l2s_kernel<<<static_cast<int>((total + 255) / 256), 256, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(L2), gscale, static_cast<__nv_bfloat16*>(l2s), N, R);
   return launch_status();
 }
 
@@ -276,14 +279,14 @@ svdq_status svdq_scale_offset(int K, int row, int kblock, size_t* out) {
 }
 
 svdq_status svdq_weight_sizes(int N, int K, int r, size_t* codes_bytes, size_t* scales_bytes, size_t* l1t_bytes,
-                              size_t* l2t_bytes) {
+                              size_t* l2s_bytes) {
   const svdq_status s = check_layer_shape(N, K, r);
   if (s != SVDQ_OK) return s;
-  if (!codes_bytes || !scales_bytes || !l1t_bytes || !l2t_bytes) return SVDQ_ERR_INVALID_ARG;
+  if (!codes_bytes || !scales_bytes || !l1t_bytes || !l2s_bytes) return SVDQ_ERR_INVALID_ARG;
   *codes_bytes = static_cast<size_t>(N) * (K / 2);
   *scales_bytes = static_cast<size_t>(N) * (K / 16);
   *l1t_bytes = static_cast<size_t>(r) * K * 2;
-  *l2t_bytes = static_cast<size_t>(N) * r * 2;
+  *l2s_bytes = static_cast<size_t>(N) * r * 2 * 2;
   return SVDQ_OK;
 }
 
@@ -305,28 +308,26 @@ svdq_status svdq_forward_workspace_size(int M, int K, int r, size_t* bytes) {
   return SVDQ_OK;
 }
 
-svdq_status svdq_pack_weight(int N, int K, int r, const void* W, const void* L1, const void* L2, void* w_codes,
-                             void* w_scales, float* g_w, void* l1t, void* l2t, void* stream) {
+svdq_status svdq_pack_weight(int N, int K, int r, const void* W, const void* L1, const void* L2, const float* g_x,
+                             void* w_codes, void* w_scales, float* gscale, void* l1t, void* l2s, void* stream) {
   svdq_status s = check_layer_shape(N, K, r);
   if (s != SVDQ_OK) return s;
-  if (!W || !L1 || !L2 || !w_codes || !w_scales || !g_w || !l1t || !l2t) return SVDQ_ERR_INVALID_ARG;
+  if (!W || !L1 || !L2 || !g_x || !w_codes || !w_scales || !gscale || !l1t || !l2s) return SVDQ_ERR_INVALID_ARG;
   if (!aligned16(W) || !aligned16(L1) || !aligned16(L2) || !aligned16(w_codes) || !aligned16(w_scales) ||
-      !aligned16(l1t) || !aligned16(l2t) || (reinterpret_cast<uintptr_t>(g_w) & 3u))
+      !aligned16(l1t) || !aligned16(l2s) || !aligned16(gscale) || (reinterpret_cast<uintptr_t>(g_x) & 3u))
     return SVDQ_ERR_MISALIGNED;
   DeviceInfo di;
   if ((s = current_device(nullptr, &di)) != SVDQ_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  // l2t = L2^T (N x r), l1t = L1^T (r x K)
-  transpose_bf16_kernel<<<dim3((N + 31) / 32, (r + 31) / 32), 256, 0, st>>>(
-      static_cast<const __nv_bfloat16*>(L2), static_cast<__nv_bfloat16*>(l2t), r, N);
+  // l1t = L1^T (r x K)
   transpose_bf16_kernel<<<dim3((r + 31) / 32, (K + 31) / 32), 256, 0, st>>>(
       static_cast<const __nv_bfloat16*>(L1), static_cast<__nv_bfloat16*>(l1t), K, r);
   if ((s = launch_status()) != SVDQ_OK) return s;
   switch (r) {
-    case 16: return launch_pack<16>(N, K, W, L1, l2t, w_codes, w_scales, g_w, st);
-    case 32: return launch_pack<32>(N, K, W, L1, l2t, w_codes, w_scales, g_w, st);
-    case 64: return launch_pack<64>(N, K, W, L1, l2t, w_codes, w_scales, g_w, st);
-    default: return launch_pack<128>(N, K, W, L1, l2t, w_codes, w_scales, g_w, st);
+    case 16: return launch_pack<16>(N, K, W, L1, L2, g_x, w_codes, w_scales, gscale, l2s, st);
+    case 32: return launch_pack<32>(N, K, W, L1, L2, g_x, w_codes, w_scales, gscale, l2s, st);
+    case 64: return launch_pack<64>(N, K, W, L1, L2, g_x, w_codes, w_scales, gscale, l2s, st);
+    default: return launch_pack<128>(N, K, W, L1, L2, g_x, w_codes, w_scales, gscale, l2s, st);
   }
 }
 
@@ -350,13 +351,14 @@ svdq_status svdq_act_global_scale(int M, int K, const void* X, int64_t ldx, floa
   return launch_status();
 }
 
-svdq_status svdq_quantize_act(int M, int K, int r, const void* X, int64_t ldx, float g_x, const void* l1t,
+svdq_status svdq_quantize_act(int M, int K, int r, const void* X, int64_t ldx, const float* g_x, const void* l1t,
                               void* codes, void* scales, void* xl1, void* stream) {
   if (M < 0 || K <= 0 || !valid_rank(r)) return SVDQ_ERR_INVALID_ARG;
   if (K % 256 != 0 || ldx < K || ldx % 8 != 0) return SVDQ_ERR_UNSUPPORTED_SHAPE;
   if (M == 0) return SVDQ_OK;
-  if (!X || !l1t || !codes || !scales || !xl1) return SVDQ_ERR_INVALID_ARG;
-  if (!aligned16(X) || !aligned16(l1t) || !aligned16(codes) || !aligned16(scales) || !aligned16(xl1))
+  if (!X || !g_x || !l1t || !codes || !scales || !xl1) return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(l1t) || !aligned16(codes) || !aligned16(scales) || !aligned16(xl1) ||
+      (reinterpret_cast<uintptr_t>(g_x) & 3u))
     return SVDQ_ERR_MISALIGNED;
   svdq_status s;
   DeviceInfo di;
@@ -366,28 +368,27 @@ svdq_status svdq_quantize_act(int M, int K, int r, const void* X, int64_t ldx, f
 }
 
 svdq_status svdq_w4a4_gemm(int M, int N, int K, int r, const void* a_codes, const void* a_scales, const void* xl1,
-                           float g_x, const void* w_codes, const void* w_scales, const float* g_w, const void* l2t,
+                           const void* w_codes, const void* w_scales, const float* gscale, const void* l2s,
                            const void* bias, void* Y, int64_t ldy, void* stream) {
   if (M < 0) return SVDQ_ERR_INVALID_ARG;
   svdq_status s = check_layer_shape(N, K, r);
   if (s != SVDQ_OK) return s;
   if (ldy < N || ldy % 8 != 0) return SVDQ_ERR_UNSUPPORTED_SHAPE;
   if (M == 0) return SVDQ_OK;
-  if (!a_codes || !a_scales || !xl1 || !w_codes || !w_scales || !g_w || !l2t || !Y) return SVDQ_ERR_INVALID_ARG;
+  if (!a_codes || !a_scales || !xl1 || !w_codes || !w_scales || !gscale || !l2s || !Y) return SVDQ_ERR_INVALID_ARG;
   if (!aligned16(a_codes) || !aligned16(a_scales) || !aligned16(xl1) || !aligned16(w_codes) ||
-      !aligned16(w_scales) || !aligned16(l2t) || !aligned16(Y) || (bias && !aligned16(bias)) ||
-      (reinterpret_cast<uintptr_t>(g_w) & 3u))
+      !aligned16(w_scales) || !aligned16(l2s) || !aligned16(Y) || (bias && !aligned16(bias)) || !aligned16(gscale))
     return SVDQ_ERR_MISALIGNED;
   DeviceInfo di;
   if ((s = current_device(nullptr, &di)) != SVDQ_OK) return s;
-  return gemm_dispatch(M, N, K, r, a_codes, a_scales, xl1, g_x, w_codes, w_scales, g_w, l2t, bias, Y, ldy,
+  return gemm_dispatch(M, N, K, r, a_codes, a_scales, xl1, w_codes, w_scales, gscale, l2s, bias, Y, ldy,
                        static_cast<cudaStream_t>(stream), di.sm_count);
 }
 
-svdq_status svdq_linear_forward(int M, int N, int K, int r, const void* X, int64_t ldx, float g_x,
-                                const void* w_codes, const void* w_scales, const float* g_w, const void* l1t,
-                                const void* l2t, const void* bias, void* Y, int64_t ldy, void* workspace,
-                                size_t workspace_bytes, void* stream) {
+svdq_status svdq_linear_forward(int M, int N, int K, int r, const void* X, int64_t ldx, const void* w_codes,
+                                const void* w_scales, const float* gscale, const void* l1t, const void* l2s,
+                                const void* bias, void* Y, int64_t ldy, void* workspace, size_t workspace_bytes,
+                                void* stream) {
   if (M < 0) return SVDQ_ERR_INVALID_ARG;
   svdq_status s = check_layer_shape(N, K, r);
   if (s != SVDQ_OK) return s;
@@ -403,9 +404,10 @@ svdq_status svdq_linear_forward(int M, int N, int K, int r, const void* X, int64
   uint8_t* a_codes = ws;
   uint8_t* a_scales = ws + round_up(c, 256);
   uint8_t* xl1 = a_scales + round_up(sc, 256);
-  s = svdq_quantize_act(M, K, r, X, ldx, g_x, l1t, a_codes, a_scales, xl1, stream);
+  if (!gscale) return SVDQ_ERR_INVALID_ARG;
+  s = svdq_quantize_act(M, K, r, X, ldx, gscale, l1t, a_codes, a_scales, xl1, stream);
   if (s != SVDQ_OK) return s;
-  return svdq_w4a4_gemm(M, N, K, r, a_codes, a_scales, xl1, g_x, w_codes, w_scales, g_w, l2t, bias, Y, ldy, stream);
+  return svdq_w4a4_gemm(M, N, K, r, a_codes, a_scales, xl1, w_codes, w_scales, gscale, l2s, bias, Y, ldy, stream);
 }
 
 svdq_status svdq_read_device_error(int* code, int clear) {
@@ -472,9 +474,9 @@ svdq_status noalloc_scratch(int dev, void** out) {
 }  // namespace svdq
 
 extern "C" svdq_status svdq_linear_forward_noalloc(int M, int N, int K, int r, const void* X, int64_t ldx,
-                                                   float g_x, const void* w_codes, const void* w_scales,
-                                                   const float* g_w, const void* l1t, const void* l2t,
-                                                   const void* bias, void* Y, int64_t ldy, void* stream) {
+                                                   const void* w_codes, const void* w_scales, const float* gscale,
+                                                   const void* l1t, const void* l2s, const void* bias, void* Y,
+                                                   int64_t ldy, void* stream) {
   if (M < 0) return SVDQ_ERR_INVALID_ARG;
   svdq_status s = check_layer_shape(N, K, r);
   if (s != SVDQ_OK) return s;
@@ -495,6 +497,6 @@ extern "C" svdq_status svdq_linear_forward_noalloc(int M, int N, int K, int r, c
   if ((s = noalloc_scratch(dev, &scratch)) != SVDQ_OK) return s;
   // Nothing in the scratch has to start at zero: the quantize kernel of this
   // call writes every byte the GEMM of this call reads.
-  return svdq_linear_forward(M, N, K, r, X, ldx, g_x, w_codes, w_scales, g_w, l1t, l2t, bias, Y, ldy, scratch,
+  return svdq_linear_forward(M, N, K, r, X, ldx, w_codes, w_scales, gscale, l1t, l2s, bias, Y, ldy, scratch,
                              kNoAllocScratchBytes, stream);
 }
