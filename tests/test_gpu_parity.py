@@ -178,3 +178,50 @@ def test_m_zero_is_noop(lib):
     X = torch.empty((0, 256), dtype=torch.bfloat16, device="cuda")
     Y = lib.svdq_linear_forward(X, pw)
     assert Y.shape == (0, 128)
+
+
+# ------------------------------------------------------------------ CTA-pair (2-SM) GEMM
+@pytest.mark.parametrize("M,K,N,r", [(1, 256, 256, 16), (129, 512, 512, 64), (300, 768, 256, 128),
+                                     (600, 1280, 768, 32), (4096, 512, 4096, 32), (2304, 256, 2560, 128)])
+def test_linear_forward_parity_pair_kernel(lib, monkeypatch, M, K, N, r):
+    """The 256x256-tile CTA-pair kernel (forced), including persistent loops over
+    several tiles per pair, partial row tiles and every rank."""
+    monkeypatch.setenv("SVDQ_GEMM_KERNEL", "2sm")
+    X, W, b, L1, L2 = _layer(M, K, N, r)
+    g_x = osv.act_global_scale(X)
+    pw = lib.svdq_pack_weight(W.cuda(), _to_dev(L1), _to_dev(L2), float(g_x))
+    Y = lib.svdq_linear_forward(X.cuda(), pw, b.cuda())
+    torch.cuda.synchronize()
+    assert lib.svdq_read_device_error() == 0
+    fwd = osv.forward(X, osv.pack_weight(W, L1, L2), b, g_x)
+    _check_y(Y, fwd)
+    # the single-CTA kernel computes the same layer
+    monkeypatch.setenv("SVDQ_GEMM_KERNEL", "1sm")
+    Y1 = lib.svdq_linear_forward(X.cuda(), pw, b.cuda())
+    torch.cuda.synchronize()
+    assert osv.rel_fro(_bf16_np(Y1), _bf16_np(Y)) <= REL_FRO
+
+
+def test_config2_full_size_sampled_rows(lib):
+    """The DiT fused-QKV workload at full size (M=4608, K=3072, N=9216, r=32) in
+    the launch configuration bench.py times; the oracle checks 96 sampled rows
+    (random ones plus the first and last) against the GPU output."""
+    spec = workloads.WORKLOADS[2].layers[0]
+    X, W, b = workloads.make_layer(spec)
+    L1, L2, _ = osv.lowrank_factors(W, spec.r)
+    g_x = osv.act_global_scale(X)
+    pw = lib.svdq_pack_weight(W.cuda(), _to_dev(L1), _to_dev(L2), float(g_x))
+    qa = lib.svdq_quantize_act(X.cuda(), pw)
+    Y = lib.svdq_w4a4_gemm(qa, pw, b.cuda())
+    torch.cuda.synchronize()
+    assert lib.svdq_read_device_error() == 0
+    rng = np.random.default_rng(17)
+    rows = np.unique(np.concatenate([[0, 1, spec.M - 1], rng.choice(spec.M, 93, replace=False)]))
+    ref_pw = osv.pack_weight(W, L1, L2)
+    codes = layouts.unpack_codes(pw.codes.cpu().numpy(), spec.N, spec.K)
+    assert np.array_equal(codes, ref_pw.codes)
+    fwd = osv.forward(X[rows], ref_pw, b, g_x)
+    act_codes = layouts.unpack_codes(qa.codes.cpu().numpy(), spec.M, spec.K)[rows]
+    act_scales = layouts.untile_scales(qa.scales.cpu().numpy(), spec.M, spec.K)[rows]
+    assert np.array_equal(act_codes, fwd.codes) and np.array_equal(act_scales, fwd.scales)
+    _check_y(Y, fwd, rows=rows)

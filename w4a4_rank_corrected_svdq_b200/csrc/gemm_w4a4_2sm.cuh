@@ -1,0 +1,426 @@
+// gemm_w4a4_2sm.cuh — the block-scaled NVFP4 GEMM of the SVDQuant W4A4 layer on
+// CTA pairs (tcgen05 cta_group::2), 256 x 256 output tiles:
+//
+//   Y[m,n] = bf16( alpha * ( sum_k (cX SX)(cR SR) + sum_j XL1[m,j] (hi + lo)[n,j] ) + b[n] )
+//
+// with alpha = g_x g_w and hi + lo = L2^T / alpha (packed at load time), so the
+// 4-bit product and the low-rank up projection share one fp32 accumulator
+// (blog "Bringing Nunchaku 4-bit Diffusion Inference to Diffusers", figure
+// caption in "Background: SVDQuant and Nunchaku": the up projection is fused
+// with the 4-bit compute kernel).
+//
+// A cluster of two CTAs on two SMs owns a 256 x 256 tile. Each CTA loads its
+// own 128 rows of A and its own 128 rows of B; one thread of the even CTA issues
+// 256x256xK MMAs that read both CTAs' shared memory and write each CTA's
+// 128 x 256 half of the accumulator into that CTA's TMEM. Per 256-wide K block
+// and SM this moves 38 KB for 8.4 MFLOP (half the bytes per FLOP of a 128 x 128
+// single-CTA tile), which keeps the L2 -> SM traffic within what L2 delivers.
+// No load uses cluster multicast: each CTA fetches every byte it stores.
+//
+// Roles (320 threads per CTA):
+//  * warp 0     TMA producer (both CTAs): per tile first r/c low-rank stages
+//               (XL1 columns, hi and lo columns of l2s; c = min(r, 32)), then
+//               K/256 stages of E2M1 codes (128-byte swizzle) and UE4M3 scale
+//               atoms. Completion bytes of both CTAs land on the even CTA's
+//               barrier (cp.async.bulk.tensor .cta_group::2).
+//  * warp 1     TMEM owner (both CTAs, 512 columns); in the even CTA lane 0
+//               issues the MMAs and the scale copies smem -> TMEM.
+//  * warps 2-9  epilogue (both CTAs): TMEM -> registers, y = alpha acc + b,
+//               bf16 stores; two warps per 32-lane TMEM quadrant, one per
+//               128-column half.
+// TMEM: accumulator 0 = columns [0,256), accumulator 1 = [208,464): the two
+// share [208,256), which the epilogue reads first and releases early, so the
+// next tile's MMAs start long before the previous tile is fully stored; scale
+// factors at [464,480) (A) and [480,512) (B, 256 rows).
+// Every wait is bounded; see mbar_wait.
+#pragma once
+
+#include "ptx.cuh"
+
+namespace svdq {
+
+// ------------------------------------------------------------------ cluster / 2-SM PTX
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// Address of the same shared-memory object in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// As mbar_wait, with cluster-scope acquire (arrivals come from both CTAs).
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  const uint32_t a = smem_u32(bar);
+  if (mbar_try_wait_cluster(a, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 32; ++i)
+      if (mbar_try_wait_cluster(a, parity)) return true;
+    if (*abort) return false;
+    if (globaltimer() - t0 > kWaitLimitNs) {
+      record_error(6);
+      *abort = 1;
+      return false;
+    }
+  }
+}
+// 2-D tiled load into this CTA's shared memory; the completion bytes are counted
+// on the barrier at `bar_cluster` (the even CTA's barrier).
+__device__ __forceinline__ void tma_load_2d_cg2(void* dst, const CUtensorMap* m, int x, int y, uint32_t bar_cluster) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+      "[%4];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(x), "r"(y), "r"(bar_cluster)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_alloc_cg2(uint32_t* dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_cg2() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_cg2(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void mma_nvf4_cg2(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                             uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+          d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+__device__ __forceinline__ void mma_bf16_cg2(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                             uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_cp_cg2(uint32_t taddr, uint64_t s_desc) {
+  asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(s_desc) : "memory");
+}
+// Arrives on the barrier at this shared-memory offset in every CTA of `mask`
+// once all prior tcgen05 operations of this thread have completed.
+__device__ __forceinline__ void tc_commit_cg2_mc(uint64_t* bar, uint16_t mask) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+                   smem_u32(bar)),
+               "h"(mask)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+}
+
+// ------------------------------------------------------------------ configuration
+constexpr int k2Threads = 320;
+constexpr int k2TileM = 256;  // per CTA pair; 128 rows per CTA
+constexpr int k2TileN = 256;  // per CTA pair; each CTA loads 128 rows of B
+constexpr int k2Acc1Col = 208;
+constexpr int k2SfaCol = 464;
+constexpr int k2SfbCol = 480;
+
+template <int R>
+struct Gemm2Cfg {
+  static constexpr int kABytes = 128 * 128;     // 128 rows x 256 E2M1
+  static constexpr int kBBytes = 128 * 128;
+  static constexpr int kSfaBytes = 2048;        // 4 atoms: 128 rows x 4 x 16 scales
+  static constexpr int kSfbBytes = 4096;        // 2 x 4 atoms: 256 rows
+  static constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;  // 38 KB
+  static constexpr int kStages = 5;
+  static constexpr int kLrCols = R < 32 ? R : 32;           // low-rank columns per stage
+  static constexpr int kLrSteps = R / kLrCols;              // low-rank stages per tile
+  static constexpr int kLrRowBytes = kLrCols * 2;
+  static constexpr int kLrTileBytes = 128 * kLrRowBytes;    // per operand per CTA
+  static constexpr SwizzleMode kLrSwizzle = kLrRowBytes == 64 ? kSwizzle64B : kSwizzle32B;
+  static constexpr uint32_t kMainTx = 2u * kStageBytes;     // both CTAs
+  static constexpr uint32_t kLrTx = 2u * 3u * kLrTileBytes;
+  static constexpr int kBarOff = kStages * kStageBytes;
+  static constexpr int kSmemBytes = kBarOff + 256 + 1024;
+};
+
+struct Gemm2Barriers {
+  uint64_t full[8];
+  uint64_t empty[8];
+  uint64_t acc_full[2];
+  uint64_t acc_empty[2];
+  uint64_t ovl_free;
+  uint64_t teardown;
+  uint32_t tmem_base;
+  int abort;
+};
+
+// One epilogue warp's 128-column half of a tile: eight 16-column chunks
+// starting at chunk FIRST (wrapping). If the warp holds the columns shared by
+// the two accumulators, it releases them after the first three chunks.
+template <int FIRST>
+__device__ __forceinline__ void epilogue_half(uint32_t taddr, const uint4 (&bv)[16], float alpha,
+                                              __nv_bfloat16* yrow, bool holds_overlap, uint32_t ovl_bar, int lane) {
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int ch = (FIRST + i) & 7;
+    uint32_t v[16];
+    tmem_ld_32x32b_x16(taddr + 16 * ch, v);
+    tmem_ld_wait();
+    if (i == 2 && holds_overlap) {
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(ovl_bar);
+    }
+    const uint32_t bw[8] = {bv[2 * ch].x,     bv[2 * ch].y,     bv[2 * ch].z,     bv[2 * ch].w,
+                            bv[2 * ch + 1].x, bv[2 * ch + 1].y, bv[2 * ch + 1].z, bv[2 * ch + 1].w};
+    uint32_t packed[8];
+#pragma unroll
+    for (int p = 0; p < 8; ++p) {
+      const float b0 = __uint_as_float(bw[p] << 16);
+      const float b1 = __uint_as_float(bw[p] & 0xFFFF0000u);
+      const float y0 = __fmaf_rn(__uint_as_float(v[2 * p]), alpha, b0);
+      const float y1 = __fmaf_rn(__uint_as_float(v[2 * p + 1]), alpha, b1);
+      const __nv_bfloat162 hv = __floats2bfloat162_rn(y0, y1);
+      packed[p] = *reinterpret_cast<const uint32_t*>(&hv);
+    }
+    if (yrow != nullptr) {
+      uint4* dst = reinterpret_cast<uint4*>(yrow + 16 * ch);
+      dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+      dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+    }
+  }
+}
+
+template <int R>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(k2Threads, 1) w4a4_gemm_2sm_kernel(
+    const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+    const __grid_constant__ CUtensorMap tm_sfa, const __grid_constant__ CUtensorMap tm_sfb,
+    const __grid_constant__ CUtensorMap tm_xl1, const __grid_constant__ CUtensorMap tm_l2s,
+    const float* __restrict__ gscale, const __nv_bfloat16* __restrict__ bias, __nv_bfloat16* __restrict__ Y,
+    int64_t ldy, int M, int N, int K) {
+  using C = Gemm2Cfg<R>;
+  constexpr int S = C::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Gemm2Barriers* bars = reinterpret_cast<Gemm2Barriers*>(smem + C::kBarOff);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+  const int num_mt = (M + k2TileM - 1) / k2TileM;
+  const int num_nt = N / k2TileN;
+  const int num_tiles = num_mt * num_nt;
+  const int pair = blockIdx.x >> 1;
+  const int num_pairs = gridDim.x >> 1;
+  const int nk = K / 256;
+  const int steps = C::kLrSteps + nk;
+  const int sf_row_stride = K / 64;  // scale atoms per 128-row block
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&bars->full[s], 1);
+      mbar_init(&bars->empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&bars->acc_full[b], 1);
+      mbar_init(&bars->acc_empty[b], 16);  // 8 epilogue warps x 2 CTAs
+    }
+    mbar_init(&bars->ovl_free, 8);         // 4 warps (the half holding the shared columns) x 2 CTAs
+    mbar_init(&bars->teardown, 1);
+    bars->abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tm_a);
+    prefetch_tmap(&tm_b);
+    prefetch_tmap(&tm_sfa);
+    prefetch_tmap(&tm_sfb);
+    prefetch_tmap(&tm_xl1);
+    prefetch_tmap(&tm_l2s);
+  }
+  if (warp == 1) {
+    tmem_alloc_cg2(&bars->tmem_base, 512);
+    tmem_relinquish_cg2();
+  }
+  tc_fence_before();
+  cluster_sync_all();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+  volatile int* abort = &bars->abort;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer (both CTAs)
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
+        const int mt = tile % num_mt, nt = tile / num_mt;
+        const int m_own = mt * k2TileM + static_cast<int>(rank) * 128;
+        const int n_own = nt * k2TileN + static_cast<int>(rank) * 128;
+        const int nblk = nt * 2;  // first 128-row block of B in this tile
+        for (int step = 0; step < steps; ++step) {
+          if (!mbar_wait(&bars->empty[s], ph ^ 1, abort)) { ok = false; break; }
+          uint8_t* st = smem + s * C::kStageBytes;
+          const uint32_t bar = mapa_shared(smem_u32(&bars->full[s]), 0);
+          if (step < C::kLrSteps) {
+            if (rank == 0) mbar_arrive_expect_tx(&bars->full[s], C::kLrTx);
+            const int x = step * C::kLrCols;
+            tma_load_2d_cg2(st, &tm_xl1, x, m_own, bar);
+            tma_load_2d_cg2(st + C::kABytes, &tm_l2s, x, n_own, bar);
+            tma_load_2d_cg2(st + C::kABytes + C::kLrTileBytes, &tm_l2s, x, N + n_own, bar);
+          } else {
+            const int kb = step - C::kLrSteps;
+            if (rank == 0) mbar_arrive_expect_tx(&bars->full[s], C::kMainTx);
+            tma_load_2d_cg2(st, &tm_a, kb * 128, m_own, bar);
+            tma_load_2d_cg2(st + C::kABytes, &tm_b, kb * 128, n_own, bar);
+            uint8_t* sf = st + C::kABytes + C::kBBytes;
+            tma_load_2d_cg2(sf, &tm_sfa, 0, ((m_own / 128) * sf_row_stride + 4 * kb) * 2, bar);
+            tma_load_2d_cg2(sf + C::kSfaBytes, &tm_sfb, 0, (nblk * sf_row_stride + 4 * kb) * 2, bar);
+            tma_load_2d_cg2(sf + C::kSfaBytes + 2048, &tm_sfb, 0, ((nblk + 1) * sf_row_stride + 4 * kb) * 2, bar);
+          }
+          if (++s == S) { s = 0; ph ^= 1; }
+        }
+      }
+      if (!ok) {
+        // error path: give copies that may still be in flight time to land
+        const uint64_t t0 = globaltimer();
+        while (globaltimer() - t0 < 2000000ull) {
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (even CTA)
+    if (rank == 0 && lane == 0) {
+      const uint32_t idesc_fp4 = (1u << 7) | (1u << 10) | (uint32_t(k2TileN >> 3) << 17) | (uint32_t(k2TileM >> 4) << 24);
+      const uint32_t idesc_bf16 =
+          (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(k2TileN >> 3) << 17) | (uint32_t(k2TileM >> 4) << 24);
+      const uint32_t t_sfa = tmem + k2SfaCol;
+      const uint32_t t_sfb = tmem + k2SfbCol;
+      int s = 0;
+      uint32_t ph = 0;
+      int it = 0;
+      bool ok = true;
+      for (int tile = pair; tile < num_tiles && ok; tile += num_pairs, ++it) {
+        const int b = it & 1;
+        const uint32_t t_acc = tmem + (b ? k2Acc1Col : 0);
+        if (!mbar_wait_cluster(&bars->acc_empty[b], ((it >> 1) & 1) ^ 1, abort)) { ok = false; break; }
+        if (it > 0 && !mbar_wait_cluster(&bars->ovl_free, (it - 1) & 1, abort)) { ok = false; break; }
+        tc_fence_after();
+        for (int step = 0; step < steps; ++step) {
+          if (!mbar_wait(&bars->full[s], ph, abort)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t st = smem_u32(smem + s * C::kStageBytes);
+          if (step < C::kLrSteps) {
+#pragma unroll
+            for (int k16 = 0; k16 < C::kLrCols / 16; ++k16) {
+              const uint64_t a = smem_desc(st + 32 * k16, 16, 8 * C::kLrRowBytes, C::kLrSwizzle);
+              const uint64_t bh = smem_desc(st + C::kABytes + 32 * k16, 16, 8 * C::kLrRowBytes, C::kLrSwizzle);
+              const uint64_t bl =
+                  smem_desc(st + C::kABytes + C::kLrTileBytes + 32 * k16, 16, 8 * C::kLrRowBytes, C::kLrSwizzle);
+              mma_bf16_cg2(t_acc, a, bh, idesc_bf16, (step | k16) != 0 ? 1u : 0u);
+              mma_bf16_cg2(t_acc, a, bl, idesc_bf16, 1u);
+            }
+          } else {
+            const uint32_t sfa = st + C::kABytes + C::kBBytes;
+            const uint32_t sfb = sfa + C::kSfaBytes;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              tmem_cp_cg2(t_sfa + 4 * j, smem_desc(sfa + 512 * j, 0, 128, kSwizzleNone));
+              tmem_cp_cg2(t_sfb + 8 * j, smem_desc(sfb + 512 * j, 0, 128, kSwizzleNone));
+              tmem_cp_cg2(t_sfb + 8 * j + 4, smem_desc(sfb + 2048 + 512 * j, 0, 128, kSwizzleNone));
+            }
+            const uint64_t adesc = smem_desc(st, 16, 1024, kSwizzle128B);
+            const uint64_t bdesc = smem_desc(st + C::kABytes, 16, 1024, kSwizzle128B);
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              mma_nvf4_cg2(t_acc, adesc + 2 * j, bdesc + 2 * j, idesc_fp4, t_sfa + 4 * j, t_sfb + 8 * j, 1u);
+          }
+          tc_commit_cg2_mc(&bars->empty[s], 0x3);
+          if (++s == S) { s = 0; ph ^= 1; }
+        }
+        if (!ok) break;
+        tc_commit_cg2_mc(&bars->acc_full[b], 0x3);
+      }
+      // every MMA this thread issued completes before TMEM is released
+      tc_commit(&bars->teardown);
+      volatile int never = 0;
+      mbar_wait(&bars->teardown, 0, &never);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (both CTAs)
+    const int e = warp - 2;
+    const int q = warp & 3;  // TMEM lane quadrant this warp may access
+    const int h = e >> 2;    // 128-column half of the tile
+    const float alpha = gscale[2];
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(32 * q) << 16);
+    const uint32_t ovl_bar = mapa_shared(smem_u32(&bars->ovl_free), 0);
+    int it = 0;
+    for (int tile = pair; tile < num_tiles; tile += num_pairs, ++it) {
+      const int mt = tile % num_mt, nt = tile / num_mt;
+      const int b = it & 1;
+      const int row = mt * k2TileM + static_cast<int>(rank) * 128 + 32 * q + lane;
+      const int col0 = nt * k2TileN + 128 * h;
+      // bias of this warp's 128 columns, fetched before the accumulator is ready
+      uint4 bv[16];
+      if (bias != nullptr) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) bv[i] = ldg_v4(bias + col0 + 8 * i);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) bv[i] = make_uint4(0u, 0u, 0u, 0u);
+      }
+      if (!mbar_wait(&bars->acc_full[b], (it >> 1) & 1, abort)) break;
+      tc_fence_after();
+      const uint32_t acc_col = (b ? k2Acc1Col : 0) + 128 * h;
+      // the half holding the shared columns [208,256) drains them first
+      const bool holds_overlap = (b == 0) ? (h == 1) : (h == 0);
+      __nv_bfloat16* yrow = (row < M) ? Y + static_cast<int64_t>(row) * ldy + col0 : nullptr;
+      if (b == 0 && h == 1)
+        epilogue_half<5>(lane_base + acc_col, bv, alpha, yrow, holds_overlap, ovl_bar, lane);
+      else
+        epilogue_half<0>(lane_base + acc_col, bv, alpha, yrow, holds_overlap, ovl_bar, lane);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&bars->acc_empty[b]), 0));
+    }
+  }
+
+  tc_fence_before();
+  cluster_sync_all();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_cg2(tmem, 512);
+  }
+}
+
+}  // namespace svdq

@@ -6,11 +6,13 @@
 
 #include <atomic>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
 #include "../../include/svdq.h"
 #include "gemm_w4a4.cuh"
+#include "gemm_w4a4_2sm.cuh"
 #include "pack_weight.cuh"
 #include "quantize_act.cuh"
 
@@ -186,16 +188,72 @@ svdq_status launch_gemm(int M, int N, int K, const void* a_codes, const void* a_
   return launch_status();
 }
 
+template <int R>
+svdq_status launch_gemm_2sm(int M, int N, int K, const void* a_codes, const void* a_scales, const void* xl1,
+                            const void* w_codes, const void* w_scales, const float* gscale, const void* l2s,
+                            const void* bias, void* Y, int64_t ldy, cudaStream_t stream, int sm_count) {
+  using C = Gemm2Cfg<R>;
+  CUtensorMap tm_a, tm_b, tm_sfa, tm_sfb, tm_x, tm_l;
+  const uint64_t kb = static_cast<uint64_t>(K / 2);
+  const uint64_t mpad = round_up(static_cast<size_t>(M), 128);
+  const CUtensorMapSwizzle lr_sw = C::kLrRowBytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B;
+  // scales as rows of 256 bytes: one 128-row x 256-K block is 8 consecutive rows
+  if (!make_tmap_2d(&tm_a, a_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, kb, M, kb, 128, 128,
+                    CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_tmap_2d(&tm_b, w_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, kb, N, kb, 128, 128,
+                    CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_tmap_2d(&tm_sfa, a_scales, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, 256, mpad * (K / 16) / 256, 256, 256, 8,
+                    CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !make_tmap_2d(&tm_sfb, w_scales, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, 256, static_cast<uint64_t>(N) * (K / 16) / 256,
+                    256, 256, 8, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !make_tmap_2d(&tm_x, xl1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, R, M, R * 2, C::kLrCols, 128, lr_sw) ||
+      !make_tmap_2d(&tm_l, l2s, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, R, 2 * static_cast<uint64_t>(N), R * 2,
+                    C::kLrCols, 128, lr_sw))
+    return SVDQ_ERR_CUDA;
+  auto kern = w4a4_gemm_2sm_kernel<R>;
+  static std::atomic<uint64_t> attr_done{0};
+  ensure_smem_attr(kern, C::kSmemBytes, attr_done);
+  const int tiles = ((M + k2TileM - 1) / k2TileM) * (N / k2TileN);
+  const int max_pairs = sm_count / 2;
+  const int pairs = tiles < max_pairs ? tiles : max_pairs;
+  kern<<<2 * pairs, k2Threads, C::kSmemBytes, stream>>>(tm_a, tm_b, tm_sfa, tm_sfb, tm_x, tm_l, gscale,
+                                                        static_cast<const __nv_bfloat16*>(bias),
+                                                        static_cast<__nv_bfloat16*>(Y), ldy, M, N, K);
+  return launch_status();
+}
+
+// Kernel choice: CTA-pair 256x256 tiles when N is a multiple of 256 and there
+// are enough rows to keep most SM pairs busy; otherwise single-CTA 128x128
+// tiles. SVDQ_GEMM_KERNEL=1sm|2sm overrides the choice (tests, benchmarks).
+bool use_2sm(int M, int N) {
+  if (N % 256 != 0) return false;
+  const char* env = std::getenv("SVDQ_GEMM_KERNEL");
+  if (env != nullptr) {
+    if (std::strcmp(env, "2sm") == 0) return true;
+    if (std::strcmp(env, "1sm") == 0) return false;
+  }
+  return M >= 512;
+}
+
 svdq_status gemm_dispatch(int M, int N, int K, int r, const void* a_codes, const void* a_scales, const void* xl1,
                           const void* w_codes, const void* w_scales, const float* gscale, const void* l2s,
                           const void* bias, void* Y, int64_t ldy, cudaStream_t st, int sms) {
-  switch (r) {
-    case 16: return launch_gemm<16>(M, N, K, a_codes, a_scales, xl1, w_codes, w_scales, gscale, l2s, bias, Y, ldy, st, sms);
-    case 32: return launch_gemm<32>(M, N, K, a_codes, a_scales, xl1, w_codes, w_scales, gscale, l2s, bias, Y, ldy, st, sms);
-    case 64: return launch_gemm<64>(M, N, K, a_codes, a_scales, xl1, w_codes, w_scales, gscale, l2s, bias, Y, ldy, st, sms);
-    default:
-      return launch_gemm<128>(M, N, K, a_codes, a_scales, xl1, w_codes, w_scales, gscale, l2s, bias, Y, ldy, st, sms);
+#define SVDQ_GEMM_ARGS M, N, K, a_codes, a_scales, xl1, w_codes, w_scales, gscale, l2s, bias, Y, ldy, st, sms
+  if (use_2sm(M, N)) {
+    switch (r) {
+      case 16: return launch_gemm_2sm<16>(SVDQ_GEMM_ARGS);
+      case 32: return launch_gemm_2sm<32>(SVDQ_GEMM_ARGS);
+      case 64: return launch_gemm_2sm<64>(SVDQ_GEMM_ARGS);
+      default: return launch_gemm_2sm<128>(SVDQ_GEMM_ARGS);
+    }
   }
+  switch (r) {
+    case 16: return launch_gemm<16>(SVDQ_GEMM_ARGS);
+    case 32: return launch_gemm<32>(SVDQ_GEMM_ARGS);
+    case 64: return launch_gemm<64>(SVDQ_GEMM_ARGS);
+    default: return launch_gemm<128>(SVDQ_GEMM_ARGS);
+  }
+#undef SVDQ_GEMM_ARGS
 }
 
 // amax|X| over an M x K bf16 matrix with row pitch ldx -> *g as fp32 bits.
