@@ -168,7 +168,9 @@ struct Gemm2Cfg {
   static constexpr SwizzleMode kLrSwizzle = kLrRowBytes == 64 ? kSwizzle64B : kSwizzle32B;
   static constexpr uint32_t kMainTx = 2u * kStageBytes;     // both CTAs
   static constexpr uint32_t kLrTx = 2u * 3u * kLrTileBytes;
-  static constexpr int kBarOff = kStages * kStageBytes;
+  static constexpr int kOutOff = kStages * kStageBytes;      // epilogue staging: 8 warps x 2 x 2 KB
+  static constexpr int kOutBytes = 8 * 2 * 2048;
+  static constexpr int kBarOff = kOutOff + kOutBytes;
   static constexpr int kSmemBytes = kBarOff + 256 + 1024;
 };
 
@@ -183,41 +185,78 @@ struct Gemm2Barriers {
   int abort;
 };
 
-// One epilogue warp's 128-column half of a tile: eight 16-column chunks
-// starting at chunk FIRST (wrapping). If the warp holds the columns shared by
-// the two accumulators, it releases them after the first three chunks.
-template <int FIRST>
-__device__ __forceinline__ void epilogue_half(uint32_t taddr, const uint4 (&bv)[16], float alpha,
-                                              __nv_bfloat16* yrow, bool holds_overlap, uint32_t ovl_bar, int lane) {
+// bf16 tile store from shared memory (TMA, async bulk group).
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* m, const void* src, int x, int y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                   reinterpret_cast<uint64_t>(m)),
+               "r"(x), "r"(y), "r"(smem_u32(src))
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// y = alpha * acc + b for one 32-column chunk of this lane's row, packed to
+// bf16 and written into a 32-row x 64-byte staging buffer in the 64-byte
+// swizzled order the Y tensor map expects; then lane 0 issues the TMA store.
+__device__ __forceinline__ void store_chunk(const uint32_t (&v)[32], const uint4 (&bv)[16], int c, float alpha,
+                                            uint8_t* stage, const CUtensorMap* tm_y, int x, int y, int lane) {
+  uint32_t packed[16];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int ch = (FIRST + i) & 7;
-    uint32_t v[16];
-    tmem_ld_32x32b_x16(taddr + 16 * ch, v);
-    tmem_ld_wait();
-    if (i == 2 && holds_overlap) {
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(ovl_bar);
-    }
-    const uint32_t bw[8] = {bv[2 * ch].x,     bv[2 * ch].y,     bv[2 * ch].z,     bv[2 * ch].w,
-                            bv[2 * ch + 1].x, bv[2 * ch + 1].y, bv[2 * ch + 1].z, bv[2 * ch + 1].w};
-    uint32_t packed[8];
-#pragma unroll
-    for (int p = 0; p < 8; ++p) {
-      const float b0 = __uint_as_float(bw[p] << 16);
-      const float b1 = __uint_as_float(bw[p] & 0xFFFF0000u);
-      const float y0 = __fmaf_rn(__uint_as_float(v[2 * p]), alpha, b0);
-      const float y1 = __fmaf_rn(__uint_as_float(v[2 * p + 1]), alpha, b1);
-      const __nv_bfloat162 hv = __floats2bfloat162_rn(y0, y1);
-      packed[p] = *reinterpret_cast<const uint32_t*>(&hv);
-    }
-    if (yrow != nullptr) {
-      uint4* dst = reinterpret_cast<uint4*>(yrow + 16 * ch);
-      dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-      dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
-    }
+  for (int p = 0; p < 16; ++p) {
+    const uint4 bq = bv[4 * c + p / 4];
+    const uint32_t bw = (p % 4 == 0) ? bq.x : (p % 4 == 1) ? bq.y : (p % 4 == 2) ? bq.z : bq.w;
+    const float y0 = __fmaf_rn(__uint_as_float(v[2 * p]), alpha, __uint_as_float(bw << 16));
+    const float y1 = __fmaf_rn(__uint_as_float(v[2 * p + 1]), alpha, __uint_as_float(bw & 0xFFFF0000u));
+    const __nv_bfloat162 hv = __floats2bfloat162_rn(y0, y1);
+    packed[p] = *reinterpret_cast<const uint32_t*>(&hv);
   }
+  if (lane == 0) bulk_wait_read1();  // the previous store from this buffer has read it
+  __syncwarp();
+  const int sw = (lane >> 1) & 3;
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+    *reinterpret_cast<uint4*>(stage + lane * 64 + ((j ^ sw) << 4)) =
+        make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0) {
+    tma_store_2d(tm_y, stage, x, y);
+    bulk_commit();
+  }
+}
+
+// One epilogue warp's 128-column half of a tile, in four 32-column chunks.
+// If the warp holds the columns shared by the two accumulators (chunks 2,3 of
+// accumulator 0's upper half; chunks 0,1 of accumulator 1's lower half), it
+// reads those first and releases them before doing any other work.
+template <int FIRST>
+__device__ __forceinline__ void epilogue_half(uint32_t taddr, const uint4 (&bv)[16], float alpha, uint8_t* stage,
+                                              int& nbuf, const CUtensorMap* tm_y, int x0, int y0, bool holds_overlap,
+                                              uint32_t ovl_bar, int lane) {
+  uint32_t va[32], vb[32];
+  tmem_ld_32x32b_x32(taddr + 32 * ((FIRST + 0) & 3), va);
+  tmem_ld_32x32b_x32(taddr + 32 * ((FIRST + 1) & 3), vb);
+  tmem_ld_wait();
+  if (holds_overlap) {
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive_cluster(ovl_bar);
+  }
+  store_chunk(va, bv, (FIRST + 0) & 3, alpha, stage + 2048 * (nbuf & 1), tm_y, x0 + 32 * ((FIRST + 0) & 3), y0, lane);
+  ++nbuf;
+  store_chunk(vb, bv, (FIRST + 1) & 3, alpha, stage + 2048 * (nbuf & 1), tm_y, x0 + 32 * ((FIRST + 1) & 3), y0, lane);
+  ++nbuf;
+  tmem_ld_32x32b_x32(taddr + 32 * ((FIRST + 2) & 3), va);
+  tmem_ld_32x32b_x32(taddr + 32 * ((FIRST + 3) & 3), vb);
+  tmem_ld_wait();
+  store_chunk(va, bv, (FIRST + 2) & 3, alpha, stage + 2048 * (nbuf & 1), tm_y, x0 + 32 * ((FIRST + 2) & 3), y0, lane);
+  ++nbuf;
+  store_chunk(vb, bv, (FIRST + 3) & 3, alpha, stage + 2048 * (nbuf & 1), tm_y, x0 + 32 * ((FIRST + 3) & 3), y0, lane);
+  ++nbuf;
 }
 
 template <int R>
@@ -225,8 +264,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(k2Threads, 1) w4a4_g
     const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
     const __grid_constant__ CUtensorMap tm_sfa, const __grid_constant__ CUtensorMap tm_sfb,
     const __grid_constant__ CUtensorMap tm_xl1, const __grid_constant__ CUtensorMap tm_l2s,
-    const float* __restrict__ gscale, const __nv_bfloat16* __restrict__ bias, __nv_bfloat16* __restrict__ Y,
-    int64_t ldy, int M, int N, int K) {
+    const __grid_constant__ CUtensorMap tm_y, const float* __restrict__ gscale,
+    const __nv_bfloat16* __restrict__ bias, int M, int N, int K) {
   using C = Gemm2Cfg<R>;
   constexpr int S = C::kStages;
   extern __shared__ uint8_t smem_raw[];
@@ -266,6 +305,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(k2Threads, 1) w4a4_g
     prefetch_tmap(&tm_sfb);
     prefetch_tmap(&tm_xl1);
     prefetch_tmap(&tm_l2s);
+    prefetch_tmap(&tm_y);
   }
   if (warp == 1) {
     tmem_alloc_cg2(&bars->tmem_base, 512);
@@ -384,11 +424,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(k2Threads, 1) w4a4_g
     const float alpha = gscale[2];
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(32 * q) << 16);
     const uint32_t ovl_bar = mapa_shared(smem_u32(&bars->ovl_free), 0);
+    uint8_t* stage = smem + C::kOutOff + e * 4096;
+    int nbuf = 0;
     int it = 0;
     for (int tile = pair; tile < num_tiles; tile += num_pairs, ++it) {
       const int mt = tile % num_mt, nt = tile / num_mt;
       const int b = it & 1;
-      const int row = mt * k2TileM + static_cast<int>(rank) * 128 + 32 * q + lane;
+      const int y0 = mt * k2TileM + static_cast<int>(rank) * 128 + 32 * q;
       const int col0 = nt * k2TileN + 128 * h;
       // bias of this warp's 128 columns, fetched before the accumulator is ready
       uint4 bv[16];
@@ -401,18 +443,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(k2Threads, 1) w4a4_g
       }
       if (!mbar_wait(&bars->acc_full[b], (it >> 1) & 1, abort)) break;
       tc_fence_after();
-      const uint32_t acc_col = (b ? k2Acc1Col : 0) + 128 * h;
-      // the half holding the shared columns [208,256) drains them first
-      const bool holds_overlap = (b == 0) ? (h == 1) : (h == 0);
-      __nv_bfloat16* yrow = (row < M) ? Y + static_cast<int64_t>(row) * ldy + col0 : nullptr;
+      const uint32_t acc = lane_base + (b ? k2Acc1Col : 0) + 128 * h;
       if (b == 0 && h == 1)
-        epilogue_half<5>(lane_base + acc_col, bv, alpha, yrow, holds_overlap, ovl_bar, lane);
+        epilogue_half<2>(acc, bv, alpha, stage, nbuf, &tm_y, col0, y0, true, ovl_bar, lane);
       else
-        epilogue_half<0>(lane_base + acc_col, bv, alpha, yrow, holds_overlap, ovl_bar, lane);
+        epilogue_half<0>(acc, bv, alpha, stage, nbuf, &tm_y, col0, y0, b == 1 && h == 0, ovl_bar, lane);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&bars->acc_empty[b]), 0));
     }
+    if (lane == 0) bulk_wait_all();
+    __syncwarp();
   }
 
   tc_fence_before();

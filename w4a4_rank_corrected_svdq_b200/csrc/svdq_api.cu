@@ -193,7 +193,7 @@ svdq_status launch_gemm_2sm(int M, int N, int K, const void* a_codes, const void
                             const void* w_codes, const void* w_scales, const float* gscale, const void* l2s,
                             const void* bias, void* Y, int64_t ldy, cudaStream_t stream, int sm_count) {
   using C = Gemm2Cfg<R>;
-  CUtensorMap tm_a, tm_b, tm_sfa, tm_sfb, tm_x, tm_l;
+  CUtensorMap tm_a, tm_b, tm_sfa, tm_sfb, tm_x, tm_l, tm_y;
   const uint64_t kb = static_cast<uint64_t>(K / 2);
   const uint64_t mpad = round_up(static_cast<size_t>(M), 128);
   const CUtensorMapSwizzle lr_sw = C::kLrRowBytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B;
@@ -208,7 +208,9 @@ svdq_status launch_gemm_2sm(int M, int N, int K, const void* a_codes, const void
                     256, 256, 8, CU_TENSOR_MAP_SWIZZLE_NONE) ||
       !make_tmap_2d(&tm_x, xl1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, R, M, R * 2, C::kLrCols, 128, lr_sw) ||
       !make_tmap_2d(&tm_l, l2s, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, R, 2 * static_cast<uint64_t>(N), R * 2,
-                    C::kLrCols, 128, lr_sw))
+                    C::kLrCols, 128, lr_sw) ||
+      !make_tmap_2d(&tm_y, Y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, M, static_cast<uint64_t>(ldy) * 2, 32, 32,
+                    CU_TENSOR_MAP_SWIZZLE_64B))
     return SVDQ_ERR_CUDA;
   auto kern = w4a4_gemm_2sm_kernel<R>;
   static std::atomic<uint64_t> attr_done{0};
@@ -216,9 +218,8 @@ svdq_status launch_gemm_2sm(int M, int N, int K, const void* a_codes, const void
   const int tiles = ((M + k2TileM - 1) / k2TileM) * (N / k2TileN);
   const int max_pairs = sm_count / 2;
   const int pairs = tiles < max_pairs ? tiles : max_pairs;
-  kern<<<2 * pairs, k2Threads, C::kSmemBytes, stream>>>(tm_a, tm_b, tm_sfa, tm_sfb, tm_x, tm_l, gscale,
-                                                        static_cast<const __nv_bfloat16*>(bias),
-                                                        static_cast<__nv_bfloat16*>(Y), ldy, M, N, K);
+  kern<<<2 * pairs, k2Threads, C::kSmemBytes, stream>>>(tm_a, tm_b, tm_sfa, tm_sfb, tm_x, tm_l, tm_y, gscale,
+                                                        static_cast<const __nv_bfloat16*>(bias), M, N, K);
   return launch_status();
 }
 
