@@ -94,6 +94,28 @@ __device__ __forceinline__ void tma_load_2d_cg2(void* dst, const CUtensorMap* m,
       "l"(reinterpret_cast<uint64_t>(m)), "r"(x), "r"(y), "r"(bar_cluster)
       : "memory");
 }
+// 4-D / 5-D tiled loads with .cta_group::2 completion (used for the scale
+// factors, whose tensor maps repeat each 512-byte atom four times through a
+// zero-stride dimension, producing the replicated layout TMEM needs).
+__device__ __forceinline__ void tma_load_4d_cg2(void* dst, const CUtensorMap* m, int c0, int c1, int c2, int c3,
+                                                uint32_t bar_cluster) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, "
+      "%4, %5}], [%6];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(bar_cluster)
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_5d_cg2(void* dst, const CUtensorMap* m, int c0, int c1, int c2, int c3, int c4,
+                                                uint32_t bar_cluster) {
+  asm volatile(
+      "cp.async.bulk.tensor.5d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, "
+      "%4, %5, %6}], [%7];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4), "r"(bar_cluster)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_cp_128x256b_cg2(uint32_t taddr, uint64_t s_desc) {
+  asm volatile("tcgen05.cp.cta_group::2.128x256b [%0], %1;" ::"r"(taddr), "l"(s_desc) : "memory");
+}
 __device__ __forceinline__ void tmem_alloc_cg2(uint32_t* dst_smem, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
                "r"(ncols)
@@ -157,10 +179,13 @@ template <int R>
 struct Gemm2Cfg {
   static constexpr int kABytes = 128 * 128;     // 128 rows x 256 E2M1
   static constexpr int kBBytes = 128 * 128;
-  static constexpr int kSfaBytes = 2048;        // 4 atoms: 128 rows x 4 x 16 scales
-  static constexpr int kSfbBytes = 4096;        // 2 x 4 atoms: 256 rows
-  static constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;  // 38 KB
-  static constexpr int kStages = 5;
+  // Scale factors are staged in smem already replicated four times (the
+  // layout TMEM needs), so that each tcgen05.cp 128x256b moves 32 bytes per
+  // lane: two K-steps of A scales, or one K-step of both 128-row halves of B.
+  static constexpr int kSfaBytes = 4 * 2048;    // 4 K-steps x 4 replicas x 512 B (128 rows)
+  static constexpr int kSfbBytes = 2 * 4 * 2048;  // 2 row blocks x 4 K-steps x 4 replicas x 512 B
+  static constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;  // 56 KB
+  static constexpr int kStages = 3;
   static constexpr int kLrCols = R < 32 ? R : 32;           // low-rank columns per stage
   static constexpr int kLrSteps = R / kLrCols;              // low-rank stages per tile
   static constexpr int kLrRowBytes = kLrCols * 2;
@@ -344,9 +369,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(k2Threads, 1) w4a4_g
             tma_load_2d_cg2(st, &tm_a, kb * 128, m_own, bar);
             tma_load_2d_cg2(st + C::kABytes, &tm_b, kb * 128, n_own, bar);
             uint8_t* sf = st + C::kABytes + C::kBBytes;
-            tma_load_2d_cg2(sf, &tm_sfa, 0, ((m_own / 128) * sf_row_stride + 4 * kb) * 2, bar);
-            tma_load_2d_cg2(sf + C::kSfaBytes, &tm_sfb, 0, (nblk * sf_row_stride + 4 * kb) * 2, bar);
-            tma_load_2d_cg2(sf + C::kSfaBytes + 2048, &tm_sfb, 0, ((nblk + 1) * sf_row_stride + 4 * kb) * 2, bar);
+            tma_load_4d_cg2(sf, &tm_sfa, 0, 0, 0, (m_own / 128) * sf_row_stride + 4 * kb, bar);
+            tma_load_5d_cg2(sf + C::kSfaBytes, &tm_sfb, 0, 0, 0, 4 * kb, nblk, bar);
           }
           if (++s == S) { s = 0; ph ^= 1; }
         }
@@ -393,12 +417,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(k2Threads, 1) w4a4_g
           } else {
             const uint32_t sfa = st + C::kABytes + C::kBBytes;
             const uint32_t sfb = sfa + C::kSfaBytes;
+            // A: K-steps (0,1) and (2,3), 2 KB apart; B: K-step j, row blocks 8 KB apart
+            tmem_cp_128x256b_cg2(t_sfa, smem_desc(sfa, 2048, 128, kSwizzleNone));
+            tmem_cp_128x256b_cg2(t_sfa + 8, smem_desc(sfa + 4096, 2048, 128, kSwizzleNone));
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              tmem_cp_cg2(t_sfa + 4 * j, smem_desc(sfa + 512 * j, 0, 128, kSwizzleNone));
-              tmem_cp_cg2(t_sfb + 8 * j, smem_desc(sfb + 512 * j, 0, 128, kSwizzleNone));
-              tmem_cp_cg2(t_sfb + 8 * j + 4, smem_desc(sfb + 2048 + 512 * j, 0, 128, kSwizzleNone));
-            }
+            for (int j = 0; j < 4; ++j)
+              tmem_cp_128x256b_cg2(t_sfb + 8 * j, smem_desc(sfb + 2048 * j, 8192, 128, kSwizzleNone));
             const uint64_t adesc = smem_desc(st, 16, 1024, kSwizzle128B);
             const uint64_t bdesc = smem_desc(st + C::kABytes, 16, 1024, kSwizzle128B);
 #pragma unroll

@@ -115,6 +115,41 @@ bool make_tmap_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int 
   return r == CUDA_SUCCESS;
 }
 
+// Tensor map of rank 2..5 over bytes or bf16 (dims / strides in elements / bytes).
+bool make_tmap(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int rank, const uint64_t* dims,
+               const uint64_t* strides_bytes, const uint32_t* box, CUtensorMapSwizzle sw) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t d[5];
+  cuuint64_t st[4];
+  cuuint32_t b[5], es[5];
+  for (int i = 0; i < rank; ++i) {
+    d[i] = dims[i];
+    b[i] = box[i];
+    es[i] = 1;
+    if (i + 1 < rank) st[i] = strides_bytes[i];
+  }
+  return fn(m, dt, rank, const_cast<void*>(base), d, st, b, es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Scale atoms (512 B) read four times each through a zero-stride dimension:
+// SFA: {256 B, 2 halves, 4 replicas, atoms}; box = 4 consecutive atoms (one
+// 256-wide K block of one 128-row block). SFB adds the row-block dimension;
+// box = 4 atoms of two consecutive 128-row blocks.
+bool make_sf_tmaps(CUtensorMap* sfa, const void* a_scales, uint64_t a_rows_pad, CUtensorMap* sfb,
+                   const void* w_scales, uint64_t n_rows, int K) {
+  const uint64_t atoms_per_rb = static_cast<uint64_t>(K / 64);
+  const uint64_t da[4] = {256, 2, 4, (a_rows_pad / 128) * atoms_per_rb};
+  const uint64_t sa[3] = {256, 0, 512};
+  const uint32_t ba[4] = {256, 2, 4, 4};
+  const uint64_t db[5] = {256, 2, 4, atoms_per_rb, n_rows / 128};
+  const uint64_t sb[4] = {256, 0, 512, atoms_per_rb * 512};
+  const uint32_t bb[5] = {256, 2, 4, 4, 2};
+  return make_tmap(sfa, a_scales, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, da, sa, ba, CU_TENSOR_MAP_SWIZZLE_NONE) &&
+         make_tmap(sfb, w_scales, CU_TENSOR_MAP_DATA_TYPE_UINT8, 5, db, sb, bb, CU_TENSOR_MAP_SWIZZLE_NONE);
+}
+
 CUtensorMapSwizzle lr_swizzle(int r) {
   const int row_bytes = (r < 64 ? r : 64) * 2;
   return row_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
@@ -197,15 +232,11 @@ svdq_status launch_gemm_2sm(int M, int N, int K, const void* a_codes, const void
   const uint64_t kb = static_cast<uint64_t>(K / 2);
   const uint64_t mpad = round_up(static_cast<size_t>(M), 128);
   const CUtensorMapSwizzle lr_sw = C::kLrRowBytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B;
-  // scales as rows of 256 bytes: one 128-row x 256-K block is 8 consecutive rows
   if (!make_tmap_2d(&tm_a, a_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, kb, M, kb, 128, 128,
                     CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_tmap_2d(&tm_b, w_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, kb, N, kb, 128, 128,
                     CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_tmap_2d(&tm_sfa, a_scales, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, 256, mpad * (K / 16) / 256, 256, 256, 8,
-                    CU_TENSOR_MAP_SWIZZLE_NONE) ||
-      !make_tmap_2d(&tm_sfb, w_scales, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, 256, static_cast<uint64_t>(N) * (K / 16) / 256,
-                    256, 256, 8, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !make_sf_tmaps(&tm_sfa, a_scales, mpad, &tm_sfb, w_scales, static_cast<uint64_t>(N), K) ||
       !make_tmap_2d(&tm_x, xl1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, R, M, R * 2, C::kLrCols, 128, lr_sw) ||
       !make_tmap_2d(&tm_l, l2s, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, R, 2 * static_cast<uint64_t>(N), R * 2,
                     C::kLrCols, 128, lr_sw) ||
