@@ -62,9 +62,24 @@ def _check_act(lib, X, L1, r, g_x, qa, M, K):
     if mpad > M:   # padding rows must hold zero scales
         pad = layouts.untile_scales(scales_buf, mpad, K)[M:]
         assert not pad.any()
-    xl1_ref = osv.down_proj(X, L1)
-    ulps = layouts.bf16_ulp_distance(_bf16_np(qa.xl1), xl1_ref)
-    assert ulps.max() <= 1, f"XL1 max ulp {ulps.max()}"
+    _check_xl1(_bf16_np(qa.xl1), X, L1)
+
+
+def _check_xl1(xl1_gpu, X, L1):
+    """XL1 = bf16(X . L1) accumulated in fp32: |gpu - exact| <= 1/2 ulp_bf16(gpu)
+    (the final rounding) + 2 K 2^-24 sum_k |x_k L1_kj| (fp32 summation in any
+    order, Higham's bound with a factor 2 of slack for tensor-core accumulation).
+    Where the sum does not cancel this is within one bf16 ulp of the oracle."""
+    X64, L164 = osv.to_f64(X), osv.to_f64(L1)
+    exact = X64 @ L164
+    absum = np.abs(X64) @ np.abs(L164)
+    K = X64.shape[1]
+    half_ulp = np.ldexp(1.0, np.frexp(np.abs(xl1_gpu))[1] - 9)
+    bound = half_ulp + 2.0 * K * 2.0 ** -24 * absum
+    err = np.abs(xl1_gpu - exact)
+    assert np.all(err <= bound), f"XL1 error {np.max(err / bound):.2f} x bound"
+    ulps = layouts.bf16_ulp_distance(xl1_gpu, osv.down_proj(X, L1))
+    assert np.mean(ulps > 1) < 1e-3, f"XL1: {np.mean(ulps > 1):.2e} of elements beyond 1 ulp"
 
 
 def _check_y(Y, fwd, rows=None):

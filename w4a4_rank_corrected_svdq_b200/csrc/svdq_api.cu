@@ -161,28 +161,47 @@ template <int R>
 svdq_status launch_quantize(int M, int K, const void* X, int64_t ldx, const float* g_x, const void* l1t, void* codes,
                             void* scales, void* xl1, cudaStream_t stream, int sm_count) {
   const int row_tiles = (M + kQuantRows - 1) / kQuantRows;
-  int ks = 1;
-  while (ks < 8 && row_tiles * ks < 2 * sm_count && (K / (2 * ks)) % 32 == 0 && K / (2 * ks) >= 128) ks *= 2;
-  const int kchunk = K / ks;
-  const size_t smem = static_cast<size_t>(kQuantRows) * R * sizeof(float);
   auto kern = quantize_act_kernel<R>;
   static std::atomic<uint64_t> attr_done{0};
-  ensure_smem_attr(kern, static_cast<int>(smem), attr_done);
+  ensure_smem_attr(kern, 227 * 1024, attr_done);
+  CUtensorMap tm_x, tm_l;
+  if (!make_tmap_2d(&tm_x, X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, M, static_cast<uint64_t>(ldx) * 2, 64,
+                    kQuantRows, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_tmap_2d(&tm_l, l1t, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, R, static_cast<uint64_t>(K) * 2, 64, R,
+                    CU_TENSOR_MAP_SWIZZLE_128B))
+    return SVDQ_ERR_CUDA;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(ks, row_tiles, 1);
   cfg.blockDim = dim3(kQuantThreads, 1, 1);
-  cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = ks;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaLaunchKernelEx(&cfg, kern, static_cast<const __nv_bfloat16*>(X), ldx, M, K, g_x,
-                     static_cast<const __nv_bfloat16*>(l1t), static_cast<uint8_t*>(codes),
-                     static_cast<uint8_t*>(scales), static_cast<__nv_bfloat16*>(xl1), kchunk);
+  // K-split into clusters of ks CTAs: grow ks (1, 2, 4) while the grid stays
+  // within one wave of co-resident clusters and there are fewer CTAs than SMs.
+  auto fits = [&](int ks_try) {
+    cfg.gridDim = dim3(ks_try, row_tiles, 1);
+    cfg.dynamicSmemBytes = quantize_smem_bytes<R>(K / ks_try);
+    attr[0].val.clusterDim.x = ks_try;
+    int clusters = 0;
+    if (cfg.dynamicSmemBytes > 227 * 1024) return false;
+    if (cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg) != cudaSuccess) {
+      cudaGetLastError();
+      return false;
+    }
+    return clusters >= row_tiles;
+  };
+  int ks = 1;
+  while (ks < 4 && row_tiles * ks < sm_count && fits(ks * 2)) ks *= 2;
+  if (quantize_smem_bytes<R>(K / ks) > 227 * 1024) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+  const int kchunk = K / ks;
+  cfg.gridDim = dim3(ks, row_tiles, 1);
+  cfg.dynamicSmemBytes = quantize_smem_bytes<R>(kchunk);
+  attr[0].val.clusterDim.x = ks;
+  cudaLaunchKernelEx(&cfg, kern, tm_x, tm_l, M, K, g_x, static_cast<uint8_t*>(codes), static_cast<uint8_t*>(scales),
+                     static_cast<__nv_bfloat16*>(xl1), kchunk);
   return launch_status();
 }
 
