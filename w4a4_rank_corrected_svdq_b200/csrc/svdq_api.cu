@@ -68,8 +68,49 @@ void ensure_smem_attr(Kernel kern, int bytes, std::atomic<uint64_t>& done) {
   const uint64_t bit = 1ull << (dev & 63);
   if (done.load(std::memory_order_acquire) & bit) return;
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  // Every kernel here stages through shared memory and barely uses L1: ask for
+  // the largest shared-memory carveout so that the occupancy queries (and the
+  // launches) count every CTA that fits.
+  cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
   done.fetch_or(bit, std::memory_order_acq_rel);
 }
+
+// cudaOccupancyMaxActiveClusters costs far more host time than a launch; its
+// answer depends only on (kernel, device, cluster size, dynamic shared memory),
+// so each answer is kept. A full table simply stops caching.
+class ClusterOccupancyCache {
+ public:
+  template <typename Kernel>
+  int get(Kernel kern, cudaLaunchConfig_t* cfg, int dev) {
+    const uint64_t key = (static_cast<uint64_t>(dev & 0xFF) << 56) |
+                         (static_cast<uint64_t>(cfg->attrs[0].val.clusterDim.x & 0xFF) << 48) |
+                         (static_cast<uint64_t>(cfg->dynamicSmemBytes) & 0xFFFFFFFFull);
+    {
+      std::lock_guard<std::mutex> lock(mu_);
+      for (int i = 0; i < n_; ++i)
+        if (keys_[i] == key) return vals_[i];
+    }
+    int clusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&clusters, kern, cfg) != cudaSuccess) {
+      cudaGetLastError();
+      clusters = 0;
+    }
+    std::lock_guard<std::mutex> lock(mu_);
+    if (n_ < kSlots) {
+      keys_[n_] = key;
+      vals_[n_] = clusters;
+      ++n_;
+    }
+    return clusters;
+  }
+
+ private:
+  static constexpr int kSlots = 64;
+  uint64_t keys_[kSlots] = {};
+  int vals_[kSlots] = {};
+  int n_ = 0;
+  std::mutex mu_;
+};
 
 svdq_status launch_status() {
   const cudaError_t e = cudaGetLastError();
@@ -179,22 +220,34 @@ svdq_status launch_quantize(int M, int K, const void* X, int64_t ldx, const floa
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  // K-split into clusters of ks CTAs: grow ks (1, 2, 4) while the grid stays
-  // within one wave of co-resident clusters and there are fewer CTAs than SMs.
+  // K-split into clusters of ks CTAs: the largest ks in {8, 4, 2} whose grid
+  // keeps at most one CTA per SM, whose CTAs keep whole 64-column steps, and
+  // whose clusters are all resident at once. Clusters are placed within a GPC,
+  // so at about one CTA per SM a few clusters find no whole free group of SMs
+  // and must share SMs with running CTAs. cudaOccupancyMaxActiveClusters
+  // counts one CTA per SM for any kernel that allocates tensor memory (on B200
+  // it reports 33 clusters of four, yet 36 start together when two CTAs'
+  // shared memory fits an SM; registers are bounded for two CTAs by
+  // __launch_bounds__). A grid is accepted if either bound admits it.
+  static ClusterOccupancyCache occupancy;
+  int dev = 0;
+  cudaGetDevice(&dev);
   auto fits = [&](int ks_try) {
+    if (K % (kQuantStep * ks_try) != 0 || row_tiles * ks_try > sm_count) return false;
+    const size_t smem = quantize_smem_bytes<R>(K / ks_try);
+    if (smem > 227 * 1024) return false;
+    if (2 * (smem + 1024) <= 228 * 1024) return true;
     cfg.gridDim = dim3(ks_try, row_tiles, 1);
-    cfg.dynamicSmemBytes = quantize_smem_bytes<R>(K / ks_try);
+    cfg.dynamicSmemBytes = smem;
     attr[0].val.clusterDim.x = ks_try;
-    int clusters = 0;
-    if (cfg.dynamicSmemBytes > 227 * 1024) return false;
-    if (cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg) != cudaSuccess) {
-      cudaGetLastError();
-      return false;
-    }
-    return clusters >= row_tiles;
+    return occupancy.get(kern, &cfg, dev) >= row_tiles;
   };
   int ks = 1;
-  while (ks < 4 && row_tiles * ks < sm_count && fits(ks * 2)) ks *= 2;
+  for (int cand = 8; cand > 1; cand /= 2)
+    if (fits(cand)) {
+      ks = cand;
+      break;
+    }
   if (quantize_smem_bytes<R>(K / ks) > 227 * 1024) return SVDQ_ERR_UNSUPPORTED_SHAPE;
   const int kchunk = K / ks;
   cfg.gridDim = dim3(ks, row_tiles, 1);
