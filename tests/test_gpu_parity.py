@@ -114,6 +114,26 @@ def test_quantize_act_bitexact(lib, M, K, r):
     _check_act(lib, X, L1, r, g_x, qa, M, K)
 
 
+@pytest.mark.parametrize("rows", [64, 128])
+@pytest.mark.parametrize("ks", [1, 2, 4, 8])
+@pytest.mark.parametrize("r", [16, 32, 64, 128])
+def test_quantize_act_every_launch_plan(lib, monkeypatch, rows, ks, r):
+    """Every launch plan of the activation kernel: 64- or 128-row tiles, K split
+    over a cluster of 1, 2, 4 or 8 CTAs, every rank; M = 200 leaves a ragged
+    last tile for both heights and an odd count of 64-row tiles."""
+    M, K = 200, 1024
+    monkeypatch.setenv("SVDQ_QUANT_PLAN", f"{rows},{ks}")
+    X, W, b, L1, L2 = _layer(M, K, 128, r)
+    g_x = osv.act_global_scale(X)
+    pw = _act_only_weight(lib, K, r, L1, g_x)
+    qa = lib.QuantAct(M, K, r, "cuda")
+    for buf in (qa.codes, qa.scales, qa.xl1.view(torch.uint8)):
+        buf.fill_(0xA5)   # every output byte, padding included, must be written
+    lib.svdq_quantize_act(X.cuda(), pw, out=qa)
+    torch.cuda.synchronize()
+    _check_act(lib, X, L1, r, g_x, qa, M, K)
+
+
 def test_quantize_act_zero_rows_and_strided_input(lib):
     M, K, r = 130, 512, 32
     X, W, b, L1, L2 = _layer(M, K, 128, r)

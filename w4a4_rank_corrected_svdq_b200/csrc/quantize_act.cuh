@@ -6,33 +6,37 @@
 // projection is fused with the quantisation kernel, so the 16-bit branch adds
 // no extra pass over the activations.
 //
-// A CTA owns 128 rows and a K-range; the KS K-ranges of one 128-row block form
-// a thread-block cluster. Roles (288 threads; two CTAs fit an SM, so clusters
-// of four still fill the GPU in one wave):
+// A CTA owns ROWS (64 or 128) rows and a K-range; the KS K-ranges of one row
+// block form a thread-block cluster. Roles (288 threads):
 //  * warp 0      barrier setup and TMEM allocation; then lane 0 is both the
-//                TMA producer (per 64-column step one X tile, 128 rows x 128 B
-//                with 128-byte swizzle, and one L1^T tile, r rows x 128 B, into
-//                a ring of shared-memory stages) and the MMA issuer (four
-//                128 x r x 16 bf16 tcgen05 MMAs per step, XL1 accumulating in
-//                TMEM). The first stages are requested before the CTA-wide
-//                sync so the setup hides under their latency;
-//  * warps 1-8   quantisers, two steps per iteration for independent work in
-//                flight: thread t takes row t/2 and 32 columns (two NVFP4
-//                blocks) of each step, read from the swizzled tile with
-//                conflict-free 16-byte loads; per block one divide gives the
-//                scale and a 127-entry table of correctly rounded reciprocals
-//                (dec(S) g takes at most 127 values) gives 1/sd; products are
-//                formed two at a time (packed fp32); 16 code bytes per thread
-//                go out in one store and the scale bytes into staged 512-byte
-//                atoms that are written once.
+//                TMA producer (per 64-column step one X tile, ROWS rows x
+//                128 B with 128-byte swizzle, and one L1^T tile, r rows x
+//                128 B, into a ring of shared-memory stages) and the MMA issuer
+//                (four 128 x r x 16 bf16 tcgen05 MMAs per step, XL1
+//                accumulating in TMEM). With 64-row tiles the MMA still has
+//                M = 128: its rows 64-127 read the bytes after the tile (the
+//                ring is padded so they stay inside the allocation) and land in
+//                TMEM lanes that are never read. The first stages are requested
+//                before the CTA-wide sync so the setup hides under their
+//                latency;
+//  * warps 1-8   quantisers, several steps per iteration for independent work
+//                in flight: each thread takes one row and ROWS/64 NVFP4 blocks
+//                (16 columns each) of every step, read from the swizzled tile
+//                with conflict-free 16-byte loads; per block one divide gives
+//                the scale and a 127-entry table of correctly rounded
+//                reciprocals (dec(S) g takes at most 127 values) gives 1/sd;
+//                products are formed two at a time (packed fp32); code bytes go
+//                out in one store per step and the scale bytes into staged
+//                512-byte atoms written out after the K-range (a 64-row tile
+//                owns half of every atom).
 // XL1 reduction over the cluster (deterministic): CTA q finishes rows
-// [q*128/KS, (q+1)*128/KS). After one cluster barrier (every ring is drained),
-// each CTA reads its TMEM partial row by row and sends it with asynchronous
-// 16-byte stores into the owning CTA's shared memory (slot = source rank);
-// the stores count their bytes on the owner's mbarrier, which was armed with
-// the total at setup, so no thread waits for its own stores to land. The owner
-// adds the KS slots in rank order. Every mbarrier wait is bounded (see
-// mbar_wait).
+// [q*ROWS/KS, (q+1)*ROWS/KS) of the tile. After one cluster barrier (every
+// ring is drained), each CTA reads its TMEM partial row by row and sends it
+// with asynchronous 16-byte stores into the owning CTA's shared memory
+// (slot = source rank); the stores count their bytes on the owner's mbarrier,
+// which was armed with the total at setup, so no thread waits for its own
+// stores to land. The owner adds the KS slots in rank order. Every mbarrier
+// wait is bounded (see mbar_wait).
 #pragma once
 
 #include "nvfp4.cuh"
@@ -41,27 +45,34 @@ namespace svdq {
 
 constexpr int kQuantThreads = 288;
 constexpr int kQuantWarps = 8;     // quantiser warps (1..8)
-constexpr int kQuantRows = 128;
 constexpr int kQuantStep = 64;     // columns per step (128 bytes of bf16)
+constexpr int kQuantMaxStages = 8;
 
-template <int R>
+template <int R, int ROWS>
 struct QuantCfg {
-  static constexpr int kXBytes = kQuantRows * 128;        // 16 KB
+  static_assert(ROWS == 64 || ROWS == 128, "row tile");
+  static constexpr int kXBytes = ROWS * 128;
   static constexpr int kLBytes = R * 128;                  // L1^T tile
   static constexpr int kStageBytes = kXBytes + kLBytes;
-  static constexpr int kStages = (R >= 128) ? 3 : (R >= 64 ? 4 : 5);
+  static constexpr int kStages = ROWS == 128 ? ((R >= 128) ? 3 : (R >= 64 ? 4 : 5))
+                                             : ((R >= 128) ? 4 : (R >= 64 ? 6 : 8));
   static constexpr int kTmemCols = R < 32 ? 32 : R;
-  static constexpr int kRingBytes = kStages * kStageBytes;
-  // Partial-sum slots [KS][128/KS rows][R] fp32 = 128 x R x 4 bytes whatever
+  // MMA rows past a 64-row tile read up to 8 KB beyond the last stage.
+  static constexpr int kRingBytes = kStages * kStageBytes + (ROWS == 64 ? 8192 : 0);
+  // Partial-sum slots [KS][ROWS/KS rows][R] fp32 = ROWS x R x 4 bytes whatever
   // KS is; they alias the ring once every CTA of the cluster has drained it.
-  static constexpr int kPartBytes = kQuantRows * R * 4;
+  static constexpr int kPartBytes = ROWS * R * 4;
   static constexpr int kBody = kRingBytes > kPartBytes ? kRingBytes : kPartBytes;
   static constexpr int kSwzMask = (R / 4 < 8 ? R / 4 : 8) - 1;  // 16-byte chunk swizzle of a partial row
+  static constexpr int kBpt = ROWS / 64;   // NVFP4 blocks per quantiser thread per step
+  static constexpr int kTpr = 4 / kBpt;    // quantiser threads per row
+  static constexpr int kBatch = 4 / kBpt;  // steps per quantiser iteration
+  static_assert(kStages <= kQuantMaxStages, "barrier arrays");
 };
 
 struct QuantBarriers {
-  uint64_t full[5];
-  uint64_t empty[5];
+  uint64_t full[kQuantMaxStages];
+  uint64_t empty[kQuantMaxStages];
   uint64_t acc_done;
   uint64_t xl1_in;   // every partial row for this CTA's output rows has arrived
   uint32_t tmem_base;
@@ -70,28 +81,29 @@ struct QuantBarriers {
 
 // Dynamic shared memory: stage ring (later XL1 partial slots), scale staging
 // for the CTA's K-range, reciprocal table, barriers, alignment slack.
-template <int R>
+template <int R, int ROWS>
 __host__ __device__ constexpr size_t quantize_smem_bytes(int kchunk) {
-  return static_cast<size_t>(QuantCfg<R>::kBody) + static_cast<size_t>(kchunk / 64) * 512 + 512 + 128 + 1024;
+  return static_cast<size_t>(QuantCfg<R, ROWS>::kBody) + static_cast<size_t>(kchunk / 64) * 512 + 512 + 256 + 1024;
 }
 
-// Two NVFP4 blocks (32 bf16 values, four 16-byte words) -> 16 code bytes and
-// the two scale bytes (low byte = first block). Every step is one correctly
-// rounded fp32 operation: S = e4m3(amax / (6 g)), q = x * (1 / fp32(dec(S) g)).
-__device__ __forceinline__ void quantize_32(const uint4 (&v)[4], float d, const float* inv_tab, uint4& codes,
-                                            uint32_t& sc2) {
-  uint32_t c[4];
-  sc2 = 0;
+// NB NVFP4 blocks (16 bf16 values = two 16-byte words each) -> 8 code bytes
+// per block in c[2b], c[2b+1] and the scale bytes in sc (block b in byte b).
+// Every step is one correctly rounded fp32 operation:
+// S = e4m3(amax / (6 g)), q = x * (1 / fp32(dec(S) g)).
+template <int NB>
+__device__ __forceinline__ void quantize_blocks(const uint4 (&v)[2 * NB], float d, const float* inv_tab,
+                                                uint32_t (&c)[2 * NB], uint32_t& sc) {
+  sc = 0;
 #pragma unroll
-  for (int blk = 0; blk < 2; ++blk) {
+  for (int blk = 0; blk < NB; ++blk) {
     float f[8], e[8];
     bf16x8_to_f32(v[2 * blk], f);
     bf16x8_to_f32(v[2 * blk + 1], e);
     float am = 0.0f;
 #pragma unroll
     for (int i = 0; i < 8; ++i) am = fmaxf(am, fmaxf(fabsf(f[i]), fabsf(e[i])));
-    const uint32_t sc = f32_to_e4m3(__fdiv_rn(am, d));
-    const float inv = inv_tab[sc];
+    const uint32_t s = f32_to_e4m3(__fdiv_rn(am, d));
+    const float inv = inv_tab[s];
 #pragma unroll
     for (int i = 0; i < 8; i += 2) {
       mul2_rn(f[i], f[i + 1], inv);
@@ -99,18 +111,18 @@ __device__ __forceinline__ void quantize_32(const uint4 (&v)[4], float d, const 
     }
     c[2 * blk] = f32x8_to_e2m1(f);
     c[2 * blk + 1] = f32x8_to_e2m1(e);
-    sc2 |= sc << (8 * blk);
+    sc |= s << (8 * blk);
   }
-  codes = make_uint4(c[0], c[1], c[2], c[3]);
 }
 
-template <int R>
+template <int R, int ROWS>
 __global__ void __launch_bounds__(kQuantThreads, 2) quantize_act_kernel(
     const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_l1t, int M, int K,
     const float* __restrict__ g_x, uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
     __nv_bfloat16* __restrict__ xl1, int kchunk) {
-  using C = QuantCfg<R>;
+  using C = QuantCfg<R, ROWS>;
   constexpr int S = C::kStages;
+  constexpr int BPT = C::kBpt;
   extern __shared__ uint8_t qsmem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(qsmem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sc_stage = smem + C::kBody;
@@ -122,10 +134,10 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quantize_act_kernel(
   const int ks = static_cast<int>(cluster_rank());
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int m0 = blockIdx.y * kQuantRows;
+  const int m0 = blockIdx.y * ROWS;
   const int k_begin = ks * kchunk;
   const int nsteps = kchunk / kQuantStep;
-  const int rpc = kQuantRows / KS;  // output rows finished by each CTA of the cluster
+  const int rpc = ROWS / KS;  // output rows finished by each CTA of the cluster
   const float g = *g_x;
 
   if (threadIdx.x == 0) {
@@ -137,7 +149,7 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quantize_act_kernel(
     mbar_init(&bars->xl1_in, 1);
     bars->abort = 0;
     fence_barrier_init();
-    // rpc rows of R fp32 from each of the KS CTAs = 128 x R x 4 bytes
+    // rpc rows of R fp32 from each of the KS CTAs = ROWS x R x 4 bytes
     mbar_arrive_expect_tx(&bars->xl1_in, C::kPartBytes);
     prefetch_tmap(&tm_x);
     prefetch_tmap(&tm_l1t);
@@ -162,6 +174,8 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quantize_act_kernel(
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
   volatile int* abort = &bars->abort;
+  // Warps whose TMEM lane quarter (warp % 4) holds the tile's rows read XL1.
+  const bool xl1_reader = warp >= 4 && warp < 4 + ROWS / 32;
 
   if (warp == 0) {
     // ------------------------------------------------- producer + XL1 MMA issuer
@@ -194,43 +208,53 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quantize_act_kernel(
   } else {
     // ------------------------------------------------------------ quantisers
     const int t = threadIdx.x - 32;
-    const int rl = t >> 1;     // local row
-    const int h = t & 1;       // which 32 columns of the step
+    const int rl = t / C::kTpr;            // local row
+    const int b0 = (t % C::kTpr) * BPT;    // first NVFP4 block of the step
+    const int r128 = (m0 & 127) + rl;      // row inside its 128-row scale atom
     const int row = m0 + rl;
     const bool valid = row < M;
     const float d = __fmul_rn(6.0f, g);
-    uint8_t* cp = codes + static_cast<int64_t>(valid ? row : 0) * (K / 2) + k_begin / 2 + 16 * h;
-    uint8_t* sp = sc_stage + (rl & 31) * 16 + (rl >> 5) * 4 + 2 * h;
+    uint8_t* cp = codes + static_cast<int64_t>(valid ? row : 0) * (K / 2) + k_begin / 2 + 8 * b0;
+    uint8_t* sp = sc_stage + (r128 & 31) * 16 + (r128 >> 5) * 4 + b0;
     const int swz = rl & 7;
-    auto load_stage = [&](int st, uint4 (&v)[4]) -> bool {
+    auto load_stage = [&](int st, uint4 (&v)[2 * BPT]) -> bool {
       const int s = st % S;
       if (!mbar_wait(&bars->full[s], (st / S) & 1, abort)) return false;
       const uint8_t* tile = smem + s * C::kStageBytes + rl * 128;
 #pragma unroll
-      for (int j = 0; j < 4; ++j) v[j] = *reinterpret_cast<const uint4*>(tile + (((4 * h + j) ^ swz) << 4));
+      for (int j = 0; j < 2 * BPT; ++j) v[j] = *reinterpret_cast<const uint4*>(tile + (((2 * b0 + j) ^ swz) << 4));
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->empty[s]);  // this warp is done reading the stage
       return true;
     };
-    auto emit = [&](int st, const uint4 (&v)[4]) {
-      uint4 c;
-      uint32_t sc2;
-      quantize_32(v, d, inv_tab, c, sc2);
-      if (valid) *reinterpret_cast<uint4*>(cp + st * (kQuantStep / 2)) = c;
-      *reinterpret_cast<uint16_t*>(sp + st * 512) = static_cast<uint16_t>(sc2);
+    auto emit = [&](int st, const uint4 (&v)[2 * BPT]) {
+      uint32_t c[2 * BPT];
+      uint32_t sc;
+      quantize_blocks<BPT>(v, d, inv_tab, c, sc);
+      if constexpr (BPT == 2) {
+        if (valid) *reinterpret_cast<uint4*>(cp + st * (kQuantStep / 2)) = make_uint4(c[0], c[1], c[2], c[3]);
+        *reinterpret_cast<uint16_t*>(sp + st * 512) = static_cast<uint16_t>(sc);
+      } else {
+        if (valid) *reinterpret_cast<uint2*>(cp + st * (kQuantStep / 2)) = make_uint2(c[0], c[1]);
+        sp[st * 512] = static_cast<uint8_t>(sc);
+      }
     };
     int st = 0;
-    for (; st + 1 < nsteps; st += 2) {
-      uint4 v0[4], v1[4];
-      if (!load_stage(st, v0) || !load_stage(st + 1, v1)) break;
-      emit(st, v0);
-      emit(st + 1, v1);
+    for (; st + C::kBatch <= nsteps; st += C::kBatch) {
+      uint4 v[C::kBatch][2 * BPT];
+      bool ok = true;
+#pragma unroll
+      for (int i = 0; i < C::kBatch; ++i) ok = ok && load_stage(st + i, v[i]);
+      if (!ok) break;
+#pragma unroll
+      for (int i = 0; i < C::kBatch; ++i) emit(st + i, v[i]);
     }
-    if (st + 1 == nsteps) {
-      uint4 v0[4];
-      if (load_stage(st, v0)) emit(st, v0);
+    for (; st < nsteps; ++st) {
+      uint4 v[2 * BPT];
+      if (!load_stage(st, v)) break;
+      emit(st, v);
     }
-    if (warp <= 4) {  // warps 1-4 read XL1 from TMEM below: every MMA must have completed
+    if (xl1_reader) {  // XL1 is read from TMEM below: every MMA must have completed
       volatile int never = 0;
       mbar_wait(&bars->acc_done, 0, &never);
     }
@@ -245,7 +269,7 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quantize_act_kernel(
   cluster_arrive_relaxed();
   cluster_wait();
   tc_fence_after();
-  if (warp >= 1 && warp <= 4) {
+  if (xl1_reader) {
     const int q = warp & 3;          // TMEM lane quarter this warp may read
     const int rloc = 32 * q + lane;  // local row held by this thread
     const int owner = rloc / rpc;
@@ -266,9 +290,22 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quantize_act_kernel(
     }
   }
   {
+    // Scale atoms of this K-range: whole 512-byte atoms, or this tile's half
+    // (8 bytes of every 16-byte line) for a 64-row tile.
     uint8_t* dst = scales + (static_cast<size_t>(m0 / 128) * (K / 64) + k_begin / 64) * 512;
-    for (int i = threadIdx.x; i < nsteps * 32; i += kQuantThreads)
-      reinterpret_cast<uint4*>(dst)[i] = reinterpret_cast<const uint4*>(sc_stage)[i];
+    if (ROWS == 128) {
+      for (int i = threadIdx.x; i < nsteps * 32; i += kQuantThreads)
+        reinterpret_cast<uint4*>(dst)[i] = reinterpret_cast<const uint4*>(sc_stage)[i];
+    } else {
+      const int half = (m0 & 127) >> 6;
+      // The last tile of an odd count also zeroes the padding half of its atoms.
+      const bool pad_other = half == 0 && m0 + 64 >= M;
+      for (int i = threadIdx.x; i < nsteps * 32; i += kQuantThreads) {
+        const int off = (i >> 5) * 512 + (i & 31) * 16 + 8 * half;
+        *reinterpret_cast<uint2*>(dst + off) = *reinterpret_cast<const uint2*>(sc_stage + off);
+        if (pad_other) *reinterpret_cast<uint2*>(dst + off + 8) = make_uint2(0u, 0u);
+      }
+    }
   }
   tc_fence_before();
   __syncthreads();

@@ -198,73 +198,150 @@ CUtensorMapSwizzle lr_swizzle(int r) {
 }
 
 // ------------------------------------------------------------------ launches
+// Launch plan of the quantiser: row-tile height (64 or 128) and K-split ks
+// (CTAs per cluster).
+struct QuantPlan {
+  int rows = 128;
+  int ks = 1;
+};
+
+// Is (ROWS, ks) a one-wave grid of at most one CTA per SM whose clusters are
+// all resident at once? Clusters are placed within a GPC, so at about one CTA
+// per SM a few clusters may find no whole free group of SMs and then share SMs
+// with running CTAs (*shares = true), which needs two CTAs' shared memory to
+// fit an SM (registers are bounded for two CTAs by __launch_bounds__).
+// cudaOccupancyMaxActiveClusters counts one CTA per SM for any kernel that
+// allocates tensor memory: on B200 it reports 33 clusters of four, yet 36
+// start together when two CTAs' shared memory fits an SM.
+template <int R, int ROWS>
+bool quant_candidate(int M, int K, int ks, int sm_count, int dev, bool* shares) {
+  static ClusterOccupancyCache occupancy;
+  const int tiles = (M + ROWS - 1) / ROWS;
+  if (K % (kQuantStep * ks) != 0 || tiles * ks > sm_count) return false;
+  const size_t smem = quantize_smem_bytes<R, ROWS>(K / ks);
+  if (smem > 227 * 1024) return false;
+  *shares = false;
+  if (ks == 1) return true;
+  auto kern = quantize_act_kernel<R, ROWS>;
+  static std::atomic<uint64_t> attr_done{0};
+  ensure_smem_attr(kern, 227 * 1024, attr_done);
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = ks;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cfg.blockDim = dim3(kQuantThreads, 1, 1);
+  cfg.gridDim = dim3(ks, tiles, 1);
+  cfg.dynamicSmemBytes = smem;
+  if (occupancy.get(kern, &cfg, dev) >= tiles) return true;
+  *shares = true;
+  return 2 * (smem + 1024) <= 228 * 1024;
+}
+
+// Most CTAs (up to one per SM) wins; ties go to the taller tile (fewer L1^T
+// tile reloads and half the steps: on B200, 36 x 128-row tiles split four ways
+// run 10 % faster than 72 x 64-row tiles split two ways although three of
+// their clusters share SMs). With
+// no one-wave plan (very large M, or K too long for the shared-memory
+// staging) the smallest K-split whose shared memory fits, 128-row tiles.
+// SVDQ_QUANT_PLAN="rows,ks" (tests, benchmarks) forces a plan when K splits
+// into whole 64-column steps and its shared memory fits; otherwise it is
+// ignored.
 template <int R>
-svdq_status launch_quantize(int M, int K, const void* X, int64_t ldx, const float* g_x, const void* l1t, void* codes,
-                            void* scales, void* xl1, cudaStream_t stream, int sm_count) {
-  const int row_tiles = (M + kQuantRows - 1) / kQuantRows;
-  auto kern = quantize_act_kernel<R>;
+QuantPlan plan_quantize(int M, int K, int sm_count) {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  QuantPlan best;
+  if (const char* env = std::getenv("SVDQ_QUANT_PLAN")) {
+    int rows = 0, ks = 0;
+    if (std::sscanf(env, "%d,%d", &rows, &ks) == 2 && (rows == 64 || rows == 128) &&
+        (ks == 1 || ks == 2 || ks == 4 || ks == 8) && K % (kQuantStep * ks) == 0) {
+      const size_t smem =
+          rows == 64 ? quantize_smem_bytes<R, 64>(K / ks) : quantize_smem_bytes<R, 128>(K / ks);
+      if (smem <= 227 * 1024) {
+        best.rows = rows;
+        best.ks = ks;
+        return best;
+      }
+    }
+  }
+  long best_score = -1;
+  for (int rows : {128, 64})
+    for (int ks : {1, 2, 4, 8}) {
+      bool shares = false;  // clusters may share SMs; measured not to cost more than the extra steps
+      const bool ok = rows == 128 ? quant_candidate<R, 128>(M, K, ks, sm_count, dev, &shares)
+                                  : quant_candidate<R, 64>(M, K, ks, sm_count, dev, &shares);
+      if (!ok) continue;
+      const long ctas = static_cast<long>((M + rows - 1) / rows) * ks;
+      const long score = ctas;
+      if (score > best_score) {
+        best_score = score;
+        best.rows = rows;
+        best.ks = ks;
+      }
+    }
+  if (best_score < 0) {
+    best.rows = 128;
+    best.ks = 1;
+    while (best.ks < 8 && K % (kQuantStep * best.ks * 2) == 0 &&
+           quantize_smem_bytes<R, 128>(K / best.ks) > 227 * 1024)
+      best.ks *= 2;
+  }
+  return best;
+}
+
+template <int R, int ROWS>
+svdq_status launch_quantize(int M, int K, int ks, const void* X, int64_t ldx, const float* g_x, const void* l1t,
+                            void* codes, void* scales, void* xl1, cudaStream_t stream) {
+  const int row_tiles = (M + ROWS - 1) / ROWS;
+  const int kchunk = K / ks;
+  const size_t smem = quantize_smem_bytes<R, ROWS>(kchunk);
+  if (smem > 227 * 1024) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+  auto kern = quantize_act_kernel<R, ROWS>;
   static std::atomic<uint64_t> attr_done{0};
   ensure_smem_attr(kern, 227 * 1024, attr_done);
   CUtensorMap tm_x, tm_l;
-  if (!make_tmap_2d(&tm_x, X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, M, static_cast<uint64_t>(ldx) * 2, 64,
-                    kQuantRows, CU_TENSOR_MAP_SWIZZLE_128B) ||
+  if (!make_tmap_2d(&tm_x, X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, M, static_cast<uint64_t>(ldx) * 2, 64, ROWS,
+                    CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_tmap_2d(&tm_l, l1t, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, R, static_cast<uint64_t>(K) * 2, 64, R,
                     CU_TENSOR_MAP_SWIZZLE_128B))
     return SVDQ_ERR_CUDA;
   cudaLaunchConfig_t cfg = {};
   cfg.blockDim = dim3(kQuantThreads, 1, 1);
+  cfg.gridDim = dim3(ks, row_tiles, 1);
+  cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = ks;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  // K-split into clusters of ks CTAs: the largest ks in {8, 4, 2} whose grid
-  // keeps at most one CTA per SM, whose CTAs keep whole 64-column steps, and
-  // whose clusters are all resident at once. Clusters are placed within a GPC,
-  // so at about one CTA per SM a few clusters find no whole free group of SMs
-  // and must share SMs with running CTAs. cudaOccupancyMaxActiveClusters
-  // counts one CTA per SM for any kernel that allocates tensor memory (on B200
-  // it reports 33 clusters of four, yet 36 start together when two CTAs'
-  // shared memory fits an SM; registers are bounded for two CTAs by
-  // __launch_bounds__). A grid is accepted if either bound admits it.
-  static ClusterOccupancyCache occupancy;
-  int dev = 0;
-  cudaGetDevice(&dev);
-  auto fits = [&](int ks_try) {
-    if (K % (kQuantStep * ks_try) != 0 || row_tiles * ks_try > sm_count) return false;
-    const size_t smem = quantize_smem_bytes<R>(K / ks_try);
-    if (smem > 227 * 1024) return false;
-    if (2 * (smem + 1024) <= 228 * 1024) return true;
-    cfg.gridDim = dim3(ks_try, row_tiles, 1);
-    cfg.dynamicSmemBytes = smem;
-    attr[0].val.clusterDim.x = ks_try;
-    return occupancy.get(kern, &cfg, dev) >= row_tiles;
-  };
-  int ks = 1;
-  for (int cand = 8; cand > 1; cand /= 2)
-    if (fits(cand)) {
-      ks = cand;
-      break;
-    }
-  if (quantize_smem_bytes<R>(K / ks) > 227 * 1024) return SVDQ_ERR_UNSUPPORTED_SHAPE;
-  const int kchunk = K / ks;
-  cfg.gridDim = dim3(ks, row_tiles, 1);
-  cfg.dynamicSmemBytes = quantize_smem_bytes<R>(kchunk);
-  attr[0].val.clusterDim.x = ks;
   cudaLaunchKernelEx(&cfg, kern, tm_x, tm_l, M, K, g_x, static_cast<uint8_t*>(codes), static_cast<uint8_t*>(scales),
                      static_cast<__nv_bfloat16*>(xl1), kchunk);
   return launch_status();
 }
 
+template <int R>
+svdq_status launch_quantize_planned(int M, int K, const void* X, int64_t ldx, const float* g_x, const void* l1t,
+                                    void* codes, void* scales, void* xl1, cudaStream_t st, int sms) {
+  const QuantPlan plan = plan_quantize<R>(M, K, sms);
+  if (plan.rows == 64)
+    return launch_quantize<R, 64>(M, K, plan.ks, X, ldx, g_x, l1t, codes, scales, xl1, st);
+  return launch_quantize<R, 128>(M, K, plan.ks, X, ldx, g_x, l1t, codes, scales, xl1, st);
+}
+
 svdq_status quantize_dispatch(int M, int K, int r, const void* X, int64_t ldx, const float* g_x, const void* l1t,
                               void* codes, void* scales, void* xl1, cudaStream_t st, int sms) {
   switch (r) {
-    case 16: return launch_quantize<16>(M, K, X, ldx, g_x, l1t, codes, scales, xl1, st, sms);
-    case 32: return launch_quantize<32>(M, K, X, ldx, g_x, l1t, codes, scales, xl1, st, sms);
-    case 64: return launch_quantize<64>(M, K, X, ldx, g_x, l1t, codes, scales, xl1, st, sms);
-    default: return launch_quantize<128>(M, K, X, ldx, g_x, l1t, codes, scales, xl1, st, sms);
+    case 16: return launch_quantize_planned<16>(M, K, X, ldx, g_x, l1t, codes, scales, xl1, st, sms);
+    case 32: return launch_quantize_planned<32>(M, K, X, ldx, g_x, l1t, codes, scales, xl1, st, sms);
+    case 64: return launch_quantize_planned<64>(M, K, X, ldx, g_x, l1t, codes, scales, xl1, st, sms);
+    default: return launch_quantize_planned<128>(M, K, X, ldx, g_x, l1t, codes, scales, xl1, st, sms);
   }
 }
 
