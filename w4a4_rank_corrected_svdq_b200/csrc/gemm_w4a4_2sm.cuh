@@ -212,10 +212,10 @@ __device__ __forceinline__ void epilogue_half(uint32_t taddr, const uint4 (&bv)[
   tmem_ld_32x32b_x32(taddr + 32 * ((FIRST + 0) & 3), va);
   tmem_ld_32x32b_x32(taddr + 32 * ((FIRST + 1) & 3), vb);
   tmem_ld_wait();
-  if (holds_overlap) {
+  if (holds_overlap) {  // the loads above have completed (tcgen05.wait::ld): nothing else to publish
     tc_fence_before();
     __syncwarp();
-    if (lane == 0) mbar_arrive_cluster(ovl_bar);
+    if (lane == 0) mbar_arrive_cluster_relaxed(ovl_bar);
   }
   store_chunk(va, bv, (FIRST + 0) & 3, alpha, stage + 2048 * (nbuf & 1), tm_y, x0 + 32 * ((FIRST + 0) & 3), y0, lane);
   ++nbuf;
@@ -420,7 +420,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(k2Threads, 1) w4a4_g
         epilogue_half<0>(acc, bv, alpha, stage, nbuf, &tm_y, col0, y0, b == 1 && h == 0, ovl_bar, lane);
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&bars->acc_empty[b]), 0));
+      // every TMEM load of this accumulator has completed; the MMAs read nothing this warp wrote
+      if (lane == 0) mbar_arrive_cluster_relaxed(mapa_shared(smem_u32(&bars->acc_empty[b]), 0));
     }
     if (lane == 0) bulk_wait_all();
     __syncwarp();
