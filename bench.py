@@ -37,7 +37,13 @@ import workloads  # noqa: E402
 
 METRIC = "W4A4 linear TFLOP/s and tokens/s on 1 B200; % of NVFP4 tensor peak / HBM roofline"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+WORKLOAD = workloads.WORKLOADS[2]   # DiT fused QKV, M=4608, K=3072, N=9216, r=32
 FP4_PER_BF16 = 4.0   # nominal dense fp4 / bf16 tensor throughput ratio (9 / 2.25 PFLOP/s)
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch of the
+# dominant kernel on this workload, from the ncu capture summarised in
+# profiles/w4a4_gemm_2sm_kernel_qkv_4608x3072x9216_r32.md. Valid only for the
+# kernel as captured: set to None whenever the kernel changes.
+NCU_TRAFFIC_BYTES = {("dit_qkv_4608x3072x9216_r32", "w4a4_gemm_2sm_kernel"): 25425664 + 35224576}
 
 
 def _peaks():
@@ -57,7 +63,7 @@ def _quant_bytes(M, K, r):
 
 
 class ClockSampler:
-    """nvidia-smi clocks / throttle reasons sampled every 200 ms while running."""
+    """nvidia-smi clocks / throttle reasons sampled every 50 ms while running."""
 
     FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
               "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
@@ -70,7 +76,7 @@ class ClockSampler:
     def __enter__(self):
         try:
             self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200",
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "50",
                  "-i", str(self.index)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
@@ -184,7 +190,7 @@ def run_reference(args, spec):
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": spec.name, "M": spec.M, "K": spec.K, "N": spec.N, "r": spec.r},
+        "config": {"workload": WORKLOAD.name, "M": spec.M, "K": spec.K, "N": spec.N, "r": spec.r},
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": _cores(), "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }))
@@ -296,14 +302,14 @@ def run_ours(args, spec):
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "nvfp4", "data": "synthetic",
-        "config": {"workload": spec.name, "M": M, "K": K, "N": N, "r": r, "global_batch_tokens": world * M,
+        "config": {"workload": WORKLOAD.name, "M": M, "K": K, "N": N, "r": r, "global_batch_tokens": world * M,
                    "parallelism": f"replicas x{world}" if world > 1 else "single",
                    "l2": (f"inputs larger than L2: {n_sets} rotating copies of X and the packed weight "
                           f"({n_sets * set_bytes / 2**20:.0f} MiB, L2 {l2_bytes / 2**20:.0f} MiB); no flush kernel"),
                    "factors": "seeded stand-in low-rank factors (timing does not depend on their values)"},
         "tokens_per_s": tokens,
         "roofline": {"bound": "tensor", "achieved": gemm_tflops, "peak": fp4_peak, "unit": "TFLOP/s",
-                     "frac": gemm_tflops / fp4_peak, "traffic": None,
+                     "frac": gemm_tflops / fp4_peak, "traffic": NCU_TRAFFIC_BYTES.get((WORKLOAD.name, gemm_name)),
                      "kernel": gemm_name, "peak_source": f"{kind} bf16 burst x {FP4_PER_BF16:g} (fp4/bf16)"},
         "ms_per_step_loop": loop_ms,
         "kernels": {
@@ -339,7 +345,7 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
-    spec = workloads.WORKLOADS[2].layers[0]
+    spec = WORKLOAD.layers[0]
     if args.impl == "reference":
         return run_reference(args, spec)
     return run_ours(args, spec)
