@@ -116,6 +116,32 @@ svdq_status svdq_pack_weight(int N, int K, int r, const void* W, const void* L1,
                              const float* g_x, void* w_codes, void* w_scales, float* gscale, void* l1t,
                              void* l2s, void* stream);
 
+/* Load time (S0): the rank-r factors of the 16-bit branch from a truncated
+ * SVD of W^T (blog, section "Background: SVDQuant and Nunchaku": the branch
+ * holds the weight's dominant singular directions). With W^T = U S V^T:
+ *     L1 = bf16(U_r S_r)   (K x r, row-major)
+ *     L2 = bf16(V_r^T)     (r x N, row-major)
+ * computed in float64 by randomized subspace iteration (Halko, Martinsson and
+ * Tropp 2011): a Gaussian sketch of r + 32 columns drawn from `seed` by a
+ * counter-based generator, `power_iters` power iterations (each re-
+ * orthonormalised by shifted Cholesky QR), then the exact SVD of the sketched
+ * problem (two-sided Jacobi on its Gram matrix). The result is deterministic
+ * for a given seed. It approaches the optimal rank-r factors as power_iters
+ * grows: separated singular values converge fast; on a flat spectrum with
+ * power_iters = 32 the residual energy ||W^T - L1 L2||_F^2 is within about
+ * 2e-4 of the Eckart-Young minimum (rank 128; 1e-6 at rank 32). sigma
+ * (device, r doubles, may be NULL) receives S_r in decreasing order.
+ * Shapes: r in {16, 32, 64, 128}, r <= min(N, K), K % 8 == 0 (N and K need not
+ * satisfy the GEMM's rules). W, L1, L2 16-byte aligned, sigma 8-byte aligned,
+ * workspace 256-byte aligned and at least svdq_lowrank_workspace_size bytes
+ * (SVDQ_ERR_WORKSPACE otherwise); power_iters in [0, 64].
+ * The blog does not say how the SVD is computed; this is the load-time step
+ * that feeds svdq_pack_weight. */
+svdq_status svdq_lowrank_workspace_size(int N, int K, int r, size_t* bytes);
+svdq_status svdq_lowrank_init(int N, int K, int r, const void* W, void* L1, void* L2, double* sigma,
+                              unsigned long long seed, int power_iters, void* workspace, size_t ws_bytes,
+                              void* stream);
+
 /* Calibrated (static) activation scale: *g_out = fp32(amax|X| / 2688), or 1
  * for an all-zero X. X bf16 [M][ldx]; g_out is a device float. */
 svdq_status svdq_act_global_scale(int M, int K, const void* X, int64_t ldx, float* g_out,

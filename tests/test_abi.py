@@ -93,11 +93,31 @@ def test_validation_happens_before_device_checks(L):
                             None) == 0
 
 
+def test_lowrank_sizes_and_validation(L):
+    p = ctypes.c_void_p(0x10000)
+    odd = ctypes.c_void_p(0x10008)
+    ws = _lib.svdq_lowrank_workspace_size(9216, 3072, 32)
+    assert ws >= 8 * (2 * 9216 + 2 * 3072) * 64        # two N x p and two K x p float64 buffers, p = r + 32
+    assert _lib.svdq_lowrank_workspace_size(200, 1000, 16) > 0   # no GEMM shape rules
+    out = ctypes.c_size_t()
+    assert L.svdq_lowrank_workspace_size(128, 256, 24, ctypes.byref(out)) == 1    # rank
+    assert L.svdq_lowrank_workspace_size(16, 256, 32, ctypes.byref(out)) == 2     # r > min(N, K)
+    big = ctypes.c_size_t(1 << 40)
+    # rank, then shape, then alignment, then workspace size, all before any device check
+    assert L.svdq_lowrank_init(128, 256, 24, p, p, p, None, 0, 4, p, big, None) == 1
+    assert L.svdq_lowrank_init(128, 256, 32, p, p, p, None, 0, 65, p, big, None) == 1   # power_iters
+    assert L.svdq_lowrank_init(128, 252, 32, p, p, p, None, 0, 4, p, big, None) == 2    # K % 8
+    assert L.svdq_lowrank_init(128, 256, 32, odd, p, p, None, 0, 4, p, big, None) == 3
+    assert L.svdq_lowrank_init(128, 256, 32, p, p, p, ctypes.c_void_p(0x10004), 0, 4, p, big, None) == 3
+    assert L.svdq_lowrank_init(128, 256, 32, p, p, p, None, 0, 4, p, ctypes.c_size_t(16), None) == 7
+
+
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU path")
 def test_no_gpu_is_unsupported_device(L):
     p = ctypes.c_void_p(0x10000)
     assert L.svdq_quantize_act(4, 256, 32, p, 256, p, p, p, p, p, None) == 4
     assert L.svdq_pack_weight(128, 256, 32, p, p, p, p, p, p, p, p, p, None) == 4
+    assert L.svdq_lowrank_init(128, 256, 32, p, p, p, None, 0, 4, p, ctypes.c_size_t(1 << 40), None) == 4
     code = ctypes.c_int()
     assert L.svdq_read_device_error(ctypes.byref(code), 0) == 4
 

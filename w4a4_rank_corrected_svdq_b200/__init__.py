@@ -14,6 +14,8 @@ from ._lib import (  # noqa: F401
     svdq_act_sizes,
     svdq_forward_workspace_size,
     svdq_linear_forward,
+    svdq_lowrank_init,
+    svdq_lowrank_workspace_size,
     svdq_pack_weight,
     svdq_quantize_act,
     svdq_read_device_error,

@@ -38,6 +38,8 @@ SIGNATURES = {
     "svdq_linear_forward": (_i, [_i, _i, _i, _i, _p, _i64, _p, _p, _p, _p, _p, _p, _p, _i64, _p, _sz, _p]),
     "svdq_read_device_error": (_i, [_pi, _i]),
     "svdq_linear_forward_noalloc": (_i, [_i, _i, _i, _i, _p, _i64, _p, _p, _p, _p, _p, _p, _p, _i64, _p]),
+    "svdq_lowrank_workspace_size": (_i, [_i, _i, _i, _psz]),
+    "svdq_lowrank_init": (_i, [_i, _i, _i, _p, _p, _p, _p, ctypes.c_ulonglong, _i, _p, _sz, _p]),
 }
 
 
@@ -119,6 +121,32 @@ def svdq_forward_workspace_size(M: int, K: int, r: int) -> int:
     out = ctypes.c_size_t()
     _check("svdq_forward_workspace_size", lib().svdq_forward_workspace_size(M, K, r, ctypes.byref(out)))
     return out.value
+
+
+def svdq_lowrank_workspace_size(N: int, K: int, r: int) -> int:
+    out = ctypes.c_size_t()
+    _check("svdq_lowrank_workspace_size", lib().svdq_lowrank_workspace_size(N, K, r, ctypes.byref(out)))
+    return out.value
+
+
+def svdq_lowrank_init(W: torch.Tensor, r: int, seed: int = 0, power_iters: int = 32,
+                      workspace: torch.Tensor | None = None):
+    """Rank-r factors of the 16-bit branch from a truncated SVD of W^T on the GPU:
+    returns (L1 [K, r] bf16, L2 [r, N] bf16, sigma [r] float64)."""
+    _dev(W, "W", torch.bfloat16)
+    if not W.is_contiguous():
+        raise ValueError("W must be contiguous")
+    N, K = W.shape
+    need = svdq_lowrank_workspace_size(N, K, r)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=W.device)
+    L1 = torch.empty((K, r), dtype=torch.bfloat16, device=W.device)
+    L2 = torch.empty((r, N), dtype=torch.bfloat16, device=W.device)
+    sigma = torch.empty(r, dtype=torch.float64, device=W.device)
+    _check("svdq_lowrank_init", lib().svdq_lowrank_init(
+        N, K, r, _ptr(W), _ptr(L1), _ptr(L2), _ptr(sigma), seed, power_iters, _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(W)))
+    return L1, L2, sigma
 
 
 # ------------------------------------------------------------------ packed weight

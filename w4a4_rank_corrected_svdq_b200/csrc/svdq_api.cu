@@ -13,6 +13,7 @@
 #include "../../include/svdq.h"
 #include "gemm_w4a4.cuh"
 #include "gemm_w4a4_2sm.cuh"
+#include "lowrank_svd.cuh"
 #include "pack_weight.cuh"
 #include "quantize_act.cuh"
 
@@ -486,6 +487,156 @@ svdq_status check_layer_shape(int N, int K, int r) {
   return SVDQ_OK;
 }
 
+// ------------------------------------------------------------------ truncated SVD (load time)
+// Sketch width p = r + 32 oversampling columns (a multiple of 16, at most 160).
+int svd_width(int r) { return r + 32; }
+
+// Split of the long dimension for the tall-skinny GEMM: enough CTAs for about
+// two per SM of a 148-SM B200 (fixed, so that workspace sizes do not depend
+// on the device), slices of at least 64.
+int ts_splits(int M, int L) {
+  const int mtiles = (M + kTsRows - 1) / kTsRows;
+  int splits = (296 + mtiles - 1) / mtiles;
+  const int max_splits = L / 64 > 0 ? L / 64 : 1;
+  if (splits > max_splits) splits = max_splits;
+  return splits < 1 ? 1 : splits;
+}
+
+size_t ts_part_elems(int M, int L, int P) {
+  const int sp = ts_splits(M, L);
+  return sp > 1 ? static_cast<size_t>(sp) * M * P : 0;
+}
+
+// Workspace layout (float64 buffers, each 256-byte aligned).
+struct SvdLayout {
+  size_t om, zt, y, yt, part, g, rr, rinv, c, v, lam, m1, m2, u1, v2, total;
+};
+
+SvdLayout svd_layout(int N, int K, int r) {
+  const int p = svd_width(r);
+  SvdLayout l{};
+  size_t off = 0;
+  auto take = [&](size_t elems) {
+    const size_t at = off;
+    off = round_up(off + elems * sizeof(double), 256);
+    return at;
+  };
+  size_t part = 0;
+  const int shapes[][3] = {{K, N, p}, {N, K, p}, {p, K, p}, {p, N, p}, {K, p, p}, {N, p, p}, {K, p, r}, {N, p, r}};
+  for (const auto& sh : shapes) {
+    const size_t e = ts_part_elems(sh[0], sh[1], sh[2]);
+    if (e > part) part = e;
+  }
+  l.om = take(static_cast<size_t>(N) * p);
+  l.zt = take(static_cast<size_t>(N) * p);
+  l.y = take(static_cast<size_t>(K) * p);
+  l.yt = take(static_cast<size_t>(K) * p);
+  l.part = take(part > 0 ? part : 1);
+  l.g = take(static_cast<size_t>(p) * p);
+  l.rr = take(static_cast<size_t>(p) * p);
+  l.rinv = take(static_cast<size_t>(p) * p);
+  l.c = take(static_cast<size_t>(p) * p);
+  l.v = take(static_cast<size_t>(p) * p);
+  l.lam = take(p);
+  l.m1 = take(static_cast<size_t>(p) * r);
+  l.m2 = take(static_cast<size_t>(p) * r);
+  l.u1 = take(static_cast<size_t>(K) * r);
+  l.v2 = take(static_cast<size_t>(N) * r);
+  l.total = off;
+  return l;
+}
+
+// C (M x P) = op(A) B with op(A) = A (M x L) or A^T (A: L x M); B: L x P.
+template <bool TRANS_A, typename TA>
+svdq_status ts_gemm(int M, int L, int P, const TA* A, int64_t lda, const double* B, double* C, double* part,
+                    cudaStream_t st) {
+  const int splits = ts_splits(M, L);
+  const int lchunk = (L + splits - 1) / splits;
+  const dim3 grid((M + kTsRows - 1) / kTsRows, splits);
+  static std::atomic<uint64_t> attr_done{0};  // static tile + up to 40 KB of B slice exceed the 48 KB default
+  ensure_smem_attr(ts_gemm_kernel<TRANS_A, TA>, kTsL * kSvdMaxP * static_cast<int>(sizeof(double)), attr_done);
+  ts_gemm_kernel<TRANS_A, TA><<<grid, kTsThreads, kTsL * P * sizeof(double), st>>>(M, L, P, A, lda, B,
+                                                                                    splits > 1 ? part : C, lchunk);
+  if (splits > 1) {
+    const int64_t n = static_cast<int64_t>(M) * P;
+    split_sum_kernel<<<static_cast<int>((n + 255) / 256 < 1184 ? (n + 255) / 256 : 1184), 256, 0, st>>>(
+        part, splits, n, C);
+  }
+  return launch_status();
+}
+
+// T (L x p, float64) <- an orthonormal basis of its column space: Cholesky QR
+// three times, the first with the diagonal shift 11 (L p + p (p + 1)) u ||T||^2
+// of Fukaya et al. (||T||_2^2 estimated by the largest squared column norm),
+// the others with only a floor against breakdown. `tmp` is L x p.
+svdq_status orth(double* T, double* tmp, int L, int p, const SvdLayout& lay, uint8_t* ws, cudaStream_t st) {
+  double* G = reinterpret_cast<double*>(ws + lay.g);
+  double* R = reinterpret_cast<double*>(ws + lay.rr);
+  double* Rinv = reinterpret_cast<double*>(ws + lay.rinv);
+  double* part = reinterpret_cast<double*>(ws + lay.part);
+  const double shift_rel = 11.0 * (static_cast<double>(L) * p + static_cast<double>(p) * (p + 1)) * 0x1.0p-53;
+  double* src = T;
+  double* dst = tmp;
+  svdq_status s;
+  for (int pass = 0; pass < 3; ++pass) {
+    if ((s = ts_gemm<true, double>(p, L, p, src, p, src, G, part, st)) != SVDQ_OK) return s;
+    chol_inv_kernel<<<1, 1024, 0, st>>>(G, p, pass == 0 ? shift_rel : 0.0, R, Rinv);
+    if ((s = launch_status()) != SVDQ_OK) return s;
+    if ((s = ts_gemm<false, double>(L, p, p, src, p, Rinv, dst, part, st)) != SVDQ_OK) return s;
+    double* t = src;
+    src = dst;
+    dst = t;
+  }
+  // three passes: the result is in tmp; copy it back
+  if (cudaMemcpyAsync(T, src, static_cast<size_t>(L) * p * sizeof(double), cudaMemcpyDeviceToDevice, st) !=
+      cudaSuccess)
+    return launch_status();
+  return SVDQ_OK;
+}
+
+svdq_status run_lowrank(int N, int K, int r, const __nv_bfloat16* W, __nv_bfloat16* L1, __nv_bfloat16* L2,
+                        double* sigma, uint64_t seed, int power_iters, uint8_t* ws, cudaStream_t st) {
+  const int p = svd_width(r);
+  const SvdLayout lay = svd_layout(N, K, r);
+  double* Om = reinterpret_cast<double*>(ws + lay.om);   // N x p: Omega, later Z
+  double* Zt = reinterpret_cast<double*>(ws + lay.zt);   // N x p scratch
+  double* Y = reinterpret_cast<double*>(ws + lay.y);     // K x p
+  double* Yt = reinterpret_cast<double*>(ws + lay.yt);   // K x p scratch
+  double* part = reinterpret_cast<double*>(ws + lay.part);
+  double* C = reinterpret_cast<double*>(ws + lay.c);
+  double* V = reinterpret_cast<double*>(ws + lay.v);
+  double* lam = reinterpret_cast<double*>(ws + lay.lam);
+  double* M1 = reinterpret_cast<double*>(ws + lay.m1);
+  double* M2 = reinterpret_cast<double*>(ws + lay.m2);
+  double* U1 = reinterpret_cast<double*>(ws + lay.u1);
+  double* V2 = reinterpret_cast<double*>(ws + lay.v2);
+  svdq_status s;
+  const int64_t n_om = static_cast<int64_t>(N) * p;
+  gauss_fill_kernel<<<static_cast<int>(((n_om + 1) / 2 + 255) / 256 < 1184 ? ((n_om + 1) / 2 + 255) / 256 : 1184),
+                      256, 0, st>>>(Om, n_om, seed);
+  if ((s = launch_status()) != SVDQ_OK) return s;
+  // Y = A Omega = W^T Omega
+  if ((s = ts_gemm<true, __nv_bfloat16>(K, N, p, W, K, Om, Y, part, st)) != SVDQ_OK) return s;
+  for (int it = 0; it < power_iters; ++it) {
+    if ((s = orth(Y, Yt, K, p, lay, ws, st)) != SVDQ_OK) return s;
+    if ((s = ts_gemm<false, __nv_bfloat16>(N, K, p, W, K, Y, Om, part, st)) != SVDQ_OK) return s;  // Z = W Y
+    if ((s = orth(Om, Zt, N, p, lay, ws, st)) != SVDQ_OK) return s;
+    if ((s = ts_gemm<true, __nv_bfloat16>(K, N, p, W, K, Om, Y, part, st)) != SVDQ_OK) return s;  // Y = W^T Z
+  }
+  if ((s = orth(Y, Yt, K, p, lay, ws, st)) != SVDQ_OK) return s;                                    // Q
+  if ((s = ts_gemm<false, __nv_bfloat16>(N, K, p, W, K, Y, Om, part, st)) != SVDQ_OK) return s;    // Z = W Q = B^T
+  if ((s = ts_gemm<true, double>(p, N, p, Om, p, Om, C, part, st)) != SVDQ_OK) return s;          // B B^T = Z^T Z
+  jacobi_eig_kernel<<<1, 1024, 0, st>>>(C, p, V, lam, 60);
+  svd_coeff_kernel<<<1, 256, 0, st>>>(lam, V, p, r, M1, M2, sigma);
+  if ((s = launch_status()) != SVDQ_OK) return s;
+  if ((s = ts_gemm<false, double>(K, p, r, Y, p, M1, U1, part, st)) != SVDQ_OK) return s;   // U_r S_r = Q U_B,r S_r
+  if ((s = ts_gemm<false, double>(N, p, r, Om, p, M2, V2, part, st)) != SVDQ_OK) return s;  // V_r = B^T U_B,r / S_r
+  const int64_t tot = static_cast<int64_t>(K + N) * r;
+  svd_store_kernel<<<static_cast<int>((tot + 255) / 256 < 1184 ? (tot + 255) / 256 : 1184), 256, 0, st>>>(
+      U1, K, V2, N, r, L1, L2);
+  return launch_status();
+}
+
 }  // namespace
 }  // namespace svdq
 
@@ -568,6 +719,31 @@ svdq_status svdq_pack_weight(int N, int K, int r, const void* W, const void* L1,
     case 64: return launch_pack<64>(N, K, W, L1, L2, g_x, w_codes, w_scales, gscale, l2s, st);
     default: return launch_pack<128>(N, K, W, L1, L2, g_x, w_codes, w_scales, gscale, l2s, st);
   }
+}
+
+svdq_status svdq_lowrank_workspace_size(int N, int K, int r, size_t* bytes) {
+  if (N <= 0 || K <= 0 || !valid_rank(r) || !bytes) return SVDQ_ERR_INVALID_ARG;
+  if (r > N || r > K) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+  *bytes = svd_layout(N, K, r).total;
+  return SVDQ_OK;
+}
+
+svdq_status svdq_lowrank_init(int N, int K, int r, const void* W, void* L1, void* L2, double* sigma,
+                              unsigned long long seed, int power_iters, void* workspace, size_t ws_bytes,
+                              void* stream) {
+  if (N <= 0 || K <= 0 || !valid_rank(r) || !W || !L1 || !L2 || !workspace || power_iters < 0 || power_iters > 64)
+    return SVDQ_ERR_INVALID_ARG;
+  if (r > N || r > K || K % 8 != 0) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(W) || !aligned16(L1) || !aligned16(L2) || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
+      (reinterpret_cast<uintptr_t>(sigma) & 7u))
+    return SVDQ_ERR_MISALIGNED;
+  if (ws_bytes < svd_layout(N, K, r).total) return SVDQ_ERR_WORKSPACE;
+  svdq_status s;
+  DeviceInfo di;
+  if ((s = current_device(nullptr, &di)) != SVDQ_OK) return s;
+  return run_lowrank(N, K, r, static_cast<const __nv_bfloat16*>(W), static_cast<__nv_bfloat16*>(L1),
+                     static_cast<__nv_bfloat16*>(L2), sigma, seed, power_iters, static_cast<uint8_t*>(workspace),
+                     static_cast<cudaStream_t>(stream));
 }
 
 svdq_status svdq_act_global_scale(int M, int K, const void* X, int64_t ldx, float* g_out, void* stream) {
