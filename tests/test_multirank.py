@@ -1,0 +1,66 @@
+"""The N > 1 host path of bench.py on CPU: two gloo ranks on 127.0.0.1.
+
+The layer shards by tokens with no exchange, so multi-GPU runs are independent
+replicas; what the ranks share is the timing protocol: a barrier on both sides
+of the timed region, the step time taken as the maximum over ranks, rank 0
+alone printing, and the reference arm running on rank 0 only.
+"""
+import os
+import socket
+import sys
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
+    sys.path.insert(0, ROOT)
+    import bench
+    import datetime
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        bench._barrier(world)
+        # each rank "measured" a different time; every rank must see the slowest
+        out[rank] = bench._max_over_ranks(1.5 + rank, world)
+        bench._barrier(world)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_and_barrier_two_gloo_ranks():
+    world = 2
+    out = mp.get_context("spawn").Manager().dict()
+    mp.start_processes(_rank_main, args=(world, _free_port(), out), nprocs=world, start_method="spawn", join=True)
+    assert dict(out) == {0: 2.5, 1: 2.5}
+
+
+def test_reference_arm_runs_on_rank_zero_only(monkeypatch, capsys):
+    sys.path.insert(0, ROOT)
+    import bench
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    monkeypatch.setenv("RANK", "1")
+
+    class Args:
+        steps, warmup = 1, 3
+
+    # rank 1 returns at once: no oracle work, nothing printed
+    assert bench.run_reference(Args, bench.WORKLOAD.layers[0]) == 0
+    assert capsys.readouterr().out == ""
+
+
+def test_single_rank_needs_no_process_group():
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench._max_over_ranks(3.25, 1) == 3.25
+    bench._barrier(1)

@@ -163,13 +163,3 @@ def small_layer(M: int, K: int, N: int, r: int, seed: int = 1234, outliers: int 
                      x_outlier_count=min(outliers, K), x_outlier_gain=gain,
                      w_std=w_std, bias_std=bias_std)
     return spec, make_layer(spec)
-
-
-def factor_stand_ins(spec: LayerSpec):
-    """Seeded Gaussian stand-ins for the low-rank factors (L1: K x r, L2: r x N),
-    bf16, of the magnitude a rank-r decomposition of W would have. Only for
-    timing runs, whose work does not depend on the factor values."""
-    rng = np.random.default_rng([*spec.seed, 99])
-    l1 = rng.normal(0.0, spec.w_std * np.sqrt(spec.N), size=(spec.K, spec.r)).astype(np.float32)
-    l2 = rng.normal(0.0, 1.0 / np.sqrt(spec.N), size=(spec.r, spec.N)).astype(np.float32)
-    return _to_bf16(l1), _to_bf16(l2)
