@@ -125,6 +125,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) w4a4_gemm_kernel(
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  pdl_wait();  // the prologue above overlaps the previous kernel (programmatic dependent launch)
   const uint32_t tmem = bars->tmem_base;
   volatile int* abort = &bars->abort;
 

@@ -287,6 +287,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(k2Threads, 1) w4a4_g
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
   volatile int* abort = &bars->abort;
+  // Everything above overlaps the previous kernel of the stream (programmatic
+  // dependent launch); nothing global is read or written before this wait.
+  pdl_wait();
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer (both CTAs)

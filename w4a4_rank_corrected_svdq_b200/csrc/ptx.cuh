@@ -149,6 +149,16 @@ __device__ __forceinline__ void st_async_v4(uint32_t cluster_addr, uint32_t v0, 
                : "memory");
 }
 
+// ------------------------------------------------------------------ programmatic dependent launch
+// Lets the next kernel of the stream, if it was launched with programmatic
+// stream serialization, be scheduled now (it still waits in pdl_wait).
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+// Waits until the preceding kernel of the stream has completed and its memory
+// operations are visible; returns at once for a launch without that attribute.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ------------------------------------------------------------------ TMA / bulk copies
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* m) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");

@@ -139,6 +139,9 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quantize_act_kernel(
   const int nsteps = kchunk / kQuantStep;
   const int rpc = ROWS / KS;  // output rows finished by each CTA of the cluster
   const float g = *g_x;
+  // The GEMM that consumes this kernel's output may be scheduled now: it
+  // prepares its shared memory and TMEM, then waits for this grid to finish.
+  pdl_launch_dependents();
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {

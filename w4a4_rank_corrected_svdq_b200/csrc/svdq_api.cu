@@ -113,6 +113,24 @@ class ClusterOccupancyCache {
   std::mutex mu_;
 };
 
+// Launch attributes for a kernel that may start while the previous kernel of
+// the stream is finishing (programmatic dependent launch); the kernel itself
+// waits (griddepcontrol.wait) before touching global memory.
+struct PdlLaunch {
+  cudaLaunchAttribute attr[1];
+  cudaLaunchConfig_t cfg = {};
+  PdlLaunch(dim3 grid, dim3 block, size_t smem, cudaStream_t st) {
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+  }
+};
+
 svdq_status launch_status() {
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
@@ -367,9 +385,10 @@ svdq_status launch_gemm(int M, int N, int K, const void* a_codes, const void* a_
   ensure_smem_attr(kern, C::kSmemBytes, attr_done);
   const int tiles = ((M + kBM - 1) / kBM) * (N / kBN);
   const int grid = tiles < sm_count ? tiles : sm_count;
-  kern<<<grid, kGemmThreads, C::kSmemBytes, stream>>>(
-      tm_a, tm_b, tm_x, tm_l, static_cast<const uint8_t*>(a_scales), static_cast<const uint8_t*>(w_scales), gscale,
-      static_cast<const __nv_bfloat16*>(bias), static_cast<__nv_bfloat16*>(Y), ldy, M, N, K);
+  PdlLaunch pl(dim3(grid), dim3(kGemmThreads), C::kSmemBytes, stream);
+  cudaLaunchKernelEx(&pl.cfg, kern, tm_a, tm_b, tm_x, tm_l, static_cast<const uint8_t*>(a_scales),
+                     static_cast<const uint8_t*>(w_scales), gscale, static_cast<const __nv_bfloat16*>(bias),
+                     static_cast<__nv_bfloat16*>(Y), ldy, M, N, K);
   return launch_status();
 }
 
@@ -399,8 +418,9 @@ svdq_status launch_gemm_2sm(int M, int N, int K, const void* a_codes, const void
   const int tiles = ((M + k2TileM - 1) / k2TileM) * (N / k2TileN);
   const int max_pairs = sm_count / 2;
   const int pairs = tiles < max_pairs ? tiles : max_pairs;
-  kern<<<2 * pairs, k2Threads, C::kSmemBytes, stream>>>(tm_a, tm_b, tm_sfa, tm_sfb, tm_x, tm_l, tm_y, gscale,
-                                                        static_cast<const __nv_bfloat16*>(bias), M, N, K);
+  PdlLaunch pl(dim3(2 * pairs), dim3(k2Threads), C::kSmemBytes, stream);
+  cudaLaunchKernelEx(&pl.cfg, kern, tm_a, tm_b, tm_sfa, tm_sfb, tm_x, tm_l, tm_y, gscale,
+                     static_cast<const __nv_bfloat16*>(bias), M, N, K);
   return launch_status();
 }
 
