@@ -23,6 +23,11 @@ Functions, in the order the method applies them:
   quantize_act      NVFP4 of X                        (every call)
   down_proj         XL1 = bf16(X . L1)                (every call)
   forward           Y                                  (every call)
+  qkv_norm_rope     per-head RMSNorm of Q and K and rotary embedding on a
+                    fused QKV output (section "Quantizing models with
+                    structural rewrites": the fused operator consumes the QKV
+                    projection, the Q/K normalisation and the rotary embedding
+                    together)
 """
 from __future__ import annotations
 
@@ -130,6 +135,50 @@ def forward(X, pw: PackedWeight, bias, g_x) -> Forward:
     if bias is not None:
         y = y + to_f64(bias)[None, :]
     return Forward(codes, scales, xl1, y, nvfp4.bf16_round(y))
+
+
+# ------------------------------------------------------------------ fused QKV post-processing
+def rms_norm_heads(y, heads: int, head_dim: int, weight, eps: float) -> np.ndarray:
+    """Per-head RMSNorm of an [M, heads * head_dim] block, float64:
+    x / sqrt(mean over the head of x^2 + eps) * weight (weight: head_dim)."""
+    y = np.asarray(y, dtype=np.float64)
+    M = y.shape[0]
+    x = y.reshape(M, heads, head_dim)
+    ms = np.mean(x * x, axis=2, keepdims=True)
+    out = x / np.sqrt(ms + eps) * to_f64(weight)[None, None, :]
+    return out.reshape(M, heads * head_dim)
+
+
+def rotary_pairs(y, heads: int, head_dim: int, cos, sin) -> np.ndarray:
+    """Rotary embedding of every head on adjacent pairs (2j, 2j+1), float64:
+    (x0, x1) -> (x0 cos[2j] - x1 sin[2j], x1 cos[2j+1] + x0 sin[2j+1]), with
+    cos, sin: [M, head_dim] per token position."""
+    y = np.asarray(y, dtype=np.float64)
+    M = y.shape[0]
+    x = y.reshape(M, heads, head_dim)
+    c = np.asarray(cos, dtype=np.float64)[:, None, :]
+    s = np.asarray(sin, dtype=np.float64)[:, None, :]
+    x0, x1 = x[..., 0::2], x[..., 1::2]
+    out = np.empty_like(x)
+    out[..., 0::2] = x0 * c[..., 0::2] - x1 * s[..., 0::2]
+    out[..., 1::2] = x1 * c[..., 1::2] + x0 * s[..., 1::2]
+    return out.reshape(M, heads * head_dim)
+
+
+def qkv_norm_rope(y_ref, heads: int, head_dim: int, w_q, w_k, eps: float, cos, sin):
+    """The fused QKV post-processing of a [M, 3 * heads * head_dim] projection
+    output laid out [Q | K | V]: Q and K get per-head RMSNorm (weights w_q, w_k)
+    then the rotary embedding; V passes through. The input is the layer output
+    rounded to bf16 (what the unfused sequence hands to the norm). Returns
+    (float64 result, the result rounded to bf16)."""
+    y = np.asarray(y_ref, dtype=np.float64)
+    hd = heads * head_dim
+    out = y.copy()
+    for blk, w in ((0, w_q), (1, w_k)):
+        part = y[:, blk * hd:(blk + 1) * hd]
+        out[:, blk * hd:(blk + 1) * hd] = rotary_pairs(rms_norm_heads(part, heads, head_dim, w, eps),
+                                                        heads, head_dim, cos, sin)
+    return out, nvfp4.bf16_round(out)
 
 
 # ------------------------------------------------------------------ metrics

@@ -212,3 +212,64 @@ def test_low_rank_correction_beats_plain_w4a4_on_outliers(outlier_gain):
     L10, L20, _ = svdq.lowrank_factors(W64, 0)
     e_naive = svdq.rel_fro(svdq.forward(X64, svdq.pack_weight(W64, L10, L20), b64, g_x).y64, exact)
     assert e_svdq < e_naive
+
+
+# ------------------------------------------------------------------ fused QKV norm + rotary
+def test_rms_norm_closed_forms():
+    rng = np.random.default_rng(41)
+    y = rng.standard_normal((5, 3 * 16)) * 7.0
+    out = svdq.rms_norm_heads(y, 3, 16, np.ones(16), 0.0)
+    ms = np.mean(out.reshape(5, 3, 16) ** 2, axis=2)
+    assert np.allclose(ms, 1.0, rtol=0, atol=1e-12)           # unit RMS per head with eps = 0
+    c = np.full((2, 16), -2.5)
+    w = np.arange(1, 17, dtype=np.float64)
+    assert np.allclose(svdq.rms_norm_heads(c, 1, 16, w, 0.0), -w[None, :], atol=1e-12)  # constant row -> sign * w
+    # eps dominates a zero row: the result stays zero
+    assert not svdq.rms_norm_heads(np.zeros((1, 16)), 1, 16, w, 1e-6).any()
+
+
+def test_rotary_is_complex_multiplication():
+    """With cos[2j] = cos[2j+1] = cos(theta_j) (and likewise sin), each pair is the
+    complex product (x0 + i x1) e^(i theta_j): an independent formulation."""
+    rng = np.random.default_rng(42)
+    M, H, D = 4, 2, 8
+    y = rng.standard_normal((M, H * D))
+    theta = rng.uniform(-np.pi, np.pi, (M, D // 2))
+    cos = np.repeat(np.cos(theta), 2, axis=1)
+    sin = np.repeat(np.sin(theta), 2, axis=1)
+    out = svdq.rotary_pairs(y, H, D, cos, sin).reshape(M, H, D)
+    z = y.reshape(M, H, D)[..., 0::2] + 1j * y.reshape(M, H, D)[..., 1::2]
+    ref = z * np.exp(1j * theta)[:, None, :]
+    assert np.allclose(out[..., 0::2], ref.real, atol=1e-13)
+    assert np.allclose(out[..., 1::2], ref.imag, atol=1e-13)
+    # pair norms are preserved, rotating back by -theta restores the input, cos = 1 / sin = 0 is the identity
+    assert np.allclose(np.abs(ref), np.abs(z), atol=1e-13)
+    back = svdq.rotary_pairs(out.reshape(M, H * D), H, D, cos, -sin)
+    assert np.allclose(back, y, atol=1e-13)
+    assert np.array_equal(svdq.rotary_pairs(y, H, D, np.ones((M, D)), np.zeros((M, D))), y)
+
+
+def test_qkv_norm_rope_against_loops():
+    """The fused post-processing against per-element Python loops on a tiny case;
+    V passes through unchanged; the bf16 output is the float64 result rounded."""
+    rng = np.random.default_rng(43)
+    M, H, D = 3, 2, 4
+    y = nvfp4.bf16_round(rng.standard_normal((M, 3 * H * D)) * 3.0)
+    wq, wk = rng.uniform(0.5, 1.5, D), rng.uniform(0.5, 1.5, D)
+    cos, sin = rng.uniform(-1, 1, (M, D)), rng.uniform(-1, 1, (M, D))
+    eps = 1e-6
+    out, out_bf16 = svdq.qkv_norm_rope(y, H, D, wq, wk, eps, cos, sin)
+    ref = y.copy()
+    for blk, w in ((0, wq), (1, wk)):
+        for m in range(M):
+            for h in range(H):
+                base = blk * H * D + h * D
+                x = [y[m, base + i] for i in range(D)]
+                rstd = 1.0 / np.sqrt(sum(v * v for v in x) / D + eps)
+                n = [x[i] * rstd * w[i] for i in range(D)]
+                for j in range(D // 2):
+                    ref[m, base + 2 * j] = n[2 * j] * cos[m, 2 * j] - n[2 * j + 1] * sin[m, 2 * j]
+                    ref[m, base + 2 * j + 1] = n[2 * j + 1] * cos[m, 2 * j + 1] + n[2 * j] * sin[m, 2 * j + 1]
+    assert np.allclose(out, ref, rtol=0, atol=1e-12)
+    assert np.array_equal(out[:, 2 * H * D:], y[:, 2 * H * D:])
+    assert np.array_equal(out_bf16, nvfp4.bf16_round(out))
