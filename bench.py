@@ -310,6 +310,35 @@ def run_ours(args, spec):
     if svdq.svdq_read_device_error() != 0:
         raise RuntimeError("device error during timing")
 
+    # Fused QKV post-processing (per-head RMSNorm of Q/K + rotary embedding in the
+    # GEMM epilogue) against the plain layer, same inputs, same public API path.
+    heads = N // 384
+    qkv = None
+    if N == heads * 384:
+        wq = torch.ones(128, dtype=torch.bfloat16, device=dev)
+        wk = torch.ones(128, dtype=torch.bfloat16, device=dev)
+        cos_np, sin_np = workloads.rope_tables(M, 128)
+        cos_t, sin_t = torch.from_numpy(cos_np).to(dev), torch.from_numpy(sin_np).to(dev)
+        n_q = min(args.steps, 200)
+
+        def timed(fn):
+            for i in range(3):
+                fn(i)
+            torch.cuda.synchronize()
+            a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for i in range(n_q):
+                fn(i)
+            z.record(stream)
+            torch.cuda.synchronize()
+            return _max_over_ranks(a.elapsed_time(z), world) / n_q
+
+        plain_ms = timed(lambda i: svdq.svdq_linear_forward(Xs[i % n_sets], pws[i % n_sets], bd, out=Y, workspace=ws))
+        fused_ms = timed(lambda i: svdq.svdq_linear_forward_qkv(Xs[i % n_sets], pws[i % n_sets], bd, heads, wq, wk,
+                                                               1e-6, cos_t, sin_t, out=Y, workspace=ws))
+        qkv = {"heads": heads, "head_dim": 128, "ms_per_step": fused_ms, "plain_ms_per_step": plain_ms,
+               "overhead": fused_ms / plain_ms - 1.0, "steps": n_q}
+
     peaks, kind = _peaks()
     gemm_name = _gemm_kernel_name(M, N)
     fp4_peak = peaks["bf16_tflops"] * FP4_PER_BF16
@@ -340,6 +369,7 @@ def run_ours(args, spec):
         },
         "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2, "ms_per_step": e2e_ms},
+        "qkv_norm_rope": qkv,
         "gpu_launches": 2 * args.steps,
         "clocks": clk.summary(),
     }

@@ -116,6 +116,31 @@ svdq_status svdq_pack_weight(int N, int K, int r, const void* W, const void* L1,
                              const float* g_x, void* w_codes, void* w_scales, float* gscale, void* l1t,
                              void* l2s, void* stream);
 
+/* The layer followed by FLUX's fused QKV post-processing (blog, section
+ * "Quantizing models with structural rewrites": one fused operator takes the
+ * grouped QKV projection, the Q/K normalisation and the rotary embedding).
+ * W is the grouped [Q; K; V] weight, N = 3 * heads * 128 (head_dim 128), and
+ * Y is laid out [Q | K | V]. With q = bf16(layer output) per head row:
+ *     n_i = q_i / sqrt(mean_i(q_i^2) + eps) * w_i       (w = norm_q_weight for
+ *                                                        Q heads, norm_k_weight
+ *                                                        for K heads; bf16[128])
+ *     (n_2j, n_2j+1) -> (n_2j c_j - n_2j+1 s_j,  n_2j+1 c_j + n_2j s_j)
+ * (each pair rotated by the angle theta_j of its token), with c_j =
+ * rope_cos[m][j] = cos(theta_j), s_j = rope_sin[m][j] (float32 [M][ld_rope],
+ * 64 used per token), computed in fp32 and rounded to bf16 once; V columns
+ * are the plain layer output. Other arguments, the workspace and the shape
+ * rules are those of svdq_linear_forward; additionally N == 3 * heads * 128,
+ * ld_rope >= 64 and ld_rope % 4 == 0, norm weights and rope tables 16-byte
+ * aligned, 0 <= eps. The normalisation and rotation happen in the GEMM's
+ * epilogue (no extra pass over Y). */
+svdq_status svdq_linear_forward_qkv(int M, int N, int K, int r, const void* X, int64_t ldx,
+                                    const void* w_codes, const void* w_scales, const float* gscale,
+                                    const void* l1t, const void* l2s, const void* bias, int heads,
+                                    const void* norm_q_weight, const void* norm_k_weight, float eps,
+                                    const float* rope_cos, const float* rope_sin, int64_t ld_rope,
+                                    void* Y, int64_t ldy, void* workspace, size_t workspace_bytes,
+                                    void* stream);
+
 /* Load time (S0): the rank-r factors of the 16-bit branch from a truncated
  * SVD of W^T (blog, section "Background: SVDQuant and Nunchaku": the branch
  * holds the weight's dominant singular directions). With W^T = U S V^T:

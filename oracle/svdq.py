@@ -151,8 +151,9 @@ def rms_norm_heads(y, heads: int, head_dim: int, weight, eps: float) -> np.ndarr
 
 def rotary_pairs(y, heads: int, head_dim: int, cos, sin) -> np.ndarray:
     """Rotary embedding of every head on adjacent pairs (2j, 2j+1), float64:
-    (x0, x1) -> (x0 cos[2j] - x1 sin[2j], x1 cos[2j+1] + x0 sin[2j+1]), with
-    cos, sin: [M, head_dim] per token position."""
+    each pair is rotated by the angle theta_j of its token position,
+    (x0, x1) -> (x0 cos_j - x1 sin_j, x1 cos_j + x0 sin_j), with
+    cos, sin: [M, head_dim // 2] (cos and sin of theta_j per token and pair)."""
     y = np.asarray(y, dtype=np.float64)
     M = y.shape[0]
     x = y.reshape(M, heads, head_dim)
@@ -160,8 +161,8 @@ def rotary_pairs(y, heads: int, head_dim: int, cos, sin) -> np.ndarray:
     s = np.asarray(sin, dtype=np.float64)[:, None, :]
     x0, x1 = x[..., 0::2], x[..., 1::2]
     out = np.empty_like(x)
-    out[..., 0::2] = x0 * c[..., 0::2] - x1 * s[..., 0::2]
-    out[..., 1::2] = x1 * c[..., 1::2] + x0 * s[..., 1::2]
+    out[..., 0::2] = x0 * c - x1 * s
+    out[..., 1::2] = x1 * c + x0 * s
     return out.reshape(M, heads * head_dim)
 
 

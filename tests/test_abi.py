@@ -112,6 +112,23 @@ def test_lowrank_sizes_and_validation(L):
     assert L.svdq_lowrank_init(128, 256, 32, p, p, p, None, 0, 4, p, ctypes.c_size_t(16), None) == 7
 
 
+def test_qkv_forward_validation(L):
+    p = ctypes.c_void_p(0x10000)
+    odd = ctypes.c_void_p(0x10008)
+    f = ctypes.c_float
+    ws = ctypes.c_size_t(1 << 40)
+    args = lambda N, heads, eps, cs, ld: (4, N, 256, 32, p, 256, p, p, p, p, p, None, heads, p, p, f(eps), cs, p, ld,
+                                          p, N, p, ws, None)
+    assert L.svdq_linear_forward_qkv(*args(768, 2, 1e-6, p, 128)) in (0, 4)     # valid (no GPU here: 4)
+    assert L.svdq_linear_forward_qkv(*args(768, 1, 1e-6, p, 128)) == 2          # N != 3 * heads * 128
+    assert L.svdq_linear_forward_qkv(*args(768, 2, -1.0, p, 128)) == 1          # eps < 0
+    assert L.svdq_linear_forward_qkv(*args(768, 2, 1e-6, p, 64)) in (0, 4)      # 64 angles per token suffice
+    assert L.svdq_linear_forward_qkv(*args(768, 2, 1e-6, p, 60)) == 2           # ld_rope < 64
+    assert L.svdq_linear_forward_qkv(*args(768, 2, 1e-6, p, 66)) == 2           # ld_rope % 4 != 0
+    assert L.svdq_linear_forward_qkv(*args(768, 2, 1e-6, odd, 128)) == 3        # misaligned rope table
+    assert L.svdq_linear_forward_qkv(*args(768, 0, 1e-6, p, 128)) == 1          # heads
+
+
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU path")
 def test_no_gpu_is_unsupported_device(L):
     p = ctypes.c_void_p(0x10000)

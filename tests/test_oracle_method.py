@@ -229,24 +229,26 @@ def test_rms_norm_closed_forms():
 
 
 def test_rotary_is_complex_multiplication():
-    """With cos[2j] = cos[2j+1] = cos(theta_j) (and likewise sin), each pair is the
-    complex product (x0 + i x1) e^(i theta_j): an independent formulation."""
+    """Each pair is the complex product (x0 + i x1) e^(i theta_j): an independent
+    formulation of the rotation by theta_j."""
     rng = np.random.default_rng(42)
     M, H, D = 4, 2, 8
     y = rng.standard_normal((M, H * D))
     theta = rng.uniform(-np.pi, np.pi, (M, D // 2))
-    cos = np.repeat(np.cos(theta), 2, axis=1)
-    sin = np.repeat(np.sin(theta), 2, axis=1)
-    out = svdq.rotary_pairs(y, H, D, cos, sin).reshape(M, H, D)
+    out = svdq.rotary_pairs(y, H, D, np.cos(theta), np.sin(theta)).reshape(M, H, D)
     z = y.reshape(M, H, D)[..., 0::2] + 1j * y.reshape(M, H, D)[..., 1::2]
     ref = z * np.exp(1j * theta)[:, None, :]
     assert np.allclose(out[..., 0::2], ref.real, atol=1e-13)
     assert np.allclose(out[..., 1::2], ref.imag, atol=1e-13)
     # pair norms are preserved, rotating back by -theta restores the input, cos = 1 / sin = 0 is the identity
     assert np.allclose(np.abs(ref), np.abs(z), atol=1e-13)
-    back = svdq.rotary_pairs(out.reshape(M, H * D), H, D, cos, -sin)
+    back = svdq.rotary_pairs(out.reshape(M, H * D), H, D, np.cos(theta), -np.sin(theta))
     assert np.allclose(back, y, atol=1e-13)
-    assert np.array_equal(svdq.rotary_pairs(y, H, D, np.ones((M, D)), np.zeros((M, D))), y)
+    assert np.array_equal(svdq.rotary_pairs(y, H, D, np.ones((M, D // 2)), np.zeros((M, D // 2))), y)
+    # a quarter turn maps (x0, x1) to (-x1, x0)
+    q = svdq.rotary_pairs(y, H, D, np.zeros((M, D // 2)), np.ones((M, D // 2))).reshape(M, H, D)
+    assert np.array_equal(q[..., 0::2], -y.reshape(M, H, D)[..., 1::2])
+    assert np.array_equal(q[..., 1::2], y.reshape(M, H, D)[..., 0::2])
 
 
 def test_qkv_norm_rope_against_loops():
@@ -256,7 +258,7 @@ def test_qkv_norm_rope_against_loops():
     M, H, D = 3, 2, 4
     y = nvfp4.bf16_round(rng.standard_normal((M, 3 * H * D)) * 3.0)
     wq, wk = rng.uniform(0.5, 1.5, D), rng.uniform(0.5, 1.5, D)
-    cos, sin = rng.uniform(-1, 1, (M, D)), rng.uniform(-1, 1, (M, D))
+    cos, sin = rng.uniform(-1, 1, (M, D // 2)), rng.uniform(-1, 1, (M, D // 2))
     eps = 1e-6
     out, out_bf16 = svdq.qkv_norm_rope(y, H, D, wq, wk, eps, cos, sin)
     ref = y.copy()
@@ -268,8 +270,8 @@ def test_qkv_norm_rope_against_loops():
                 rstd = 1.0 / np.sqrt(sum(v * v for v in x) / D + eps)
                 n = [x[i] * rstd * w[i] for i in range(D)]
                 for j in range(D // 2):
-                    ref[m, base + 2 * j] = n[2 * j] * cos[m, 2 * j] - n[2 * j + 1] * sin[m, 2 * j]
-                    ref[m, base + 2 * j + 1] = n[2 * j + 1] * cos[m, 2 * j + 1] + n[2 * j] * sin[m, 2 * j + 1]
+                    ref[m, base + 2 * j] = n[2 * j] * cos[m, j] - n[2 * j + 1] * sin[m, j]
+                    ref[m, base + 2 * j + 1] = n[2 * j + 1] * cos[m, j] + n[2 * j] * sin[m, j]
     assert np.allclose(out, ref, rtol=0, atol=1e-12)
     assert np.array_equal(out[:, 2 * H * D:], y[:, 2 * H * D:])
     assert np.array_equal(out_bf16, nvfp4.bf16_round(out))

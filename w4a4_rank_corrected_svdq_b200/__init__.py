@@ -14,6 +14,7 @@ from ._lib import (  # noqa: F401
     svdq_act_sizes,
     svdq_forward_workspace_size,
     svdq_linear_forward,
+    svdq_linear_forward_qkv,
     svdq_lowrank_init,
     svdq_lowrank_workspace_size,
     svdq_pack_weight,

@@ -38,6 +38,8 @@ SIGNATURES = {
     "svdq_linear_forward": (_i, [_i, _i, _i, _i, _p, _i64, _p, _p, _p, _p, _p, _p, _p, _i64, _p, _sz, _p]),
     "svdq_read_device_error": (_i, [_pi, _i]),
     "svdq_linear_forward_noalloc": (_i, [_i, _i, _i, _i, _p, _i64, _p, _p, _p, _p, _p, _p, _p, _i64, _p]),
+    "svdq_linear_forward_qkv": (_i, [_i, _i, _i, _i, _p, _i64, _p, _p, _p, _p, _p, _p, _i, _p, _p, _f, _p, _p,
+                                     _i64, _p, _i64, _p, _sz, _p]),
     "svdq_lowrank_workspace_size": (_i, [_i, _i, _i, _psz]),
     "svdq_lowrank_init": (_i, [_i, _i, _i, _p, _p, _p, _p, ctypes.c_ulonglong, _i, _p, _sz, _p]),
 }
@@ -255,6 +257,38 @@ def svdq_linear_forward(X: torch.Tensor, pw: PackedWeight, bias: torch.Tensor | 
     _check("svdq_linear_forward", lib().svdq_linear_forward(
         M, N, K, r, _ptr(X), ldx, _ptr(pw.codes), _ptr(pw.scales), _ptr(pw.gscale), _ptr(pw.l1t),
         _ptr(pw.l2s), _ptr(bias), _ptr(Y), ldy, _ptr(ws), ws.numel(), _stream(X)))
+    return Y
+
+
+def svdq_linear_forward_qkv(X: torch.Tensor, pw: PackedWeight, bias: torch.Tensor | None, heads: int,
+                            norm_q_weight: torch.Tensor, norm_k_weight: torch.Tensor, eps: float,
+                            rope_cos: torch.Tensor, rope_sin: torch.Tensor, out: torch.Tensor | None = None,
+                            workspace: torch.Tensor | None = None) -> torch.Tensor:
+    """The layer with the fused QKV post-processing (per-head RMSNorm of Q and K,
+    rotary embedding; head_dim 128). rope_cos / rope_sin: float32 [M, >=64],
+    cos / sin of each token's angle per pair (2j, 2j+1)."""
+    _dev(X, "X", torch.bfloat16)
+    M, K = X.shape
+    ldx = _rows(X, "X", K)
+    N = pw.N
+    for t, n in ((norm_q_weight, "norm_q_weight"), (norm_k_weight, "norm_k_weight")):
+        _dev(t, n, torch.bfloat16, (128,))
+    for t, n in ((rope_cos, "rope_cos"), (rope_sin, "rope_sin")):
+        _dev(t, n, torch.float32)
+        if t.dim() != 2 or t.shape[0] != M or t.stride(1) != 1:
+            raise ValueError(f"{n} must be [M, >=64] with unit column stride")
+    if rope_cos.stride(0) != rope_sin.stride(0):
+        raise ValueError("rope_cos and rope_sin must share a row stride")
+    if bias is not None:
+        _dev(bias, "bias", torch.bfloat16, (N,))
+    Y = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=X.device)
+    ldy = _rows(Y, "Y", N)
+    if workspace is None:
+        workspace = torch.empty(max(1, svdq_forward_workspace_size(M, K, pw.r)), dtype=torch.uint8, device=X.device)
+    _check("svdq_linear_forward_qkv", lib().svdq_linear_forward_qkv(
+        M, N, K, pw.r, _ptr(X), ldx, _ptr(pw.codes), _ptr(pw.scales), _ptr(pw.gscale), _ptr(pw.l1t), _ptr(pw.l2s),
+        _ptr(bias), heads, _ptr(norm_q_weight), _ptr(norm_k_weight), float(eps), _ptr(rope_cos), _ptr(rope_sin),
+        rope_cos.stride(0), _ptr(Y), ldy, _ptr(workspace), workspace.numel(), _stream(X)))
     return Y
 
 

@@ -33,6 +33,7 @@
 #pragma once
 
 #include "ptx.cuh"
+#include "qkv_post.cuh"
 
 namespace svdq {
 
@@ -73,13 +74,13 @@ struct GemmBarriers {
   int abort;
 };
 
-template <int R>
+template <int R, bool QKV>
 __global__ void __launch_bounds__(kGemmThreads, 1) w4a4_gemm_kernel(
     const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
     const __grid_constant__ CUtensorMap tm_xl1, const __grid_constant__ CUtensorMap tm_l2s,
     const uint8_t* __restrict__ a_scales, const uint8_t* __restrict__ w_scales,
     const float* __restrict__ gscale, const __nv_bfloat16* __restrict__ bias, __nv_bfloat16* __restrict__ Y,
-    int64_t ldy, int M, int N, int K) {
+    int64_t ldy, int M, int N, int K, const QkvPost post) {
   using C = GemmCfg<R>;
   constexpr int S = C::kStages;
   extern __shared__ uint8_t smem_raw[];
@@ -246,44 +247,84 @@ __global__ void __launch_bounds__(kGemmThreads, 1) w4a4_gemm_kernel(
       tc_fence_after();
       const int row = mb * kBM + 32 * q + lane;
       const uint32_t lane_base = tmem + (static_cast<uint32_t>(32 * q) << 16);
-#pragma unroll 1
-      for (int c = 0; c < kBN / 32; ++c) {
-        uint32_t va[32], vl[32];
-        tmem_ld_32x32b_x32(lane_base + b * kBN + 32 * c, va);
-        tmem_ld_32x32b_x32(lane_base + 256 + 32 * c, vl);
-        tmem_ld_wait();
-        const int n0 = nb * kBN + 32 * c;
-        float bf[32];
-        if (bias != nullptr) {
+      if constexpr (QKV) {
+        // The tile is one 128-column head of Q, K or V: gather the row, then
+        // normalise and rotate Q / K rows before storing.
+        const int n_tile = nb * kBN;
+        const int seg = n_tile / post.hd;
+        const __nv_bfloat16* w = seg == 0 ? post.w_q : (seg == 1 ? post.w_k : nullptr);
+        uint32_t pk[64];
+#pragma unroll
+        for (int c = 0; c < kBN / 32; ++c) {
+          uint32_t va[32], vl[32];
+          tmem_ld_32x32b_x32(lane_base + b * kBN + 32 * c, va);
+          tmem_ld_32x32b_x32(lane_base + 256 + 32 * c, vl);
+          tmem_ld_wait();
+          uint32_t bw[16];
 #pragma unroll
           for (int v = 0; v < 4; ++v) {
-            const uint4 u = ldg_v4(bias + n0 + 8 * v);
-            const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              bf[8 * v + 2 * i] = __uint_as_float(w4[i] << 16);
-              bf[8 * v + 2 * i + 1] = __uint_as_float(w4[i] & 0xFFFF0000u);
-            }
+            const uint4 u = bias != nullptr ? ldg_v4(bias + n_tile + 32 * c + 8 * v) : make_uint4(0u, 0u, 0u, 0u);
+            bw[4 * v] = u.x;
+            bw[4 * v + 1] = u.y;
+            bw[4 * v + 2] = u.z;
+            bw[4 * v + 3] = u.w;
           }
-        } else {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) bf[i] = 0.0f;
+          for (int i = 0; i < 16; ++i) {
+            const float s0 = __fadd_rn(__uint_as_float(va[2 * i]), __uint_as_float(vl[2 * i]));
+            const float s1 = __fadd_rn(__uint_as_float(va[2 * i + 1]), __uint_as_float(vl[2 * i + 1]));
+            pk[16 * c + i] = pack_bf16(__fmaf_rn(s0, alpha, bf16_lo(bw[i])), __fmaf_rn(s1, alpha, bf16_hi(bw[i])));
+          }
         }
-        uint32_t packed[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float s0 = __fadd_rn(__uint_as_float(va[2 * i]), __uint_as_float(vl[2 * i]));
-          const float s1 = __fadd_rn(__uint_as_float(va[2 * i + 1]), __uint_as_float(vl[2 * i + 1]));
-          const float y0 = __fmaf_rn(s0, alpha, bf[2 * i]);
-          const float y1 = __fmaf_rn(s1, alpha, bf[2 * i + 1]);
-          const __nv_bfloat162 h = __floats2bfloat162_rn(y0, y1);
-          packed[i] = *reinterpret_cast<const uint32_t*>(&h);
+        if (w != nullptr) {
+          const int64_t rr = row < M ? row : M - 1;
+          qk_norm_rope_row(pk, w, post.cos + rr * post.ld_rope, post.sin + rr * post.ld_rope, post.eps);
         }
         if (row < M) {
-          uint4* dst = reinterpret_cast<uint4*>(Y + static_cast<int64_t>(row) * ldy + n0);
+          uint4* dst = reinterpret_cast<uint4*>(Y + static_cast<int64_t>(row) * ldy + n_tile);
 #pragma unroll
-          for (int v = 0; v < 4; ++v)
-            dst[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
+          for (int v = 0; v < 16; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+        }
+      } else {
+#pragma unroll 1
+        for (int c = 0; c < kBN / 32; ++c) {
+          uint32_t va[32], vl[32];
+          tmem_ld_32x32b_x32(lane_base + b * kBN + 32 * c, va);
+          tmem_ld_32x32b_x32(lane_base + 256 + 32 * c, vl);
+          tmem_ld_wait();
+          const int n0 = nb * kBN + 32 * c;
+          float bf[32];
+          if (bias != nullptr) {
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              const uint4 u = ldg_v4(bias + n0 + 8 * v);
+              const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                bf[8 * v + 2 * i] = __uint_as_float(w4[i] << 16);
+                bf[8 * v + 2 * i + 1] = __uint_as_float(w4[i] & 0xFFFF0000u);
+              }
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) bf[i] = 0.0f;
+          }
+          uint32_t packed[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float s0 = __fadd_rn(__uint_as_float(va[2 * i]), __uint_as_float(vl[2 * i]));
+            const float s1 = __fadd_rn(__uint_as_float(va[2 * i + 1]), __uint_as_float(vl[2 * i + 1]));
+            const float y0 = __fmaf_rn(s0, alpha, bf[2 * i]);
+            const float y1 = __fmaf_rn(s1, alpha, bf[2 * i + 1]);
+            const __nv_bfloat162 h = __floats2bfloat162_rn(y0, y1);
+            packed[i] = *reinterpret_cast<const uint32_t*>(&h);
+          }
+          if (row < M) {
+            uint4* dst = reinterpret_cast<uint4*>(Y + static_cast<int64_t>(row) * ldy + n0);
+#pragma unroll
+            for (int v = 0; v < 4; ++v)
+              dst[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
+          }
         }
       }
       tc_fence_before();

@@ -36,6 +36,7 @@
 #pragma once
 
 #include "ptx.cuh"
+#include "qkv_post.cuh"
 
 namespace svdq {
 
@@ -121,7 +122,7 @@ constexpr int k2Acc1Col = 208;
 constexpr int k2SfaCol = 464;
 constexpr int k2SfbCol = 480;
 
-template <int R>
+template <int R, bool QKV = false>
 struct Gemm2Cfg {
   static constexpr int kABytes = 128 * 128;     // 128 rows x 256 E2M1
   static constexpr int kBBytes = 128 * 128;
@@ -139,9 +140,15 @@ struct Gemm2Cfg {
   static constexpr SwizzleMode kLrSwizzle = kLrRowBytes == 64 ? kSwizzle64B : kSwizzle32B;
   static constexpr uint32_t kMainTx = 2u * kStageBytes;     // both CTAs
   static constexpr uint32_t kLrTx = 2u * 3u * kLrTileBytes;
-  static constexpr int kOutOff = kStages * kStageBytes;      // epilogue staging: 8 warps x 2 x 2 KB
-  static constexpr int kOutBytes = 8 * 2 * 2048;
-  static constexpr int kBarOff = kOutOff + kOutBytes;
+  // Epilogue staging per warp: two 2 KB bf16 TMA-store buffers.
+  static constexpr int kOutPerWarp = 4096;
+  static constexpr int kOutOff = kStages * kStageBytes;
+  static constexpr int kOutBytes = 8 * kOutPerWarp;
+  // Fused QKV: per warp, partial sums of squares of its rows for the two heads
+  // of a tile, double-buffered (2 x 2 x 32 floats).
+  static constexpr int kXchgOff = kOutOff + kOutBytes;
+  static constexpr int kXchgBytes = QKV ? 8 * 512 : 0;
+  static constexpr int kBarOff = kXchgOff + kXchgBytes;
   static constexpr int kSmemBytes = kBarOff + 256 + 1024;
 };
 
@@ -152,6 +159,7 @@ struct Gemm2Barriers {
   uint64_t acc_empty[2];
   uint64_t ovl_free;
   uint64_t teardown;
+  uint64_t xchg[4];  // fused QKV: the two epilogue warps of a TMEM lane quadrant (64 arrivals)
   uint32_t tmem_base;
   int abort;
 };
@@ -165,6 +173,7 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap* m, const void* s
 }
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_read1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -230,14 +239,221 @@ __device__ __forceinline__ void epilogue_half(uint32_t taddr, const uint4 (&bv)[
   ++nbuf;
 }
 
-template <int R>
+// ------------------------------------------------------------------ fused QKV epilogue
+// For the fused QKV variant the two epilogue warps of a TMEM lane quadrant
+// split a 256-column tile (two 128-column heads) by chunks rather than by
+// heads: warp h takes chunks 2h, 2h+1 of both heads, so the rotary angles it
+// needs (pairs 32h..32h+31 of its rows) are the same for both heads and are
+// fetched once, before the accumulator is ready. The per-row sums of squares
+// of the two warps are combined through shared memory.
+
+// Writes / reads this lane's row of 16 packed bf16 pairs in a 2 KB staging
+// buffer (32 rows x 64 bytes, the 64-byte swizzle of the store map).
+__device__ __forceinline__ void stage_row16(uint8_t* buf, const uint32_t (&pk)[16], int lane) {
+  const int sw = (lane >> 1) & 3;
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+    *reinterpret_cast<uint4*>(buf + lane * 64 + ((j ^ sw) << 4)) =
+        make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+}
+__device__ __forceinline__ void load_row16(const uint8_t* buf, uint32_t (&pk)[16], int lane) {
+  const int sw = (lane >> 1) & 3;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint4 v = *reinterpret_cast<const uint4*>(buf + lane * 64 + ((j ^ sw) << 4));
+    pk[4 * j] = v.x;
+    pk[4 * j + 1] = v.y;
+    pk[4 * j + 2] = v.z;
+    pk[4 * j + 3] = v.w;
+  }
+}
+// This lane's row of 16 rotary angles (cos at cr, sin at sr; 16-byte aligned).
+__device__ __forceinline__ void load_angles16(const float* cr, const float* sr, float (&tc)[16], float (&ts)[16]) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float4 c = reinterpret_cast<const float4*>(cr)[i];
+    const float4 sv = reinterpret_cast<const float4*>(sr)[i];
+    tc[4 * i] = c.x;
+    tc[4 * i + 1] = c.y;
+    tc[4 * i + 2] = c.z;
+    tc[4 * i + 3] = c.w;
+    ts[4 * i] = sv.x;
+    ts[4 * i + 1] = sv.y;
+    ts[4 * i + 2] = sv.z;
+    ts[4 * i + 3] = sv.w;
+  }
+}
+
+// Publishes a staged buffer to the async proxy and stores it with TMA.
+__device__ __forceinline__ void store_staged(const uint8_t* buf, const CUtensorMap* tm_y, int x, int y, int lane) {
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0) {
+    tma_store_2d(tm_y, buf, x, y);
+    bulk_commit();
+  }
+}
+
+// bf16 pairs of alpha * acc + b for one 32-column chunk (bias at bcol, or none).
+__device__ __forceinline__ void pack32(const uint32_t (&v)[32], const __nv_bfloat16* bcol, float alpha,
+                                       uint32_t (&pk)[16]) {
+  pack_chunk(v, bcol, alpha, pk);
+}
+
+// Sum of squares of 16 packed bf16 pairs, added to ss in element order.
+__device__ __forceinline__ float sumsq16(const uint32_t (&pk)[16], float ss) {
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const float a = bf16_lo(pk[i]), b = bf16_hi(pk[i]);
+    ss = __fmaf_rn(a, a, ss);
+    ss = __fmaf_rn(b, b, ss);
+  }
+  return ss;
+}
+
+// RMSNorm (rstd, weights wcol: the chunk's 32 bf16) and rotation of the 16
+// pairs of a chunk of this lane's row by their angles (tc, ts: cos, sin), in
+// fp32, one rounding to bf16.
+__device__ __forceinline__ void qk_rot16(uint32_t (&pk)[16], float rstd, const __nv_bfloat16* __restrict__ wcol,
+                                         const float (&tc)[16], const float (&ts)[16]) {
+#pragma unroll
+  for (int q4 = 0; q4 < 4; ++q4) {
+    const uint4 wv = *reinterpret_cast<const uint4*>(wcol + 8 * q4);
+    const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      const int j = 4 * q4 + t;
+      const float c = tc[j], sn = ts[j];
+      const float n0 = bf16_lo(pk[j]) * rstd * bf16_lo(ww[t]);
+      const float n1 = bf16_hi(pk[j]) * rstd * bf16_hi(ww[t]);
+      pk[j] = pack_bf16(__fmaf_rn(n0, c, -n1 * sn), __fmaf_rn(n1, c, n0 * sn));
+    }
+  }
+}
+
+// One fused-QKV tile for one epilogue warp: chunks c0 = 2h, c0 + 1 of head F
+// (read first: it holds the columns shared by the two accumulators when
+// holds_overlap) and of head 1 - F. tacc: the accumulator's TMEM address for
+// this lane quadrant. For a Q/K tile (w_f, w_s the norm weights of heads F
+// and 1 - F)
+// tc0/ts0 hold the angles of chunk c0's pairs (fetched before the
+// accumulator was ready), cr/sr point at those of chunk c0 + 1 (fetched once
+// the first head is read) and xs_* are the exchange slots; a V tile
+// (w_f == nullptr) is stored as computed. Returns false on abort.
+__device__ __forceinline__ bool epilogue_qkv_tile(uint32_t tacc, int F, int h, const __nv_bfloat16* btile, float alpha,
+                                                  uint8_t* stage, const CUtensorMap* tm_y, int xt, int y0,
+                                                  bool holds_overlap, uint32_t ovl_bar, int lane,
+                                                  const __nv_bfloat16* w_f, const __nv_bfloat16* w_s,
+                                                  const float (&tc0)[16],
+                                                  const float (&ts0)[16], const float* cr, const float* sr,
+                                                  float* xs_mine, const float* xs_peer,
+                                                  uint64_t* xbar, uint32_t xpar, float eps, volatile int* abort) {
+  const int S = 1 - F;
+  const bool qk = w_f != nullptr;
+  const int c0 = 2 * h;
+  const auto bcol = [&](int head, int c) { return btile != nullptr ? btile + 128 * head + 32 * c : nullptr; };
+  float ssf = 0.0f, sss = 0.0f;  // this warp's part of the rows' sums of squares
+  if (lane == 0) bulk_wait_read0();  // both staging buffers are free
+  __syncwarp();
+  {
+    uint32_t va[32], vb[32];
+    tmem_ld_32x32b_x32(tacc + 128 * F + 32 * c0, va);
+    tmem_ld_32x32b_x32(tacc + 128 * F + 32 * (c0 + 1), vb);
+    tmem_ld_wait();
+    if (holds_overlap) {  // the loads above have completed (tcgen05.wait::ld): nothing else to publish
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster_relaxed(ovl_bar);
+    }
+    uint32_t pk[16];
+    pack32(va, bcol(F, c0), alpha, pk);
+    ssf = sumsq16(pk, ssf);
+    stage_row16(stage, pk, lane);
+    if (!qk) store_staged(stage, tm_y, xt + 128 * F + 32 * c0, y0, lane);
+    pack32(vb, bcol(F, c0 + 1), alpha, pk);
+    ssf = sumsq16(pk, ssf);
+    stage_row16(stage + 2048, pk, lane);
+    if (!qk) store_staged(stage + 2048, tm_y, xt + 128 * F + 32 * (c0 + 1), y0, lane);
+  }
+  float tc1[16], ts1[16];
+  if (qk) {
+    load_angles16(cr, sr, tc1, ts1);
+    // head 1 - F never holds shared columns: read it for its sums now and
+    // again, to store it, after the exchange
+#pragma unroll 1
+    for (int k = 0; k < 2; ++k) {
+      uint32_t va[32], pk[16];
+      tmem_ld_32x32b_x32(tacc + 128 * S + 32 * (c0 + k), va);
+      tmem_ld_wait();
+      pack32(va, bcol(S, c0 + k), alpha, pk);
+      sss = sumsq16(pk, sss);
+    }
+    // this warp's partial sums for heads 0 / 1, then the partner's
+    xs_mine[32 * F + lane] = ssf;
+    xs_mine[32 * S + lane] = sss;
+    mbar_arrive(xbar);
+    if (!mbar_wait(xbar, xpar, abort)) return false;
+    const float pf = xs_peer[32 * F + lane], pss = xs_peer[32 * S + lane];
+    // rows' sums in chunk order: warp 0's chunks 0, 1 then warp 1's chunks 2, 3
+    const float tf = h == 0 ? ssf + pf : pf + ssf;
+    const float tsum = h == 0 ? sss + pss : pss + sss;
+    const float rs_f = 1.0f / sqrtf(__fmaf_rn(tf, 1.0f / kHeadDim, eps));
+    const float rs_s = 1.0f / sqrtf(__fmaf_rn(tsum, 1.0f / kHeadDim, eps));
+    uint32_t pk[16];
+    load_row16(stage, pk, lane);
+    qk_rot16(pk, rs_f, w_f + 32 * c0, tc0, ts0);
+    stage_row16(stage, pk, lane);
+    store_staged(stage, tm_y, xt + 128 * F + 32 * c0, y0, lane);
+    load_row16(stage + 2048, pk, lane);
+    qk_rot16(pk, rs_f, w_f + 32 * (c0 + 1), tc1, ts1);
+    stage_row16(stage + 2048, pk, lane);
+    store_staged(stage + 2048, tm_y, xt + 128 * F + 32 * (c0 + 1), y0, lane);
+    {
+      uint32_t va[32];
+      tmem_ld_32x32b_x32(tacc + 128 * S + 32 * c0, va);
+      tmem_ld_wait();
+      pack32(va, bcol(S, c0), alpha, pk);
+    }
+    qk_rot16(pk, rs_s, w_s + 32 * c0, tc0, ts0);
+    if (lane == 0) bulk_wait_read1();  // the store from buffer 0 has read it
+    __syncwarp();
+    stage_row16(stage, pk, lane);
+    store_staged(stage, tm_y, xt + 128 * S + 32 * c0, y0, lane);
+    {
+      uint32_t va[32];
+      tmem_ld_32x32b_x32(tacc + 128 * S + 32 * (c0 + 1), va);
+      tmem_ld_wait();
+      pack32(va, bcol(S, c0 + 1), alpha, pk);
+    }
+    qk_rot16(pk, rs_s, w_s + 32 * (c0 + 1), tc1, ts1);
+    if (lane == 0) bulk_wait_read1();
+    __syncwarp();
+    stage_row16(stage + 2048, pk, lane);
+    store_staged(stage + 2048, tm_y, xt + 128 * S + 32 * (c0 + 1), y0, lane);
+    return true;
+  }
+#pragma unroll 1
+  for (int k = 0; k < 2; ++k) {  // V: head 1 - F as computed
+    uint32_t va[32], pk[16];
+    tmem_ld_32x32b_x32(tacc + 128 * S + 32 * (c0 + k), va);
+    tmem_ld_wait();
+    pack32(va, bcol(S, c0 + k), alpha, pk);
+    if (lane == 0) bulk_wait_read1();
+    __syncwarp();
+    stage_row16(stage + 2048 * k, pk, lane);
+    store_staged(stage + 2048 * k, tm_y, xt + 128 * S + 32 * (c0 + k), y0, lane);
+  }
+  return true;
+}
+
+template <int R, bool QKV>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(k2Threads, 1) w4a4_gemm_2sm_kernel(
     const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
     const __grid_constant__ CUtensorMap tm_sfa, const __grid_constant__ CUtensorMap tm_sfb,
     const __grid_constant__ CUtensorMap tm_xl1, const __grid_constant__ CUtensorMap tm_l2s,
     const __grid_constant__ CUtensorMap tm_y, const float* __restrict__ gscale,
-    const __nv_bfloat16* __restrict__ bias, int M, int N, int K) {
-  using C = Gemm2Cfg<R>;
+    const __nv_bfloat16* __restrict__ bias, int M, int N, int K, const QkvPost post) {
+  using C = Gemm2Cfg<R, QKV>;
   constexpr int S = C::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -266,6 +482,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(k2Threads, 1) w4a4_g
     }
     mbar_init(&bars->ovl_free, 8);         // 4 warps (the half holding the shared columns) x 2 CTAs
     mbar_init(&bars->teardown, 1);
+    for (int i = 0; i < 4; ++i) mbar_init(&bars->xchg[i], 64);
     bars->abort = 0;
     fence_barrier_init();
   }
@@ -397,14 +614,51 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(k2Threads, 1) w4a4_g
     const float alpha = gscale[2];
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(32 * q) << 16);
     const uint32_t ovl_bar = mapa_shared(smem_u32(&bars->ovl_free), 0);
-    uint8_t* stage = smem + C::kOutOff + e * 4096;
+    uint8_t* stage = smem + C::kOutOff + e * C::kOutPerWarp;
     int nbuf = 0;
+    uint32_t nx = 0;  // fused QKV: exchanges of row sums done by this warp
     int it = 0;
     for (int tile = pair; tile < num_tiles; tile += num_pairs, ++it) {
       const int mt = tile % num_mt, nt = tile / num_mt;
       const int b = it & 1;
       const int y0 = mt * k2TileM + static_cast<int>(rank) * 128 + 32 * q;
       const int col0 = nt * k2TileN + 128 * h;
+      if constexpr (QKV) {
+        // Q / K tiles: this lane's rotary angles for the warp's first chunk,
+        // fetched before the accumulator is ready. A tile is all Q/K or all V (the
+        // V block starts at 2 * hd, a multiple of 256).
+        const int xt = nt * k2TileN;
+        const bool qk = xt < 2 * post.hd;
+        float tc0[16], ts0[16];
+        const int64_t row = (y0 + lane < M) ? y0 + lane : M - 1;
+        const float* cr = post.cos + row * post.ld_rope + 32 * h;
+        const float* sr = post.sin + row * post.ld_rope + 32 * h;
+        if (qk) {
+          load_angles16(cr, sr, tc0, ts0);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) tc0[i] = ts0[i] = 0.0f;
+        }
+        const __nv_bfloat16* w0 = qk ? (xt < post.hd ? post.w_q : post.w_k) : nullptr;
+        const __nv_bfloat16* w1 = qk ? (xt + 128 < post.hd ? post.w_q : post.w_k) : nullptr;
+        if (!mbar_wait(&bars->acc_full[b], (it >> 1) & 1, abort)) break;
+        tc_fence_after();
+        const uint32_t tacc = lane_base + (b ? k2Acc1Col : 0);
+        const __nv_bfloat16* btile = bias != nullptr ? bias + xt : nullptr;
+        float* xs = reinterpret_cast<float*>(smem + C::kXchgOff) + 128 * (2 * q + h) + 64 * (nx & 1);
+        const float* xp = reinterpret_cast<const float*>(smem + C::kXchgOff) + 128 * (2 * q + (h ^ 1)) + 64 * (nx & 1);
+        // accumulator 0's shared columns lie in head 1 (warp 1's chunks),
+        // accumulator 1's in head 0 (warp 0's chunks)
+        const bool ok = epilogue_qkv_tile(tacc, b == 0 ? 1 : 0, h, btile, alpha, stage, &tm_y, xt, y0, h == (b == 0),
+                                          ovl_bar, lane, b == 0 ? w1 : w0, b == 0 ? w0 : w1, tc0, ts0, cr + 16, sr + 16, xs, xp, &bars->xchg[q], nx & 1,
+                                          post.eps, abort);
+        if (!ok) break;
+        if (qk) ++nx;
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster_relaxed(mapa_shared(smem_u32(&bars->acc_empty[b]), 0));
+        continue;
+      }
       // bias of this warp's 128 columns, fetched before the accumulator is ready
       uint4 bv[16];
       if (bias != nullptr) {

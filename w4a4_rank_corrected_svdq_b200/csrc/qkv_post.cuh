@@ -1,0 +1,100 @@
+// qkv_post.cuh — fused QKV post-processing in the GEMM epilogue: per-head
+// RMSNorm of the Q and K heads and the rotary embedding, applied to the
+// layer's bf16 output before it is stored.
+//
+// Blog "Bringing Nunchaku 4-bit Diffusion Inference to Diffusers", section
+// "Quantizing models with structural rewrites": the Q, K and V projections
+// are fused into one to_qkv layer, and the fused operator consumes that
+// projection, the Q/K normalisation and the rotary embedding together.
+// For a [M, 3 * H * 128] output laid out [Q | K | V] (head_dim 128):
+//   q = bf16(alpha * acc + b)                       (the layer output)
+//   n_i = q_i / sqrt(mean_i(q_i^2) + eps) * w_i     (RMSNorm per head, fp32)
+//   (n0, n1) -> (n0 c_j - n1 s_j, n1 c_j + n0 s_j)  (pair 2j, 2j+1 rotated by theta_j)
+// rounded to bf16 once; V is stored unchanged. An epilogue warp holds 32 rows
+// of one 128-column head, so each thread owns a whole head row: the norm is
+// thread-local and each rotation pair lies in one 32-column chunk.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cstdint>
+
+namespace svdq {
+
+constexpr int kHeadDim = 128;
+
+struct QkvPost {
+  const __nv_bfloat16* w_q;  // [128] RMSNorm weight of the Q heads
+  const __nv_bfloat16* w_k;  // [128] RMSNorm weight of the K heads
+  const float* cos;          // [M][ld_rope] cos(theta_j) per token and pair (64 used)
+  const float* sin;          // [M][ld_rope] sin(theta_j)
+  int64_t ld_rope;
+  int hd;                    // columns of each of Q, K and V (heads * 128)
+  float eps;
+};
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+// One head row held as 64 packed bf16 pairs (element 2j in the low half of
+// p[j]): RMSNorm with weight w, then the rotation of each pair j by this
+// row's angle (cs[j], sn[j]: 64 floats each, 16-byte aligned), in place.
+__device__ __forceinline__ void qk_norm_rope_row(uint32_t (&p)[64], const __nv_bfloat16* __restrict__ w,
+                                                 const float* __restrict__ cs, const float* __restrict__ sn,
+                                                 float eps) {
+  float ss = 0.0f;
+#pragma unroll
+  for (int j = 0; j < 64; ++j) {
+    const float x0 = bf16_lo(p[j]), x1 = bf16_hi(p[j]);
+    ss = __fmaf_rn(x0, x0, ss);
+    ss = __fmaf_rn(x1, x1, ss);
+  }
+  const float rstd = 1.0f / sqrtf(__fmaf_rn(ss, 1.0f / kHeadDim, eps));
+#pragma unroll
+  for (int g = 0; g < 16; ++g) {  // 8 columns = 4 pairs per group
+    const uint4 wv = *reinterpret_cast<const uint4*>(w + 8 * g);
+    const float4 c4 = *reinterpret_cast<const float4*>(cs + 4 * g);
+    const float4 s4 = *reinterpret_cast<const float4*>(sn + 4 * g);
+    const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
+    const float cc[4] = {c4.x, c4.y, c4.z, c4.w};
+    const float ssn[4] = {s4.x, s4.y, s4.z, s4.w};
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      const int j = 4 * g + t;
+      const float n0 = bf16_lo(p[j]) * rstd * bf16_lo(ww[t]);
+      const float n1 = bf16_hi(p[j]) * rstd * bf16_hi(ww[t]);
+      p[j] = pack_bf16(__fmaf_rn(n0, cc[t], -n1 * ssn[t]), __fmaf_rn(n1, cc[t], n0 * ssn[t]));
+    }
+  }
+}
+
+// bf16 pairs of y = alpha * acc + b for one 32-column chunk (bias: 32 bf16 at
+// bcol, or none).
+__device__ __forceinline__ void pack_chunk(const uint32_t (&v)[32], const __nv_bfloat16* __restrict__ bcol,
+                                           float alpha, uint32_t* out) {
+  uint32_t bw[16];
+  if (bcol != nullptr) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const uint4 u = *reinterpret_cast<const uint4*>(bcol + 8 * q);
+      bw[4 * q] = u.x;
+      bw[4 * q + 1] = u.y;
+      bw[4 * q + 2] = u.z;
+      bw[4 * q + 3] = u.w;
+    }
+  } else {
+#pragma unroll
+    for (int q = 0; q < 16; ++q) bw[q] = 0u;
+  }
+#pragma unroll
+  for (int p = 0; p < 16; ++p) {
+    const float y0 = __fmaf_rn(__uint_as_float(v[2 * p]), alpha, bf16_lo(bw[p]));
+    const float y1 = __fmaf_rn(__uint_as_float(v[2 * p + 1]), alpha, bf16_hi(bw[p]));
+    out[p] = pack_bf16(y0, y1);
+  }
+}
+
+}  // namespace svdq

@@ -364,10 +364,11 @@ svdq_status quantize_dispatch(int M, int K, int r, const void* X, int64_t ldx, c
   }
 }
 
-template <int R>
+template <int R, bool QKV>
 svdq_status launch_gemm(int M, int N, int K, const void* a_codes, const void* a_scales, const void* xl1,
                         const void* w_codes, const void* w_scales, const float* gscale, const void* l2s,
-                        const void* bias, void* Y, int64_t ldy, cudaStream_t stream, int sm_count) {
+                        const void* bias, void* Y, int64_t ldy, cudaStream_t stream, int sm_count,
+                        const QkvPost& post) {
   using C = GemmCfg<R>;
   CUtensorMap tm_a, tm_b, tm_x, tm_l;
   const uint64_t kb = static_cast<uint64_t>(K / 2);
@@ -380,7 +381,7 @@ svdq_status launch_gemm(int M, int N, int K, const void* a_codes, const void* a_
       !make_tmap_2d(&tm_l, l2s, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, R, 2 * static_cast<uint64_t>(N), R * 2,
                     C::kLrAtomCols, kBN, lr_swizzle(R)))
     return SVDQ_ERR_CUDA;
-  auto kern = w4a4_gemm_kernel<R>;
+  auto kern = w4a4_gemm_kernel<R, QKV>;
   static std::atomic<uint64_t> attr_done{0};
   ensure_smem_attr(kern, C::kSmemBytes, attr_done);
   const int tiles = ((M + kBM - 1) / kBM) * (N / kBN);
@@ -388,15 +389,16 @@ svdq_status launch_gemm(int M, int N, int K, const void* a_codes, const void* a_
   PdlLaunch pl(dim3(grid), dim3(kGemmThreads), C::kSmemBytes, stream);
   cudaLaunchKernelEx(&pl.cfg, kern, tm_a, tm_b, tm_x, tm_l, static_cast<const uint8_t*>(a_scales),
                      static_cast<const uint8_t*>(w_scales), gscale, static_cast<const __nv_bfloat16*>(bias),
-                     static_cast<__nv_bfloat16*>(Y), ldy, M, N, K);
+                     static_cast<__nv_bfloat16*>(Y), ldy, M, N, K, post);
   return launch_status();
 }
 
-template <int R>
+template <int R, bool QKV>
 svdq_status launch_gemm_2sm(int M, int N, int K, const void* a_codes, const void* a_scales, const void* xl1,
                             const void* w_codes, const void* w_scales, const float* gscale, const void* l2s,
-                            const void* bias, void* Y, int64_t ldy, cudaStream_t stream, int sm_count) {
-  using C = Gemm2Cfg<R>;
+                            const void* bias, void* Y, int64_t ldy, cudaStream_t stream, int sm_count,
+                            const QkvPost& post) {
+  using C = Gemm2Cfg<R, QKV>;
   CUtensorMap tm_a, tm_b, tm_sfa, tm_sfb, tm_x, tm_l, tm_y;
   const uint64_t kb = static_cast<uint64_t>(K / 2);
   const uint64_t mpad = round_up(static_cast<size_t>(M), 128);
@@ -412,7 +414,7 @@ svdq_status launch_gemm_2sm(int M, int N, int K, const void* a_codes, const void
       !make_tmap_2d(&tm_y, Y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, M, static_cast<uint64_t>(ldy) * 2, 32, 32,
                     CU_TENSOR_MAP_SWIZZLE_64B))
     return SVDQ_ERR_CUDA;
-  auto kern = w4a4_gemm_2sm_kernel<R>;
+  auto kern = w4a4_gemm_2sm_kernel<R, QKV>;
   static std::atomic<uint64_t> attr_done{0};
   ensure_smem_attr(kern, C::kSmemBytes, attr_done);
   const int tiles = ((M + k2TileM - 1) / k2TileM) * (N / k2TileN);
@@ -420,7 +422,7 @@ svdq_status launch_gemm_2sm(int M, int N, int K, const void* a_codes, const void
   const int pairs = tiles < max_pairs ? tiles : max_pairs;
   PdlLaunch pl(dim3(2 * pairs), dim3(k2Threads), C::kSmemBytes, stream);
   cudaLaunchKernelEx(&pl.cfg, kern, tm_a, tm_b, tm_sfa, tm_sfb, tm_x, tm_l, tm_y, gscale,
-                     static_cast<const __nv_bfloat16*>(bias), M, N, K);
+                     static_cast<const __nv_bfloat16*>(bias), M, N, K, post);
   return launch_status();
 }
 
@@ -437,24 +439,28 @@ bool use_2sm(int M, int N) {
   return M >= 512;
 }
 
+// post == nullptr: the plain layer; otherwise the fused QKV post-processing.
 svdq_status gemm_dispatch(int M, int N, int K, int r, const void* a_codes, const void* a_scales, const void* xl1,
                           const void* w_codes, const void* w_scales, const float* gscale, const void* l2s,
-                          const void* bias, void* Y, int64_t ldy, cudaStream_t st, int sms) {
-#define SVDQ_GEMM_ARGS M, N, K, a_codes, a_scales, xl1, w_codes, w_scales, gscale, l2s, bias, Y, ldy, st, sms
+                          const void* bias, void* Y, int64_t ldy, cudaStream_t st, int sms,
+                          const QkvPost* post = nullptr) {
+  const QkvPost none{};
+  const QkvPost& pp = post != nullptr ? *post : none;
+#define SVDQ_GEMM_ARGS M, N, K, a_codes, a_scales, xl1, w_codes, w_scales, gscale, l2s, bias, Y, ldy, st, sms, pp
+#define SVDQ_GEMM_CASES(F, Q)                 \
+  switch (r) {                                \
+    case 16: return F<16, Q>(SVDQ_GEMM_ARGS); \
+    case 32: return F<32, Q>(SVDQ_GEMM_ARGS); \
+    case 64: return F<64, Q>(SVDQ_GEMM_ARGS); \
+    default: return F<128, Q>(SVDQ_GEMM_ARGS); \
+  }
   if (use_2sm(M, N)) {
-    switch (r) {
-      case 16: return launch_gemm_2sm<16>(SVDQ_GEMM_ARGS);
-      case 32: return launch_gemm_2sm<32>(SVDQ_GEMM_ARGS);
-      case 64: return launch_gemm_2sm<64>(SVDQ_GEMM_ARGS);
-      default: return launch_gemm_2sm<128>(SVDQ_GEMM_ARGS);
-    }
+    if (post != nullptr) SVDQ_GEMM_CASES(launch_gemm_2sm, true)
+    SVDQ_GEMM_CASES(launch_gemm_2sm, false)
   }
-  switch (r) {
-    case 16: return launch_gemm<16>(SVDQ_GEMM_ARGS);
-    case 32: return launch_gemm<32>(SVDQ_GEMM_ARGS);
-    case 64: return launch_gemm<64>(SVDQ_GEMM_ARGS);
-    default: return launch_gemm<128>(SVDQ_GEMM_ARGS);
-  }
+  if (post != nullptr) SVDQ_GEMM_CASES(launch_gemm, true)
+  SVDQ_GEMM_CASES(launch_gemm, false)
+#undef SVDQ_GEMM_CASES
 #undef SVDQ_GEMM_ARGS
 }
 
@@ -657,6 +663,10 @@ svdq_status run_lowrank(int N, int K, int r, const __nv_bfloat16* W, __nv_bfloat
   return launch_status();
 }
 
+svdq_status gemm_checked(int M, int N, int K, int r, const void* a_codes, const void* a_scales, const void* xl1,
+                         const void* w_codes, const void* w_scales, const float* gscale, const void* l2s,
+                         const void* bias, void* Y, int64_t ldy, void* stream, const QkvPost* post);
+
 }  // namespace
 }  // namespace svdq
 
@@ -805,6 +815,57 @@ svdq_status svdq_quantize_act(int M, int K, int r, const void* X, int64_t ldx, c
 svdq_status svdq_w4a4_gemm(int M, int N, int K, int r, const void* a_codes, const void* a_scales, const void* xl1,
                            const void* w_codes, const void* w_scales, const float* gscale, const void* l2s,
                            const void* bias, void* Y, int64_t ldy, void* stream) {
+  return gemm_checked(M, N, K, r, a_codes, a_scales, xl1, w_codes, w_scales, gscale, l2s, bias, Y, ldy, stream,
+                      nullptr);
+}
+
+svdq_status svdq_linear_forward_qkv(int M, int N, int K, int r, const void* X, int64_t ldx, const void* w_codes,
+                                    const void* w_scales, const float* gscale, const void* l1t, const void* l2s,
+                                    const void* bias, int heads, const void* norm_q_weight,
+                                    const void* norm_k_weight, float eps, const float* rope_cos,
+                                    const float* rope_sin, int64_t ld_rope, void* Y, int64_t ldy, void* workspace,
+                                    size_t workspace_bytes, void* stream) {
+  if (M < 0 || heads <= 0 || !(eps >= 0.0f && eps < 1e30f)) return SVDQ_ERR_INVALID_ARG;
+  svdq_status s = check_layer_shape(N, K, r);
+  if (s != SVDQ_OK) return s;
+  if (static_cast<int64_t>(N) != 3ll * heads * kHeadDim) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+  if (ldx < K || ldx % 8 != 0 || ldy < N || ldy % 8 != 0 || ld_rope < kHeadDim / 2 || ld_rope % 4 != 0)
+    return SVDQ_ERR_UNSUPPORTED_SHAPE;
+  if (M == 0) return SVDQ_OK;
+  if (!norm_q_weight || !norm_k_weight || !rope_cos || !rope_sin || !workspace || !gscale)
+    return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(norm_q_weight) || !aligned16(norm_k_weight) || !aligned16(rope_cos) || !aligned16(rope_sin) ||
+      !aligned16(workspace))
+    return SVDQ_ERR_MISALIGNED;
+  size_t need = 0, c = 0, sc = 0, x = 0;
+  svdq_forward_workspace_size(M, K, r, &need);
+  svdq_act_sizes(M, K, r, &c, &sc, &x);
+  if (workspace_bytes < need) return SVDQ_ERR_WORKSPACE;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint8_t* a_codes = ws;
+  uint8_t* a_scales = ws + round_up(c, 256);
+  uint8_t* xl1 = a_scales + round_up(sc, 256);
+  s = svdq_quantize_act(M, K, r, X, ldx, gscale, l1t, a_codes, a_scales, xl1, stream);
+  if (s != SVDQ_OK) return s;
+  QkvPost post{};
+  post.w_q = static_cast<const __nv_bfloat16*>(norm_q_weight);
+  post.w_k = static_cast<const __nv_bfloat16*>(norm_k_weight);
+  post.cos = rope_cos;
+  post.sin = rope_sin;
+  post.ld_rope = ld_rope;
+  post.hd = heads * kHeadDim;
+  post.eps = eps;
+  return gemm_checked(M, N, K, r, a_codes, a_scales, xl1, w_codes, w_scales, gscale, l2s, bias, Y, ldy, stream,
+                      &post);
+}
+
+}  // extern "C"
+
+namespace svdq {
+namespace {
+svdq_status gemm_checked(int M, int N, int K, int r, const void* a_codes, const void* a_scales, const void* xl1,
+                         const void* w_codes, const void* w_scales, const float* gscale, const void* l2s,
+                         const void* bias, void* Y, int64_t ldy, void* stream, const QkvPost* post) {
   if (M < 0) return SVDQ_ERR_INVALID_ARG;
   svdq_status s = check_layer_shape(N, K, r);
   if (s != SVDQ_OK) return s;
@@ -817,8 +878,12 @@ svdq_status svdq_w4a4_gemm(int M, int N, int K, int r, const void* a_codes, cons
   DeviceInfo di;
   if ((s = current_device(nullptr, &di)) != SVDQ_OK) return s;
   return gemm_dispatch(M, N, K, r, a_codes, a_scales, xl1, w_codes, w_scales, gscale, l2s, bias, Y, ldy,
-                       static_cast<cudaStream_t>(stream), di.sm_count);
+                       static_cast<cudaStream_t>(stream), di.sm_count, post);
 }
+}  // namespace
+}  // namespace svdq
+
+extern "C" {
 
 svdq_status svdq_linear_forward(int M, int N, int K, int r, const void* X, int64_t ldx, const void* w_codes,
                                 const void* w_scales, const float* gscale, const void* l1t, const void* l2s,

@@ -163,3 +163,15 @@ def small_layer(M: int, K: int, N: int, r: int, seed: int = 1234, outliers: int 
                      x_outlier_count=min(outliers, K), x_outlier_gain=gain,
                      w_std=w_std, bias_std=bias_std)
     return spec, make_layer(spec)
+
+
+def rope_tables(M: int, head_dim: int = 128, base: float = 10000.0, seed: int = 0):
+    """Rotary tables for token positions: cos and sin of theta[m, j] = pos[m] *
+    base^(-2j/head_dim), [M, head_dim // 2] float32, one angle per pair
+    (2j, 2j+1); pos is a seeded permutation of 0..M-1, so the tables are not
+    monotone in the row index."""
+    rng = np.random.default_rng([seed, M, head_dim])
+    pos = rng.permutation(M).astype(np.float64)
+    freq = base ** (-np.arange(0, head_dim, 2, dtype=np.float64) / head_dim)
+    ang = pos[:, None] * freq[None, :]
+    return np.cos(ang).astype(np.float32), np.sin(ang).astype(np.float32)
