@@ -13,10 +13,17 @@ Lite": 4-bit weights and activations). Written as one formula:
 
 with L1: K x r and L2: r x N in bfloat16 (the figure caption in that section:
 the down projection X.L1 is fused with the activation quantiser, the up
-projection (X.L1).L2 with the 4-bit GEMM). Smoothing is the identity here
-(lambda = 1), which is exactly the formula above.
+projection (X.L1).L2 with the 4-bit GEMM).
+
+Smoothing ("moving activation outliers into the weights", same section) is a
+per-input-channel factor lambda: the 4-bit branch sees X^ = X diag(1/lambda)
+and W^ = W diag(lambda), so X^ W^T = X W^T. lambda = 1 (smooth=None) is
+exactly the formula above. With smoothing the low-rank factors approximate
+W^T scaled by lambda, and L1 is stored with 1/lambda folded in, so the
+16-bit branch reads the raw X: X . L1 = X^ . (U_r S_r).
 
 Functions, in the order the method applies them:
+  smooth_factors    lambda from channel amaxima       (calibration)
   lowrank_factors   truncated SVD of W^T             (load time)
   residual          R = W - (L1 L2)^T                 (load time)
   pack_weight       NVFP4 of R, its global scale      (load time)
@@ -47,27 +54,58 @@ def to_f64(t) -> np.ndarray:
 
 
 # ------------------------------------------------------------------ load time
-def lowrank_factors(W, r: int):
+def smooth_factors(X, W, alpha: float = 0.5) -> np.ndarray:
+    """Per-input-channel smoothing factors (calibration), float32 [K]:
+    lambda_k = amax_m|X[m,k]|^alpha / amax_n|W[n,k]|^(1-alpha), in float64
+    and rounded once to fp32 (alpha = 0.5: sqrt(ax) / sqrt(aw), each step
+    correctly rounded); lambda_k = 1 where either amax is 0. The pages say
+    only that outliers move into the weights; this is SmoothQuant's rule
+    (Xiao et al. 2023), which balances the two channel ranges."""
+    ax = np.max(np.abs(to_f64(X)), axis=0)
+    aw = np.max(np.abs(to_f64(W)), axis=0)
+    lam = np.ones(ax.shape, dtype=np.float64)
+    ok = (ax > 0) & (aw > 0)
+    if alpha == 0.5:
+        lam[ok] = np.sqrt(ax[ok]) / np.sqrt(aw[ok])
+    else:
+        lam[ok] = ax[ok] ** alpha / aw[ok] ** (1.0 - alpha)
+    return lam.astype(np.float32)
+
+
+def inv_smooth(lam) -> np.ndarray:
+    """fp32(1 / lambda), the factor the activation quantiser applies."""
+    return (np.float32(1.0) / np.asarray(lam, dtype=np.float32)).astype(np.float32)
+
+
+def lowrank_factors(W, r: int, smooth=None):
     """Rank-r factors of W^T (K x N) from a float64 SVD.
 
     W^T = U diag(s) V^T; L1 = bf16(U_r diag(s_r)) (K x r), L2 = bf16(V_r^T)
     (r x N). The pages do not say how the singular values are split between
     the factors; any split is valid because everything downstream uses these
-    exact bf16 factors. Returns (L1, L2, s) with s all singular values (float64).
+    exact bf16 factors. With smoothing (lambda = smooth) the SVD is of
+    diag(lambda) W^T and L1 = bf16(diag(1/lambda) U_r diag(s_r)), the
+    division in float64. Returns (L1, L2, s) with s all singular values
+    (float64) of the matrix decomposed.
     """
     Wt = to_f64(W).T
+    if smooth is not None:
+        Wt = Wt * to_f64(smooth)[:, None]
     U, s, Vt = np.linalg.svd(Wt, full_matrices=False)
-    L1 = nvfp4.bf16_round(U[:, :r] * s[:r])
-    L2 = nvfp4.bf16_round(Vt[:r, :])
-    return L1, L2, s
+    L1 = U[:, :r] * s[:r]
+    if smooth is not None:
+        L1 = L1 / to_f64(smooth)[:, None]
+    return nvfp4.bf16_round(L1), nvfp4.bf16_round(Vt[:r, :]), s
 
 
-def residual(W, L1, L2) -> np.ndarray:
+def residual(W, L1, L2, smooth=None) -> np.ndarray:
     """R[n,k] = W[n,k] - sum_j L1[k,j] L2[j,n], float64, j ascending, then fp32 RN.
 
     Each product of two bf16 numbers is exact in float64; the running sum is
     rounded after each addition in the stated order, so the result is fully
-    determined.
+    determined. With smoothing the float64 difference is multiplied by
+    lambda_k (one more float64 rounding) before the fp32 rounding: the
+    residual of W^ = W diag(lambda) against the folded factors.
     """
     W = to_f64(W)
     L1 = to_f64(L1)
@@ -75,7 +113,10 @@ def residual(W, L1, L2) -> np.ndarray:
     s = np.zeros_like(W)
     for j in range(L1.shape[1]):
         s += np.outer(L2[j, :], L1[:, j])
-    return (W - s).astype(np.float32)
+    d = W - s
+    if smooth is not None:
+        d = d * to_f64(smooth)[None, :]
+    return d.astype(np.float32)
 
 
 @dataclass
@@ -85,24 +126,35 @@ class PackedWeight:
     g_w: np.float32      # global decode scale of R
     L1: np.ndarray       # float64 [K, r] (bf16 values)
     L2: np.ndarray       # float64 [r, N] (bf16 values)
+    inv_smooth: np.ndarray | None = None   # float32 [K] = fp32(1/lambda), or None
 
 
-def pack_weight(W, L1, L2) -> PackedWeight:
-    R = residual(W, L1, L2)
+def pack_weight(W, L1, L2, smooth=None) -> PackedWeight:
+    R = residual(W, L1, L2, smooth)
     g_w = nvfp4.global_scale(R)
     codes, scales = nvfp4.quantize_rows(R, g_w)
-    return PackedWeight(codes, scales, g_w, to_f64(L1), to_f64(L2))
+    inv = inv_smooth(smooth) if smooth is not None else None
+    return PackedWeight(codes, scales, g_w, to_f64(L1), to_f64(L2), inv)
 
 
 # ------------------------------------------------------------------ per call
-def act_global_scale(X) -> np.float32:
-    """Static (calibrated) activation decode scale, g_X = fp32(amax|X| / 2688)."""
-    return nvfp4.global_scale(to_f64(X).astype(np.float32))
+def smooth_act(X, inv=None) -> np.ndarray:
+    """X^ = fp32(fp32(x) * inv[k]) (one fp32 rounding), or fp32(X) without smoothing."""
+    x = to_f64(X).astype(np.float32)
+    if inv is None:
+        return x
+    return (x * np.asarray(inv, dtype=np.float32)[None, :]).astype(np.float32)
 
 
-def quantize_act(X, g_x):
-    """NVFP4 of the activation rows: (codes [M, K], scales [M, K/16])."""
-    return nvfp4.quantize_rows(to_f64(X).astype(np.float32), g_x)
+def act_global_scale(X, inv=None) -> np.float32:
+    """Activation decode scale, g_X = fp32(amax|X^| / 2688): static (calibrated
+    once) or computed every call (dynamic), the same formula."""
+    return nvfp4.global_scale(smooth_act(X, inv))
+
+
+def quantize_act(X, g_x, inv=None):
+    """NVFP4 of the (smoothed) activation rows: (codes [M, K], scales [M, K/16])."""
+    return nvfp4.quantize_rows(smooth_act(X, inv), g_x)
 
 
 def down_proj(X, L1) -> np.ndarray:
@@ -127,8 +179,9 @@ def gemm_4bit(codes_x, scales_x, codes_w, scales_w) -> np.ndarray:
 
 
 def forward(X, pw: PackedWeight, bias, g_x) -> Forward:
-    """Y = acc * g_X * g_W + XL1 . L2 + b, float64; y_ref = bf16(Y)."""
-    codes, scales = quantize_act(X, g_x)
+    """Y = acc * g_X * g_W + XL1 . L2 + b, float64; y_ref = bf16(Y). The 4-bit
+    branch quantises the smoothed X^ (pw.inv_smooth), the 16-bit branch reads X."""
+    codes, scales = quantize_act(X, g_x, pw.inv_smooth)
     xl1 = down_proj(X, pw.L1)
     acc = gemm_4bit(codes, scales, pw.codes, pw.scales)
     y = acc * float(g_x) * float(pw.g_w) + xl1 @ pw.L2
