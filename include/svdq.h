@@ -103,18 +103,41 @@ svdq_status svdq_forward_workspace_size(int M, int K, int r, size_t* bytes);
  * remaining residual is quantised to 4 bits.
  *   W   bf16 [N][K], L1 bf16 [K][r], L2 bf16 [r][N]   (L1.L2 is the rank-r
  *       factorisation of W^T)
+ *   smooth  device float [K] smoothing factors lambda (positive, finite), or
+ *       NULL for none (lambda = 1). With smoothing (same section: outliers
+ *       move from the activations into the weights) L1 must be the factor
+ *       with 1/lambda folded in (svdq_lowrank_init with the same smooth), and
+ *       the per-call functions must be given inv_smooth.
  *   g_x device float: the layer's calibrated (static) activation decode scale,
- *       e.g. from svdq_act_global_scale on calibration activations.
+ *       e.g. from svdq_act_global_scale on calibration activations (with the
+ *       same inv_smooth).
  *   Writes: w_codes [N][K/2], w_scales (tiled), gscale[4], l1t [r][K],
- *           l2s [2][N][r] (layouts above).
- * R[n,k] = W[n,k] - sum_j L1[k,j] L2[j,n] is formed in float64 (j ascending,
- * products exact) and rounded once to float32; g_w = fp32(amax|R| / 2688)
+ *           l2s [2][N][r] (layouts above), and with smoothing inv_smooth
+ *           [K] = fp32(1 / lambda) (16-byte aligned; NULL exactly when smooth
+ *           is NULL, SVDQ_ERR_INVALID_ARG otherwise; a lambda that is not a
+ *           positive finite number records SVDQ_ERR_INVALID_ARG in the device
+ *           error word).
+ * R[n,k] = lambda_k (W[n,k] - sum_j L1[k,j] L2[j,n]) is formed in float64
+ * (j ascending, products exact; the multiplication by lambda_k is one more
+ * float64 rounding) and rounded once to float32; g_w = fp32(amax|R| / 2688)
  * (1 if R == 0); then R is quantised with the NVFP4 rule of svdq_quantize_act.
  * Requires alpha = g_x g_w >= 2^-100 (so L2 / alpha stays finite in bf16).
  * The output buffers must not overlap the inputs. */
 svdq_status svdq_pack_weight(int N, int K, int r, const void* W, const void* L1, const void* L2,
-                             const float* g_x, void* w_codes, void* w_scales, float* gscale, void* l1t,
-                             void* l2s, void* stream);
+                             const float* smooth, const float* g_x, void* w_codes, void* w_scales,
+                             float* gscale, void* l1t, void* l2s, float* inv_smooth, void* stream);
+
+/* Smoothing calibration (load time): per input channel k,
+ *     lambda_k = amax_m|X[m,k]|^alpha / amax_n|W[n,k]|^(1 - alpha)
+ * in float64, clamped to [2^-32, 2^32], rounded once to fp32; lambda_k = 1
+ * where either amax is 0. The blog (section "Background: SVDQuant and
+ * Nunchaku") says outliers move from the activations into the weights but not
+ * how the factors are chosen; this is SmoothQuant's rule (Xiao et al. 2023).
+ * alpha = 0.5 is computed as sqrt(ax) / sqrt(aw), each step correctly rounded.
+ * X bf16 [M][ldx] (calibration activations), W bf16 [N][K]; alpha in [0, 1];
+ * lambda: device float [K]. */
+svdq_status svdq_smooth_factors(int M, int N, int K, const void* X, int64_t ldx, const void* W, float alpha,
+                                float* lambda, void* stream);
 
 /* The layer followed by FLUX's fused QKV post-processing (blog, section
  * "Quantizing models with structural rewrites": one fused operator takes the
@@ -135,7 +158,8 @@ svdq_status svdq_pack_weight(int N, int K, int r, const void* W, const void* L1,
  * epilogue (no extra pass over Y). */
 svdq_status svdq_linear_forward_qkv(int M, int N, int K, int r, const void* X, int64_t ldx,
                                     const void* w_codes, const void* w_scales, const float* gscale,
-                                    const void* l1t, const void* l2s, const void* bias, int heads,
+                                    const void* l1t, const void* l2s, const float* inv_smooth,
+                                    const void* bias, int heads,
                                     const void* norm_q_weight, const void* norm_k_weight, float eps,
                                     const float* rope_cos, const float* rope_sin, int64_t ld_rope,
                                     void* Y, int64_t ldy, void* workspace, size_t workspace_bytes,
@@ -160,30 +184,39 @@ svdq_status svdq_linear_forward_qkv(int M, int N, int K, int r, const void* X, i
  * satisfy the GEMM's rules). W, L1, L2 16-byte aligned, sigma 8-byte aligned,
  * workspace 256-byte aligned and at least svdq_lowrank_workspace_size bytes
  * (SVDQ_ERR_WORKSPACE otherwise); power_iters in [0, 64].
+ * With smoothing (smooth: device float [K] lambda, 16-byte aligned, or NULL)
+ * the matrix decomposed is diag(lambda) W^T and L1 = bf16(U_r S_r / lambda_k
+ * per row, in float64), so X . L1 = X^ . U_r S_r for X^ = X diag(1/lambda).
  * The blog does not say how the SVD is computed; this is the load-time step
  * that feeds svdq_pack_weight. */
 svdq_status svdq_lowrank_workspace_size(int N, int K, int r, size_t* bytes);
-svdq_status svdq_lowrank_init(int N, int K, int r, const void* W, void* L1, void* L2, double* sigma,
-                              unsigned long long seed, int power_iters, void* workspace, size_t ws_bytes,
-                              void* stream);
+svdq_status svdq_lowrank_init(int N, int K, int r, const void* W, const float* smooth, void* L1, void* L2,
+                              double* sigma, unsigned long long seed, int power_iters, void* workspace,
+                              size_t ws_bytes, void* stream);
 
-/* Calibrated (static) activation scale: *g_out = fp32(amax|X| / 2688), or 1
- * for an all-zero X. X bf16 [M][ldx]; g_out is a device float. */
-svdq_status svdq_act_global_scale(int M, int K, const void* X, int64_t ldx, float* g_out,
-                                  void* stream);
+/* Activation scale: *g_out = fp32(amax|X^| / 2688), or 1 for an all-zero X,
+ * with X^ = fp32(x * inv_smooth[k]) (inv_smooth: device float [K], 16-byte
+ * aligned, or NULL for X^ = X). X bf16 [M][ldx]; g_out is a device float.
+ * Run once on calibration activations it gives the static g_x. */
+svdq_status svdq_act_global_scale(int M, int K, const void* X, int64_t ldx, const float* inv_smooth,
+                                  float* g_out, void* stream);
 
 /* ------------------------------------------------------------ per call */
 /* Activation quantisation fused with the low-rank down projection (blog
  * figure caption in "Background: SVDQuant and Nunchaku": the down projection
  * is fused with the quantisation kernel). One pass over X [M][ldx] (bf16):
- *   per 16-element block: S = e4m3_rn_sat(amax / fp32(6 g_x)),
- *   sd = fp32(dec(S) g_x), code = e2m1_rn_sat(fp32(x * fp32(1/sd))) (0 if sd == 0);
- *   xl1 = bf16(X . L1) with fp32 accumulation (L1 given as l1t [r][K]).
- * g_x is a device float (gscale[0] of a packed layer).
+ *   x^ = fp32(x * inv_smooth[k]) with smoothing, else x;
+ *   per 16-element block of x^: S = e4m3_rn_sat(amax / fp32(6 g_x)),
+ *   sd = fp32(dec(S) g_x), code = e2m1_rn_sat(fp32(x^ * fp32(1/sd))) (0 if sd == 0);
+ *   xl1 = bf16(X . L1) of the raw X, with fp32 accumulation (L1 given as
+ *   l1t [r][K]; with smoothing it carries 1/lambda).
+ * g_x is a device float (gscale[0] of a packed layer); inv_smooth is the
+ * packed layer's [K] floats (16-byte aligned) or NULL.
  * Writes codes [M][K/2], scales (tiled, rows padded to 128; padding rows are
  * written as zero scales), xl1 [M][r]. Deterministic. */
 svdq_status svdq_quantize_act(int M, int K, int r, const void* X, int64_t ldx, const float* g_x,
-                              const void* l1t, void* codes, void* scales, void* xl1, void* stream);
+                              const void* l1t, const float* inv_smooth, void* codes, void* scales, void* xl1,
+                              void* stream);
 
 /* The block-scaled FP4 GEMM with the low-rank up projection and bias fused in
  * its epilogue (blog figure caption: the up projection is fused with the 4-bit
@@ -197,14 +230,14 @@ svdq_status svdq_w4a4_gemm(int M, int N, int K, int r, const void* a_codes, cons
                            const void* xl1, const void* w_codes, const void* w_scales, const float* gscale,
                            const void* l2s, const void* bias, void* Y, int64_t ldy, void* stream);
 
-/* The whole layer: svdq_quantize_act (with g_x = gscale[0]) into `workspace`,
- * then svdq_w4a4_gemm.
+/* The whole layer: svdq_quantize_act (with g_x = gscale[0] and inv_smooth)
+ * into `workspace`, then svdq_w4a4_gemm.
  * workspace_bytes must be >= svdq_forward_workspace_size(M, K, r). */
 svdq_status svdq_linear_forward(int M, int N, int K, int r, const void* X, int64_t ldx,
                                 const void* w_codes, const void* w_scales, const float* gscale,
-                                const void* l1t, const void* l2s, const void* bias, void* Y,
-                                int64_t ldy, void* workspace, size_t workspace_bytes,
-                                void* stream);
+                                const void* l1t, const void* l2s, const float* inv_smooth,
+                                const void* bias, void* Y, int64_t ldy, void* workspace,
+                                size_t workspace_bytes, void* stream);
 
 /* Same computation as svdq_linear_forward, for callers that cannot supply a
  * workspace: plugin interfaces of inference runtimes that pass only a layer's
@@ -226,8 +259,8 @@ svdq_status svdq_linear_forward(int M, int N, int K, int r, const void* X, int64
  * Arguments, layouts and errors otherwise as svdq_linear_forward. */
 svdq_status svdq_linear_forward_noalloc(int M, int N, int K, int r, const void* X, int64_t ldx,
                                         const void* w_codes, const void* w_scales, const float* gscale,
-                                        const void* l1t, const void* l2s, const void* bias, void* Y,
-                                        int64_t ldy, void* stream);
+                                        const void* l1t, const void* l2s, const float* inv_smooth,
+                                        const void* bias, void* Y, int64_t ldy, void* stream);
 
 /* ------------------------------------------------------------ errors */
 /* Reads (and, if clear != 0, resets) the device error word of the current

@@ -56,11 +56,13 @@ def to_f64(t) -> np.ndarray:
 # ------------------------------------------------------------------ load time
 def smooth_factors(X, W, alpha: float = 0.5) -> np.ndarray:
     """Per-input-channel smoothing factors (calibration), float32 [K]:
-    lambda_k = amax_m|X[m,k]|^alpha / amax_n|W[n,k]|^(1-alpha), in float64
-    and rounded once to fp32 (alpha = 0.5: sqrt(ax) / sqrt(aw), each step
-    correctly rounded); lambda_k = 1 where either amax is 0. The pages say
-    only that outliers move into the weights; this is SmoothQuant's rule
-    (Xiao et al. 2023), which balances the two channel ranges."""
+    lambda_k = amax_m|X[m,k]|^alpha / amax_n|W[n,k]|^(1-alpha), in float64,
+    clamped to [2^-32, 2^32] and rounded once to fp32 (alpha = 0.5:
+    sqrt(ax) / sqrt(aw), each step correctly rounded); lambda_k = 1 where
+    either amax is 0. alpha is taken as an fp32 value. The pages say only that
+    outliers move into the weights; this is SmoothQuant's rule (Xiao et al.
+    2023), which balances the two channel ranges."""
+    alpha = float(np.float32(alpha))
     ax = np.max(np.abs(to_f64(X)), axis=0)
     aw = np.max(np.abs(to_f64(W)), axis=0)
     lam = np.ones(ax.shape, dtype=np.float64)
@@ -69,6 +71,7 @@ def smooth_factors(X, W, alpha: float = 0.5) -> np.ndarray:
         lam[ok] = np.sqrt(ax[ok]) / np.sqrt(aw[ok])
     else:
         lam[ok] = ax[ok] ** alpha / aw[ok] ** (1.0 - alpha)
+    lam[ok] = np.clip(lam[ok], 2.0 ** -32, 2.0 ** 32)
     return lam.astype(np.float32)
 
 

@@ -79,15 +79,16 @@ def test_validation_happens_before_device_checks(L):
     p = ctypes.c_void_p(0x10000)          # never dereferenced: validation fails first
     odd = ctypes.c_void_p(0x10008)
     # bad K
-    assert L.svdq_quantize_act(4, 100, 32, p, 100, p, p, p, p, p, None) == 2
+    assert L.svdq_quantize_act(4, 100, 32, p, 100, p, p, None, p, p, p, None) == 2
     # null pointer
-    assert L.svdq_quantize_act(4, 256, 32, None, 256, p, p, p, p, p, None) == 1
+    assert L.svdq_quantize_act(4, 256, 32, None, 256, p, p, None, p, p, p, None) == 1
     # misaligned pointer
-    assert L.svdq_quantize_act(4, 256, 32, odd, 256, p, p, p, p, p, None) == 3
+    assert L.svdq_quantize_act(4, 256, 32, odd, 256, p, p, None, p, p, p, None) == 3
+    assert L.svdq_quantize_act(4, 256, 32, p, 256, p, p, ctypes.c_void_p(0x10004), p, p, p, None) == 3  # inv_smooth
     # bad leading dimension
     assert L.svdq_w4a4_gemm(4, 128, 256, 32, p, p, p, p, p, p, p, None, p, 100, None) == 2
     # workspace too small
-    assert L.svdq_linear_forward(4, 128, 256, 32, p, 256, p, p, p, p, p, None, p, 128, p, 16, None) == 7
+    assert L.svdq_linear_forward(4, 128, 256, 32, p, 256, p, p, p, p, p, None, None, p, 128, p, 16, None) == 7
     # M == 0 is a valid no-op
     assert L.svdq_w4a4_gemm(0, 128, 256, 32, None, None, None, None, None, None, None, None, None, 128,
                             None) == 0
@@ -104,12 +105,29 @@ def test_lowrank_sizes_and_validation(L):
     assert L.svdq_lowrank_workspace_size(16, 256, 32, ctypes.byref(out)) == 2     # r > min(N, K)
     big = ctypes.c_size_t(1 << 40)
     # rank, then shape, then alignment, then workspace size, all before any device check
-    assert L.svdq_lowrank_init(128, 256, 24, p, p, p, None, 0, 4, p, big, None) == 1
-    assert L.svdq_lowrank_init(128, 256, 32, p, p, p, None, 0, 65, p, big, None) == 1   # power_iters
-    assert L.svdq_lowrank_init(128, 252, 32, p, p, p, None, 0, 4, p, big, None) == 2    # K % 8
-    assert L.svdq_lowrank_init(128, 256, 32, odd, p, p, None, 0, 4, p, big, None) == 3
-    assert L.svdq_lowrank_init(128, 256, 32, p, p, p, ctypes.c_void_p(0x10004), 0, 4, p, big, None) == 3
-    assert L.svdq_lowrank_init(128, 256, 32, p, p, p, None, 0, 4, p, ctypes.c_size_t(16), None) == 7
+    assert L.svdq_lowrank_init(128, 256, 24, p, None, p, p, None, 0, 4, p, big, None) == 1
+    assert L.svdq_lowrank_init(128, 256, 32, p, None, p, p, None, 0, 65, p, big, None) == 1   # power_iters
+    assert L.svdq_lowrank_init(128, 252, 32, p, None, p, p, None, 0, 4, p, big, None) == 2    # K % 8
+    assert L.svdq_lowrank_init(128, 256, 32, odd, None, p, p, None, 0, 4, p, big, None) == 3
+    assert L.svdq_lowrank_init(128, 256, 32, p, None, p, p, ctypes.c_void_p(0x10004), 0, 4, p, big, None) == 3
+    assert L.svdq_lowrank_init(128, 256, 32, p, odd, p, p, None, 0, 4, p, big, None) == 3     # smooth
+    assert L.svdq_lowrank_init(128, 256, 32, p, None, p, p, None, 0, 4, p, ctypes.c_size_t(16), None) == 7
+
+
+def test_smoothing_validation(L):
+    p = ctypes.c_void_p(0x10000)
+    odd = ctypes.c_void_p(0x10008)
+    f = ctypes.c_float
+    # smooth and inv_smooth come together
+    assert L.svdq_pack_weight(128, 256, 32, p, p, p, p, p, p, p, p, p, p, None, None) == 1
+    assert L.svdq_pack_weight(128, 256, 32, p, p, p, None, p, p, p, p, p, p, p, None) == 1
+    assert L.svdq_pack_weight(128, 256, 32, p, p, p, odd, p, p, p, p, p, p, p, None) == 3
+    # calibration: alpha in [0, 1], K % 8, alignment
+    assert L.svdq_smooth_factors(4, 128, 256, p, 256, p, f(1.5), p, None) == 1
+    assert L.svdq_smooth_factors(4, 128, 256, p, 256, p, f(-0.1), p, None) == 1
+    assert L.svdq_smooth_factors(4, 128, 252, p, 256, p, f(0.5), p, None) == 2
+    assert L.svdq_smooth_factors(4, 128, 256, odd, 256, p, f(0.5), p, None) == 3
+    assert L.svdq_act_global_scale(4, 256, p, 256, odd, p, None) == 3
 
 
 def test_qkv_forward_validation(L):
@@ -117,8 +135,8 @@ def test_qkv_forward_validation(L):
     odd = ctypes.c_void_p(0x10008)
     f = ctypes.c_float
     ws = ctypes.c_size_t(1 << 40)
-    args = lambda N, heads, eps, cs, ld: (4, N, 256, 32, p, 256, p, p, p, p, p, None, heads, p, p, f(eps), cs, p, ld,
-                                          p, N, p, ws, None)
+    args = lambda N, heads, eps, cs, ld: (4, N, 256, 32, p, 256, p, p, p, p, p, None, None, heads, p, p, f(eps), cs,
+                                          p, ld, p, N, p, ws, None)
     assert L.svdq_linear_forward_qkv(*args(768, 2, 1e-6, p, 128)) in (0, 4)     # valid (no GPU here: 4)
     assert L.svdq_linear_forward_qkv(*args(768, 1, 1e-6, p, 128)) == 2          # N != 3 * heads * 128
     assert L.svdq_linear_forward_qkv(*args(768, 2, -1.0, p, 128)) == 1          # eps < 0
@@ -132,9 +150,10 @@ def test_qkv_forward_validation(L):
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU path")
 def test_no_gpu_is_unsupported_device(L):
     p = ctypes.c_void_p(0x10000)
-    assert L.svdq_quantize_act(4, 256, 32, p, 256, p, p, p, p, p, None) == 4
-    assert L.svdq_pack_weight(128, 256, 32, p, p, p, p, p, p, p, p, p, None) == 4
-    assert L.svdq_lowrank_init(128, 256, 32, p, p, p, None, 0, 4, p, ctypes.c_size_t(1 << 40), None) == 4
+    assert L.svdq_quantize_act(4, 256, 32, p, 256, p, p, None, p, p, p, None) == 4
+    assert L.svdq_pack_weight(128, 256, 32, p, p, p, None, p, p, p, p, p, p, None, None) == 4
+    assert L.svdq_lowrank_init(128, 256, 32, p, None, p, p, None, 0, 4, p, ctypes.c_size_t(1 << 40), None) == 4
+    assert L.svdq_smooth_factors(4, 128, 256, p, 256, p, ctypes.c_float(0.5), p, None) == 4
     code = ctypes.c_int()
     assert L.svdq_read_device_error(ctypes.byref(code), 0) == 4
 

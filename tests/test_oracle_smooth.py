@@ -80,6 +80,12 @@ def test_calibration_closed_forms():
     assert np.allclose((ax / svdq.smooth_factors(X, W, 1.0))[ok], 1.0, rtol=1e-6, atol=0)
     assert np.allclose((aw * svdq.smooth_factors(X, W, 0.0))[ok], 1.0, rtol=1e-6, atol=0)
     assert svdq.smooth_factors(X, W).dtype == np.float32
+    # the factors are clamped to [2^-32, 2^32]: an extreme channel ratio of 2^160 saturates
+    Xe, We = X.copy(), W.copy()
+    Xe[:, 0], We[:, 0] = 2.0 ** 80, 2.0 ** -80
+    Xe[:, 1], We[:, 1] = 2.0 ** -80, 2.0 ** 80
+    le = svdq.smooth_factors(Xe, We)
+    assert le[0] == np.float32(2.0 ** 32) and le[1] == np.float32(2.0 ** -32)
 
 
 def test_smoothed_factors_satisfy_eckart_young_on_the_smoothed_weight():

@@ -35,8 +35,8 @@ def _noalloc(L, X, pw, bias, Y):
     M, K = X.shape
     stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
     return L.svdq_linear_forward_noalloc(M, pw.N, K, pw.r, _p(X), X.stride(0), _p(pw.codes), _p(pw.scales),
-                                         _p(pw.gscale), _p(pw.l1t), _p(pw.l2s), _p(bias), _p(Y), Y.stride(0),
-                                         stream)
+                                         _p(pw.gscale), _p(pw.l1t), _p(pw.l2s), _p(pw.inv_smooth), _p(bias), _p(Y),
+                                         Y.stride(0), stream)
 
 
 @pytest.mark.parametrize("M,K,N,r", [(256, 1024, 1024, 32), (333, 768, 384, 64)])
@@ -67,4 +67,4 @@ def test_noalloc_rejects_shapes_beyond_the_scratch_limit(lib):
     p = ctypes.c_void_p(0x10000)             # never dereferenced: the size check fails first
     M, K, N, r = 18432, 3072, 128, 32        # workspace about 33 MB > 16 MiB
     assert lib.svdq_forward_workspace_size(M, K, r) > (16 << 20)
-    assert L.svdq_linear_forward_noalloc(M, N, K, r, p, K, p, p, p, p, p, None, p, N, None) == 7
+    assert L.svdq_linear_forward_noalloc(M, N, K, r, p, K, p, p, p, p, p, None, None, p, N, None) == 7

@@ -31,17 +31,18 @@ SIGNATURES = {
     "svdq_weight_sizes": (_i, [_i, _i, _i, _psz, _psz, _psz, _psz]),
     "svdq_act_sizes": (_i, [_i, _i, _i, _psz, _psz, _psz]),
     "svdq_forward_workspace_size": (_i, [_i, _i, _i, _psz]),
-    "svdq_pack_weight": (_i, [_i, _i, _i, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p]),
-    "svdq_act_global_scale": (_i, [_i, _i, _p, _i64, _p, _p]),
-    "svdq_quantize_act": (_i, [_i, _i, _i, _p, _i64, _p, _p, _p, _p, _p, _p]),
+    "svdq_pack_weight": (_i, [_i, _i, _i, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p]),
+    "svdq_smooth_factors": (_i, [_i, _i, _i, _p, _i64, _p, _f, _p, _p]),
+    "svdq_act_global_scale": (_i, [_i, _i, _p, _i64, _p, _p, _p]),
+    "svdq_quantize_act": (_i, [_i, _i, _i, _p, _i64, _p, _p, _p, _p, _p, _p, _p]),
     "svdq_w4a4_gemm": (_i, [_i, _i, _i, _i, _p, _p, _p, _p, _p, _p, _p, _p, _p, _i64, _p]),
-    "svdq_linear_forward": (_i, [_i, _i, _i, _i, _p, _i64, _p, _p, _p, _p, _p, _p, _p, _i64, _p, _sz, _p]),
+    "svdq_linear_forward": (_i, [_i, _i, _i, _i, _p, _i64, _p, _p, _p, _p, _p, _p, _p, _p, _i64, _p, _sz, _p]),
     "svdq_read_device_error": (_i, [_pi, _i]),
-    "svdq_linear_forward_noalloc": (_i, [_i, _i, _i, _i, _p, _i64, _p, _p, _p, _p, _p, _p, _p, _i64, _p]),
-    "svdq_linear_forward_qkv": (_i, [_i, _i, _i, _i, _p, _i64, _p, _p, _p, _p, _p, _p, _i, _p, _p, _f, _p, _p,
-                                     _i64, _p, _i64, _p, _sz, _p]),
+    "svdq_linear_forward_noalloc": (_i, [_i, _i, _i, _i, _p, _i64, _p, _p, _p, _p, _p, _p, _p, _p, _i64, _p]),
+    "svdq_linear_forward_qkv": (_i, [_i, _i, _i, _i, _p, _i64, _p, _p, _p, _p, _p, _p, _p, _i, _p, _p, _f, _p,
+                                     _p, _i64, _p, _i64, _p, _sz, _p]),
     "svdq_lowrank_workspace_size": (_i, [_i, _i, _i, _psz]),
-    "svdq_lowrank_init": (_i, [_i, _i, _i, _p, _p, _p, _p, ctypes.c_ulonglong, _i, _p, _sz, _p]),
+    "svdq_lowrank_init": (_i, [_i, _i, _i, _p, _p, _p, _p, _p, ctypes.c_ulonglong, _i, _p, _sz, _p]),
 }
 
 
@@ -131,14 +132,24 @@ def svdq_lowrank_workspace_size(N: int, K: int, r: int) -> int:
     return out.value
 
 
+def _smooth_vec(t: torch.Tensor | None, K: int, name: str):
+    if t is not None:
+        _dev(t, name, torch.float32, (K,))
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    return t
+
+
 def svdq_lowrank_init(W: torch.Tensor, r: int, seed: int = 0, power_iters: int = 32,
-                      workspace: torch.Tensor | None = None):
-    """Rank-r factors of the 16-bit branch from a truncated SVD of W^T on the GPU:
+                      workspace: torch.Tensor | None = None, smooth: torch.Tensor | None = None):
+    """Rank-r factors of the 16-bit branch from a truncated SVD of W^T on the GPU
+    (of diag(smooth) W^T with L1 carrying 1/smooth when smoothing):
     returns (L1 [K, r] bf16, L2 [r, N] bf16, sigma [r] float64)."""
     _dev(W, "W", torch.bfloat16)
     if not W.is_contiguous():
         raise ValueError("W must be contiguous")
     N, K = W.shape
+    _smooth_vec(smooth, K, "smooth")
     need = svdq_lowrank_workspace_size(N, K, r)
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=W.device)
@@ -146,7 +157,7 @@ def svdq_lowrank_init(W: torch.Tensor, r: int, seed: int = 0, power_iters: int =
     L2 = torch.empty((r, N), dtype=torch.bfloat16, device=W.device)
     sigma = torch.empty(r, dtype=torch.float64, device=W.device)
     _check("svdq_lowrank_init", lib().svdq_lowrank_init(
-        N, K, r, _ptr(W), _ptr(L1), _ptr(L2), _ptr(sigma), seed, power_iters, _ptr(workspace),
+        N, K, r, _ptr(W), _ptr(smooth), _ptr(L1), _ptr(L2), _ptr(sigma), seed, power_iters, _ptr(workspace),
         workspace.numel() * workspace.element_size(), _stream(W)))
     return L1, L2, sigma
 
@@ -155,7 +166,8 @@ def svdq_lowrank_init(W: torch.Tensor, r: int, seed: int = 0, power_iters: int =
 class PackedWeight:
     """Device buffers of one packed layer (allocated by torch, filled by svdq_pack_weight).
 
-    gscale = [g_x, g_w, g_x*g_w, 0]; l2s = [2, N, r] bf16 hi / lo parts of L2^T / (g_x g_w)."""
+    gscale = [g_x, g_w, g_x*g_w, 0]; l2s = [2, N, r] bf16 hi / lo parts of L2^T / (g_x g_w);
+    inv_smooth = fp32(1 / lambda) [K] of a smoothed layer, else None."""
 
     def __init__(self, N: int, K: int, r: int, device):
         cb, sb, lb1, lb2 = svdq_weight_sizes(N, K, r)
@@ -165,6 +177,7 @@ class PackedWeight:
         self.gscale = torch.empty(4, dtype=torch.float32, device=device)
         self.l1t = torch.empty((r, K), dtype=torch.bfloat16, device=device)
         self.l2s = torch.empty((2, N, r), dtype=torch.bfloat16, device=device)
+        self.inv_smooth = None
 
     @property
     def g_x(self) -> torch.Tensor:
@@ -175,9 +188,12 @@ class PackedWeight:
         return self.gscale[1:2]
 
 
-def svdq_pack_weight(W: torch.Tensor, L1: torch.Tensor, L2: torch.Tensor, g_x, out: PackedWeight | None = None):
+def svdq_pack_weight(W: torch.Tensor, L1: torch.Tensor, L2: torch.Tensor, g_x, out: PackedWeight | None = None,
+                     smooth: torch.Tensor | None = None):
     """Pack one layer. g_x: the calibrated activation scale, a CUDA float32 tensor of
-    one element (e.g. from svdq_act_global_scale) or a Python float."""
+    one element (e.g. from svdq_act_global_scale) or a Python float. smooth: the
+    smoothing factors lambda [K] float32 (L1 then from svdq_lowrank_init with the
+    same smooth), or None."""
     N, K = W.shape
     r = L1.shape[1]
     _dev(W, "W", torch.bfloat16)
@@ -189,19 +205,41 @@ def svdq_pack_weight(W: torch.Tensor, L1: torch.Tensor, L2: torch.Tensor, g_x, o
     if not isinstance(g_x, torch.Tensor):
         g_x = torch.tensor([float(g_x)], dtype=torch.float32, device=W.device)
     _dev(g_x, "g_x", torch.float32)
+    _smooth_vec(smooth, K, "smooth")
     pw = out if out is not None else PackedWeight(N, K, r, W.device)
+    pw.inv_smooth = None if smooth is None else torch.empty(K, dtype=torch.float32, device=W.device)
     _check("svdq_pack_weight", lib().svdq_pack_weight(
-        N, K, r, _ptr(W), _ptr(L1), _ptr(L2), _ptr(g_x), _ptr(pw.codes), _ptr(pw.scales), _ptr(pw.gscale),
-        _ptr(pw.l1t), _ptr(pw.l2s), _stream(W)))
+        N, K, r, _ptr(W), _ptr(L1), _ptr(L2), _ptr(smooth), _ptr(g_x), _ptr(pw.codes), _ptr(pw.scales),
+        _ptr(pw.gscale), _ptr(pw.l1t), _ptr(pw.l2s), _ptr(pw.inv_smooth), _stream(W)))
     return pw
 
 
-def svdq_act_global_scale(X: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
+def svdq_smooth_factors(X: torch.Tensor, W: torch.Tensor, alpha: float = 0.5,
+                        out: torch.Tensor | None = None) -> torch.Tensor:
+    """Smoothing factors lambda [K] (float32) from calibration activations X [M, K]
+    and the weight W [N, K]."""
+    _dev(X, "X", torch.bfloat16)
+    _dev(W, "W", torch.bfloat16)
+    M, K = X.shape
+    ldx = _rows(X, "X", K)
+    if W.dim() != 2 or W.shape[1] != K or not W.is_contiguous():
+        raise ValueError("W must be contiguous [N, K]")
+    lam = out if out is not None else torch.empty(K, dtype=torch.float32, device=X.device)
+    _check("svdq_smooth_factors", lib().svdq_smooth_factors(M, W.shape[0], K, _ptr(X), ldx, _ptr(W), float(alpha),
+                                                            _ptr(lam), _stream(X)))
+    return lam
+
+
+def svdq_act_global_scale(X: torch.Tensor, out: torch.Tensor | None = None,
+                          inv_smooth: torch.Tensor | None = None) -> torch.Tensor:
+    """fp32(amax|X^| / 2688) with X^ = X * inv_smooth (or X), on the device."""
     _dev(X, "X", torch.bfloat16)
     M, K = X.shape
     ldx = _rows(X, "X", K)
+    _smooth_vec(inv_smooth, K, "inv_smooth")
     g = out if out is not None else torch.empty(1, dtype=torch.float32, device=X.device)
-    _check("svdq_act_global_scale", lib().svdq_act_global_scale(M, K, _ptr(X), ldx, _ptr(g), _stream(X)))
+    _check("svdq_act_global_scale", lib().svdq_act_global_scale(M, K, _ptr(X), ldx, _ptr(inv_smooth), _ptr(g),
+                                                                _stream(X)))
     return g
 
 
@@ -222,8 +260,8 @@ def svdq_quantize_act(X: torch.Tensor, pw: PackedWeight, out: QuantAct | None = 
     ldx = _rows(X, "X", K)
     qa = out if out is not None else QuantAct(M, K, pw.r, X.device)
     _check("svdq_quantize_act", lib().svdq_quantize_act(
-        M, K, pw.r, _ptr(X), ldx, _ptr(pw.gscale), _ptr(pw.l1t), _ptr(qa.codes), _ptr(qa.scales), _ptr(qa.xl1),
-        _stream(X)))
+        M, K, pw.r, _ptr(X), ldx, _ptr(pw.gscale), _ptr(pw.l1t), _ptr(pw.inv_smooth), _ptr(qa.codes),
+        _ptr(qa.scales), _ptr(qa.xl1), _stream(X)))
     return qa
 
 
@@ -256,7 +294,7 @@ def svdq_linear_forward(X: torch.Tensor, pw: PackedWeight, bias: torch.Tensor | 
     ws = workspace if workspace is not None else torch.empty(max(need, 16), dtype=torch.uint8, device=X.device)
     _check("svdq_linear_forward", lib().svdq_linear_forward(
         M, N, K, r, _ptr(X), ldx, _ptr(pw.codes), _ptr(pw.scales), _ptr(pw.gscale), _ptr(pw.l1t),
-        _ptr(pw.l2s), _ptr(bias), _ptr(Y), ldy, _ptr(ws), ws.numel(), _stream(X)))
+        _ptr(pw.l2s), _ptr(pw.inv_smooth), _ptr(bias), _ptr(Y), ldy, _ptr(ws), ws.numel(), _stream(X)))
     return Y
 
 
@@ -287,7 +325,7 @@ def svdq_linear_forward_qkv(X: torch.Tensor, pw: PackedWeight, bias: torch.Tenso
         workspace = torch.empty(max(1, svdq_forward_workspace_size(M, K, pw.r)), dtype=torch.uint8, device=X.device)
     _check("svdq_linear_forward_qkv", lib().svdq_linear_forward_qkv(
         M, N, K, pw.r, _ptr(X), ldx, _ptr(pw.codes), _ptr(pw.scales), _ptr(pw.gscale), _ptr(pw.l1t), _ptr(pw.l2s),
-        _ptr(bias), heads, _ptr(norm_q_weight), _ptr(norm_k_weight), float(eps), _ptr(rope_cos), _ptr(rope_sin),
+        _ptr(pw.inv_smooth), _ptr(bias), heads, _ptr(norm_q_weight), _ptr(norm_k_weight), float(eps), _ptr(rope_cos), _ptr(rope_sin),
         rope_cos.stride(0), _ptr(Y), ldy, _ptr(workspace), workspace.numel(), _stream(X)))
     return Y
 

@@ -70,13 +70,16 @@ __device__ __forceinline__ double to_f64(__nv_bfloat16 x) { return static_cast<d
 // Partial products over one slice of the long dimension L:
 //   TRANS_A = false: C[m][j] = sum_l A[m][l] B[l][j]   (A: M x L, row-major, lda)
 //   TRANS_A = true:  C[m][j] = sum_l A[l][m] B[l][j]   (A: L x M, row-major, lda)
-// B: L x P float64 (ldb = P). Grid (ceil(M / 32), splits); split s covers
+// B: L x P float64 (ldb = P). colscale (or nullptr) multiplies each element
+// of the row-major A by the factor of its column: A[.][c] * colscale[c] (the
+// smoothing of W's input channels). Grid (ceil(M / 32), splits); split s covers
 // l in [s*lchunk, min(L, (s+1)*lchunk)) in ascending order and writes
 // part[s][m][j]. P <= kSvdMaxP and a multiple of 16; dynamic shared memory
 // holds the B slice (kTsL x P doubles).
 template <bool TRANS_A, typename TA>
 __global__ void __launch_bounds__(kTsThreads) ts_gemm_kernel(int M, int L, int P, const TA* __restrict__ A,
-                                                            int64_t lda, const double* __restrict__ B,
+                                                            int64_t lda, const float* __restrict__ colscale,
+                                                            const double* __restrict__ B,
                                                             double* __restrict__ part, int lchunk) {
   __shared__ double a_s[kTsL][kTsRows + 1];
   extern __shared__ double ts_dyn[];
@@ -98,9 +101,11 @@ __global__ void __launch_bounds__(kTsThreads) ts_gemm_kernel(int M, int L, int P
       const int li = TRANS_A ? i / kTsRows : i % kTsL;
       const int mi = TRANS_A ? i % kTsRows : i / kTsL;
       double v = 0.0;
-      if (li < lt && m0 + mi < M)
+      if (li < lt && m0 + mi < M) {
         v = TRANS_A ? to_f64(A[static_cast<int64_t>(l0 + li) * lda + m0 + mi])
                     : to_f64(A[static_cast<int64_t>(m0 + mi) * lda + l0 + li]);
+        if (colscale != nullptr) v *= static_cast<double>(colscale[TRANS_A ? m0 + mi : l0 + li]);
+      }
       a_s[li][mi] = v;
     }
     for (int i = threadIdx.x; i < kTsL * P; i += kTsThreads) {
@@ -334,14 +339,16 @@ __global__ void svd_coeff_kernel(const double* __restrict__ lam, const double* _
     if (sigma_out != nullptr) sigma_out[i] = sig[i];
 }
 
-// bf16 outputs: L1[k][i] = bf16(U1[k][i]) (K x r) and L2[i][n] = bf16(V2[n][i]) (r x N).
+// bf16 outputs: L1[k][i] = bf16(U1[k][i] / lambda_k) (K x r; the division in
+// float64, none when smooth is nullptr) and L2[i][n] = bf16(V2[n][i]) (r x N).
 __global__ void svd_store_kernel(const double* __restrict__ U1, int K, const double* __restrict__ V2, int N, int r,
-                                 __nv_bfloat16* __restrict__ L1, __nv_bfloat16* __restrict__ L2) {
+                                 const float* __restrict__ smooth, __nv_bfloat16* __restrict__ L1,
+                                 __nv_bfloat16* __restrict__ L2) {
   const int64_t n1 = static_cast<int64_t>(K) * r, n2 = static_cast<int64_t>(N) * r;
   for (int64_t t = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; t < n1 + n2;
        t += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     if (t < n1) {
-      L1[t] = __double2bfloat16(U1[t]);
+      L1[t] = __double2bfloat16(smooth != nullptr ? U1[t] / static_cast<double>(smooth[t / r]) : U1[t]);
     } else {
       const int64_t u = t - n1;  // output index in L2 (r x N)
       const int64_t i = u / N, n = u % N;

@@ -9,7 +9,10 @@
 // is formed in float64 with j ascending (each bf16 x bf16 product is exact in
 // float64, so a fused multiply-add gives the same value) and rounded once to
 // float32; g_w = fp32(amax|R| / 2688) (1 if R == 0); R is then quantised with
-// the same NVFP4 rule as the activations, blocks of 16 along K.
+// the same NVFP4 rule as the activations, blocks of 16 along K. With smoothing
+// (outliers moved into the weights, same section) the float64 difference is
+// multiplied by lambda_k before the fp32 rounding: the residual of
+// W diag(lambda) against factors whose L1 carries 1/lambda.
 //
 // Work split: a warp owns 32 consecutive K-columns (two 16-element blocks) and
 // walks `rows_per_warp` rows n; each lane keeps its column's L1 row in
@@ -42,7 +45,8 @@ __global__ void transpose_bf16_kernel(const __nv_bfloat16* __restrict__ in, __nv
 
 template <int R>
 __device__ __forceinline__ float residual_at(const __nv_bfloat16* __restrict__ W, const float (&l1row)[R],
-                                             const __nv_bfloat16* __restrict__ l2t, int N, int K, int n, int k) {
+                                             const __nv_bfloat16* __restrict__ l2t, int N, int K, int n, int k,
+                                             double lam) {
   double s = 0.0;
   const __nv_bfloat16* l2 = l2t + static_cast<int64_t>(n) * R;
 #pragma unroll
@@ -54,7 +58,7 @@ __device__ __forceinline__ float residual_at(const __nv_bfloat16* __restrict__ W
     for (int i = 0; i < 8; ++i) s = __dadd_rn(s, __dmul_rn(static_cast<double>(l1row[j8 + i]), static_cast<double>(f[i])));
   }
   const double w = static_cast<double>(__bfloat162float(W[static_cast<int64_t>(n) * K + k]));
-  return __double2float_rn(__dsub_rn(w, s));
+  return __double2float_rn(__dmul_rn(__dsub_rn(w, s), lam));
 }
 
 template <int R>
@@ -75,7 +79,8 @@ template <int R>
 __global__ void __launch_bounds__(kPackThreads) residual_amax_kernel(const __nv_bfloat16* __restrict__ W,
                                                                       const __nv_bfloat16* __restrict__ L1,
                                                                       const __nv_bfloat16* __restrict__ l2t,
-                                                                      int N, int K, unsigned* amax_bits) {
+                                                                      const float* __restrict__ smooth, int N,
+                                                                      int K, unsigned* amax_bits) {
   const int lane = threadIdx.x & 31;
   const int gw = blockIdx.x * (kPackThreads / 32) + (threadIdx.x >> 5);
   const int slabs = K / 32;
@@ -85,9 +90,10 @@ __global__ void __launch_bounds__(kPackThreads) residual_amax_kernel(const __nv_
   const int k = slab * 32 + lane;
   float l1row[R];
   load_l1_row<R>(L1, k, l1row);
+  const double lam = smooth != nullptr ? static_cast<double>(smooth[k]) : 1.0;
   float am = 0.0f;
   const int n_end = min(N, n_begin + kPackRowsPerWarp);
-  for (int n = n_begin; n < n_end; ++n) am = fmaxf(am, fabsf(residual_at<R>(W, l1row, l2t, N, K, n, k)));
+  for (int n = n_begin; n < n_end; ++n) am = fmaxf(am, fabsf(residual_at<R>(W, l1row, l2t, N, K, n, k, lam)));
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
   if (lane == 0) atomicMax(amax_bits, __float_as_uint(am));
@@ -131,8 +137,8 @@ __global__ void make_l2s_kernel(const __nv_bfloat16* __restrict__ L2, const floa
 template <int R>
 __global__ void __launch_bounds__(kPackThreads) residual_quant_kernel(
     const __nv_bfloat16* __restrict__ W, const __nv_bfloat16* __restrict__ L1,
-    const __nv_bfloat16* __restrict__ l2t, int N, int K, const float* __restrict__ gscale,
-    uint8_t* __restrict__ codes, uint8_t* __restrict__ scales) {
+    const __nv_bfloat16* __restrict__ l2t, const float* __restrict__ smooth, int N, int K,
+    const float* __restrict__ gscale, uint8_t* __restrict__ codes, uint8_t* __restrict__ scales) {
   const int lane = threadIdx.x & 31;
   const int gw = blockIdx.x * (kPackThreads / 32) + (threadIdx.x >> 5);
   const int slabs = K / 32;
@@ -142,11 +148,12 @@ __global__ void __launch_bounds__(kPackThreads) residual_quant_kernel(
   const int k = slab * 32 + lane;
   float l1row[R];
   load_l1_row<R>(L1, k, l1row);
+  const double lam = smooth != nullptr ? static_cast<double>(smooth[k]) : 1.0;
   const float g = gscale[1];
   const float d = __fmul_rn(6.0f, g);
   const int n_end = min(N, n_begin + kPackRowsPerWarp);
   for (int n = n_begin; n < n_end; ++n) {
-    const float x = residual_at<R>(W, l1row, l2t, N, K, n, k);
+    const float x = residual_at<R>(W, l1row, l2t, N, K, n, k, lam);
     float am = fabsf(x);
 #pragma unroll
     for (int o = 8; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));

@@ -290,8 +290,18 @@ __device__ __forceinline__ float e4m3_to_f32(uint32_t code) {
   return __half2float(__ushort_as_half(static_cast<unsigned short>(h2 & 0xFFFFu)));
 }
 
-// x0 *= s, x1 *= s as two IEEE round-to-nearest fp32 products (no flush to
-// zero) in one packed sm_100 instruction: the same results as two __fmul_rn.
+// (x0, x1) *= (s0, s1): two IEEE round-to-nearest fp32 products (no flush to
+// zero) in one packed sm_100 instruction, the same results as two __fmul_rn.
+__device__ __forceinline__ void mul2x2_rn(float& x0, float& x1, float s0, float s1) {
+  asm("{\n\t.reg .b64 pa, pb, pd;\n\t"
+      "mov.b64 pa, {%0, %1};\n\t"
+      "mov.b64 pb, {%2, %3};\n\t"
+      "mul.rn.f32x2 pd, pa, pb;\n\t"
+      "mov.b64 {%0, %1}, pd;\n\t}"
+      : "+f"(x0), "+f"(x1)
+      : "f"(s0), "f"(s1));
+}
+// x0 *= s, x1 *= s (as mul2x2_rn with s0 = s1 = s).
 __device__ __forceinline__ void mul2_rn(float& x0, float& x1, float s) {
   asm("{\n\t.reg .b64 pa, pb, pd;\n\t"
       "mov.b64 pa, {%0, %1};\n\t"

@@ -89,16 +89,29 @@ __host__ __device__ constexpr size_t quantize_smem_bytes(int kchunk) {
 // NB NVFP4 blocks (16 bf16 values = two 16-byte words each) -> 8 code bytes
 // per block in c[2b], c[2b+1] and the scale bytes in sc (block b in byte b).
 // Every step is one correctly rounded fp32 operation:
-// S = e4m3(amax / (6 g)), q = x * (1 / fp32(dec(S) g)).
+// x^ = x * inv_smooth[k] (when smoothing), S = e4m3(amax / (6 g)),
+// q = x^ * (1 / fp32(dec(S) g)). sm: the blocks' 16 * NB smoothing factors
+// (16-byte aligned), or nullptr.
 template <int NB>
 __device__ __forceinline__ void quantize_blocks(const uint4 (&v)[2 * NB], float d, const float* inv_tab,
-                                                uint32_t (&c)[2 * NB], uint32_t& sc) {
+                                                const float* __restrict__ sm, uint32_t (&c)[2 * NB], uint32_t& sc) {
   sc = 0;
 #pragma unroll
   for (int blk = 0; blk < NB; ++blk) {
     float f[8], e[8];
     bf16x8_to_f32(v[2 * blk], f);
     bf16x8_to_f32(v[2 * blk + 1], e);
+    if (sm != nullptr) {
+      const float4* s4 = reinterpret_cast<const float4*>(sm + 16 * blk);
+      const float4 a = __ldg(s4), b = __ldg(s4 + 1), cc = __ldg(s4 + 2), dd = __ldg(s4 + 3);
+      const float fa[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+      const float fe[8] = {cc.x, cc.y, cc.z, cc.w, dd.x, dd.y, dd.z, dd.w};
+#pragma unroll
+      for (int i = 0; i < 8; i += 2) {
+        mul2x2_rn(f[i], f[i + 1], fa[i], fa[i + 1]);
+        mul2x2_rn(e[i], e[i + 1], fe[i], fe[i + 1]);
+      }
+    }
     float am = 0.0f;
 #pragma unroll
     for (int i = 0; i < 8; ++i) am = fmaxf(am, fmaxf(fabsf(f[i]), fabsf(e[i])));
@@ -115,11 +128,13 @@ __device__ __forceinline__ void quantize_blocks(const uint4 (&v)[2 * NB], float 
   }
 }
 
-template <int R, int ROWS>
+// SMOOTH: the 4-bit branch quantises x * inv_smooth[k] (smoothing); the plain
+// instantiation ignores inv_smooth.
+template <int R, int ROWS, bool SMOOTH>
 __global__ void __launch_bounds__(kQuantThreads, 2) quantize_act_kernel(
     const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_l1t, int M, int K,
-    const float* __restrict__ g_x, uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
-    __nv_bfloat16* __restrict__ xl1, int kchunk) {
+    const float* __restrict__ g_x, const float* __restrict__ inv_smooth, uint8_t* __restrict__ codes,
+    uint8_t* __restrict__ scales, __nv_bfloat16* __restrict__ xl1, int kchunk) {
   using C = QuantCfg<R, ROWS>;
   constexpr int S = C::kStages;
   constexpr int BPT = C::kBpt;
@@ -233,7 +248,8 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quantize_act_kernel(
     auto emit = [&](int st, const uint4 (&v)[2 * BPT]) {
       uint32_t c[2 * BPT];
       uint32_t sc;
-      quantize_blocks<BPT>(v, d, inv_tab, c, sc);
+      quantize_blocks<BPT>(v, d, inv_tab, SMOOTH ? inv_smooth + k_begin + st * kQuantStep + 16 * b0 : nullptr, c,
+                           sc);
       if constexpr (BPT == 2) {
         if (valid) *reinterpret_cast<uint4*>(cp + st * (kQuantStep / 2)) = make_uint4(c[0], c[1], c[2], c[3]);
         *reinterpret_cast<uint16_t*>(sp + st * 512) = static_cast<uint16_t>(sc);

@@ -15,6 +15,7 @@
 #include "gemm_w4a4_2sm.cuh"
 #include "lowrank_svd.cuh"
 #include "pack_weight.cuh"
+#include "smooth.cuh"
 #include "quantize_act.cuh"
 
 namespace svdq {
@@ -241,7 +242,7 @@ bool quant_candidate(int M, int K, int ks, int sm_count, int dev, bool* shares) 
   if (smem > 227 * 1024) return false;
   *shares = false;
   if (ks == 1) return true;
-  auto kern = quantize_act_kernel<R, ROWS>;
+  auto kern = quantize_act_kernel<R, ROWS, false>;
   static std::atomic<uint64_t> attr_done{0};
   ensure_smem_attr(kern, 227 * 1024, attr_done);
   cudaLaunchConfig_t cfg = {};
@@ -314,14 +315,14 @@ QuantPlan plan_quantize(int M, int K, int sm_count) {
 
 template <int R, int ROWS>
 svdq_status launch_quantize(int M, int K, int ks, const void* X, int64_t ldx, const float* g_x, const void* l1t,
-                            void* codes, void* scales, void* xl1, cudaStream_t stream) {
+                            const float* inv_smooth, void* codes, void* scales, void* xl1, cudaStream_t stream) {
   const int row_tiles = (M + ROWS - 1) / ROWS;
   const int kchunk = K / ks;
   const size_t smem = quantize_smem_bytes<R, ROWS>(kchunk);
   if (smem > 227 * 1024) return SVDQ_ERR_UNSUPPORTED_SHAPE;
-  auto kern = quantize_act_kernel<R, ROWS>;
-  static std::atomic<uint64_t> attr_done{0};
-  ensure_smem_attr(kern, 227 * 1024, attr_done);
+  auto kern = inv_smooth != nullptr ? quantize_act_kernel<R, ROWS, true> : quantize_act_kernel<R, ROWS, false>;
+  static std::atomic<uint64_t> attr_done[2] = {};
+  ensure_smem_attr(kern, 227 * 1024, attr_done[inv_smooth != nullptr]);
   CUtensorMap tm_x, tm_l;
   if (!make_tmap_2d(&tm_x, X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, M, static_cast<uint64_t>(ldx) * 2, 64, ROWS,
                     CU_TENSOR_MAP_SWIZZLE_128B) ||
@@ -340,28 +341,32 @@ svdq_status launch_quantize(int M, int K, int ks, const void* X, int64_t ldx, co
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaLaunchKernelEx(&cfg, kern, tm_x, tm_l, M, K, g_x, static_cast<uint8_t*>(codes), static_cast<uint8_t*>(scales),
-                     static_cast<__nv_bfloat16*>(xl1), kchunk);
+  cudaLaunchKernelEx(&cfg, kern, tm_x, tm_l, M, K, g_x, inv_smooth, static_cast<uint8_t*>(codes),
+                     static_cast<uint8_t*>(scales), static_cast<__nv_bfloat16*>(xl1), kchunk);
   return launch_status();
 }
 
 template <int R>
 svdq_status launch_quantize_planned(int M, int K, const void* X, int64_t ldx, const float* g_x, const void* l1t,
-                                    void* codes, void* scales, void* xl1, cudaStream_t st, int sms) {
+                                    const float* inv_smooth, void* codes, void* scales, void* xl1, cudaStream_t st,
+                                    int sms) {
   const QuantPlan plan = plan_quantize<R>(M, K, sms);
   if (plan.rows == 64)
-    return launch_quantize<R, 64>(M, K, plan.ks, X, ldx, g_x, l1t, codes, scales, xl1, st);
-  return launch_quantize<R, 128>(M, K, plan.ks, X, ldx, g_x, l1t, codes, scales, xl1, st);
+    return launch_quantize<R, 64>(M, K, plan.ks, X, ldx, g_x, l1t, inv_smooth, codes, scales, xl1, st);
+  return launch_quantize<R, 128>(M, K, plan.ks, X, ldx, g_x, l1t, inv_smooth, codes, scales, xl1, st);
 }
 
 svdq_status quantize_dispatch(int M, int K, int r, const void* X, int64_t ldx, const float* g_x, const void* l1t,
-                              void* codes, void* scales, void* xl1, cudaStream_t st, int sms) {
+                              const float* inv_smooth, void* codes, void* scales, void* xl1, cudaStream_t st,
+                              int sms) {
+#define SVDQ_Q_ARGS M, K, X, ldx, g_x, l1t, inv_smooth, codes, scales, xl1, st, sms
   switch (r) {
-    case 16: return launch_quantize_planned<16>(M, K, X, ldx, g_x, l1t, codes, scales, xl1, st, sms);
-    case 32: return launch_quantize_planned<32>(M, K, X, ldx, g_x, l1t, codes, scales, xl1, st, sms);
-    case 64: return launch_quantize_planned<64>(M, K, X, ldx, g_x, l1t, codes, scales, xl1, st, sms);
-    default: return launch_quantize_planned<128>(M, K, X, ldx, g_x, l1t, codes, scales, xl1, st, sms);
+    case 16: return launch_quantize_planned<16>(SVDQ_Q_ARGS);
+    case 32: return launch_quantize_planned<32>(SVDQ_Q_ARGS);
+    case 64: return launch_quantize_planned<64>(SVDQ_Q_ARGS);
+    default: return launch_quantize_planned<128>(SVDQ_Q_ARGS);
   }
+#undef SVDQ_Q_ARGS
 }
 
 template <int R, bool QKV>
@@ -464,8 +469,10 @@ svdq_status gemm_dispatch(int M, int N, int K, int r, const void* a_codes, const
 #undef SVDQ_GEMM_ARGS
 }
 
-// amax|X| over an M x K bf16 matrix with row pitch ldx -> *g as fp32 bits.
-__global__ void act_amax_kernel(const __nv_bfloat16* __restrict__ X, int64_t ldx, int M, int K, unsigned* bits) {
+// amax|X^| over an M x K bf16 matrix with row pitch ldx -> *g as fp32 bits,
+// X^ = fp32(x * inv[k]) with smoothing (inv != nullptr), else X.
+__global__ void act_amax_kernel(const __nv_bfloat16* __restrict__ X, int64_t ldx, int M, int K,
+                                const float* __restrict__ inv, unsigned* bits) {
   float am = 0.0f;
   const int vec_per_row = K / 8;
   const int64_t total = static_cast<int64_t>(M) * vec_per_row;
@@ -475,6 +482,13 @@ __global__ void act_amax_kernel(const __nv_bfloat16* __restrict__ X, int64_t ldx
     const int col = static_cast<int>(i % vec_per_row) * 8;
     float f[8];
     bf16x8_to_f32(ldg_nc_v4(X + row * ldx + col), f);
+    if (inv != nullptr) {
+      const float4 a = __ldg(reinterpret_cast<const float4*>(inv + col));
+      const float4 b = __ldg(reinterpret_cast<const float4*>(inv + col) + 1);
+      const float s8[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+      for (int j = 0; j < 8; ++j) f[j] = __fmul_rn(f[j], s8[j]);
+    }
 #pragma unroll
     for (int j = 0; j < 8; ++j) am = fmaxf(am, fabsf(f[j]));
   }
@@ -484,8 +498,8 @@ __global__ void act_amax_kernel(const __nv_bfloat16* __restrict__ X, int64_t ldx
 }
 
 template <int R>
-svdq_status launch_pack(int N, int K, const void* W, const void* L1, const void* L2, const float* g_x, void* codes,
-                        void* scales, float* gscale, void* l2s, cudaStream_t st) {
+svdq_status launch_pack(int N, int K, const void* W, const void* L1, const void* L2, const float* smooth,
+                        const float* g_x, void* codes, void* scales, float* gscale, void* l2s, cudaStream_t st) {
   // The residual kernels read L2 transposed (N x r); plane 1 of l2s serves as
   // that scratch until make_l2s_kernel overwrites both planes at the end.
   __nv_bfloat16* l2t_scratch = static_cast<__nv_bfloat16*>(l2s) + static_cast<size_t>(N) * R;
@@ -495,11 +509,11 @@ svdq_status launch_pack(int N, int K, const void* W, const void* L1, const void*
   const int blocks = (warps + kPackThreads / 32 - 1) / (kPackThreads / 32);
   if (cudaMemsetAsync(gscale, 0, 4 * sizeof(float), st) != cudaSuccess) return launch_status();
   residual_amax_kernel<R><<<blocks, kPackThreads, 0, st>>>(static_cast<const __nv_bfloat16*>(W),
-                                                           static_cast<const __nv_bfloat16*>(L1), l2t_scratch, N, K,
-                                                           reinterpret_cast<unsigned*>(gscale + 1));
+                                                           static_cast<const __nv_bfloat16*>(L1), l2t_scratch, smooth,
+                                                           N, K, reinterpret_cast<unsigned*>(gscale + 1));
   finalize_gscale_kernel<<<1, 1, 0, st>>>(gscale, g_x);
   residual_quant_kernel<R><<<blocks, kPackThreads, 0, st>>>(
-      static_cast<const __nv_bfloat16*>(W), static_cast<const __nv_bfloat16*>(L1), l2t_scratch, N, K, gscale,
+      static_cast<const __nv_bfloat16*>(W), static_cast<const __nv_bfloat16*>(L1), l2t_scratch, smooth, N, K, gscale,
       static_cast<uint8_t*>(codes), static_cast<uint8_t*>(scales));
   const int64_t total = static_cast<int64_t>(N) * R;
   make_l2s_kernel<<<static_cast<int>((total + 255) / 256), 256, 0, st>>>(
@@ -575,14 +589,14 @@ SvdLayout svd_layout(int N, int K, int r) {
 // C (M x P) = op(A) B with op(A) = A (M x L) or A^T (A: L x M); B: L x P.
 template <bool TRANS_A, typename TA>
 svdq_status ts_gemm(int M, int L, int P, const TA* A, int64_t lda, const double* B, double* C, double* part,
-                    cudaStream_t st) {
+                    cudaStream_t st, const float* colscale = nullptr) {
   const int splits = ts_splits(M, L);
   const int lchunk = (L + splits - 1) / splits;
   const dim3 grid((M + kTsRows - 1) / kTsRows, splits);
   static std::atomic<uint64_t> attr_done{0};  // static tile + up to 40 KB of B slice exceed the 48 KB default
   ensure_smem_attr(ts_gemm_kernel<TRANS_A, TA>, kTsL * kSvdMaxP * static_cast<int>(sizeof(double)), attr_done);
-  ts_gemm_kernel<TRANS_A, TA><<<grid, kTsThreads, kTsL * P * sizeof(double), st>>>(M, L, P, A, lda, B,
-                                                                                    splits > 1 ? part : C, lchunk);
+  ts_gemm_kernel<TRANS_A, TA><<<grid, kTsThreads, kTsL * P * sizeof(double), st>>>(
+      M, L, P, A, lda, colscale, B, splits > 1 ? part : C, lchunk);
   if (splits > 1) {
     const int64_t n = static_cast<int64_t>(M) * P;
     split_sum_kernel<<<static_cast<int>((n + 255) / 256 < 1184 ? (n + 255) / 256 : 1184), 256, 0, st>>>(
@@ -620,8 +634,9 @@ svdq_status orth(double* T, double* tmp, int L, int p, const SvdLayout& lay, uin
   return SVDQ_OK;
 }
 
-svdq_status run_lowrank(int N, int K, int r, const __nv_bfloat16* W, __nv_bfloat16* L1, __nv_bfloat16* L2,
-                        double* sigma, uint64_t seed, int power_iters, uint8_t* ws, cudaStream_t st) {
+svdq_status run_lowrank(int N, int K, int r, const __nv_bfloat16* W, const float* smooth, __nv_bfloat16* L1,
+                        __nv_bfloat16* L2, double* sigma, uint64_t seed, int power_iters, uint8_t* ws,
+                        cudaStream_t st) {
   const int p = svd_width(r);
   const SvdLayout lay = svd_layout(N, K, r);
   double* Om = reinterpret_cast<double*>(ws + lay.om);   // N x p: Omega, later Z
@@ -641,16 +656,17 @@ svdq_status run_lowrank(int N, int K, int r, const __nv_bfloat16* W, __nv_bfloat
   gauss_fill_kernel<<<static_cast<int>(((n_om + 1) / 2 + 255) / 256 < 1184 ? ((n_om + 1) / 2 + 255) / 256 : 1184),
                       256, 0, st>>>(Om, n_om, seed);
   if ((s = launch_status()) != SVDQ_OK) return s;
-  // Y = A Omega = W^T Omega
-  if ((s = ts_gemm<true, __nv_bfloat16>(K, N, p, W, K, Om, Y, part, st)) != SVDQ_OK) return s;
+  // A = diag(lambda) W^T (lambda = 1 without smoothing): every read of W scales its column k by lambda_k.
+  // Y = A Omega
+  if ((s = ts_gemm<true, __nv_bfloat16>(K, N, p, W, K, Om, Y, part, st, smooth)) != SVDQ_OK) return s;
   for (int it = 0; it < power_iters; ++it) {
     if ((s = orth(Y, Yt, K, p, lay, ws, st)) != SVDQ_OK) return s;
-    if ((s = ts_gemm<false, __nv_bfloat16>(N, K, p, W, K, Y, Om, part, st)) != SVDQ_OK) return s;  // Z = W Y
+    if ((s = ts_gemm<false, __nv_bfloat16>(N, K, p, W, K, Y, Om, part, st, smooth)) != SVDQ_OK) return s;  // Z = A^T Y
     if ((s = orth(Om, Zt, N, p, lay, ws, st)) != SVDQ_OK) return s;
-    if ((s = ts_gemm<true, __nv_bfloat16>(K, N, p, W, K, Om, Y, part, st)) != SVDQ_OK) return s;  // Y = W^T Z
+    if ((s = ts_gemm<true, __nv_bfloat16>(K, N, p, W, K, Om, Y, part, st, smooth)) != SVDQ_OK) return s;  // Y = A Z
   }
-  if ((s = orth(Y, Yt, K, p, lay, ws, st)) != SVDQ_OK) return s;                                    // Q
-  if ((s = ts_gemm<false, __nv_bfloat16>(N, K, p, W, K, Y, Om, part, st)) != SVDQ_OK) return s;    // Z = W Q = B^T
+  if ((s = orth(Y, Yt, K, p, lay, ws, st)) != SVDQ_OK) return s;                                            // Q
+  if ((s = ts_gemm<false, __nv_bfloat16>(N, K, p, W, K, Y, Om, part, st, smooth)) != SVDQ_OK) return s;  // B^T = A^T Q
   if ((s = ts_gemm<true, double>(p, N, p, Om, p, Om, C, part, st)) != SVDQ_OK) return s;          // B B^T = Z^T Z
   jacobi_eig_kernel<<<1, 1024, 0, st>>>(C, p, V, lam, 60);
   svd_coeff_kernel<<<1, 256, 0, st>>>(lam, V, p, r, M1, M2, sigma);
@@ -659,7 +675,7 @@ svdq_status run_lowrank(int N, int K, int r, const __nv_bfloat16* W, __nv_bfloat
   if ((s = ts_gemm<false, double>(N, p, r, Om, p, M2, V2, part, st)) != SVDQ_OK) return s;  // V_r = B^T U_B,r / S_r
   const int64_t tot = static_cast<int64_t>(K + N) * r;
   svd_store_kernel<<<static_cast<int>((tot + 255) / 256 < 1184 ? (tot + 255) / 256 : 1184), 256, 0, st>>>(
-      U1, K, V2, N, r, L1, L2);
+      U1, K, V2, N, r, smooth, L1, L2);
   return launch_status();
 }
 
@@ -728,26 +744,33 @@ svdq_status svdq_forward_workspace_size(int M, int K, int r, size_t* bytes) {
   return SVDQ_OK;
 }
 
-svdq_status svdq_pack_weight(int N, int K, int r, const void* W, const void* L1, const void* L2, const float* g_x,
-                             void* w_codes, void* w_scales, float* gscale, void* l1t, void* l2s, void* stream) {
+svdq_status svdq_pack_weight(int N, int K, int r, const void* W, const void* L1, const void* L2, const float* smooth,
+                             const float* g_x, void* w_codes, void* w_scales, float* gscale, void* l1t, void* l2s,
+                             float* inv_smooth, void* stream) {
   svdq_status s = check_layer_shape(N, K, r);
   if (s != SVDQ_OK) return s;
   if (!W || !L1 || !L2 || !g_x || !w_codes || !w_scales || !gscale || !l1t || !l2s) return SVDQ_ERR_INVALID_ARG;
+  if ((smooth == nullptr) != (inv_smooth == nullptr)) return SVDQ_ERR_INVALID_ARG;
   if (!aligned16(W) || !aligned16(L1) || !aligned16(L2) || !aligned16(w_codes) || !aligned16(w_scales) ||
-      !aligned16(l1t) || !aligned16(l2s) || !aligned16(gscale) || (reinterpret_cast<uintptr_t>(g_x) & 3u))
+      !aligned16(l1t) || !aligned16(l2s) || !aligned16(gscale) || (reinterpret_cast<uintptr_t>(g_x) & 3u) ||
+      (smooth && (!aligned16(smooth) || !aligned16(inv_smooth))))
     return SVDQ_ERR_MISALIGNED;
   DeviceInfo di;
   if ((s = current_device(nullptr, &di)) != SVDQ_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (smooth != nullptr) {
+    inv_smooth_kernel<<<(K + 255) / 256, 256, 0, st>>>(smooth, inv_smooth, K);
+    if ((s = launch_status()) != SVDQ_OK) return s;
+  }
   // l1t = L1^T (r x K)
   transpose_bf16_kernel<<<dim3((r + 31) / 32, (K + 31) / 32), 256, 0, st>>>(
       static_cast<const __nv_bfloat16*>(L1), static_cast<__nv_bfloat16*>(l1t), K, r);
   if ((s = launch_status()) != SVDQ_OK) return s;
   switch (r) {
-    case 16: return launch_pack<16>(N, K, W, L1, L2, g_x, w_codes, w_scales, gscale, l2s, st);
-    case 32: return launch_pack<32>(N, K, W, L1, L2, g_x, w_codes, w_scales, gscale, l2s, st);
-    case 64: return launch_pack<64>(N, K, W, L1, L2, g_x, w_codes, w_scales, gscale, l2s, st);
-    default: return launch_pack<128>(N, K, W, L1, L2, g_x, w_codes, w_scales, gscale, l2s, st);
+    case 16: return launch_pack<16>(N, K, W, L1, L2, smooth, g_x, w_codes, w_scales, gscale, l2s, st);
+    case 32: return launch_pack<32>(N, K, W, L1, L2, smooth, g_x, w_codes, w_scales, gscale, l2s, st);
+    case 64: return launch_pack<64>(N, K, W, L1, L2, smooth, g_x, w_codes, w_scales, gscale, l2s, st);
+    default: return launch_pack<128>(N, K, W, L1, L2, smooth, g_x, w_codes, w_scales, gscale, l2s, st);
   }
 }
 
@@ -758,28 +781,30 @@ svdq_status svdq_lowrank_workspace_size(int N, int K, int r, size_t* bytes) {
   return SVDQ_OK;
 }
 
-svdq_status svdq_lowrank_init(int N, int K, int r, const void* W, void* L1, void* L2, double* sigma,
-                              unsigned long long seed, int power_iters, void* workspace, size_t ws_bytes,
-                              void* stream) {
+svdq_status svdq_lowrank_init(int N, int K, int r, const void* W, const float* smooth, void* L1, void* L2,
+                              double* sigma, unsigned long long seed, int power_iters, void* workspace,
+                              size_t ws_bytes, void* stream) {
   if (N <= 0 || K <= 0 || !valid_rank(r) || !W || !L1 || !L2 || !workspace || power_iters < 0 || power_iters > 64)
     return SVDQ_ERR_INVALID_ARG;
   if (r > N || r > K || K % 8 != 0) return SVDQ_ERR_UNSUPPORTED_SHAPE;
   if (!aligned16(W) || !aligned16(L1) || !aligned16(L2) || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
-      (reinterpret_cast<uintptr_t>(sigma) & 7u))
+      (reinterpret_cast<uintptr_t>(sigma) & 7u) || (smooth && !aligned16(smooth)))
     return SVDQ_ERR_MISALIGNED;
   if (ws_bytes < svd_layout(N, K, r).total) return SVDQ_ERR_WORKSPACE;
   svdq_status s;
   DeviceInfo di;
   if ((s = current_device(nullptr, &di)) != SVDQ_OK) return s;
-  return run_lowrank(N, K, r, static_cast<const __nv_bfloat16*>(W), static_cast<__nv_bfloat16*>(L1),
+  return run_lowrank(N, K, r, static_cast<const __nv_bfloat16*>(W), smooth, static_cast<__nv_bfloat16*>(L1),
                      static_cast<__nv_bfloat16*>(L2), sigma, seed, power_iters, static_cast<uint8_t*>(workspace),
                      static_cast<cudaStream_t>(stream));
 }
 
-svdq_status svdq_act_global_scale(int M, int K, const void* X, int64_t ldx, float* g_out, void* stream) {
+svdq_status svdq_act_global_scale(int M, int K, const void* X, int64_t ldx, const float* inv_smooth, float* g_out,
+                                  void* stream) {
   if (M < 0 || K <= 0 || !X || !g_out) return SVDQ_ERR_INVALID_ARG;
   if (K % 8 != 0 || ldx < K || ldx % 8 != 0) return SVDQ_ERR_UNSUPPORTED_SHAPE;
-  if (!aligned16(X) || (reinterpret_cast<uintptr_t>(g_out) & 3u)) return SVDQ_ERR_MISALIGNED;
+  if (!aligned16(X) || (reinterpret_cast<uintptr_t>(g_out) & 3u) || (inv_smooth && !aligned16(inv_smooth)))
+    return SVDQ_ERR_MISALIGNED;
   svdq_status s;
   DeviceInfo di;
   if ((s = current_device(nullptr, &di)) != SVDQ_OK) return s;
@@ -790,26 +815,42 @@ svdq_status svdq_act_global_scale(int M, int K, const void* X, int64_t ldx, floa
     int64_t blocks = (vecs + 255) / 256;
     if (blocks > 8 * di.sm_count) blocks = 8 * di.sm_count;
     act_amax_kernel<<<static_cast<int>(blocks), 256, 0, st>>>(static_cast<const __nv_bfloat16*>(X), ldx, M, K,
-                                                                reinterpret_cast<unsigned*>(g_out));
+                                                                inv_smooth, reinterpret_cast<unsigned*>(g_out));
   }
   finalize_global_scale_kernel<<<1, 1, 0, st>>>(g_out);
   return launch_status();
 }
 
+svdq_status svdq_smooth_factors(int M, int N, int K, const void* X, int64_t ldx, const void* W, float alpha,
+                                float* lambda, void* stream) {
+  if (M < 0 || N <= 0 || K <= 0 || !X || !W || !lambda || !(alpha >= 0.0f && alpha <= 1.0f))
+    return SVDQ_ERR_INVALID_ARG;
+  if (K % 8 != 0 || ldx < K || ldx % 8 != 0) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(X) || !aligned16(W) || (reinterpret_cast<uintptr_t>(lambda) & 3u)) return SVDQ_ERR_MISALIGNED;
+  svdq_status s;
+  DeviceInfo di;
+  if ((s = current_device(nullptr, &di)) != SVDQ_OK) return s;
+  smooth_factors_kernel<<<(K + kSmoothCols - 1) / kSmoothCols, kSmoothThreads, 0,
+                          static_cast<cudaStream_t>(stream)>>>(static_cast<const __nv_bfloat16*>(X), ldx, M,
+                                                               static_cast<const __nv_bfloat16*>(W), N, K, alpha,
+                                                               lambda);
+  return launch_status();
+}
+
 svdq_status svdq_quantize_act(int M, int K, int r, const void* X, int64_t ldx, const float* g_x, const void* l1t,
-                              void* codes, void* scales, void* xl1, void* stream) {
+                              const float* inv_smooth, void* codes, void* scales, void* xl1, void* stream) {
   if (M < 0 || K <= 0 || !valid_rank(r)) return SVDQ_ERR_INVALID_ARG;
   if (K % 256 != 0 || ldx < K || ldx % 8 != 0) return SVDQ_ERR_UNSUPPORTED_SHAPE;
   if (M == 0) return SVDQ_OK;
   if (!X || !g_x || !l1t || !codes || !scales || !xl1) return SVDQ_ERR_INVALID_ARG;
   if (!aligned16(X) || !aligned16(l1t) || !aligned16(codes) || !aligned16(scales) || !aligned16(xl1) ||
-      (reinterpret_cast<uintptr_t>(g_x) & 3u))
+      (reinterpret_cast<uintptr_t>(g_x) & 3u) || (inv_smooth && !aligned16(inv_smooth)))
     return SVDQ_ERR_MISALIGNED;
   svdq_status s;
   DeviceInfo di;
   if ((s = current_device(nullptr, &di)) != SVDQ_OK) return s;
-  return quantize_dispatch(M, K, r, X, ldx, g_x, l1t, codes, scales, xl1, static_cast<cudaStream_t>(stream),
-                           di.sm_count);
+  return quantize_dispatch(M, K, r, X, ldx, g_x, l1t, inv_smooth, codes, scales, xl1,
+                           static_cast<cudaStream_t>(stream), di.sm_count);
 }
 
 svdq_status svdq_w4a4_gemm(int M, int N, int K, int r, const void* a_codes, const void* a_scales, const void* xl1,
@@ -821,7 +862,7 @@ svdq_status svdq_w4a4_gemm(int M, int N, int K, int r, const void* a_codes, cons
 
 svdq_status svdq_linear_forward_qkv(int M, int N, int K, int r, const void* X, int64_t ldx, const void* w_codes,
                                     const void* w_scales, const float* gscale, const void* l1t, const void* l2s,
-                                    const void* bias, int heads, const void* norm_q_weight,
+                                    const float* inv_smooth, const void* bias, int heads, const void* norm_q_weight,
                                     const void* norm_k_weight, float eps, const float* rope_cos,
                                     const float* rope_sin, int64_t ld_rope, void* Y, int64_t ldy, void* workspace,
                                     size_t workspace_bytes, void* stream) {
@@ -845,7 +886,7 @@ svdq_status svdq_linear_forward_qkv(int M, int N, int K, int r, const void* X, i
   uint8_t* a_codes = ws;
   uint8_t* a_scales = ws + round_up(c, 256);
   uint8_t* xl1 = a_scales + round_up(sc, 256);
-  s = svdq_quantize_act(M, K, r, X, ldx, gscale, l1t, a_codes, a_scales, xl1, stream);
+  s = svdq_quantize_act(M, K, r, X, ldx, gscale, l1t, inv_smooth, a_codes, a_scales, xl1, stream);
   if (s != SVDQ_OK) return s;
   QkvPost post{};
   post.w_q = static_cast<const __nv_bfloat16*>(norm_q_weight);
@@ -887,8 +928,8 @@ extern "C" {
 
 svdq_status svdq_linear_forward(int M, int N, int K, int r, const void* X, int64_t ldx, const void* w_codes,
                                 const void* w_scales, const float* gscale, const void* l1t, const void* l2s,
-                                const void* bias, void* Y, int64_t ldy, void* workspace, size_t workspace_bytes,
-                                void* stream) {
+                                const float* inv_smooth, const void* bias, void* Y, int64_t ldy, void* workspace,
+                                size_t workspace_bytes, void* stream) {
   if (M < 0) return SVDQ_ERR_INVALID_ARG;
   svdq_status s = check_layer_shape(N, K, r);
   if (s != SVDQ_OK) return s;
@@ -905,7 +946,7 @@ svdq_status svdq_linear_forward(int M, int N, int K, int r, const void* X, int64
   uint8_t* a_scales = ws + round_up(c, 256);
   uint8_t* xl1 = a_scales + round_up(sc, 256);
   if (!gscale) return SVDQ_ERR_INVALID_ARG;
-  s = svdq_quantize_act(M, K, r, X, ldx, gscale, l1t, a_codes, a_scales, xl1, stream);
+  s = svdq_quantize_act(M, K, r, X, ldx, gscale, l1t, inv_smooth, a_codes, a_scales, xl1, stream);
   if (s != SVDQ_OK) return s;
   return svdq_w4a4_gemm(M, N, K, r, a_codes, a_scales, xl1, w_codes, w_scales, gscale, l2s, bias, Y, ldy, stream);
 }
@@ -975,8 +1016,8 @@ svdq_status noalloc_scratch(int dev, void** out) {
 
 extern "C" svdq_status svdq_linear_forward_noalloc(int M, int N, int K, int r, const void* X, int64_t ldx,
                                                    const void* w_codes, const void* w_scales, const float* gscale,
-                                                   const void* l1t, const void* l2s, const void* bias, void* Y,
-                                                   int64_t ldy, void* stream) {
+                                                   const void* l1t, const void* l2s, const float* inv_smooth,
+                                                   const void* bias, void* Y, int64_t ldy, void* stream) {
   if (M < 0) return SVDQ_ERR_INVALID_ARG;
   svdq_status s = check_layer_shape(N, K, r);
   if (s != SVDQ_OK) return s;
@@ -997,6 +1038,6 @@ extern "C" svdq_status svdq_linear_forward_noalloc(int M, int N, int K, int r, c
   if ((s = noalloc_scratch(dev, &scratch)) != SVDQ_OK) return s;
   // Nothing in the scratch has to start at zero: the quantize kernel of this
   // call writes every byte the GEMM of this call reads.
-  return svdq_linear_forward(M, N, K, r, X, ldx, w_codes, w_scales, gscale, l1t, l2s, bias, Y, ldy, scratch,
-                             kNoAllocScratchBytes, stream);
+  return svdq_linear_forward(M, N, K, r, X, ldx, w_codes, w_scales, gscale, l1t, l2s, inv_smooth, bias, Y, ldy,
+                             scratch, kNoAllocScratchBytes, stream);
 }
