@@ -205,6 +205,7 @@ def _clone_packed(svdq, pw, dev):
     c = svdq.PackedWeight(pw.N, pw.K, pw.r, dev)
     for name in ("codes", "scales", "gscale", "l1t", "l2s"):
         getattr(c, name).copy_(getattr(pw, name))
+    c.inv_smooth = None if pw.inv_smooth is None else pw.inv_smooth.clone()
     return c
 
 
@@ -310,8 +311,26 @@ def run_ours(args, spec):
     if svdq.svdq_read_device_error() != 0:
         raise RuntimeError("device error during timing")
 
-    # Fused QKV post-processing (per-head RMSNorm of Q/K + rotary embedding in the
-    # GEMM epilogue) against the plain layer, same inputs, same public API path.
+    # Variants of the layer through the public API, same rotating inputs, each
+    # against the plain forward: the fused QKV post-processing (per-head RMSNorm
+    # of Q/K + rotary embedding in the GEMM epilogue), smoothing (lambda from
+    # calibration on X; the quantiser multiplies by inv_smooth), and the dynamic
+    # activation scale (an amax pass over X every call).
+    n_q = min(args.steps, 200)
+
+    def timed(fn):
+        for i in range(3):
+            fn(i)
+        torch.cuda.synchronize()
+        a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for i in range(n_q):
+            fn(i)
+        z.record(stream)
+        torch.cuda.synchronize()
+        return _max_over_ranks(a.elapsed_time(z), world) / n_q
+
+    plain_ms = timed(lambda i: svdq.svdq_linear_forward(Xs[i % n_sets], pws[i % n_sets], bd, out=Y, workspace=ws))
     heads = N // 384
     qkv = None
     if N == heads * 384:
@@ -319,25 +338,27 @@ def run_ours(args, spec):
         wk = torch.ones(128, dtype=torch.bfloat16, device=dev)
         cos_np, sin_np = workloads.rope_tables(M, 128)
         cos_t, sin_t = torch.from_numpy(cos_np).to(dev), torch.from_numpy(sin_np).to(dev)
-        n_q = min(args.steps, 200)
-
-        def timed(fn):
-            for i in range(3):
-                fn(i)
-            torch.cuda.synchronize()
-            a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            for i in range(n_q):
-                fn(i)
-            z.record(stream)
-            torch.cuda.synchronize()
-            return _max_over_ranks(a.elapsed_time(z), world) / n_q
-
-        plain_ms = timed(lambda i: svdq.svdq_linear_forward(Xs[i % n_sets], pws[i % n_sets], bd, out=Y, workspace=ws))
         fused_ms = timed(lambda i: svdq.svdq_linear_forward_qkv(Xs[i % n_sets], pws[i % n_sets], bd, heads, wq, wk,
                                                                1e-6, cos_t, sin_t, out=Y, workspace=ws))
         qkv = {"heads": heads, "head_dim": 128, "ms_per_step": fused_ms, "plain_ms_per_step": plain_ms,
                "overhead": fused_ms / plain_ms - 1.0, "steps": n_q}
+    Wv = W.to(dev)
+    lam = svdq.svdq_smooth_factors(Xd, Wv, 0.5)
+    L1s, L2s, _ = svdq.svdq_lowrank_init(Wv, r, smooth=lam)
+    pw_s = svdq.svdq_pack_weight(Wv, L1s, L2s, 1.0, smooth=lam)
+    g_s = svdq.svdq_act_global_scale(Xd, inv_smooth=pw_s.inv_smooth)
+    pw_s = svdq.svdq_pack_weight(Wv, L1s, L2s, g_s, smooth=lam)
+    del Wv
+    pws_s = [pw_s] + [_clone_packed(svdq, pw_s, dev) for _ in range(n_sets - 1)]
+    smooth_ms = timed(lambda i: svdq.svdq_linear_forward(Xs[i % n_sets], pws_s[i % n_sets], bd, out=Y, workspace=ws))
+    ws_d = torch.empty(svdq.svdq_dynamic_workspace_size(M, N, K, r), dtype=torch.uint8, device=dev)
+    dyn_ms = timed(lambda i: svdq.svdq_linear_forward_dynamic(Xs[i % n_sets], pws[i % n_sets], bd, out=Y,
+                                                              workspace=ws_d))
+    if svdq.svdq_read_device_error() != 0:
+        raise RuntimeError("device error during the variant timings")
+    variants = {"note": "public-API forward, same rotating inputs, one event pair around all steps",
+                "steps": n_q, "plain_ms_per_step": plain_ms,
+                "smoothed_ms_per_step": smooth_ms, "dynamic_scale_ms_per_step": dyn_ms}
 
     peaks, kind = _peaks()
     gemm_name = _gemm_kernel_name(M, N)
@@ -370,6 +391,7 @@ def run_ours(args, spec):
         "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2, "ms_per_step": e2e_ms},
         "qkv_norm_rope": qkv,
+        "variants": variants,
         "gpu_launches": 2 * args.steps,
         "clocks": clk.summary(),
     }

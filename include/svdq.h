@@ -239,6 +239,28 @@ svdq_status svdq_linear_forward(int M, int N, int K, int r, const void* X, int64
                                 const void* bias, void* Y, int64_t ldy, void* workspace,
                                 size_t workspace_bytes, void* stream);
 
+/* The whole layer with a dynamic activation scale: g_x is computed from this
+ * call's X instead of the calibrated gscale[0]:
+ *     g = fp32(amax|X^| / 2688)  (1 for an all-zero X^; X^ = X * inv_smooth),
+ *     alpha' = fp32(g g_w),
+ * and the packed hi/lo planes of L2^T / alpha are re-expressed for alpha'
+ * (v = hi + lo, v' = fp32(v fp32(alpha / alpha')), hi' = bf16(v'),
+ * lo' = bf16(v' - hi'); unchanged when alpha' == alpha). Then the layer runs as
+ * svdq_linear_forward with these scales. This costs one more read of X (the
+ * amax pass) and a pass over the N x r planes. The blog does not say whether
+ * the activation scale is calibrated or per call; this entry point is the
+ * per-call reading, svdq_linear_forward the calibrated one.
+ * Workspace: svdq_dynamic_workspace_size(M, N, K, r) bytes, 256-byte aligned;
+ * after the call it holds, at offset svdq_forward_workspace_size(M, K, r),
+ * the floats {g, g_w, alpha', amax}. Other arguments as
+ * svdq_linear_forward. */
+svdq_status svdq_dynamic_workspace_size(int M, int N, int K, int r, size_t* bytes);
+svdq_status svdq_linear_forward_dynamic(int M, int N, int K, int r, const void* X, int64_t ldx,
+                                        const void* w_codes, const void* w_scales, const float* gscale,
+                                        const void* l1t, const void* l2s, const float* inv_smooth,
+                                        const void* bias, void* Y, int64_t ldy, void* workspace,
+                                        size_t workspace_bytes, void* stream);
+
 /* Same computation as svdq_linear_forward, for callers that cannot supply a
  * workspace: plugin interfaces of inference runtimes that pass only a layer's
  * inputs and outputs, and code running after the process has fixed its device

@@ -130,6 +130,23 @@ def test_smoothing_validation(L):
     assert L.svdq_act_global_scale(4, 256, p, 256, odd, p, None) == 3
 
 
+def test_dynamic_forward_sizes_and_validation(L):
+    p = ctypes.c_void_p(0x10000)
+    odd = ctypes.c_void_p(0x10008)
+    base = _lib.svdq_forward_workspace_size(300, 512, 32)
+    assert _lib.svdq_dynamic_workspace_size(300, 384, 512, 32) == base + 8192 + 384 * 32 * 4
+    with pytest.raises(_lib.SvdqError):
+        _lib.svdq_dynamic_workspace_size(300, 100, 512, 32)     # N % 128
+    need = _lib.svdq_dynamic_workspace_size(4, 128, 256, 32)
+    args = lambda ws, wsb, x: (4, 128, 256, 32, x, 256, p, p, p, p, p, None, None, p, 128, ws, ctypes.c_size_t(wsb),
+                               None)
+    assert L.svdq_linear_forward_dynamic(*args(p, need - 1, p)) == 7     # workspace too small
+    assert L.svdq_linear_forward_dynamic(*args(odd, need, p)) == 3       # misaligned workspace
+    assert L.svdq_linear_forward_dynamic(*args(p, need, None)) == 1      # no X
+    assert L.svdq_linear_forward_dynamic(0, 128, 256, 32, None, 256, None, None, None, None, None, None, None, None,
+                                         128, None, 0, None) == 0          # M == 0: no-op
+
+
 def test_qkv_forward_validation(L):
     p = ctypes.c_void_p(0x10000)
     odd = ctypes.c_void_p(0x10008)

@@ -12,8 +12,10 @@ from ._lib import (  # noqa: F401
     lib,
     svdq_act_global_scale,
     svdq_act_sizes,
+    svdq_dynamic_workspace_size,
     svdq_forward_workspace_size,
     svdq_linear_forward,
+    svdq_linear_forward_dynamic,
     svdq_linear_forward_qkv,
     svdq_lowrank_init,
     svdq_lowrank_workspace_size,

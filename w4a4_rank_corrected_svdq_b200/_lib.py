@@ -41,6 +41,9 @@ SIGNATURES = {
     "svdq_linear_forward_noalloc": (_i, [_i, _i, _i, _i, _p, _i64, _p, _p, _p, _p, _p, _p, _p, _p, _i64, _p]),
     "svdq_linear_forward_qkv": (_i, [_i, _i, _i, _i, _p, _i64, _p, _p, _p, _p, _p, _p, _p, _i, _p, _p, _f, _p,
                                      _p, _i64, _p, _i64, _p, _sz, _p]),
+    "svdq_dynamic_workspace_size": (_i, [_i, _i, _i, _i, _psz]),
+    "svdq_linear_forward_dynamic": (_i, [_i, _i, _i, _i, _p, _i64, _p, _p, _p, _p, _p, _p, _p, _p, _i64, _p, _sz,
+                                         _p]),
     "svdq_lowrank_workspace_size": (_i, [_i, _i, _i, _psz]),
     "svdq_lowrank_init": (_i, [_i, _i, _i, _p, _p, _p, _p, _p, ctypes.c_ulonglong, _i, _p, _sz, _p]),
 }
@@ -327,6 +330,32 @@ def svdq_linear_forward_qkv(X: torch.Tensor, pw: PackedWeight, bias: torch.Tenso
         M, N, K, pw.r, _ptr(X), ldx, _ptr(pw.codes), _ptr(pw.scales), _ptr(pw.gscale), _ptr(pw.l1t), _ptr(pw.l2s),
         _ptr(pw.inv_smooth), _ptr(bias), heads, _ptr(norm_q_weight), _ptr(norm_k_weight), float(eps), _ptr(rope_cos), _ptr(rope_sin),
         rope_cos.stride(0), _ptr(Y), ldy, _ptr(workspace), workspace.numel(), _stream(X)))
+    return Y
+
+
+def svdq_dynamic_workspace_size(M: int, N: int, K: int, r: int) -> int:
+    out = ctypes.c_size_t()
+    _check("svdq_dynamic_workspace_size", lib().svdq_dynamic_workspace_size(M, N, K, r, ctypes.byref(out)))
+    return out.value
+
+
+def svdq_linear_forward_dynamic(X: torch.Tensor, pw: PackedWeight, bias: torch.Tensor | None = None,
+                                out: torch.Tensor | None = None, workspace: torch.Tensor | None = None) -> torch.Tensor:
+    """The layer with the activation scale computed from this call's X."""
+    _dev(X, "X", torch.bfloat16)
+    M, K = X.shape
+    N, r = pw.N, pw.r
+    ldx = _rows(X, "X", K)
+    if bias is not None:
+        _dev(bias, "bias", torch.bfloat16, (N,))
+    Y = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=X.device)
+    _dev(Y, "Y", torch.bfloat16)
+    ldy = _rows(Y, "Y", N)
+    need = svdq_dynamic_workspace_size(M, N, K, r)
+    ws = workspace if workspace is not None else torch.empty(need, dtype=torch.uint8, device=X.device)
+    _check("svdq_linear_forward_dynamic", lib().svdq_linear_forward_dynamic(
+        M, N, K, r, _ptr(X), ldx, _ptr(pw.codes), _ptr(pw.scales), _ptr(pw.gscale), _ptr(pw.l1t),
+        _ptr(pw.l2s), _ptr(pw.inv_smooth), _ptr(bias), _ptr(Y), ldy, _ptr(ws), ws.numel(), _stream(X)))
     return Y
 
 

@@ -63,11 +63,18 @@ struct QuantCfg {
   // KS is; they alias the ring once every CTA of the cluster has drained it.
   static constexpr int kPartBytes = ROWS * R * 4;
   static constexpr int kBody = kRingBytes > kPartBytes ? kRingBytes : kPartBytes;
+  // Smoothing factors of each step (64 floats), loaded with the step's tiles
+  // into a ring of 2 x kStages slots: the slot of step st is rewritten only
+  // with step st + 2 kStages, whose load waits for every quantiser warp to
+  // release step st + kStages, which each does after quantising step st.
+  static constexpr int kSmoothSlots = 2 * kStages;
+  static constexpr int kSmoothBytes = kSmoothSlots * kQuantStep * 4;
   static constexpr int kSwzMask = (R / 4 < 8 ? R / 4 : 8) - 1;  // 16-byte chunk swizzle of a partial row
   static constexpr int kBpt = ROWS / 64;   // NVFP4 blocks per quantiser thread per step
   static constexpr int kTpr = 4 / kBpt;    // quantiser threads per row
   static constexpr int kBatch = 4 / kBpt;  // steps per quantiser iteration
   static_assert(kStages <= kQuantMaxStages, "barrier arrays");
+  static_assert(kStages >= kBatch, "the smoothing ring needs a step's release to follow its quantisation");
 };
 
 struct QuantBarriers {
@@ -79,11 +86,14 @@ struct QuantBarriers {
   int abort;
 };
 
-// Dynamic shared memory: stage ring (later XL1 partial slots), scale staging
-// for the CTA's K-range, reciprocal table, barriers, alignment slack.
+// Dynamic shared memory: stage ring (later XL1 partial slots), smoothing-factor
+// ring, scale staging for the CTA's K-range, reciprocal table, barriers,
+// alignment slack. (Both instantiations reserve the smoothing ring, so the
+// launch plan does not depend on smoothing.)
 template <int R, int ROWS>
 __host__ __device__ constexpr size_t quantize_smem_bytes(int kchunk) {
-  return static_cast<size_t>(QuantCfg<R, ROWS>::kBody) + static_cast<size_t>(kchunk / 64) * 512 + 512 + 256 + 1024;
+  return static_cast<size_t>(QuantCfg<R, ROWS>::kBody) + QuantCfg<R, ROWS>::kSmoothBytes +
+         static_cast<size_t>(kchunk / 64) * 512 + 512 + 256 + 1024;
 }
 
 // NB NVFP4 blocks (16 bf16 values = two 16-byte words each) -> 8 code bytes
@@ -91,7 +101,7 @@ __host__ __device__ constexpr size_t quantize_smem_bytes(int kchunk) {
 // Every step is one correctly rounded fp32 operation:
 // x^ = x * inv_smooth[k] (when smoothing), S = e4m3(amax / (6 g)),
 // q = x^ * (1 / fp32(dec(S) g)). sm: the blocks' 16 * NB smoothing factors
-// (16-byte aligned), or nullptr.
+// (16-byte aligned, in shared memory), or nullptr.
 template <int NB>
 __device__ __forceinline__ void quantize_blocks(const uint4 (&v)[2 * NB], float d, const float* inv_tab,
                                                 const float* __restrict__ sm, uint32_t (&c)[2 * NB], uint32_t& sc) {
@@ -103,7 +113,7 @@ __device__ __forceinline__ void quantize_blocks(const uint4 (&v)[2 * NB], float 
     bf16x8_to_f32(v[2 * blk + 1], e);
     if (sm != nullptr) {
       const float4* s4 = reinterpret_cast<const float4*>(sm + 16 * blk);
-      const float4 a = __ldg(s4), b = __ldg(s4 + 1), cc = __ldg(s4 + 2), dd = __ldg(s4 + 3);
+      const float4 a = s4[0], b = s4[1], cc = s4[2], dd = s4[3];
       const float fa[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
       const float fe[8] = {cc.x, cc.y, cc.z, cc.w, dd.x, dd.y, dd.z, dd.w};
 #pragma unroll
@@ -140,7 +150,8 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quantize_act_kernel(
   constexpr int BPT = C::kBpt;
   extern __shared__ uint8_t qsmem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(qsmem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sc_stage = smem + C::kBody;
+  float* sm_ring = reinterpret_cast<float*>(smem + C::kBody);
+  uint8_t* sc_stage = smem + C::kBody + C::kSmoothBytes;
   float* inv_tab = reinterpret_cast<float*>(sc_stage + (kchunk / 64) * 512);
   QuantBarriers* bars = reinterpret_cast<QuantBarriers*>(inv_tab + 128);
   float* part = reinterpret_cast<float*>(smem);  // slots, valid after the cluster barrier
@@ -153,11 +164,11 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quantize_act_kernel(
   const int k_begin = ks * kchunk;
   const int nsteps = kchunk / kQuantStep;
   const int rpc = ROWS / KS;  // output rows finished by each CTA of the cluster
-  const float g = *g_x;
-  // The GEMM that consumes this kernel's output may be scheduled now: it
-  // prepares its shared memory and TMEM, then waits for this grid to finish.
-  pdl_launch_dependents();
 
+  // The prologue reads only X, L1^T and the smoothing factors, which no kernel
+  // of the layer writes; g_x may come from the kernel before this one (the
+  // dynamic scale), so it is read after griddepcontrol.wait (a no-op unless
+  // this grid was launched as a programmatic dependent).
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(&bars->full[s], 1);
@@ -173,11 +184,19 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quantize_act_kernel(
     prefetch_tmap(&tm_l1t);
     for (int st = 0; st < S && st < nsteps; ++st) {
       uint8_t* dst = smem + st * C::kStageBytes;
-      mbar_arrive_expect_tx(&bars->full[st], C::kStageBytes);
+      mbar_arrive_expect_tx(&bars->full[st], C::kStageBytes + (SMOOTH ? kQuantStep * 4 : 0));
       tma_load_2d(dst, &tm_x, k_begin + st * kQuantStep, m0, &bars->full[st]);
       tma_load_2d(dst + C::kXBytes, &tm_l1t, k_begin + st * kQuantStep, 0, &bars->full[st]);
+      if (SMOOTH)
+        bulk_load(sm_ring + (st % C::kSmoothSlots) * kQuantStep, inv_smooth + k_begin + st * kQuantStep,
+                  kQuantStep * 4, &bars->full[st]);
     }
   }
+  pdl_wait();
+  const float g = *g_x;
+  // The GEMM that consumes this kernel's output may be scheduled now: it
+  // prepares its shared memory and TMEM, then waits for this grid to finish.
+  pdl_launch_dependents();
   if (warp == 0) {
     __syncwarp();
     tmem_alloc(&bars->tmem_base, C::kTmemCols);
@@ -216,9 +235,12 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quantize_act_kernel(
         if (nx < nsteps) {
           if (!mbar_wait(&bars->empty[s], ph, abort)) break;
           uint8_t* dst = smem + s * C::kStageBytes;
-          mbar_arrive_expect_tx(&bars->full[s], C::kStageBytes);
+          mbar_arrive_expect_tx(&bars->full[s], C::kStageBytes + (SMOOTH ? kQuantStep * 4 : 0));
           tma_load_2d(dst, &tm_x, k_begin + nx * kQuantStep, m0, &bars->full[s]);
           tma_load_2d(dst + C::kXBytes, &tm_l1t, k_begin + nx * kQuantStep, 0, &bars->full[s]);
+          if (SMOOTH)
+            bulk_load(sm_ring + (nx % C::kSmoothSlots) * kQuantStep, inv_smooth + k_begin + nx * kQuantStep,
+                      kQuantStep * 4, &bars->full[s]);
         }
       }
       tc_commit(&bars->acc_done);
@@ -248,8 +270,8 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quantize_act_kernel(
     auto emit = [&](int st, const uint4 (&v)[2 * BPT]) {
       uint32_t c[2 * BPT];
       uint32_t sc;
-      quantize_blocks<BPT>(v, d, inv_tab, SMOOTH ? inv_smooth + k_begin + st * kQuantStep + 16 * b0 : nullptr, c,
-                           sc);
+      quantize_blocks<BPT>(v, d, inv_tab, SMOOTH ? sm_ring + (st % C::kSmoothSlots) * kQuantStep + 16 * b0 : nullptr,
+                           c, sc);
       if constexpr (BPT == 2) {
         if (valid) *reinterpret_cast<uint4*>(cp + st * (kQuantStep / 2)) = make_uint4(c[0], c[1], c[2], c[3]);
         *reinterpret_cast<uint16_t*>(sp + st * 512) = static_cast<uint16_t>(sc);

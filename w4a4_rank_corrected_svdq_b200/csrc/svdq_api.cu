@@ -315,7 +315,8 @@ QuantPlan plan_quantize(int M, int K, int sm_count) {
 
 template <int R, int ROWS>
 svdq_status launch_quantize(int M, int K, int ks, const void* X, int64_t ldx, const float* g_x, const void* l1t,
-                            const float* inv_smooth, void* codes, void* scales, void* xl1, cudaStream_t stream) {
+                            const float* inv_smooth, void* codes, void* scales, void* xl1, cudaStream_t stream,
+                            bool pdl) {
   const int row_tiles = (M + ROWS - 1) / ROWS;
   const int kchunk = K / ks;
   const size_t smem = quantize_smem_bytes<R, ROWS>(kchunk);
@@ -334,13 +335,17 @@ svdq_status launch_quantize(int M, int K, int ks, const void* X, int64_t ldx, co
   cfg.gridDim = dim3(ks, row_tiles, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = ks;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  // pdl: a programmatic dependent of the previous kernel on the stream (the
+  // kernel reads g_x only after griddepcontrol.wait).
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = pdl ? 2 : 1;
   cudaLaunchKernelEx(&cfg, kern, tm_x, tm_l, M, K, g_x, inv_smooth, static_cast<uint8_t*>(codes),
                      static_cast<uint8_t*>(scales), static_cast<__nv_bfloat16*>(xl1), kchunk);
   return launch_status();
@@ -349,17 +354,17 @@ svdq_status launch_quantize(int M, int K, int ks, const void* X, int64_t ldx, co
 template <int R>
 svdq_status launch_quantize_planned(int M, int K, const void* X, int64_t ldx, const float* g_x, const void* l1t,
                                     const float* inv_smooth, void* codes, void* scales, void* xl1, cudaStream_t st,
-                                    int sms) {
+                                    int sms, bool pdl) {
   const QuantPlan plan = plan_quantize<R>(M, K, sms);
   if (plan.rows == 64)
-    return launch_quantize<R, 64>(M, K, plan.ks, X, ldx, g_x, l1t, inv_smooth, codes, scales, xl1, st);
-  return launch_quantize<R, 128>(M, K, plan.ks, X, ldx, g_x, l1t, inv_smooth, codes, scales, xl1, st);
+    return launch_quantize<R, 64>(M, K, plan.ks, X, ldx, g_x, l1t, inv_smooth, codes, scales, xl1, st, pdl);
+  return launch_quantize<R, 128>(M, K, plan.ks, X, ldx, g_x, l1t, inv_smooth, codes, scales, xl1, st, pdl);
 }
 
 svdq_status quantize_dispatch(int M, int K, int r, const void* X, int64_t ldx, const float* g_x, const void* l1t,
                               const float* inv_smooth, void* codes, void* scales, void* xl1, cudaStream_t st,
-                              int sms) {
-#define SVDQ_Q_ARGS M, K, X, ldx, g_x, l1t, inv_smooth, codes, scales, xl1, st, sms
+                              int sms, bool pdl = false) {
+#define SVDQ_Q_ARGS M, K, X, ldx, g_x, l1t, inv_smooth, codes, scales, xl1, st, sms, pdl
   switch (r) {
     case 16: return launch_quantize_planned<16>(SVDQ_Q_ARGS);
     case 32: return launch_quantize_planned<32>(SVDQ_Q_ARGS);
@@ -469,32 +474,142 @@ svdq_status gemm_dispatch(int M, int N, int K, int r, const void* a_codes, const
 #undef SVDQ_GEMM_ARGS
 }
 
-// amax|X^| over an M x K bf16 matrix with row pitch ldx -> *g as fp32 bits,
-// X^ = fp32(x * inv[k]) with smoothing (inv != nullptr), else X.
-__global__ void act_amax_kernel(const __nv_bfloat16* __restrict__ X, int64_t ldx, int M, int K,
-                                const float* __restrict__ inv, unsigned* bits) {
-  float am = 0.0f;
-  const int vec_per_row = K / 8;
-  const int64_t total = static_cast<int64_t>(M) * vec_per_row;
-  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t row = i / vec_per_row;
-    const int col = static_cast<int>(i % vec_per_row) * 8;
-    float f[8];
-    bf16x8_to_f32(ldg_nc_v4(X + row * ldx + col), f);
-    if (inv != nullptr) {
-      const float4 a = __ldg(reinterpret_cast<const float4*>(inv + col));
-      const float4 b = __ldg(reinterpret_cast<const float4*>(inv + col) + 1);
-      const float s8[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+// max |fp32(x * inv[col + j])| (or |x|) over one 16-byte vector of 8 bf16.
+__device__ __forceinline__ float vec_amax(const __nv_bfloat16* p, const float* __restrict__ inv, int col, float am) {
+  float f[8];
+  bf16x8_to_f32(ldg_nc_v4(p), f);
+  if (inv != nullptr) {
+    const float4 a = __ldg(reinterpret_cast<const float4*>(inv + col));
+    const float4 b = __ldg(reinterpret_cast<const float4*>(inv + col) + 1);
+    const float s8[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
 #pragma unroll
-      for (int j = 0; j < 8; ++j) f[j] = __fmul_rn(f[j], s8[j]);
-    }
-#pragma unroll
-    for (int j = 0; j < 8; ++j) am = fmaxf(am, fabsf(f[j]));
+    for (int j = 0; j < 8; ++j) f[j] = __fmul_rn(f[j], s8[j]);
   }
 #pragma unroll
+  for (int j = 0; j < 8; ++j) am = fmaxf(am, fabsf(f[j]));
+  return am;
+}
+
+// amax|X^| over an M x K bf16 matrix with row pitch ldx, X^ = fp32(x * inv[k])
+// with smoothing (inv != nullptr), else X. A grid-stride walk over the 16-byte
+// vectors, four loads in flight per thread, then per block either one
+// atomicMax into *bits (fp32 bits: |x| >= 0, so the unsigned order of the bits
+// is the order of the values) or, with partial != nullptr, the block's
+// maximum in partial[blockIdx.x]. Idx: 32-bit indexing when the vector count
+// fits.
+template <typename Idx>
+__global__ void __launch_bounds__(256) act_amax_kernel(const __nv_bfloat16* __restrict__ X, int64_t ldx, int M,
+                                                       int K, const float* __restrict__ inv, unsigned* bits,
+                                                       float* __restrict__ partial) {
+  pdl_launch_dependents();  // a programmatic dependent waits for this grid's completion anyway
+  const Idx vpr = static_cast<Idx>(K / 8);
+  const Idx total = static_cast<Idx>(M) * vpr;
+  const Idx stride = static_cast<Idx>(gridDim.x) * blockDim.x;
+  float am = 0.0f;
+  Idx i = static_cast<Idx>(blockIdx.x) * blockDim.x + threadIdx.x;
+  auto at = [&](Idx v) { return X + static_cast<int64_t>(v / vpr) * ldx + static_cast<int64_t>(v % vpr) * 8; };
+  for (; i + 3 * stride < total; i += 4 * stride) {
+    const Idx i1 = i + stride, i2 = i + 2 * stride, i3 = i + 3 * stride;
+    const uint4 v0 = ldg_nc_v4(at(i)), v1 = ldg_nc_v4(at(i1)), v2 = ldg_nc_v4(at(i2)), v3 = ldg_nc_v4(at(i3));
+    const uint4 vv[4] = {v0, v1, v2, v3};
+    const Idx ii[4] = {i, i1, i2, i3};
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      float f[8];
+      bf16x8_to_f32(vv[u], f);
+      if (inv != nullptr) {
+        const int col = static_cast<int>(ii[u] % vpr) * 8;
+        const float4 a = __ldg(reinterpret_cast<const float4*>(inv + col));
+        const float4 b = __ldg(reinterpret_cast<const float4*>(inv + col) + 1);
+        const float s8[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+        for (int j = 0; j < 8; ++j) f[j] = __fmul_rn(f[j], s8[j]);
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) am = fmaxf(am, fabsf(f[j]));
+    }
+  }
+  for (; i < total; i += stride) am = vec_amax(at(i), inv, static_cast<int>(i % vpr) * 8, am);
+  __shared__ float warp_max[8];
+#pragma unroll
   for (int o = 16; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
-  if ((threadIdx.x & 31) == 0) atomicMax(bits, __float_as_uint(am));
+  if ((threadIdx.x & 31) == 0) warp_max[threadIdx.x >> 5] = am;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int w = 1; w < static_cast<int>(blockDim.x >> 5); ++w) am = fmaxf(am, warp_max[w]);
+    if (partial != nullptr)
+      partial[blockIdx.x] = am;
+    else
+      atomicMax(bits, __float_as_uint(am));
+  }
+}
+
+constexpr int kAmaxMaxBlocks = 1984;  // partial maxima of the dynamic scale: 8 KB block minus 256 bytes
+
+// Launches act_amax_kernel over M x K: into *bits (atomicMax; the caller
+// zeroes it) or, with partial, one maximum per block. Returns the block count.
+int launch_act_amax(const __nv_bfloat16* X, int64_t ldx, int M, int K, const float* inv, unsigned* bits,
+                    float* partial, int sm_count, cudaStream_t st) {
+  const uint64_t vecs = static_cast<uint64_t>(M) * static_cast<uint64_t>(K / 8);
+  uint64_t blocks = (vecs + 1023) / 1024;
+  if (blocks > static_cast<uint64_t>(4 * sm_count)) blocks = 4 * sm_count;
+  if (blocks > static_cast<uint64_t>(kAmaxMaxBlocks)) blocks = kAmaxMaxBlocks;
+  if (blocks == 0) blocks = 1;  // an empty X still writes its (zero) partial
+  if (vecs + 4ull * blocks * 256 < (1ull << 32))
+    act_amax_kernel<uint32_t><<<static_cast<int>(blocks), 256, 0, st>>>(X, ldx, M, K, inv, bits, partial);
+  else
+    act_amax_kernel<uint64_t><<<static_cast<int>(blocks), 256, 0, st>>>(X, ldx, M, K, inv, bits, partial);
+  return static_cast<int>(blocks);
+}
+
+// Dynamic activation scale: partial[0..nparts) hold the per-block maxima of
+// amax|X^| of this call. Writes gs_out[0..3] = {g = fp32(amax / 2688) (1 if 0),
+// g_w, alpha' = fp32(g g_w), amax} and re-expresses the packed hi/lo planes of
+// L2^T / alpha for alpha': v = hi + lo (exact in fp32), v' = fp32(v *
+// fp32(alpha / alpha')), hi' = bf16(v'), lo' = bf16(v' - hi'); when alpha' ==
+// alpha the planes are copied unchanged. Launched as a programmatic dependent
+// of the amax pass (it waits for that grid here).
+__global__ void __launch_bounds__(256) dynamic_scale_kernel(const float* __restrict__ gscale,
+                                                            const float* __restrict__ partial, int nparts,
+                                                            float* __restrict__ gs_out,
+                                                            const __nv_bfloat16* __restrict__ l2s,
+                                                            __nv_bfloat16* __restrict__ l2s_out, int64_t total) {
+  pdl_wait();
+  pdl_launch_dependents();
+  __shared__ float red[8];
+  float am = 0.0f;
+  for (int i = threadIdx.x; i < nparts; i += blockDim.x) am = fmaxf(am, partial[i]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = am;
+  __syncthreads();
+  am = red[0];
+  for (int w = 1; w < static_cast<int>(blockDim.x >> 5); ++w) am = fmaxf(am, red[w]);
+  const float g = (am == 0.0f) ? 1.0f : __fdiv_rn(am, kGlobalDivisor);
+  const float gw = gscale[1];
+  const float alpha = gscale[2];
+  const float alpha_d = __fmul_rn(g, gw);
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    gs_out[0] = g;
+    gs_out[1] = gw;
+    gs_out[2] = alpha_d;
+    gs_out[3] = am;
+  }
+  const bool same = alpha_d == alpha;
+  const float ratio = __fdiv_rn(alpha, alpha_d);
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const __nv_bfloat16 hi = l2s[i], lo = l2s[total + i];
+    if (same) {
+      l2s_out[i] = hi;
+      l2s_out[total + i] = lo;
+      continue;
+    }
+    const float v = __fmul_rn(__fadd_rn(__bfloat162float(hi), __bfloat162float(lo)), ratio);
+    const __nv_bfloat16 h2 = __float2bfloat16_rn(v);
+    l2s_out[i] = h2;
+    l2s_out[total + i] = __float2bfloat16_rn(__fsub_rn(v, __bfloat162float(h2)));
+  }
 }
 
 template <int R>
@@ -811,11 +926,8 @@ svdq_status svdq_act_global_scale(int M, int K, const void* X, int64_t ldx, cons
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(g_out, 0, sizeof(float), st) != cudaSuccess) return launch_status();
   if (M > 0) {
-    const int64_t vecs = static_cast<int64_t>(M) * (K / 8);
-    int64_t blocks = (vecs + 255) / 256;
-    if (blocks > 8 * di.sm_count) blocks = 8 * di.sm_count;
-    act_amax_kernel<<<static_cast<int>(blocks), 256, 0, st>>>(static_cast<const __nv_bfloat16*>(X), ldx, M, K,
-                                                                inv_smooth, reinterpret_cast<unsigned*>(g_out));
+    launch_act_amax(static_cast<const __nv_bfloat16*>(X), ldx, M, K, inv_smooth, reinterpret_cast<unsigned*>(g_out),
+                    nullptr, di.sm_count, st);
   }
   finalize_global_scale_kernel<<<1, 1, 0, st>>>(g_out);
   return launch_status();
@@ -949,6 +1061,74 @@ svdq_status svdq_linear_forward(int M, int N, int K, int r, const void* X, int64
   s = svdq_quantize_act(M, K, r, X, ldx, gscale, l1t, inv_smooth, a_codes, a_scales, xl1, stream);
   if (s != SVDQ_OK) return s;
   return svdq_w4a4_gemm(M, N, K, r, a_codes, a_scales, xl1, w_codes, w_scales, gscale, l2s, bias, Y, ldy, stream);
+}
+
+}  // extern "C"
+namespace svdq {
+namespace {
+// Per-call scale block of the dynamic forward: {g, g_w, alpha', amax} at 0,
+// the amax pass's per-block maxima from byte 256.
+constexpr size_t kDynScaleBytes = 8192;
+}  // namespace
+}  // namespace svdq
+extern "C" {
+
+svdq_status svdq_dynamic_workspace_size(int M, int N, int K, int r, size_t* bytes) {
+  size_t base = 0;
+  svdq_status s = check_layer_shape(N, K, r);
+  if (s != SVDQ_OK) return s;
+  if ((s = svdq_forward_workspace_size(M, K, r, &base)) != SVDQ_OK) return s;
+  if (!bytes) return SVDQ_ERR_INVALID_ARG;
+  *bytes = base + kDynScaleBytes + round_up(static_cast<size_t>(N) * r * 2 * 2, 256);
+  return SVDQ_OK;
+}
+
+svdq_status svdq_linear_forward_dynamic(int M, int N, int K, int r, const void* X, int64_t ldx, const void* w_codes,
+                                        const void* w_scales, const float* gscale, const void* l1t, const void* l2s,
+                                        const float* inv_smooth, const void* bias, void* Y, int64_t ldy,
+                                        void* workspace, size_t workspace_bytes, void* stream) {
+  if (M < 0) return SVDQ_ERR_INVALID_ARG;
+  svdq_status s = check_layer_shape(N, K, r);
+  if (s != SVDQ_OK) return s;
+  if (ldx < K || ldx % 8 != 0 || ldy < N || ldy % 8 != 0) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+  if (M == 0) return SVDQ_OK;
+  if (!workspace || !gscale || !l2s || !X || !l1t) return SVDQ_ERR_INVALID_ARG;
+  size_t need = 0, base = 0;
+  svdq_dynamic_workspace_size(M, N, K, r, &need);
+  svdq_forward_workspace_size(M, K, r, &base);
+  if (workspace_bytes < need) return SVDQ_ERR_WORKSPACE;
+  if (!aligned16(workspace) || !aligned16(gscale) || !aligned16(l2s) || !aligned16(X) || !aligned16(l1t) ||
+      (inv_smooth && !aligned16(inv_smooth)))
+    return SVDQ_ERR_MISALIGNED;
+  DeviceInfo di;
+  if ((s = current_device(nullptr, &di)) != SVDQ_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  float* gs = reinterpret_cast<float*>(ws + base);
+  float* partial = reinterpret_cast<float*>(ws + base + 256);
+  __nv_bfloat16* l2s_d = reinterpret_cast<__nv_bfloat16*>(ws + base + kDynScaleBytes);
+  // amax|X^| of this call as per-block maxima, then the per-call scales and
+  // l2 planes, then the layer; each kernel after the first is a programmatic
+  // dependent of the one before (it waits for it before reading its output).
+  const int nparts = launch_act_amax(static_cast<const __nv_bfloat16*>(X), ldx, M, K, inv_smooth, nullptr, partial,
+                                     di.sm_count, st);
+  const int64_t total = static_cast<int64_t>(N) * r;
+  const int64_t sblocks = (total + 255) / 256 < 2 * di.sm_count ? (total + 255) / 256 : 2 * di.sm_count;
+  {
+    PdlLaunch pl(static_cast<int>(sblocks), 256, 0, st);
+    cudaLaunchKernelEx(&pl.cfg, dynamic_scale_kernel, static_cast<const float*>(gscale),
+                       static_cast<const float*>(partial), nparts, gs, static_cast<const __nv_bfloat16*>(l2s), l2s_d,
+                       total);
+  }
+  if ((s = launch_status()) != SVDQ_OK) return s;
+  size_t c = 0, sc = 0, x = 0;
+  svdq_act_sizes(M, K, r, &c, &sc, &x);
+  uint8_t* a_codes = ws;
+  uint8_t* a_scales = ws + round_up(c, 256);
+  uint8_t* xl1 = a_scales + round_up(sc, 256);
+  s = quantize_dispatch(M, K, r, X, ldx, gs, l1t, inv_smooth, a_codes, a_scales, xl1, st, di.sm_count, true);
+  if (s != SVDQ_OK) return s;
+  return svdq_w4a4_gemm(M, N, K, r, a_codes, a_scales, xl1, w_codes, w_scales, gs, l2s_d, bias, Y, ldy, stream);
 }
 
 svdq_status svdq_read_device_error(int* code, int clear) {
