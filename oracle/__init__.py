@@ -1,4 +1,5 @@
-"""CPU oracle for the SVDQuant W4A4 (NVFP4) linear layer.
+"""CPU oracle for the SVDQuant W4A4 (NVFP4) linear layer and the AWQ W4A16
+weight-only layer used beside it.
 
 TEST INFRASTRUCTURE ONLY. A plain, slow, float64 restatement of what the
 layer computes, used to check the CUDA library. Only the test suite, the
@@ -11,4 +12,4 @@ than itself: the OCP FP8 anchor values and torch's float8_e4m3fn conversion,
 the E2M1 grid, brute-force nearest-value searches, the Eckart-Young theorem,
 the r = 0 and r = full special cases, and a pure-Python 16x16 triple loop.
 """
-from . import nvfp4, svdq  # noqa: F401
+from . import awq, nvfp4, svdq  # noqa: F401
