@@ -359,6 +359,30 @@ def run_ours(args, spec):
     variants = {"note": "public-API forward, same rotating inputs, one event pair around all steps",
                 "steps": n_q, "plain_ms_per_step": plain_ms,
                 "smoothed_ms_per_step": smooth_ms, "dynamic_scale_ms_per_step": dyn_ms}
+    del pws_s, pw_s
+
+    # AWQ W4A16 (the weight-only family for modulation layers): FLUX adaLN
+    # modulation, K = 3072 -> N = 18432, M = 1 and 2 rows, six rotating copies
+    # of the packed weight (larger than L2), against the HBM roofline.
+    awq_out = {}
+    Xm1, Wm, bm = workloads.modulation_layer(1)
+    Wmd = Wm.to(dev)
+    aws = [svdq.svdq_awq_pack(Wmd) for _ in range(n_sets)]
+    del Wmd
+    bmd = bm.to(dev)
+    for Mm in (1, 2):
+        Xm = workloads.modulation_layer(Mm)[0].to(dev)
+        Ym = torch.empty((Mm, Wm.shape[0]), dtype=torch.bfloat16, device=dev)
+        t_ms = timed(lambda i: svdq.svdq_awq_gemv(Xm, aws[i % n_sets], bmd, out=Ym))
+        Nm, Km = Wm.shape
+        nbytes = Nm * Km // 2 + Nm * (Km // 64) * 3 + Mm * Km * 2 + Mm * Nm * 2 + Nm * 2
+        gbs = nbytes / (t_ms * 1e-3) / 1e9
+        awq_out[f"M{Mm}"] = {"ms": t_ms, "algorithmic_bytes": nbytes, "gbs": gbs,
+                             "frac_of_hbm": gbs / _peaks()[0]["hbm_gbs"]}
+    del aws
+    if svdq.svdq_read_device_error() != 0:
+        raise RuntimeError("device error during the AWQ timing")
+    variants["awq_w4a16_modulation_3072x18432"] = awq_out
 
     peaks, kind = _peaks()
     gemm_name = _gemm_kernel_name(M, N)

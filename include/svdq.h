@@ -284,6 +284,41 @@ svdq_status svdq_linear_forward_noalloc(int M, int N, int K, int r, const void* 
                                         const void* l1t, const void* l2s, const float* inv_smooth,
                                         const void* bias, void* Y, int64_t ldy, void* stream);
 
+/* ------------------------------------------------------------ AWQ W4A16 */
+/* The second kernel family of the blog's section "Introducing Nunchaku Lite":
+ * awq_w4a16, 4-bit weights with 16-bit activations for the adaptive-
+ * normalisation and modulation projections (memory-bound, precision-
+ * sensitive); section "Native loading in Diffusers": int4, group size 64,
+ * bfloat16. Layout of a packed N x K weight (K % 64 == 0):
+ *   codes  u8 [N][K/2], element 2j in the low nibble of byte j
+ *   scales bf16 [N][K/64], zeros u8 [N][K/64] (one per row and 64-group)
+ * Sizes in bytes: */
+svdq_status svdq_awq_sizes(int N, int K, size_t* codes_bytes, size_t* scales_bytes, size_t* zeros_bytes);
+
+/* Quantise W bf16 [N][K] (load time). Per row and 64-group of w = fp32(W *
+ * act_scale[k]) (or W), the AWQ reference pseudo-quantiser's rule, every step
+ * one correctly rounded fp32 operation:
+ *   s = bf16(fp32(max(fp32(max w - min w), 1e-5) / 15)),
+ *   z = clamp(rne(fp32(-min w / s)), 0, 15),
+ *   q = clamp(rne(fp32(w / s)) + z, 0, 15).
+ * act_scale: device float [K] activation-aware factors a_k (positive, finite),
+ * or NULL; with it inv_act [K] receives fp32(1 / a_k) (NULL exactly when
+ * act_scale is NULL; both 16-byte aligned). W and codes 16-byte aligned,
+ * scales 2-byte aligned. Deterministic. */
+svdq_status svdq_awq_pack(int N, int K, const void* W, const float* act_scale, void* codes, void* scales,
+                          void* zeros, float* inv_act, void* stream);
+
+/* Y[m,n] = bf16( sum_k x^[m,k] (q[n,k] - z[n,g]) s[n,g] + b[n] ), g = k / 64,
+ * x^ = fp32(x * inv_act[k]) (or x); the dequantised weight is exact in fp32 and
+ * the sum is accumulated in fp32. X bf16 [M][ldx] (ldx % 8 == 0, 16-byte
+ * aligned), Y bf16 [M][ldy], bias bf16 [N] or NULL, inv_act float [K] or
+ * NULL. Any M >= 0 (rows are processed eight at a time); K * 4 <= 96 KB. The
+ * layer is HBM-bound for the few rows a modulation projection has: each warp
+ * streams one weight row, the activations sit in shared memory. */
+svdq_status svdq_awq_gemv(int M, int N, int K, const void* X, int64_t ldx, const void* codes, const void* scales,
+                          const void* zeros, const float* inv_act, const void* bias, void* Y, int64_t ldy,
+                          void* stream);
+
 /* ------------------------------------------------------------ errors */
 /* Reads (and, if clear != 0, resets) the device error word of the current
  * device: 0 or an svdq_status recorded by a kernel (e.g. SVDQ_ERR_TIMEOUT).

@@ -147,6 +147,20 @@ def test_dynamic_forward_sizes_and_validation(L):
                                          128, None, 0, None) == 0          # M == 0: no-op
 
 
+def test_awq_sizes_and_validation(L):
+    p = ctypes.c_void_p(0x10000)
+    odd = ctypes.c_void_p(0x10008)
+    assert _lib.svdq_awq_sizes(100, 576) == (100 * 288, 100 * 9 * 2, 100 * 9)
+    with pytest.raises(_lib.SvdqError):
+        _lib.svdq_awq_sizes(100, 500)                                  # K % 64
+    assert L.svdq_awq_pack(100, 576, p, p, p, p, p, None, None) == 1    # act_scale without inv_act
+    assert L.svdq_awq_pack(100, 576, odd, None, p, p, p, None, None) == 3
+    assert L.svdq_awq_gemv(2, 100, 576, p, 500, p, p, p, None, None, p, 100, None) == 2    # ldx < K
+    assert L.svdq_awq_gemv(2, 100, 576, odd, 576, p, p, p, None, None, p, 100, None) == 3
+    assert L.svdq_awq_gemv(2, 100, 32768, p, 32768, p, p, p, None, None, p, 100, None) == 2  # K * 4 > 96 KB
+    assert L.svdq_awq_gemv(0, 100, 576, None, 576, None, None, None, None, None, None, 100, None) == 0
+
+
 def test_qkv_forward_validation(L):
     p = ctypes.c_void_p(0x10000)
     odd = ctypes.c_void_p(0x10008)

@@ -1,0 +1,121 @@
+"""GPU parity of the AWQ W4A16 layer (svdq_awq_pack, svdq_awq_gemv) against
+oracle/awq.py.
+
+Bars: codes, scales, zero points and inv_act bit-exact; Y within half a bf16
+ulp of its own value plus the fp32 summation bound 2 K 2^-24 sum_k |x^ w'| of
+the float64 result (the dequantised weight is exact in fp32, only the order
+of the fp32 accumulation differs), and the layer bars (relative Frobenius
+<= 1e-3 against the bf16-rounded oracle output, max |err| <= 2e-2 row RMS).
+"""
+import numpy as np
+import pytest
+import torch
+
+import workloads
+from oracle import awq
+from tests import layouts
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from w4a4_rank_corrected_svdq_b200 import _lib, build
+    build.build()
+    return _lib
+
+
+def _np(t):
+    return t.detach().to(torch.float64).cpu().numpy()
+
+
+def _act(K, seed=1):
+    return np.random.default_rng(seed).uniform(0.5, 2.0, K).astype(np.float32)
+
+
+def _check_pack(aw, ref, N, K):
+    assert np.array_equal(layouts.unpack_codes(aw.codes.cpu().numpy(), N, K), ref.codes)
+    assert np.array_equal(_np(aw.scales).astype(np.float32), ref.scales)
+    assert np.array_equal(aw.zeros.cpu().numpy(), ref.zeros)
+    if ref.inv_act is not None:
+        assert np.array_equal(aw.inv_act.cpu().numpy(), ref.inv_act)
+
+
+def _check_y(Y, X, ref, bias):
+    y = _np(Y)
+    fwd = awq.forward(X, ref, bias)
+    x = X.astype(np.float32).astype(np.float64)
+    if ref.inv_act is not None:
+        x = (X.astype(np.float32) * ref.inv_act[None, :]).astype(np.float64)
+    absum = np.abs(x) @ np.abs(awq.dequantize(ref)).T
+    K = X.shape[1]
+    half_ulp = np.ldexp(1.0, np.frexp(np.abs(y))[1] - 9)
+    bound = half_ulp + 2.0 * K * 2.0 ** -24 * absum + 1e-30
+    err = np.abs(y - fwd.y64)
+    assert np.all(err <= bound), f"{np.max(err / bound):.2f} x bound"
+    assert awq_rel(y, fwd.y_ref) <= 1e-3
+    rms = np.sqrt(np.mean(fwd.y64 ** 2, axis=1, keepdims=True))
+    assert np.max(np.abs(y - fwd.y64) / rms) <= 2e-2
+
+
+def awq_rel(a, b):
+    return float(np.linalg.norm(a - b) / np.linalg.norm(b))
+
+
+@pytest.mark.parametrize("N,K,act", [(128, 256, False), (100, 64, True), (1000, 3072, True), (37, 576, False)])
+def test_pack_bitexact(lib, N, K, act):
+    X, W, b = workloads.modulation_layer(1, K, N, seed=N)
+    a = _act(K) if act else None
+    aw = lib.svdq_awq_pack(W.cuda(), None if a is None else torch.from_numpy(a).cuda())
+    torch.cuda.synchronize()
+    assert lib.svdq_read_device_error() == 0
+    _check_pack(aw, awq.quantize(_np(W), a), N, K)
+
+
+@pytest.mark.parametrize("M,N,K,act,bias", [(1, 1000, 3072, False, True), (2, 257, 576, True, True),
+                                            (3, 128, 64, False, False), (8, 640, 1024, True, True),
+                                            (13, 300, 3072, False, True), (5, 96, 12288, True, False)])
+def test_gemv_parity(lib, M, N, K, act, bias):
+    X, W, b = workloads.modulation_layer(M, K, N, seed=M + N)
+    a = _act(K, seed=2) if act else None
+    aw = lib.svdq_awq_pack(W.cuda(), None if a is None else torch.from_numpy(a).cuda())
+    Y = lib.svdq_awq_gemv(X.cuda(), aw, b.cuda() if bias else None)
+    torch.cuda.synchronize()
+    assert lib.svdq_read_device_error() == 0
+    ref = awq.quantize(_np(W), a)
+    _check_y(Y, _np(X), ref, _np(b) if bias else None)
+
+
+def test_gemv_strided_input_and_zero_rows(lib):
+    M, N, K = 4, 256, 512
+    X, W, b = workloads.modulation_layer(M, K, N, seed=3)
+    X = X.clone()
+    X[1] = 0
+    big = torch.zeros((M, K + 64), dtype=torch.bfloat16)
+    big[:, :K] = X
+    aw = lib.svdq_awq_pack(W.cuda())
+    Y = lib.svdq_awq_gemv(big.cuda()[:, :K], aw, b.cuda())
+    torch.cuda.synchronize()
+    y = _np(Y)
+    assert np.array_equal(y[1], _np(b))          # a zero row gives the bias exactly
+    _check_y(Y, _np(X), awq.quantize(_np(W)), _np(b))
+
+
+@pytest.mark.parametrize("M", [1, 2])
+def test_modulation_full_size_sampled(lib, M):
+    """FLUX adaLN modulation (K = 3072, N = 18432) at the size the bench times;
+    codes / scales / zeros and outputs of 512 sampled rows of W."""
+    X, W, b = workloads.modulation_layer(M)
+    aw = lib.svdq_awq_pack(W.cuda())
+    Y = lib.svdq_awq_gemv(X.cuda(), aw, b.cuda())
+    torch.cuda.synchronize()
+    assert lib.svdq_read_device_error() == 0
+    N, K = W.shape
+    rows = np.unique(np.concatenate([[0, N - 1], np.random.default_rng(8).choice(N, 510, replace=False)]))
+    Wn = _np(W)[rows]
+    ref = awq.quantize(Wn)
+    codes = layouts.unpack_codes(aw.codes.cpu().numpy(), N, K)[rows]
+    assert np.array_equal(codes, ref.codes)
+    assert np.array_equal(_np(aw.scales)[rows].astype(np.float32), ref.scales)
+    assert np.array_equal(aw.zeros.cpu().numpy()[rows], ref.zeros)
+    _check_y(Y[:, torch.from_numpy(rows).cuda()], _np(X), ref, _np(b)[rows])

@@ -6,12 +6,16 @@ Inference to Diffusers"). The work runs in hand-written CUDA kernels behind
 the C ABI of include/svdq.h; this package is its ctypes binding.
 """
 from ._lib import (  # noqa: F401
+    AwqWeight,
     PackedWeight,
     QuantAct,
     SvdqError,
     lib,
     svdq_act_global_scale,
     svdq_act_sizes,
+    svdq_awq_gemv,
+    svdq_awq_pack,
+    svdq_awq_sizes,
     svdq_dynamic_workspace_size,
     svdq_forward_workspace_size,
     svdq_linear_forward,

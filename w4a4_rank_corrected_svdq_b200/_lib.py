@@ -44,6 +44,9 @@ SIGNATURES = {
     "svdq_dynamic_workspace_size": (_i, [_i, _i, _i, _i, _psz]),
     "svdq_linear_forward_dynamic": (_i, [_i, _i, _i, _i, _p, _i64, _p, _p, _p, _p, _p, _p, _p, _p, _i64, _p, _sz,
                                          _p]),
+    "svdq_awq_sizes": (_i, [_i, _i, _psz, _psz, _psz]),
+    "svdq_awq_pack": (_i, [_i, _i, _p, _p, _p, _p, _p, _p, _p]),
+    "svdq_awq_gemv": (_i, [_i, _i, _i, _p, _i64, _p, _p, _p, _p, _p, _p, _i64, _p]),
     "svdq_lowrank_workspace_size": (_i, [_i, _i, _i, _psz]),
     "svdq_lowrank_init": (_i, [_i, _i, _i, _p, _p, _p, _p, _p, ctypes.c_ulonglong, _i, _p, _sz, _p]),
 }
@@ -356,6 +359,58 @@ def svdq_linear_forward_dynamic(X: torch.Tensor, pw: PackedWeight, bias: torch.T
     _check("svdq_linear_forward_dynamic", lib().svdq_linear_forward_dynamic(
         M, N, K, r, _ptr(X), ldx, _ptr(pw.codes), _ptr(pw.scales), _ptr(pw.gscale), _ptr(pw.l1t),
         _ptr(pw.l2s), _ptr(pw.inv_smooth), _ptr(bias), _ptr(Y), ldy, _ptr(ws), ws.numel(), _stream(X)))
+    return Y
+
+
+# ------------------------------------------------------------------ AWQ W4A16
+def svdq_awq_sizes(N: int, K: int):
+    a, b, c = (ctypes.c_size_t() for _ in range(3))
+    _check("svdq_awq_sizes", lib().svdq_awq_sizes(N, K, *(ctypes.byref(x) for x in (a, b, c))))
+    return a.value, b.value, c.value
+
+
+class AwqWeight:
+    """Device buffers of one INT4 group-64 weight (filled by svdq_awq_pack):
+    codes u8 [N, K/2], scales bf16 [N, K/64], zeros u8 [N, K/64], inv_act [K] or None."""
+
+    def __init__(self, N: int, K: int, device):
+        cb, sb, zb = svdq_awq_sizes(N, K)
+        self.N, self.K = N, K
+        self.codes = torch.empty(cb, dtype=torch.uint8, device=device)
+        self.scales = torch.empty((N, K // 64), dtype=torch.bfloat16, device=device)
+        self.zeros = torch.empty((N, K // 64), dtype=torch.uint8, device=device)
+        self.inv_act = None
+
+
+def svdq_awq_pack(W: torch.Tensor, act_scale: torch.Tensor | None = None, out: AwqWeight | None = None) -> AwqWeight:
+    """INT4 group-64 quantisation of W [N, K] bf16 (act_scale: activation-aware factors [K] or None)."""
+    _dev(W, "W", torch.bfloat16)
+    if W.dim() != 2 or not W.is_contiguous():
+        raise ValueError("W must be a contiguous [N, K] tensor")
+    N, K = W.shape
+    _smooth_vec(act_scale, K, "act_scale")
+    aw = out if out is not None else AwqWeight(N, K, W.device)
+    aw.inv_act = None if act_scale is None else torch.empty(K, dtype=torch.float32, device=W.device)
+    _check("svdq_awq_pack", lib().svdq_awq_pack(N, K, _ptr(W), _ptr(act_scale), _ptr(aw.codes), _ptr(aw.scales),
+                                                _ptr(aw.zeros), _ptr(aw.inv_act), _stream(W)))
+    return aw
+
+
+def svdq_awq_gemv(X: torch.Tensor, aw: AwqWeight, bias: torch.Tensor | None = None,
+                  out: torch.Tensor | None = None) -> torch.Tensor:
+    """Y = X^ . W'^T + b for an AWQ W4A16 weight (X bf16 [M, K])."""
+    _dev(X, "X", torch.bfloat16)
+    M, K = X.shape
+    N = aw.N
+    ldx = _rows(X, "X", K)
+    if bias is not None:
+        _dev(bias, "bias", torch.bfloat16, (N,))
+    Y = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=X.device)
+    _dev(Y, "Y", torch.bfloat16)
+    ldy = _rows(Y, "Y", N)
+    _check("svdq_awq_gemv", lib().svdq_awq_gemv(M, N, K, _ptr(X), ldx, _ptr(aw.codes), _ptr(aw.scales),
+                                                _ptr(aw.zeros), _ptr(aw.inv_act), _ptr(bias), _ptr(Y), ldy,
+                                                _stream(X)))
     return Y
 
 

@@ -16,6 +16,7 @@
 #include "lowrank_svd.cuh"
 #include "pack_weight.cuh"
 #include "smooth.cuh"
+#include "awq_w4a16.cuh"
 #include "quantize_act.cuh"
 
 namespace svdq {
@@ -1129,6 +1130,100 @@ svdq_status svdq_linear_forward_dynamic(int M, int N, int K, int r, const void* 
   s = quantize_dispatch(M, K, r, X, ldx, gs, l1t, inv_smooth, a_codes, a_scales, xl1, st, di.sm_count, true);
   if (s != SVDQ_OK) return s;
   return svdq_w4a4_gemm(M, N, K, r, a_codes, a_scales, xl1, w_codes, w_scales, gs, l2s_d, bias, Y, ldy, stream);
+}
+
+svdq_status svdq_awq_sizes(int N, int K, size_t* codes_bytes, size_t* scales_bytes, size_t* zeros_bytes) {
+  if (N <= 0 || K <= 0 || !codes_bytes || !scales_bytes || !zeros_bytes) return SVDQ_ERR_INVALID_ARG;
+  if (K % kAwqGroup != 0) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+  *codes_bytes = static_cast<size_t>(N) * (K / 2);
+  *scales_bytes = static_cast<size_t>(N) * (K / kAwqGroup) * 2;
+  *zeros_bytes = static_cast<size_t>(N) * (K / kAwqGroup);
+  return SVDQ_OK;
+}
+
+svdq_status svdq_awq_pack(int N, int K, const void* W, const float* act_scale, void* codes, void* scales,
+                          void* zeros, float* inv_act, void* stream) {
+  if (N <= 0 || K <= 0 || !W || !codes || !scales || !zeros) return SVDQ_ERR_INVALID_ARG;
+  if ((act_scale == nullptr) != (inv_act == nullptr)) return SVDQ_ERR_INVALID_ARG;
+  if (K % kAwqGroup != 0) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(W) || !aligned16(codes) || (reinterpret_cast<uintptr_t>(scales) & 1u) ||
+      (act_scale && (!aligned16(act_scale) || !aligned16(inv_act))))
+    return SVDQ_ERR_MISALIGNED;
+  svdq_status s;
+  DeviceInfo di;
+  if ((s = current_device(nullptr, &di)) != SVDQ_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (act_scale != nullptr) inv_smooth_kernel<<<(K + 255) / 256, 256, 0, st>>>(act_scale, inv_act, K);
+  const int64_t groups = static_cast<int64_t>(N) * (K / kAwqGroup);
+  awq_pack_kernel<<<static_cast<int>((groups + kAwqThreads - 1) / kAwqThreads), kAwqThreads, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(W), N, K, act_scale, static_cast<uint8_t*>(codes),
+      static_cast<__nv_bfloat16*>(scales), static_cast<uint8_t*>(zeros));
+  return launch_status();
+}
+
+}  // extern "C"
+namespace svdq {
+namespace {
+constexpr int kAwqSmemCap = 96 * 1024;  // activation rows staged per CTA: at most 96 KB
+
+template <int MT>
+svdq_status launch_awq_gemv(int M, int N, int K, const __nv_bfloat16* X, int64_t ldx, const uint8_t* codes,
+                            const __nv_bfloat16* scales, const uint8_t* zeros, const float* inv_act,
+                            const __nv_bfloat16* bias, __nv_bfloat16* Y, int64_t ldy, int sm_count,
+                            cudaStream_t st) {
+  const int smem = MT * K * 4;
+  static std::atomic<uint64_t> attr_done{0};  // set once to the cap, which covers every K accepted
+  ensure_smem_attr(awq_gemv_kernel<MT>, kAwqSmemCap, attr_done);
+  int per_sm = (227 * 1024) / (smem + 1024);
+  if (per_sm > 2048 / kAwqThreads) per_sm = 2048 / kAwqThreads;
+  if (per_sm < 1) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+  int blocks = (N + kAwqThreads / 32 - 1) / (kAwqThreads / 32);
+  if (blocks > per_sm * sm_count) blocks = per_sm * sm_count;
+  for (int m0 = 0; m0 < M; m0 += MT) {
+    awq_gemv_kernel<MT><<<blocks, kAwqThreads, smem, st>>>(M - m0, N, K, X + static_cast<int64_t>(m0) * ldx, ldx,
+                                                            codes, scales, zeros, inv_act, bias,
+                                                            Y + static_cast<int64_t>(m0) * ldy, ldy);
+    const svdq_status s = launch_status();
+    if (s != SVDQ_OK) return s;
+  }
+  return SVDQ_OK;
+}
+}  // namespace
+}  // namespace svdq
+extern "C" {
+
+svdq_status svdq_awq_gemv(int M, int N, int K, const void* X, int64_t ldx, const void* codes, const void* scales,
+                          const void* zeros, const float* inv_act, const void* bias, void* Y, int64_t ldy,
+                          void* stream) {
+  if (M < 0 || N <= 0 || K <= 0) return SVDQ_ERR_INVALID_ARG;
+  if (K % kAwqGroup != 0 || ldx < K || ldx % 8 != 0 || ldy < N) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+  if (M == 0) return SVDQ_OK;
+  if (!X || !codes || !scales || !zeros || !Y) return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(codes) || (reinterpret_cast<uintptr_t>(scales) & 1u) ||
+      (reinterpret_cast<uintptr_t>(Y) & 1u) || (bias && (reinterpret_cast<uintptr_t>(bias) & 1u)) ||
+      (inv_act && (reinterpret_cast<uintptr_t>(inv_act) & 3u)))
+    return SVDQ_ERR_MISALIGNED;
+  if (K * 4 > kAwqSmemCap) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+  svdq_status s;
+  DeviceInfo di;
+  if ((s = current_device(nullptr, &di)) != SVDQ_OK) return s;
+  const auto* x = static_cast<const __nv_bfloat16*>(X);
+  const auto* c = static_cast<const uint8_t*>(codes);
+  const auto* sc = static_cast<const __nv_bfloat16*>(scales);
+  const auto* z = static_cast<const uint8_t*>(zeros);
+  const auto* b = static_cast<const __nv_bfloat16*>(bias);
+  auto* y = static_cast<__nv_bfloat16*>(Y);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // rows per launch: the smallest power of two covering M (at most 8) whose
+  // staged activations fit the cap
+  int mt = 1;
+  while (mt < 8 && mt < M && 2 * mt * K * 4 <= kAwqSmemCap) mt *= 2;
+  switch (mt) {
+    case 1: return launch_awq_gemv<1>(M, N, K, x, ldx, c, sc, z, inv_act, b, y, ldy, di.sm_count, st);
+    case 2: return launch_awq_gemv<2>(M, N, K, x, ldx, c, sc, z, inv_act, b, y, ldy, di.sm_count, st);
+    case 4: return launch_awq_gemv<4>(M, N, K, x, ldx, c, sc, z, inv_act, b, y, ldy, di.sm_count, st);
+    default: return launch_awq_gemv<8>(M, N, K, x, ldx, c, sc, z, inv_act, b, y, ldy, di.sm_count, st);
+  }
 }
 
 svdq_status svdq_read_device_error(int* code, int clear) {

@@ -175,3 +175,15 @@ def rope_tables(M: int, head_dim: int = 128, base: float = 10000.0, seed: int = 
     freq = base ** (-np.arange(0, head_dim, 2, dtype=np.float64) / head_dim)
     ang = pos[:, None] * freq[None, :]
     return np.cos(ang).astype(np.float32), np.sin(ang).astype(np.float32)
+
+def modulation_layer(M: int = 1, K: int = 3072, N: int = 6 * 3072, seed: int = 0):
+    """An adaptive-normalisation modulation projection (the AWQ W4A16 layers of
+    the blog's section "Introducing Nunchaku Lite"): FLUX's adaLN modulation
+    maps the conditioning vector (K = 3072) to six 3072-wide shift / scale /
+    gate vectors (N = 18432), one row per sample (M = batch). Returns (X, W, b):
+    X ~ N(0, 1), W ~ N(0, 0.02^2), b ~ N(0, 0.01^2), bf16, drawn in that order."""
+    rng = np.random.default_rng([7, M, K, N, seed])
+    X = rng.standard_normal((M, K), dtype=np.float32)
+    W = rng.standard_normal((N, K), dtype=np.float32) * np.float32(0.02)
+    b = rng.standard_normal(N, dtype=np.float32) * np.float32(0.01)
+    return _to_bf16(X), _to_bf16(W), _to_bf16(b)
