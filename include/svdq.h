@@ -311,8 +311,8 @@ svdq_status svdq_awq_pack(int N, int K, const void* W, const float* act_scale, v
 /* Y[m,n] = bf16( sum_k x^[m,k] (q[n,k] - z[n,g]) s[n,g] + b[n] ), g = k / 64,
  * x^ = fp32(x * inv_act[k]) (or x); the dequantised weight is exact in fp32 and
  * the sum is accumulated in fp32. X bf16 [M][ldx] (ldx % 8 == 0, 16-byte
- * aligned), Y bf16 [M][ldy], bias bf16 [N] or NULL, inv_act float [K] or
- * NULL. Any M >= 0 (rows are processed eight at a time); K * 4 <= 96 KB. The
+ * aligned), Y bf16 [M][ldy], bias bf16 [N] or NULL, inv_act float [K]
+ * (16-byte aligned) or NULL. Any M >= 0 (rows are processed eight at a time); K * 4 <= 96 KB. The
  * layer is HBM-bound for the few rows a modulation projection has: each warp
  * streams one weight row, the activations sit in shared memory. */
 svdq_status svdq_awq_gemv(int M, int N, int K, const void* X, int64_t ldx, const void* codes, const void* scales,

@@ -21,8 +21,8 @@
 // The layer reads N K / 2 bytes of codes for M K multiply-adds per row block:
 // for the few activation rows of a modulation projection it is bound by HBM,
 // not by the tensor cores, so it runs on the CUDA cores: each warp streams one
-// weight row as coalesced 4-byte code words while the activations sit in
-// shared memory.
+// weight row with coalesced 16-byte loads while the activations sit in shared
+// memory.
 #pragma once
 
 #include "nvfp4.cuh"
@@ -31,6 +31,7 @@ namespace svdq {
 
 constexpr int kAwqGroup = 64;
 constexpr int kAwqThreads = 256;
+constexpr int kAwqRows = 4;  // weight rows per warp pass of the GEMV
 
 // One thread per (row, group): codes (element 2j in the low nibble of byte j),
 // bf16 scale, u8 zero point.
@@ -80,16 +81,16 @@ __global__ void __launch_bounds__(kAwqThreads) awq_pack_kernel(const __nv_bfloat
   zeros[t] = static_cast<uint8_t>(z);
 }
 
-// Y (the first min(M, MT) rows of X) = X^ . W'^T + b. Shared memory holds X^
-// as fp32 in two planes of float4 per 8-element group (elements 0-3 and 4-7),
-// so that lanes reading consecutive groups touch consecutive 16-byte words.
-// Each warp takes output rows n = warp_id, warp_id + total_warps, ...; lane l
-// takes the row's code words (8 codes, all of one 64-group) l, l + 32, ...:
-// coalesced 128-byte loads per warp. Per word the integers q - z are formed
-// exactly (2^23 + q from one byte permute, minus the exact 2^23 + z), the
-// eight products x (q - z) are summed as two fp32 pair partials and scaled by
-// s once; the row keeps two fp32 partial sums (even and odd elements), added
-// at the end. Packed f32x2 arithmetic throughout.
+// Y (the first min(M, MT) rows of X) = X^ . W'^T + b.
+// Shared memory holds X^ as fp32, per row m and 32-element chunk c as eight
+// float4 (elements 4f..4f+3), float4 f stored at slot f ^ (c & 7): lanes
+// reading consecutive chunks then touch eight different 16-byte bank groups.
+// Each warp takes kAwqRows output rows per pass (passes strided by the number
+// of warps); lane l takes the rows' chunks l, l + 32, ... (32 codes = 16 bytes,
+// half a 64-group, so one scale and zero point each). Per
+// 8-code word the integers q - z are formed exactly (2^23 + q from one byte
+// permute, minus the exact 2^23 + z), the products x (q - z) are summed as
+// fp32 pairs over the chunk and scaled by s once. Packed f32x2 arithmetic.
 template <int MT>
 __global__ void __launch_bounds__(kAwqThreads) awq_gemv_kernel(int M, int N, int K,
                                                                const __nv_bfloat16* __restrict__ X, int64_t ldx,
@@ -99,74 +100,109 @@ __global__ void __launch_bounds__(kAwqThreads) awq_gemv_kernel(int M, int N, int
                                                                const float* __restrict__ inv_act,
                                                                const __nv_bfloat16* __restrict__ bias,
                                                                __nv_bfloat16* __restrict__ Y, int64_t ldy) {
-  extern __shared__ float4 xs4[];  // [MT][2][K/8]
+  extern __shared__ float4 xs4[];  // [MT][K/32][8], swizzled
   const int rows = M < MT ? M : MT;
-  const int K8 = K / 8;
-  for (int i = threadIdx.x; i < MT * K8; i += blockDim.x) {
-    const int m = i / K8, j = i % K8;
-    float f[8];
+  const int C = K / 32;
+  for (int i = threadIdx.x; i < MT * (K / 4); i += blockDim.x) {
+    const int m = i / (K / 4), q4 = i % (K / 4);  // float4 q4 of row m: elements 4 q4 .. 4 q4 + 3
+    float4 f = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
     if (m < rows) {
-      bf16x8_to_f32(ldg_nc_v4(X + static_cast<int64_t>(m) * ldx + 8 * j), f);
+      const __nv_bfloat16* src = X + static_cast<int64_t>(m) * ldx + 4 * q4;
+      const uint2 raw = *reinterpret_cast<const uint2*>(src);
+      f = make_float4(__uint_as_float(raw.x << 16), __uint_as_float(raw.x & 0xFFFF0000u),
+                      __uint_as_float(raw.y << 16), __uint_as_float(raw.y & 0xFFFF0000u));
       if (inv_act != nullptr) {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) f[e] = __fmul_rn(f[e], inv_act[8 * j + e]);
+        const float4 iv = *reinterpret_cast<const float4*>(inv_act + 4 * q4);
+        f = make_float4(__fmul_rn(f.x, iv.x), __fmul_rn(f.y, iv.y), __fmul_rn(f.z, iv.z), __fmul_rn(f.w, iv.w));
       }
-    } else {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) f[e] = 0.0f;
     }
-    xs4[(2 * m) * K8 + j] = make_float4(f[0], f[1], f[2], f[3]);
-    xs4[(2 * m + 1) * K8 + j] = make_float4(f[4], f[5], f[6], f[7]);
+    const int c = q4 >> 3, fi = q4 & 7;
+    xs4[(m * C + c) * 8 + (fi ^ (c & 7))] = f;
   }
   __syncthreads();
   const int lane = threadIdx.x & 31;
   const int warps = static_cast<int>(gridDim.x) * (kAwqThreads / 32);
   const int G = K / kAwqGroup;
-  for (int n = blockIdx.x * (kAwqThreads / 32) + (threadIdx.x >> 5); n < N; n += warps) {
-    const uint32_t* crow = reinterpret_cast<const uint32_t*>(codes + static_cast<int64_t>(n) * (K / 2));
-    const __nv_bfloat16* srow = scales + static_cast<int64_t>(n) * G;
-    const uint8_t* zrow = zeros + static_cast<int64_t>(n) * G;
-    float2 acc[MT];
+  // kAwqRows weight rows per warp pass: each X^ value read from shared memory
+  // serves all of them (shared-memory bandwidth, not HBM, bounds a pass over
+  // one row at a time).
+  for (int n0 = (blockIdx.x * (kAwqThreads / 32) + (threadIdx.x >> 5)) * kAwqRows; n0 < N;
+       n0 += warps * kAwqRows) {
+    float2 acc[kAwqRows][MT];
 #pragma unroll
-    for (int m = 0; m < MT; ++m) acc[m] = make_float2(0.0f, 0.0f);
-#pragma unroll 4
-    for (int j = lane; j < K8; j += 32) {
-      const uint32_t v = __ldg(crow + j);
-      const int g = j >> 3;
-      const float s = __bfloat162float(srow[g]);
-      const float zf = __fadd_rn(8388608.0f, static_cast<float>(zrow[g]));  // 2^23 + z, exact
-      const float2 s2 = make_float2(s, s), nz2 = make_float2(-zf, -zf);
-      const uint32_t lo = v & 0x0F0F0F0Fu, hi = (v >> 4) & 0x0F0F0F0Fu;
-      float2 d[4];  // (q - z) of elements (2b, 2b + 1): the low and high nibble of byte b
+    for (int r = 0; r < kAwqRows; ++r)
 #pragma unroll
-      for (int b = 0; b < 4; ++b) {
-        const float2 q = make_float2(__uint_as_float(__byte_perm(lo, 0x4B000000u, 0x7650u + b)),
-                                     __uint_as_float(__byte_perm(hi, 0x4B000000u, 0x7650u + b)));
-        d[b] = __fadd2_rn(q, nz2);
+      for (int m = 0; m < MT; ++m) acc[r][m] = make_float2(0.0f, 0.0f);
+    for (int c = lane; c < C; c += 32) {
+      uint4 v[kAwqRows];
+      float sv[kAwqRows], zf[kAwqRows];
+#pragma unroll
+      for (int r = 0; r < kAwqRows; ++r) {
+        const int n = n0 + r < N ? n0 + r : N - 1;  // rows past N repeat the last one and are not stored
+        v[r] = ldg_nc_v4(codes + static_cast<int64_t>(n) * (K / 2) + 16 * c);
+        sv[r] = __bfloat162float(scales[static_cast<int64_t>(n) * G + (c >> 1)]);
+        zf[r] = __fadd_rn(8388608.0f, static_cast<float>(zeros[static_cast<int64_t>(n) * G + (c >> 1)]));
       }
+      const int sw = c & 7;
+      float2 t[kAwqRows][MT];
+#pragma unroll
+      for (int r = 0; r < kAwqRows; ++r)
+#pragma unroll
+        for (int m = 0; m < MT; ++m) t[r][m] = make_float2(0.0f, 0.0f);
+#pragma unroll
+      for (int wd = 0; wd < 4; ++wd) {
+        float2 d[kAwqRows][4];  // (q - z) of elements (2b, 2b + 1): low and high nibble of byte b of the word
+#pragma unroll
+        for (int r = 0; r < kAwqRows; ++r) {
+          const uint32_t word = wd == 0 ? v[r].x : (wd == 1 ? v[r].y : (wd == 2 ? v[r].z : v[r].w));
+          const uint32_t lo = word & 0x0F0F0F0Fu, hi = (word >> 4) & 0x0F0F0F0Fu;
+          const float2 nz2 = make_float2(-zf[r], -zf[r]);
+#pragma unroll
+          for (int b = 0; b < 4; ++b) {
+            const float2 q = make_float2(__uint_as_float(__byte_perm(lo, 0x4B000000u, 0x7650u + b)),
+                                         __uint_as_float(__byte_perm(hi, 0x4B000000u, 0x7650u + b)));
+            d[r][b] = __fadd2_rn(q, nz2);
+          }
+        }
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
+          const float4* xc = xs4 + (m * C + c) * 8;
+          const float4 a = xc[(2 * wd) ^ sw];
+          const float4 e = xc[(2 * wd + 1) ^ sw];
+          const float2 x01 = make_float2(a.x, a.y), x23 = make_float2(a.z, a.w);
+          const float2 x45 = make_float2(e.x, e.y), x67 = make_float2(e.z, e.w);
+#pragma unroll
+          for (int r = 0; r < kAwqRows; ++r) {
+            t[r][m] = __ffma2_rn(x01, d[r][0], t[r][m]);
+            t[r][m] = __ffma2_rn(x23, d[r][1], t[r][m]);
+            t[r][m] = __ffma2_rn(x45, d[r][2], t[r][m]);
+            t[r][m] = __ffma2_rn(x67, d[r][3], t[r][m]);
+          }
+        }
+      }
+#pragma unroll
+      for (int r = 0; r < kAwqRows; ++r) {
+        const float2 s2 = make_float2(sv[r], sv[r]);
+#pragma unroll
+        for (int m = 0; m < MT; ++m) acc[r][m] = __ffma2_rn(t[r][m], s2, acc[r][m]);
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < kAwqRows; ++r) {
+      const int n = n0 + r;
+      float res[MT];
 #pragma unroll
       for (int m = 0; m < MT; ++m) {
-        const float4 a = xs4[(2 * m) * K8 + j];
-        const float4 c = xs4[(2 * m + 1) * K8 + j];
-        float2 t = __fmul2_rn(make_float2(a.x, a.y), d[0]);
-        t = __ffma2_rn(make_float2(a.z, a.w), d[1], t);
-        t = __ffma2_rn(make_float2(c.x, c.y), d[2], t);
-        t = __ffma2_rn(make_float2(c.z, c.w), d[3], t);
-        acc[m] = __ffma2_rn(t, s2, acc[m]);
+        res[m] = __fadd_rn(acc[r][m].x, acc[r][m].y);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) res[m] += __shfl_xor_sync(0xffffffffu, res[m], o);
       }
-    }
-    float r[MT];
+      if (lane == 0 && n < N) {
+        const float bn = bias != nullptr ? __bfloat162float(bias[n]) : 0.0f;
 #pragma unroll
-    for (int m = 0; m < MT; ++m) {
-      r[m] = __fadd_rn(acc[m].x, acc[m].y);
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) r[m] += __shfl_xor_sync(0xffffffffu, r[m], o);
-    }
-    if (lane == 0) {
-      const float bn = bias != nullptr ? __bfloat162float(bias[n]) : 0.0f;
-#pragma unroll
-      for (int m = 0; m < MT; ++m)
-        if (m < rows) Y[static_cast<int64_t>(m) * ldy + n] = __float2bfloat16_rn(__fadd_rn(r[m], bn));
+        for (int m = 0; m < MT; ++m)
+          if (m < rows) Y[static_cast<int64_t>(m) * ldy + n] = __float2bfloat16_rn(__fadd_rn(res[m], bn));
+      }
     }
   }
 }

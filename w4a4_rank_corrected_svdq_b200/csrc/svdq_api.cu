@@ -1174,8 +1174,9 @@ svdq_status launch_awq_gemv(int M, int N, int K, const __nv_bfloat16* X, int64_t
   const int smem = MT * K * 4;
   static std::atomic<uint64_t> attr_done{0};  // set once to the cap, which covers every K accepted
   ensure_smem_attr(awq_gemv_kernel<MT>, kAwqSmemCap, attr_done);
-  int per_sm = (227 * 1024) / (smem + 1024);
-  if (per_sm > 2048 / kAwqThreads) per_sm = 2048 / kAwqThreads;
+  int per_sm = 0;  // resident blocks per SM (registers and shared memory): one wave
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, awq_gemv_kernel<MT>, kAwqThreads, smem) != cudaSuccess)
+    return launch_status();
   if (per_sm < 1) return SVDQ_ERR_UNSUPPORTED_SHAPE;
   int blocks = (N + kAwqThreads / 32 - 1) / (kAwqThreads / 32);
   if (blocks > per_sm * sm_count) blocks = per_sm * sm_count;
@@ -1201,7 +1202,7 @@ svdq_status svdq_awq_gemv(int M, int N, int K, const void* X, int64_t ldx, const
   if (!X || !codes || !scales || !zeros || !Y) return SVDQ_ERR_INVALID_ARG;
   if (!aligned16(X) || !aligned16(codes) || (reinterpret_cast<uintptr_t>(scales) & 1u) ||
       (reinterpret_cast<uintptr_t>(Y) & 1u) || (bias && (reinterpret_cast<uintptr_t>(bias) & 1u)) ||
-      (inv_act && (reinterpret_cast<uintptr_t>(inv_act) & 3u)))
+      (inv_act && !aligned16(inv_act)))
     return SVDQ_ERR_MISALIGNED;
   if (K * 4 > kAwqSmemCap) return SVDQ_ERR_UNSUPPORTED_SHAPE;
   svdq_status s;
