@@ -9,7 +9,7 @@ modulation projections (memory-bound, precision-sensitive layers); section
 "Native loading in Diffusers" fixes its parameters: precision "int4",
 group_size 64, compute dtype bfloat16.
 
-The pages give no formulas. Readings (each also listed in the design doc):
+The pages give no formulas. Readings:
 * Asymmetric INT4 per output row and group of 64 contiguous K-elements, with
   the rule of the AWQ reference implementation's pseudo-quantiser: over the
   group's values w (fp32), s = bf16(fp32(max(fp32(max w - min w), 1e-5) / 15))

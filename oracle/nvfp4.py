@@ -18,7 +18,7 @@ Source of the definitions
 * Rounding is round-to-nearest-even with saturation to the largest finite
   value (the ".rn.satfinite" conversions of the target ISA).
 
-Readings where the pages are silent (each also listed in the design doc):
+Readings where the pages are silent:
 * g = fp32(amax / 2688), 2688 = 6 * 448, so the largest block of the tensor
   maps to the largest E2M1 magnitude times the largest E4M3 scale; g = 1 when
   the tensor is all zero.
