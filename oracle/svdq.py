@@ -35,6 +35,8 @@ Functions, in the order the method applies them:
                     structural rewrites": the fused operator consumes the QKV
                     projection, the Q/K normalisation and the rotary embedding
                     together)
+  mlp_pair          up projection, GELU, down projection (the same section
+                    names fused GELU / MLP kernels)
 """
 from __future__ import annotations
 
@@ -236,6 +238,38 @@ def qkv_norm_rope(y_ref, heads: int, head_dim: int, w_q, w_k, eps: float, cos, s
         out[:, blk * hd:(blk + 1) * hd] = rotary_pairs(rms_norm_heads(part, heads, head_dim, w, eps),
                                                         heads, head_dim, cos, sin)
     return out, nvfp4.bf16_round(out)
+
+
+# ------------------------------------------------------------------ MLP pair (GELU between two layers)
+def gelu(x, approximate: bool = False) -> np.ndarray:
+    """GELU in float64: x * Phi(x) = x (1 + erf(x / sqrt 2)) / 2, or with
+    approximate=True the tanh form x (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3))) / 2
+    (the one FLUX's feed-forward blocks use)."""
+    x = np.asarray(x, dtype=np.float64)
+    if approximate:
+        return 0.5 * x * (1.0 + np.tanh(np.sqrt(2.0 / np.pi) * (x + 0.044715 * x ** 3)))
+    from scipy.special import erf
+    return 0.5 * x * (1.0 + erf(x / np.sqrt(2.0)))
+
+
+@dataclass
+class MlpPair:
+    up: Forward          # the up projection (its y_ref is the bf16 layer output)
+    h: np.ndarray        # float64 [M, K_down] (bf16 values): bf16(GELU(up.y_ref))
+    down: Forward        # the down projection of h
+
+
+def mlp_pair(X, pw_up: PackedWeight, b_up, g_up, pw_down: PackedWeight, b_down, g_h,
+             approximate: bool = False) -> MlpPair:
+    """The feed-forward pair of a transformer block as two W4A4 layers with GELU
+    between them (blog section "Quantizing models with structural rewrites":
+    the engine fuses GELU / MLP kernels): h = bf16(GELU(bf16(up(X)))), what the
+    unfused sequence hands the down projection, which quantises h with its own
+    activation scale g_h."""
+    up = forward(X, pw_up, b_up, g_up)
+    h = nvfp4.bf16_round(gelu(up.y_ref, approximate))
+    down = forward(h, pw_down, b_down, g_h)
+    return MlpPair(up, h, down)
 
 
 # ------------------------------------------------------------------ metrics
