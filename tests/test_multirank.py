@@ -64,3 +64,30 @@ def test_single_rank_needs_no_process_group():
     import bench
     assert bench._max_over_ranks(3.25, 1) == 3.25
     bench._barrier(1)
+
+
+def test_reference_arm_prints_the_contract_line(monkeypatch, capsys):
+    """Rank 0 of the reference arm (the oracle on the host cores) prints one JSON
+    line with the bench contract's keys, its own cpu_baseline and an e2e entry
+    with no host-device traffic."""
+    import json
+    sys.path.insert(0, ROOT)
+    import bench
+    monkeypatch.setenv("WORLD_SIZE", "1")
+    monkeypatch.setenv("RANK", "0")
+
+    class Args:
+        steps, warmup = 1, 3
+
+    assert bench.run_reference(Args, bench.WORKLOAD.layers[0]) == 0
+    lines = [ln for ln in capsys.readouterr().out.splitlines() if ln.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in d, key
+    assert d["impl"] == "reference" and d["value"] > 0 and d["steps"] == 1 and d["warmup"] == 3
+    assert d["config"]["workload"] == bench.WORKLOAD.name
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    assert d["cpu_baseline"]["value"] == d["value"]
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
