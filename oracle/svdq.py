@@ -243,13 +243,17 @@ def qkv_norm_rope(y_ref, heads: int, head_dim: int, w_q, w_k, eps: float, cos, s
 # ------------------------------------------------------------------ MLP pair (GELU between two layers)
 def gelu(x, approximate: bool = False) -> np.ndarray:
     """GELU in float64: x * Phi(x) = x (1 + erf(x / sqrt 2)) / 2, or with
-    approximate=True the tanh form x (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3))) / 2
-    (the one FLUX's feed-forward blocks use)."""
+    approximate=True the tanh form x (1 + tanh(u)) / 2, u = sqrt(2/pi) (x +
+    0.044715 x^3) (the one FLUX's feed-forward blocks use). Evaluated as
+    x erfc(-x / sqrt 2) / 2 and x / (1 + exp(-2u)), the same functions written
+    without the cancellation of 1 + erf and 1 + tanh for negative x."""
     x = np.asarray(x, dtype=np.float64)
     if approximate:
-        return 0.5 * x * (1.0 + np.tanh(np.sqrt(2.0 / np.pi) * (x + 0.044715 * x ** 3)))
-    from scipy.special import erf
-    return 0.5 * x * (1.0 + erf(x / np.sqrt(2.0)))
+        u = np.sqrt(2.0 / np.pi) * (x + 0.044715 * x ** 3)
+        with np.errstate(over="ignore"):
+            return x / (1.0 + np.exp(-2.0 * u))
+    from scipy.special import erfc
+    return 0.5 * x * erfc(-x / np.sqrt(2.0))
 
 
 @dataclass

@@ -18,6 +18,20 @@ def test_gelu_matches_math_erf_loops():
     assert np.allclose(svdq.gelu(x, approximate=True), ref_t, rtol=0, atol=1e-15)
 
 
+def test_gelu_negative_tail_has_no_cancellation():
+    """Far in the negative tail GELU is tiny but not zero: x Phi(x) with Phi(x)
+    from the complementary error function (math.erfc) keeps full relative
+    precision where 1 + erf(x / sqrt 2) would cancel to zero."""
+    x = np.array([-6.0, -9.0, -12.0])
+    ref = np.array([0.5 * v * math.erfc(-v / math.sqrt(2.0)) for v in x])
+    g = svdq.gelu(x)
+    assert np.all(g < 0) and np.allclose(g, ref, rtol=1e-14, atol=0)
+    # the tanh form equals x sigma(2u): its tail follows exp(2u)
+    u = math.sqrt(2.0 / math.pi) * (-9.0 + 0.044715 * (-9.0) ** 3)
+    assert np.isclose(svdq.gelu(np.array([-9.0]), approximate=True)[0], -9.0 / (1.0 + math.exp(-2.0 * u)),
+                      rtol=1e-14, atol=0)
+
+
 def test_gelu_closed_forms():
     x = np.linspace(-8, 8, 161)
     g = svdq.gelu(x)
