@@ -284,6 +284,33 @@ svdq_status svdq_linear_forward_noalloc(int M, int N, int K, int r, const void* 
                                         const void* l1t, const void* l2s, const float* inv_smooth,
                                         const void* bias, void* Y, int64_t ldy, void* stream);
 
+/* ------------------------------------------------------------ MLP pair */
+/* The up projection of a transformer block's feed-forward pair with GELU and
+ * the down projection's activation quantisation fused into its GEMM epilogue
+ * (blog section "Quantizing models with structural rewrites": the engine's
+ * fused GELU / MLP kernels). For the layer X [M][K] -> N (arguments as
+ * svdq_linear_forward):
+ *   y = bf16(layer output), h = bf16(GELU(y)) (GELU = x Phi(x), or with
+ *   approximate != 0 its tanh form; fp32, evaluated without cancellation in
+ *   the negative tail),
+ * and h is written directly as the down projection's quantised activation:
+ *   h_codes  [M][N/2], h_scales (tiled, rows padded to 128, padding zero):
+ *            the NVFP4 rule of svdq_quantize_act with g = *g_h;
+ *   h_xl1    [M][r_down] = bf16(h . L1_down), L1_down bf16 [N][r_down]
+ *            row-major; fp32 partial sums per 128-column half tile, summed in
+ *            tile order (deterministic).
+ * These are the buffers svdq_w4a4_gemm takes as a_codes, a_scales and xl1 for
+ * the down projection (a QuantAct of M rows, K = N, rank r_down). h itself is
+ * stored only when h_out (bf16 [M][ldh]) is given. Requires N % 256 == 0 (the
+ * CTA-pair GEMM) and r_down == 32. Workspace: svdq_mlp_workspace_size bytes,
+ * 16-byte aligned. */
+svdq_status svdq_mlp_workspace_size(int M, int N, int K, int r, int r_down, size_t* bytes);
+svdq_status svdq_mlp_up_forward(int M, int N, int K, int r, const void* X, int64_t ldx, const void* w_codes,
+                                const void* w_scales, const float* gscale, const void* l1t, const void* l2s,
+                                const float* inv_smooth, const void* bias, int r_down, const float* g_h,
+                                const void* l1_down, int approximate, void* h_codes, void* h_scales, void* h_xl1,
+                                void* h_out, int64_t ldh, void* workspace, size_t workspace_bytes, void* stream);
+
 /* ------------------------------------------------------------ AWQ W4A16 */
 /* The second kernel family of the blog's section "Introducing Nunchaku Lite":
  * awq_w4a16, 4-bit weights with 16-bit activations for the adaptive-

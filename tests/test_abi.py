@@ -161,6 +161,23 @@ def test_awq_sizes_and_validation(L):
     assert L.svdq_awq_gemv(0, 100, 576, None, 576, None, None, None, None, None, None, 100, None) == 0
 
 
+def test_mlp_up_sizes_and_validation(L):
+    p = ctypes.c_void_p(0x10000)
+    odd = ctypes.c_void_p(0x10008)
+    base = _lib.svdq_forward_workspace_size(300, 512, 32)
+    assert _lib.svdq_mlp_workspace_size(300, 1024, 512, 32, 32) == base + 2 * 4 * 300 * 32 * 4
+    with pytest.raises(_lib.SvdqError):
+        _lib.svdq_mlp_workspace_size(300, 1024, 512, 32, 16)          # r_down must be 32
+    with pytest.raises(_lib.SvdqError):
+        _lib.svdq_mlp_workspace_size(300, 896, 512, 32, 32)           # N % 256
+    need = _lib.svdq_mlp_workspace_size(4, 256, 256, 32, 32)
+    args = lambda ws, wsb, l1d: (4, 256, 256, 32, p, 256, p, p, p, p, p, None, None, 32, p, l1d, 0, p, p, p, None,
+                                 0, ws, ctypes.c_size_t(wsb), None)
+    assert L.svdq_mlp_up_forward(*args(p, need - 1, p)) == 7          # workspace too small
+    assert L.svdq_mlp_up_forward(*args(p, need, None)) == 1           # no L1 of the down projection
+    assert L.svdq_mlp_up_forward(*args(p, need, odd)) == 3            # misaligned L1
+
+
 def test_qkv_forward_validation(L):
     p = ctypes.c_void_p(0x10000)
     odd = ctypes.c_void_p(0x10008)

@@ -22,6 +22,8 @@ from ._lib import (  # noqa: F401
     svdq_linear_forward_dynamic,
     svdq_linear_forward_qkv,
     svdq_lowrank_init,
+    svdq_mlp_up_forward,
+    svdq_mlp_workspace_size,
     svdq_lowrank_workspace_size,
     svdq_pack_weight,
     svdq_quantize_act,

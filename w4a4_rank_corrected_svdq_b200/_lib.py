@@ -44,6 +44,9 @@ SIGNATURES = {
     "svdq_dynamic_workspace_size": (_i, [_i, _i, _i, _i, _psz]),
     "svdq_linear_forward_dynamic": (_i, [_i, _i, _i, _i, _p, _i64, _p, _p, _p, _p, _p, _p, _p, _p, _i64, _p, _sz,
                                          _p]),
+    "svdq_mlp_workspace_size": (_i, [_i, _i, _i, _i, _i, _psz]),
+    "svdq_mlp_up_forward": (_i, [_i, _i, _i, _i, _p, _i64, _p, _p, _p, _p, _p, _p, _p, _i, _p, _p, _i, _p, _p, _p,
+                                 _p, _i64, _p, _sz, _p]),
     "svdq_awq_sizes": (_i, [_i, _i, _psz, _psz, _psz]),
     "svdq_awq_pack": (_i, [_i, _i, _p, _p, _p, _p, _p, _p, _p]),
     "svdq_awq_gemv": (_i, [_i, _i, _i, _p, _i64, _p, _p, _p, _p, _p, _p, _i64, _p]),
@@ -360,6 +363,45 @@ def svdq_linear_forward_dynamic(X: torch.Tensor, pw: PackedWeight, bias: torch.T
         M, N, K, r, _ptr(X), ldx, _ptr(pw.codes), _ptr(pw.scales), _ptr(pw.gscale), _ptr(pw.l1t),
         _ptr(pw.l2s), _ptr(pw.inv_smooth), _ptr(bias), _ptr(Y), ldy, _ptr(ws), ws.numel(), _stream(X)))
     return Y
+
+
+# ------------------------------------------------------------------ MLP pair
+def svdq_mlp_workspace_size(M: int, N: int, K: int, r: int, r_down: int = 32) -> int:
+    out = ctypes.c_size_t()
+    _check("svdq_mlp_workspace_size", lib().svdq_mlp_workspace_size(M, N, K, r, r_down, ctypes.byref(out)))
+    return out.value
+
+
+def svdq_mlp_up_forward(X: torch.Tensor, pw: PackedWeight, bias: torch.Tensor | None, g_h: torch.Tensor,
+                        l1_down: torch.Tensor, approximate: bool = False, out: QuantAct | None = None,
+                        h_out: torch.Tensor | None = None, workspace: torch.Tensor | None = None) -> QuantAct:
+    """The up projection with GELU, writing h quantised for the down projection:
+    returns the down projection's QuantAct (codes, scales, xl1 of h). g_h: the
+    down projection's activation scale (CUDA float32, one element); l1_down:
+    its L1, bf16 [N, r_down]; h_out: optional bf16 [M, N] copy of h."""
+    _dev(X, "X", torch.bfloat16)
+    M, K = X.shape
+    N, r = pw.N, pw.r
+    ldx = _rows(X, "X", K)
+    _dev(g_h, "g_h", torch.float32)
+    _dev(l1_down, "l1_down", torch.bfloat16)
+    if l1_down.dim() != 2 or l1_down.shape[0] != N or not l1_down.is_contiguous():
+        raise ValueError("l1_down must be a contiguous [N, r_down] tensor")
+    rd = l1_down.shape[1]
+    if bias is not None:
+        _dev(bias, "bias", torch.bfloat16, (N,))
+    ldh = 0
+    if h_out is not None:
+        _dev(h_out, "h_out", torch.bfloat16)
+        ldh = _rows(h_out, "h_out", N)
+    qa = out if out is not None else QuantAct(M, N, rd, X.device)
+    need = svdq_mlp_workspace_size(M, N, K, r, rd)
+    ws = workspace if workspace is not None else torch.empty(need, dtype=torch.uint8, device=X.device)
+    _check("svdq_mlp_up_forward", lib().svdq_mlp_up_forward(
+        M, N, K, r, _ptr(X), ldx, _ptr(pw.codes), _ptr(pw.scales), _ptr(pw.gscale), _ptr(pw.l1t), _ptr(pw.l2s),
+        _ptr(pw.inv_smooth), _ptr(bias), rd, _ptr(g_h), _ptr(l1_down), int(approximate), _ptr(qa.codes),
+        _ptr(qa.scales), _ptr(qa.xl1), _ptr(h_out), ldh, _ptr(ws), ws.numel(), _stream(X)))
+    return qa
 
 
 # ------------------------------------------------------------------ AWQ W4A16

@@ -36,6 +36,7 @@
 #pragma once
 
 #include "ptx.cuh"
+#include "nvfp4.cuh"
 #include "qkv_post.cuh"
 
 namespace svdq {
@@ -122,8 +123,9 @@ constexpr int k2Acc1Col = 208;
 constexpr int k2SfaCol = 464;
 constexpr int k2SfbCol = 480;
 
-template <int R, bool QKV = false>
+template <int R, int EPI = 0>
 struct Gemm2Cfg {
+  static constexpr bool QKV = EPI == 1;
   static constexpr int kABytes = 128 * 128;     // 128 rows x 256 E2M1
   static constexpr int kBBytes = 128 * 128;
   // Scale factors are staged in smem already replicated four times (the
@@ -446,14 +448,144 @@ __device__ __forceinline__ bool epilogue_qkv_tile(uint32_t tacc, int F, int h, c
   return true;
 }
 
-template <int R, bool QKV>
+// ------------------------------------------------------------------ MLP up-projection epilogue
+constexpr int kMlpRank = 32;  // the down projection's rank the fused epilogue supports
+// One 32-column chunk c (columns x0 + 32 c ..) of this lane's row: y, h =
+// bf16(GELU(y)), the two NVFP4 blocks of h (the activation quantiser's rule:
+// S = e4m3(amax / fp32(6 g)), q = h * fp32(1 / fp32(dec(S) g))), their codes
+// and scales stored for the down projection, h added into the XL1 partial
+// (part[j] += h_i L1d[x0 + 32 c + i][j]), and h optionally staged for a TMA
+// store.
+template <int RD>
+__device__ __forceinline__ void mlp_chunk(const uint32_t (&v)[32], const __nv_bfloat16* bcol, float alpha, int c,
+                                          int x0, int row, int M, int N, const MlpPost& mp, float g, float d,
+                                          float (&part)[RD], uint8_t* stage, int& nbuf, const CUtensorMap* tm_y,
+                                          int y0, int lane) {
+  uint32_t pk[16];
+  pack_chunk(v, bcol != nullptr ? bcol + 32 * c : nullptr, alpha, pk);  // y, exactly as the plain epilogue
+  float hf[32];
+#pragma unroll
+  for (int p = 0; p < 16; ++p) {
+    const uint32_t hp = pack_bf16(gelu_f32(bf16_lo(pk[p]), mp.approximate != 0),
+                                  gelu_f32(bf16_hi(pk[p]), mp.approximate != 0));
+    pk[p] = hp;
+    hf[2 * p] = bf16_lo(hp);
+    hf[2 * p + 1] = bf16_hi(hp);
+  }
+  const int col = x0 + 32 * c;
+  uint32_t words[4];
+  uint32_t sc = 0;
+#pragma unroll
+  for (int blk = 0; blk < 2; ++blk) {
+    float am = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) am = fmaxf(am, fabsf(hf[16 * blk + i]));
+    const uint32_t S = f32_to_e4m3(__fdiv_rn(am, d));
+    const float sd = __fmul_rn(e4m3_to_f32(S), g);
+    const float inv = (sd == 0.0f || S >= 0x7Fu) ? 0.0f : __frcp_rn(sd);
+    float q0[8], q1[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      q0[i] = __fmul_rn(hf[16 * blk + i], inv);
+      q1[i] = __fmul_rn(hf[16 * blk + 8 + i], inv);
+    }
+    words[2 * blk] = f32x8_to_e2m1(q0);
+    words[2 * blk + 1] = f32x8_to_e2m1(q1);
+    sc |= S << (8 * blk);
+  }
+  if (row < M) {
+    *reinterpret_cast<uint4*>(mp.codes + static_cast<int64_t>(row) * (N / 2) + col / 2) =
+        make_uint4(words[0], words[1], words[2], words[3]);
+  }
+  if (row < mp.m_pad)
+    *reinterpret_cast<uint16_t*>(mp.scales + scale_offset(N, row, col / 16)) =
+        static_cast<uint16_t>(row < M ? sc : 0u);
+  // XL1 partial: the L1 rows of these 32 columns are the same for every lane (broadcast loads);
+  // fully unrolled so that hf stays in registers
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const uint4* lrow = reinterpret_cast<const uint4*>(mp.l1d + static_cast<int64_t>(col + i) * RD);
+#pragma unroll
+    for (int j8 = 0; j8 < RD / 8; ++j8) {
+      float l[8];
+      bf16x8_to_f32(__ldg(lrow + j8), l);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) part[8 * j8 + e] = __fmaf_rn(hf[i], l[e], part[8 * j8 + e]);
+    }
+  }
+  if (mp.store_h) {
+    uint8_t* out = stage + 2048 * (nbuf & 1);
+    ++nbuf;
+    if (lane == 0) bulk_wait_read1();
+    __syncwarp();
+    stage_row16(out, pk, lane);
+    store_staged(out, tm_y, col, y0, lane);
+  }
+}
+
+// The MLP variant of epilogue_half: the warp's 128-column half in four chunks
+// (the shared accumulator columns first, released at once), then its XL1
+// partial for rows y0 .. y0 + 31 written to partial slot 2 nt + h.
+template <int RD, int FIRST>
+__device__ __forceinline__ void epilogue_half_mlp(uint32_t taddr, const __nv_bfloat16* bcol, float alpha,
+                                                  uint8_t* stage, int& nbuf, const CUtensorMap* tm_y, int x0, int y0,
+                                                  bool holds_overlap, uint32_t ovl_bar, int lane, const MlpPost& mp,
+                                                  int M, int N, int slot) {
+  const int row = y0 + lane;
+  const float g = *mp.g_h;
+  const float d = __fmul_rn(6.0f, g);
+  float part[RD];
+#pragma unroll
+  for (int j = 0; j < RD; ++j) part[j] = 0.0f;
+  {
+    uint32_t va[32], vb[32];
+    tmem_ld_32x32b_x32(taddr + 32 * ((FIRST + 0) & 3), va);
+    tmem_ld_32x32b_x32(taddr + 32 * ((FIRST + 1) & 3), vb);
+    tmem_ld_wait();
+    if (holds_overlap) {  // the loads above have completed (tcgen05.wait::ld): nothing else to publish
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster_relaxed(ovl_bar);
+    }
+    mlp_chunk<RD>(va, bcol, alpha, (FIRST + 0) & 3, x0, row, M, N, mp, g, d, part, stage, nbuf, tm_y, y0, lane);
+    mlp_chunk<RD>(vb, bcol, alpha, (FIRST + 1) & 3, x0, row, M, N, mp, g, d, part, stage, nbuf, tm_y, y0, lane);
+  }
+#pragma unroll 1
+  for (int k = 2; k < 4; ++k) {
+    uint32_t va[32];
+    tmem_ld_32x32b_x32(taddr + 32 * ((FIRST + k) & 3), va);
+    tmem_ld_wait();
+    mlp_chunk<RD>(va, bcol, alpha, (FIRST + k) & 3, x0, row, M, N, mp, g, d, part, stage, nbuf, tm_y, y0, lane);
+  }
+  if (row < M) {
+    float4* dst = reinterpret_cast<float4*>(mp.partial + (static_cast<int64_t>(slot) * M + row) * RD);
+#pragma unroll
+    for (int j = 0; j < RD / 4; ++j) dst[j] = make_float4(part[4 * j], part[4 * j + 1], part[4 * j + 2], part[4 * j + 3]);
+  }
+}
+
+// Sums the XL1 partials of an MLP up projection in slot order:
+// xl1[m][j] = bf16(sum_p partial[p][m][j]) (fp32, p ascending: deterministic).
+__global__ void mlp_xl1_reduce_kernel(const float* __restrict__ partial, int slots, int M, int rd,
+                                      __nv_bfloat16* __restrict__ xl1) {
+  const int64_t total = static_cast<int64_t>(M) * rd;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    float s = 0.0f;
+    for (int p = 0; p < slots; ++p) s = __fadd_rn(s, partial[p * total + i]);
+    xl1[i] = __float2bfloat16_rn(s);
+  }
+}
+
+template <int R, int EPI>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(k2Threads, 1) w4a4_gemm_2sm_kernel(
     const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
     const __grid_constant__ CUtensorMap tm_sfa, const __grid_constant__ CUtensorMap tm_sfb,
     const __grid_constant__ CUtensorMap tm_xl1, const __grid_constant__ CUtensorMap tm_l2s,
     const __grid_constant__ CUtensorMap tm_y, const float* __restrict__ gscale,
-    const __nv_bfloat16* __restrict__ bias, int M, int N, int K, const QkvPost post) {
-  using C = Gemm2Cfg<R, QKV>;
+    const __nv_bfloat16* __restrict__ bias, int M, int N, int K, const QkvPost post, const MlpPost mlp) {
+  using C = Gemm2Cfg<R, EPI>;
+  constexpr bool QKV = EPI == 1;
   constexpr int S = C::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -654,6 +786,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(k2Threads, 1) w4a4_g
                                           post.eps, abort);
         if (!ok) break;
         if (qk) ++nx;
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster_relaxed(mapa_shared(smem_u32(&bars->acc_empty[b]), 0));
+        continue;
+      }
+      if constexpr (EPI == 2) {
+        if (!mbar_wait(&bars->acc_full[b], (it >> 1) & 1, abort)) break;
+        tc_fence_after();
+        const uint32_t acc = lane_base + (b ? k2Acc1Col : 0) + 128 * h;
+        const __nv_bfloat16* bcol = bias != nullptr ? bias + col0 : nullptr;
+        const int slot = 2 * nt + h;
+        if (b == 0 && h == 1)
+          epilogue_half_mlp<kMlpRank, 2>(acc, bcol, alpha, stage, nbuf, &tm_y, col0, y0, true, ovl_bar, lane, mlp, M,
+                                         N, slot);
+        else
+          epilogue_half_mlp<kMlpRank, 0>(acc, bcol, alpha, stage, nbuf, &tm_y, col0, y0, b == 1 && h == 0, ovl_bar,
+                                         lane, mlp, M, N, slot);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster_relaxed(mapa_shared(smem_u32(&bars->acc_empty[b]), 0));

@@ -32,6 +32,33 @@ struct QkvPost {
   float eps;
 };
 
+// Epilogue of an MLP pair's up projection: h = bf16(GELU(bf16(alpha acc + b)))
+// quantised in place for the down projection (NVFP4 codes and tiled block
+// scales with the down projection's activation scale g_h) and its fp32 partial
+// products with the down projection's L1 (XL1 partials per 128-column half
+// tile, summed afterwards in tile order).
+struct MlpPost {
+  const float* g_h;           // device float: the down projection's activation decode scale
+  const __nv_bfloat16* l1d;   // [N][r_down] row-major: the down projection's L1 (its K = this layer's N)
+  uint8_t* codes;             // [M][N/2]
+  uint8_t* scales;            // tiled, rows padded to 128 (padding rows get zero scales)
+  float* partial;             // [2 N / 256][M][r_down] fp32
+  int m_pad;                  // M rounded up to 128
+  int store_h;                // also store h (bf16) through the output map
+  int approximate;            // tanh form of GELU
+};
+
+// GELU in fp32: x Phi(x) = x erfc(-x / sqrt 2) / 2, or the tanh form
+// x (1 + tanh u) / 2 = x / (1 + exp(-2u)), u = sqrt(2/pi) (x + 0.044715 x^3);
+// both written without the cancellation of 1 + erf / 1 + tanh for negative x.
+__device__ __forceinline__ float gelu_f32(float x, bool approximate) {
+  if (approximate) {
+    const float u = __fmul_rn(0.7978845608028654f, __fmaf_rn(__fmul_rn(0.044715f, x), __fmul_rn(x, x), x));
+    return __fdiv_rn(x, __fadd_rn(1.0f, expf(__fmul_rn(-2.0f, u))));
+  }
+  return __fmul_rn(__fmul_rn(0.5f, x), erfcf(__fmul_rn(x, -0.7071067811865476f)));
+}
+
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {

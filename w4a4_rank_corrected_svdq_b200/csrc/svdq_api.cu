@@ -404,12 +404,12 @@ svdq_status launch_gemm(int M, int N, int K, const void* a_codes, const void* a_
   return launch_status();
 }
 
-template <int R, bool QKV>
+template <int R, int EPI>
 svdq_status launch_gemm_2sm(int M, int N, int K, const void* a_codes, const void* a_scales, const void* xl1,
                             const void* w_codes, const void* w_scales, const float* gscale, const void* l2s,
                             const void* bias, void* Y, int64_t ldy, cudaStream_t stream, int sm_count,
-                            const QkvPost& post) {
-  using C = Gemm2Cfg<R, QKV>;
+                            const QkvPost& post, const MlpPost& mlp) {
+  using C = Gemm2Cfg<R, EPI>;
   CUtensorMap tm_a, tm_b, tm_sfa, tm_sfb, tm_x, tm_l, tm_y;
   const uint64_t kb = static_cast<uint64_t>(K / 2);
   const uint64_t mpad = round_up(static_cast<size_t>(M), 128);
@@ -425,7 +425,7 @@ svdq_status launch_gemm_2sm(int M, int N, int K, const void* a_codes, const void
       !make_tmap_2d(&tm_y, Y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, M, static_cast<uint64_t>(ldy) * 2, 32, 32,
                     CU_TENSOR_MAP_SWIZZLE_64B))
     return SVDQ_ERR_CUDA;
-  auto kern = w4a4_gemm_2sm_kernel<R, QKV>;
+  auto kern = w4a4_gemm_2sm_kernel<R, EPI>;
   static std::atomic<uint64_t> attr_done{0};
   ensure_smem_attr(kern, C::kSmemBytes, attr_done);
   const int tiles = ((M + k2TileM - 1) / k2TileM) * (N / k2TileN);
@@ -433,7 +433,7 @@ svdq_status launch_gemm_2sm(int M, int N, int K, const void* a_codes, const void
   const int pairs = tiles < max_pairs ? tiles : max_pairs;
   PdlLaunch pl(dim3(2 * pairs), dim3(k2Threads), C::kSmemBytes, stream);
   cudaLaunchKernelEx(&pl.cfg, kern, tm_a, tm_b, tm_sfa, tm_sfb, tm_x, tm_l, tm_y, gscale,
-                     static_cast<const __nv_bfloat16*>(bias), M, N, K, post);
+                     static_cast<const __nv_bfloat16*>(bias), M, N, K, post, mlp);
   return launch_status();
 }
 
@@ -454,9 +454,21 @@ bool use_2sm(int M, int N) {
 svdq_status gemm_dispatch(int M, int N, int K, int r, const void* a_codes, const void* a_scales, const void* xl1,
                           const void* w_codes, const void* w_scales, const float* gscale, const void* l2s,
                           const void* bias, void* Y, int64_t ldy, cudaStream_t st, int sms,
-                          const QkvPost* post = nullptr) {
+                          const QkvPost* post = nullptr, const MlpPost* mlp = nullptr) {
   const QkvPost none{};
   const QkvPost& pp = post != nullptr ? *post : none;
+  const MlpPost mnone{};
+  const MlpPost& mp = mlp != nullptr ? *mlp : mnone;
+  if (mlp != nullptr) {  // the MLP up-projection epilogue exists for the CTA-pair GEMM only
+    if (N % 256 != 0) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+#define SVDQ_GEMM2_ARGS M, N, K, a_codes, a_scales, xl1, w_codes, w_scales, gscale, l2s, bias, Y, ldy, st, sms, pp, mp
+    switch (r) {
+      case 16: return launch_gemm_2sm<16, 2>(SVDQ_GEMM2_ARGS);
+      case 32: return launch_gemm_2sm<32, 2>(SVDQ_GEMM2_ARGS);
+      case 64: return launch_gemm_2sm<64, 2>(SVDQ_GEMM2_ARGS);
+      default: return launch_gemm_2sm<128, 2>(SVDQ_GEMM2_ARGS);
+    }
+  }
 #define SVDQ_GEMM_ARGS M, N, K, a_codes, a_scales, xl1, w_codes, w_scales, gscale, l2s, bias, Y, ldy, st, sms, pp
 #define SVDQ_GEMM_CASES(F, Q)                 \
   switch (r) {                                \
@@ -466,13 +478,26 @@ svdq_status gemm_dispatch(int M, int N, int K, int r, const void* a_codes, const
     default: return F<128, Q>(SVDQ_GEMM_ARGS); \
   }
   if (use_2sm(M, N)) {
-    if (post != nullptr) SVDQ_GEMM_CASES(launch_gemm_2sm, true)
-    SVDQ_GEMM_CASES(launch_gemm_2sm, false)
+    if (post != nullptr) {
+      switch (r) {
+        case 16: return launch_gemm_2sm<16, 1>(SVDQ_GEMM2_ARGS);
+        case 32: return launch_gemm_2sm<32, 1>(SVDQ_GEMM2_ARGS);
+        case 64: return launch_gemm_2sm<64, 1>(SVDQ_GEMM2_ARGS);
+        default: return launch_gemm_2sm<128, 1>(SVDQ_GEMM2_ARGS);
+      }
+    }
+    switch (r) {
+      case 16: return launch_gemm_2sm<16, 0>(SVDQ_GEMM2_ARGS);
+      case 32: return launch_gemm_2sm<32, 0>(SVDQ_GEMM2_ARGS);
+      case 64: return launch_gemm_2sm<64, 0>(SVDQ_GEMM2_ARGS);
+      default: return launch_gemm_2sm<128, 0>(SVDQ_GEMM2_ARGS);
+    }
   }
   if (post != nullptr) SVDQ_GEMM_CASES(launch_gemm, true)
   SVDQ_GEMM_CASES(launch_gemm, false)
 #undef SVDQ_GEMM_CASES
 #undef SVDQ_GEMM_ARGS
+#undef SVDQ_GEMM2_ARGS
 }
 
 // max |fp32(x * inv[col + j])| (or |x|) over one 16-byte vector of 8 bf16.
@@ -1011,6 +1036,69 @@ svdq_status svdq_linear_forward_qkv(int M, int N, int K, int r, const void* X, i
   post.eps = eps;
   return gemm_checked(M, N, K, r, a_codes, a_scales, xl1, w_codes, w_scales, gscale, l2s, bias, Y, ldy, stream,
                       &post);
+}
+
+svdq_status svdq_mlp_workspace_size(int M, int N, int K, int r, int r_down, size_t* bytes) {
+  size_t base = 0;
+  svdq_status s = check_layer_shape(N, K, r);
+  if (s != SVDQ_OK) return s;
+  if (r_down != kMlpRank || N % 256 != 0) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+  if ((s = svdq_forward_workspace_size(M, K, r, &base)) != SVDQ_OK) return s;
+  if (!bytes) return SVDQ_ERR_INVALID_ARG;
+  *bytes = base + round_up(static_cast<size_t>(2 * (N / 256)) * M * r_down * 4, 256);
+  return SVDQ_OK;
+}
+
+svdq_status svdq_mlp_up_forward(int M, int N, int K, int r, const void* X, int64_t ldx, const void* w_codes,
+                                const void* w_scales, const float* gscale, const void* l1t, const void* l2s,
+                                const float* inv_smooth, const void* bias, int r_down, const float* g_h,
+                                const void* l1_down, int approximate, void* h_codes, void* h_scales, void* h_xl1,
+                                void* h_out, int64_t ldh, void* workspace, size_t workspace_bytes, void* stream) {
+  if (M < 0) return SVDQ_ERR_INVALID_ARG;
+  svdq_status s = check_layer_shape(N, K, r);
+  if (s != SVDQ_OK) return s;
+  if (r_down != kMlpRank || N % 256 != 0 || ldx < K || ldx % 8 != 0 || (h_out && (ldh < N || ldh % 8 != 0)))
+    return SVDQ_ERR_UNSUPPORTED_SHAPE;
+  if (M == 0) return SVDQ_OK;
+  if (!X || !gscale || !l1t || !g_h || !l1_down || !h_codes || !h_scales || !h_xl1 || !workspace)
+    return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(l1_down) || !aligned16(h_codes) || !aligned16(h_scales) || !aligned16(h_xl1) ||
+      !aligned16(workspace) || (h_out && !aligned16(h_out)) || (reinterpret_cast<uintptr_t>(g_h) & 3u))
+    return SVDQ_ERR_MISALIGNED;
+  size_t need = 0, base = 0, c = 0, sc = 0, x = 0;
+  svdq_mlp_workspace_size(M, N, K, r, r_down, &need);
+  svdq_forward_workspace_size(M, K, r, &base);
+  svdq_act_sizes(M, K, r, &c, &sc, &x);
+  if (workspace_bytes < need) return SVDQ_ERR_WORKSPACE;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint8_t* a_codes = ws;
+  uint8_t* a_scales = ws + round_up(c, 256);
+  uint8_t* xl1 = a_scales + round_up(sc, 256);
+  float* partial = reinterpret_cast<float*>(ws + base);
+  s = svdq_quantize_act(M, K, r, X, ldx, gscale, l1t, inv_smooth, a_codes, a_scales, xl1, stream);
+  if (s != SVDQ_OK) return s;
+  DeviceInfo di;
+  if ((s = current_device(nullptr, &di)) != SVDQ_OK) return s;
+  MlpPost mp{};
+  mp.g_h = g_h;
+  mp.l1d = static_cast<const __nv_bfloat16*>(l1_down);
+  mp.codes = static_cast<uint8_t*>(h_codes);
+  mp.scales = static_cast<uint8_t*>(h_scales);
+  mp.partial = partial;
+  mp.m_pad = static_cast<int>(round_up(static_cast<size_t>(M), 128));
+  mp.store_h = h_out != nullptr;
+  mp.approximate = approximate != 0;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // without h_out nothing is stored through the output map; it is built on h_codes only to be valid
+  s = gemm_dispatch(M, N, K, r, a_codes, a_scales, xl1, w_codes, w_scales, gscale, l2s, bias,
+                    h_out ? h_out : h_codes, h_out ? ldh : N, st, di.sm_count, nullptr, &mp);
+  if (s != SVDQ_OK) return s;
+  const int64_t tot = static_cast<int64_t>(M) * r_down;
+  int64_t blocks = (tot + 255) / 256;
+  if (blocks > 4 * di.sm_count) blocks = 4 * di.sm_count;
+  mlp_xl1_reduce_kernel<<<static_cast<int>(blocks), 256, 0, st>>>(partial, 2 * (N / 256), M, r_down,
+                                                                    static_cast<__nv_bfloat16*>(h_xl1));
+  return launch_status();
 }
 
 }  // extern "C"
