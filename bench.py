@@ -414,6 +414,56 @@ def run_ours(args, spec):
         raise RuntimeError("device error during the AWQ timing")
     variants["awq_w4a16_modulation_3072x18432"] = awq_out
 
+    # MLP pair (the DiT feed-forward shapes, 3072 -> 12288 -> 3072, M = 4608):
+    # the fused up projection (GELU and the down projection's activation
+    # quantisation in its GEMM epilogue) plus the down GEMM, against the
+    # unfused pair without a GELU pass (the up projection writing y in bf16,
+    # the down projection reading it back), a lower bound of the unfused cost.
+    try:
+        up_s, dn_s = workloads.WORKLOADS[3].layers[:2]
+        Xu, Wu, bu = workloads.make_layer(up_s)
+        Wdn, bdn = workloads.make_layer(dn_s, rows=1)[1:]
+        Xud, bud, bdd = Xu.to(dev), bu.to(dev), bdn.to(dev)
+        Wud = Wu.to(dev)
+        Lu1, Lu2, _ = svdq.svdq_lowrank_init(Wud, up_s.r)
+        pw_u = svdq.svdq_pack_weight(Wud, Lu1, Lu2, svdq.svdq_act_global_scale(Xud))
+        del Wud
+        Wdd = Wdn.to(dev)
+        Ld1, Ld2, _ = svdq.svdq_lowrank_init(Wdd, dn_s.r)
+        Mu, Fu = up_s.M, up_s.N
+        Hd = torch.empty((Mu, Fu), dtype=torch.bfloat16, device=dev)
+        one = torch.ones(1, dtype=torch.float32, device=dev)
+        svdq.svdq_mlp_up_forward(Xud, pw_u, bud, one, Ld1, h_out=Hd)   # calibration pass for h's scale
+        g_h = svdq.svdq_act_global_scale(Hd)
+        pw_d = svdq.svdq_pack_weight(Wdd, Ld1, Ld2, g_h)
+        del Wdd
+        qa_h = svdq.QuantAct(Mu, Fu, dn_s.r, dev)
+        ws_m = torch.empty(svdq.svdq_mlp_workspace_size(Mu, Fu, up_s.K, up_s.r, dn_s.r), dtype=torch.uint8,
+                           device=dev)
+        ws_u = torch.empty(svdq.svdq_forward_workspace_size(Mu, up_s.K, up_s.r), dtype=torch.uint8, device=dev)
+        ws_d = torch.empty(svdq.svdq_forward_workspace_size(Mu, Fu, dn_s.r), dtype=torch.uint8, device=dev)
+        Yd = torch.empty((Mu, dn_s.N), dtype=torch.bfloat16, device=dev)
+
+        def fused(i):
+            svdq.svdq_mlp_up_forward(Xud, pw_u, bud, g_h, Ld1, out=qa_h, workspace=ws_m)
+            svdq.svdq_w4a4_gemm(qa_h, pw_d, bdd, out=Yd)
+
+        def unfused(i):
+            svdq.svdq_linear_forward(Xud, pw_u, bud, out=Hd, workspace=ws_u)
+            svdq.svdq_linear_forward(Hd, pw_d, bdd, out=Yd, workspace=ws_d)
+
+        fused_ms, unfused_ms = timed(fused), timed(unfused)
+        if svdq.svdq_read_device_error() != 0:
+            raise RuntimeError("device error during the MLP pair timing")
+        pair_flops = _flops(Mu, Fu, up_s.K, up_s.r) + _flops(Mu, dn_s.N, Fu, dn_s.r)
+        variants["mlp_pair_4608x3072x12288_r32"] = {
+            "fused_ms_per_step": fused_ms, "unfused_without_gelu_ms_per_step": unfused_ms,
+            "fused_tflops": pair_flops / (fused_ms * 1e-3) / 1e12,
+            "note": "one input set; the per-step working set (about 150 MB) exceeds L2"}
+        del pw_u, pw_d, qa_h, ws_m, ws_u, ws_d, Hd, Yd
+    except Exception as exc:  # reported, not fatal: the headline line above is complete without it
+        variants["mlp_pair_4608x3072x12288_r32"] = {"error": f"{type(exc).__name__}: {str(exc)[:160]}"}
+
     peaks, kind = _peaks()
     gemm_name = _gemm_kernel_name(M, N)
     fp4_peak = peaks["bf16_tflops"] * FP4_PER_BF16
