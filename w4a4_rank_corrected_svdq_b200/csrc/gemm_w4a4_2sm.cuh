@@ -27,7 +27,12 @@
 //               issues the MMAs and the scale copies smem -> TMEM.
 //  * warps 2-9  epilogue (both CTAs): TMEM -> registers, y = alpha acc + b,
 //               bf16 stores; two warps per 32-lane TMEM quadrant, one per
-//               128-column half.
+//               128-column half. The epilogue mode EPI selects the plain
+//               layer (0), the fused QKV post-processing (1: per-head RMSNorm
+//               of Q/K and the rotary embedding; the two warps of a quadrant
+//               then split a tile by chunks) or the MLP up projection (2:
+//               GELU and the down projection's NVFP4 codes, scales and XL1
+//               partials instead of y).
 // TMEM: accumulator 0 = columns [0,256), accumulator 1 = [208,464): the two
 // share [208,256), which the epilogue reads first and releases early, so the
 // next tile's MMAs start long before the previous tile is fully stored; scale

@@ -450,7 +450,8 @@ bool use_2sm(int M, int N) {
   return M >= 512;
 }
 
-// post == nullptr: the plain layer; otherwise the fused QKV post-processing.
+// The plain layer, or with post the fused QKV post-processing, or with mlp the
+// MLP up projection (CTA-pair GEMM only).
 svdq_status gemm_dispatch(int M, int N, int K, int r, const void* a_codes, const void* a_scales, const void* xl1,
                           const void* w_codes, const void* w_scales, const float* gscale, const void* l2s,
                           const void* bias, void* Y, int64_t ldy, cudaStream_t st, int sms,
