@@ -53,6 +53,21 @@
  *          low-rank product then share one fp32 accumulator, which the
  *          epilogue multiplies by alpha once.)
  *  xl1     bf16 [M][r]   = bf16(X . L1), fp32 accumulation
+ *  inv_smooth  fp32 [K]  = fp32(1 / lambda), the smoothing factors of a
+ *          smoothed layer (written by svdq_pack_weight), or NULL
+ *
+ * Entry points
+ * ------------
+ *  load time   svdq_smooth_factors (calibration of the smoothing), svdq_lowrank_init
+ *              (truncated SVD on the GPU), svdq_act_global_scale (calibrated g_x),
+ *              svdq_pack_weight
+ *  per call    svdq_quantize_act + svdq_w4a4_gemm, or svdq_linear_forward (both),
+ *              svdq_linear_forward_dynamic (g_x from each call's X),
+ *              svdq_linear_forward_noalloc (no workspace argument),
+ *              svdq_linear_forward_qkv (fused QKV: per-head RMSNorm + rotary),
+ *              svdq_mlp_up_forward (MLP pair: GELU and the down projection's
+ *              quantised input in the up projection's epilogue)
+ *  AWQ W4A16   svdq_awq_pack, svdq_awq_gemv (weight-only INT4, group 64)
  */
 #ifndef SVDQ_H_
 #define SVDQ_H_
