@@ -91,3 +91,22 @@ def test_reference_arm_prints_the_contract_line(monkeypatch, capsys):
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
     assert d["cpu_baseline"]["value"] == d["value"]
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
+
+
+def test_clock_sampler_summary_parses_nvidia_smi_lines():
+    """The clocks record of the bench line: median SM clock under load, the
+    largest max clock, and every throttle reason seen Active in any sample."""
+    sys.path.insert(0, ROOT)
+    import bench
+    cs = bench.ClockSampler(0)
+    cs.out = "\n".join([
+        "1965, 1965, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active",
+        "1800, 1965, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+        "1900, 1965, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active",
+        "[N/A], [N/A], [N/A], [N/A], [N/A], [N/A], [N/A]",
+    ])
+    s = cs.summary()
+    assert s["sm_mhz"] == 1900.0 and s["sm_max_mhz"] == 1965.0
+    assert s["reasons"] == ["sw_power_cap"] and s["samples"] == 4
+    cs.out = ""
+    assert cs.summary()["reasons"] == ["unavailable"]
