@@ -176,6 +176,9 @@ def test_mlp_up_sizes_and_validation(L):
     assert L.svdq_mlp_up_forward(*args(p, need - 1, p)) == 7          # workspace too small
     assert L.svdq_mlp_up_forward(*args(p, need, None)) == 1           # no L1 of the down projection
     assert L.svdq_mlp_up_forward(*args(p, need, odd)) == 3            # misaligned L1
+    bad_bias = (4, 256, 256, 32, p, 256, p, p, p, p, p, None, odd, 32, p, p, 0, p, p, p, None, 0, p,
+                ctypes.c_size_t(need), None)
+    assert L.svdq_mlp_up_forward(*bad_bias) == 3                       # misaligned bias
 
 
 def test_qkv_forward_validation(L):

@@ -1061,10 +1061,13 @@ svdq_status svdq_mlp_up_forward(int M, int N, int K, int r, const void* X, int64
   if (r_down != kMlpRank || N % 256 != 0 || ldx < K || ldx % 8 != 0 || (h_out && (ldh < N || ldh % 8 != 0)))
     return SVDQ_ERR_UNSUPPORTED_SHAPE;
   if (M == 0) return SVDQ_OK;
-  if (!X || !gscale || !l1t || !g_h || !l1_down || !h_codes || !h_scales || !h_xl1 || !workspace)
+  if (!X || !gscale || !l1t || !g_h || !l1_down || !h_codes || !h_scales || !h_xl1 || !workspace || !w_codes ||
+      !w_scales || !l2s)
     return SVDQ_ERR_INVALID_ARG;
   if (!aligned16(l1_down) || !aligned16(h_codes) || !aligned16(h_scales) || !aligned16(h_xl1) ||
-      !aligned16(workspace) || (h_out && !aligned16(h_out)) || (reinterpret_cast<uintptr_t>(g_h) & 3u))
+      !aligned16(workspace) || (h_out && !aligned16(h_out)) || (reinterpret_cast<uintptr_t>(g_h) & 3u) ||
+      !aligned16(w_codes) || !aligned16(w_scales) || !aligned16(l2s) || !aligned16(gscale) ||
+      (bias && !aligned16(bias)))
     return SVDQ_ERR_MISALIGNED;
   size_t need = 0, base = 0, c = 0, sc = 0, x = 0;
   svdq_mlp_workspace_size(M, N, K, r, r_down, &need);
