@@ -2,8 +2,10 @@
 
 This module only draws random tensors of the shapes and value distributions
 that the workload definitions below describe. It holds none of the method's
-arithmetic (no quantisation, no decomposition, no matmul); both the CPU
-oracle and the CUDA path take their inputs from here.
+arithmetic (no quantisation, no SVD of the weight, no layer product; the one
+product here builds a planted low-rank weight part from random orthonormal
+bases, part of the input recipe); both the CPU oracle and the CUDA path take
+their inputs from here.
 
 Shapes come from the benchmark set built for the layer described in the
 Hugging Face blog "Bringing Nunchaku 4-bit Diffusion Inference to Diffusers"
