@@ -144,3 +144,18 @@ def test_nibble_packing_order():
     packed = nvfp4.pack_nibbles(codes)
     assert packed.tolist() == [[0x21, 0x43]]
     assert np.array_equal(nvfp4.unpack_nibbles(packed), codes)
+
+
+def test_e4m3_encode_exhaustive_over_fp32_binades():
+    """Every fp32 value from 2^-20 up to 512 (29 binades, 2^23 values each)
+    against torch's float8_e4m3fn conversion (round to nearest even, an
+    independent library routine) where it is in range, and saturation to the
+    largest finite code 0x7E above 448 (the .satfinite rule)."""
+    m = np.arange(1 << 23, dtype=np.uint32)
+    for e in range(-20, 9):
+        v = ((np.uint32(e + 127) << np.uint32(23)) | m).view(np.float32)
+        ours = nvfp4.e4m3_encode(v)
+        inr = v <= 448.0
+        ref = torch.from_numpy(np.ascontiguousarray(v[inr])).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+        assert np.array_equal(ours[inr], ref), e
+        assert np.all(ours[~inr] == 0x7E), e
