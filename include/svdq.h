@@ -102,6 +102,13 @@ int svdq_version(void);
  * UNSUPPORTED_SHAPE if K % 64 != 0. */
 svdq_status svdq_scale_offset(int K, int row, int kblock, size_t* out);
 
+/* The device rule every entry point applies (host only, no device needed):
+ * SVDQ_OK for compute capability 10.0 (B200; the kernels are built for
+ * sm_100a), SVDQ_ERR_UNSUPPORTED_DEVICE for any other capability. The blog's
+ * hardware section: the GPU's capability is checked up front and an
+ * unsupported GPU gets a clear error instead of wrong outputs. */
+svdq_status svdq_device_supported(int major, int minor);
+
 /* ------------------------------------------------------------ sizes (host) */
 /* Bytes of each packed-weight buffer for an N x K weight with rank r. */
 svdq_status svdq_weight_sizes(int N, int K, int r, size_t* codes_bytes, size_t* scales_bytes,

@@ -198,6 +198,15 @@ def test_qkv_forward_validation(L):
     assert L.svdq_linear_forward_qkv(*args(768, 0, 1e-6, p, 128)) == 1          # heads
 
 
+def test_device_rule_on_simulated_capabilities(L):
+    """The capability rule the entry points apply, fed simulated devices: only
+    compute capability 10.0 (B200) is supported; Hopper, Ada, Ampere, other
+    Blackwell parts and later families get SVDQ_ERR_UNSUPPORTED_DEVICE."""
+    assert L.svdq_device_supported(10, 0) == 0
+    for major, minor in ((9, 0), (8, 9), (8, 0), (7, 5), (10, 3), (12, 0), (11, 0), (0, 0)):
+        assert L.svdq_device_supported(major, minor) == 4, (major, minor)
+
+
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU path")
 def test_no_gpu_is_unsupported_device(L):
     p = ctypes.c_void_p(0x10000)

@@ -28,6 +28,7 @@ SIGNATURES = {
     "svdq_status_string": (ctypes.c_char_p, [_i]),
     "svdq_version": (_i, []),
     "svdq_scale_offset": (_i, [_i, _i, _i, _psz]),
+    "svdq_device_supported": (_i, [_i, _i]),
     "svdq_weight_sizes": (_i, [_i, _i, _i, _psz, _psz, _psz, _psz]),
     "svdq_act_sizes": (_i, [_i, _i, _i, _psz, _psz, _psz]),
     "svdq_forward_workspace_size": (_i, [_i, _i, _i, _psz]),

@@ -29,6 +29,17 @@ bool valid_rank(int r) { return r == 16 || r == 32 || r == 64 || r == 128; }
 size_t round_up(size_t x, size_t m) { return (x + m - 1) / m * m; }
 
 // ------------------------------------------------------------------ device checks
+}  // namespace
+}  // namespace svdq
+
+// The kernels are built for sm_100a (tcgen05, TMEM, mxf4nvf4 block-scaled MMA):
+// compute capability 10.0 exactly.
+extern "C" svdq_status svdq_device_supported(int major, int minor) {
+  return (major == 10 && minor == 0) ? SVDQ_OK : SVDQ_ERR_UNSUPPORTED_DEVICE;
+}
+
+namespace svdq {
+namespace {
 struct DeviceInfo {
   int sm_count = 0;
   int ok = -1;  // -1 unknown, 0 unsupported, 1 supported
@@ -55,7 +66,7 @@ svdq_status current_device(int* dev_out, DeviceInfo* info_out) {
       return SVDQ_ERR_UNSUPPORTED_DEVICE;
     }
     di.sm_count = sms;
-    di.ok = (major == 10 && minor == 0) ? 1 : 0;
+    di.ok = svdq_device_supported(major, minor) == SVDQ_OK ? 1 : 0;
   }
   if (di.ok != 1) return SVDQ_ERR_UNSUPPORTED_DEVICE;
   if (dev_out) *dev_out = dev;
