@@ -19,10 +19,21 @@
 #include "awq_w4a16.cuh"
 #include "quantize_act.cuh"
 
+#include <nvtx3/nvToolsExt.h>
+
 namespace svdq {
 namespace {
 
 constexpr int kVersion = 100;  // 0.1.0
+
+// NVTX range around one entry point (for timeline profilers; a no-op when no
+// tool is attached).
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool valid_rank(int r) { return r == 16 || r == 32 || r == 64 || r == 128; }
@@ -900,6 +911,7 @@ svdq_status svdq_forward_workspace_size(int M, int K, int r, size_t* bytes) {
 svdq_status svdq_pack_weight(int N, int K, int r, const void* W, const void* L1, const void* L2, const float* smooth,
                              const float* g_x, void* w_codes, void* w_scales, float* gscale, void* l1t, void* l2s,
                              float* inv_smooth, void* stream) {
+  NvtxRange nvtx_range("svdq_pack_weight");
   svdq_status s = check_layer_shape(N, K, r);
   if (s != SVDQ_OK) return s;
   if (!W || !L1 || !L2 || !g_x || !w_codes || !w_scales || !gscale || !l1t || !l2s) return SVDQ_ERR_INVALID_ARG;
@@ -937,6 +949,7 @@ svdq_status svdq_lowrank_workspace_size(int N, int K, int r, size_t* bytes) {
 svdq_status svdq_lowrank_init(int N, int K, int r, const void* W, const float* smooth, void* L1, void* L2,
                               double* sigma, unsigned long long seed, int power_iters, void* workspace,
                               size_t ws_bytes, void* stream) {
+  NvtxRange nvtx_range("svdq_lowrank_init");
   if (N <= 0 || K <= 0 || !valid_rank(r) || !W || !L1 || !L2 || !workspace || power_iters < 0 || power_iters > 64)
     return SVDQ_ERR_INVALID_ARG;
   if (r > N || r > K || K % 8 != 0) return SVDQ_ERR_UNSUPPORTED_SHAPE;
@@ -954,6 +967,7 @@ svdq_status svdq_lowrank_init(int N, int K, int r, const void* W, const float* s
 
 svdq_status svdq_act_global_scale(int M, int K, const void* X, int64_t ldx, const float* inv_smooth, float* g_out,
                                   void* stream) {
+  NvtxRange nvtx_range("svdq_act_global_scale");
   if (M < 0 || K <= 0 || !X || !g_out) return SVDQ_ERR_INVALID_ARG;
   if (K % 8 != 0 || ldx < K || ldx % 8 != 0) return SVDQ_ERR_UNSUPPORTED_SHAPE;
   if (!aligned16(X) || (reinterpret_cast<uintptr_t>(g_out) & 3u) || (inv_smooth && !aligned16(inv_smooth)))
@@ -973,6 +987,7 @@ svdq_status svdq_act_global_scale(int M, int K, const void* X, int64_t ldx, cons
 
 svdq_status svdq_smooth_factors(int M, int N, int K, const void* X, int64_t ldx, const void* W, float alpha,
                                 float* lambda, void* stream) {
+  NvtxRange nvtx_range("svdq_smooth_factors");
   if (M < 0 || N <= 0 || K <= 0 || !X || !W || !lambda || !(alpha >= 0.0f && alpha <= 1.0f))
     return SVDQ_ERR_INVALID_ARG;
   if (K % 8 != 0 || ldx < K || ldx % 8 != 0) return SVDQ_ERR_UNSUPPORTED_SHAPE;
@@ -989,6 +1004,7 @@ svdq_status svdq_smooth_factors(int M, int N, int K, const void* X, int64_t ldx,
 
 svdq_status svdq_quantize_act(int M, int K, int r, const void* X, int64_t ldx, const float* g_x, const void* l1t,
                               const float* inv_smooth, void* codes, void* scales, void* xl1, void* stream) {
+  NvtxRange nvtx_range("svdq_quantize_act");
   if (M < 0 || K <= 0 || !valid_rank(r)) return SVDQ_ERR_INVALID_ARG;
   if (K % 256 != 0 || ldx < K || ldx % 8 != 0) return SVDQ_ERR_UNSUPPORTED_SHAPE;
   if (M == 0) return SVDQ_OK;
@@ -1006,6 +1022,7 @@ svdq_status svdq_quantize_act(int M, int K, int r, const void* X, int64_t ldx, c
 svdq_status svdq_w4a4_gemm(int M, int N, int K, int r, const void* a_codes, const void* a_scales, const void* xl1,
                            const void* w_codes, const void* w_scales, const float* gscale, const void* l2s,
                            const void* bias, void* Y, int64_t ldy, void* stream) {
+  NvtxRange nvtx_range("svdq_w4a4_gemm");
   return gemm_checked(M, N, K, r, a_codes, a_scales, xl1, w_codes, w_scales, gscale, l2s, bias, Y, ldy, stream,
                       nullptr);
 }
@@ -1016,6 +1033,7 @@ svdq_status svdq_linear_forward_qkv(int M, int N, int K, int r, const void* X, i
                                     const void* norm_k_weight, float eps, const float* rope_cos,
                                     const float* rope_sin, int64_t ld_rope, void* Y, int64_t ldy, void* workspace,
                                     size_t workspace_bytes, void* stream) {
+  NvtxRange nvtx_range("svdq_linear_forward_qkv");
   if (M < 0 || heads <= 0 || !(eps >= 0.0f && eps < 1e30f)) return SVDQ_ERR_INVALID_ARG;
   svdq_status s = check_layer_shape(N, K, r);
   if (s != SVDQ_OK) return s;
@@ -1066,6 +1084,7 @@ svdq_status svdq_mlp_up_forward(int M, int N, int K, int r, const void* X, int64
                                 const float* inv_smooth, const void* bias, int r_down, const float* g_h,
                                 const void* l1_down, int approximate, void* h_codes, void* h_scales, void* h_xl1,
                                 void* h_out, int64_t ldh, void* workspace, size_t workspace_bytes, void* stream) {
+  NvtxRange nvtx_range("svdq_mlp_up_forward");
   if (M < 0) return SVDQ_ERR_INVALID_ARG;
   svdq_status s = check_layer_shape(N, K, r);
   if (s != SVDQ_OK) return s;
@@ -1146,6 +1165,7 @@ svdq_status svdq_linear_forward(int M, int N, int K, int r, const void* X, int64
                                 const void* w_scales, const float* gscale, const void* l1t, const void* l2s,
                                 const float* inv_smooth, const void* bias, void* Y, int64_t ldy, void* workspace,
                                 size_t workspace_bytes, void* stream) {
+  NvtxRange nvtx_range("svdq_linear_forward");
   if (M < 0) return SVDQ_ERR_INVALID_ARG;
   svdq_status s = check_layer_shape(N, K, r);
   if (s != SVDQ_OK) return s;
@@ -1191,6 +1211,7 @@ svdq_status svdq_linear_forward_dynamic(int M, int N, int K, int r, const void* 
                                         const void* w_scales, const float* gscale, const void* l1t, const void* l2s,
                                         const float* inv_smooth, const void* bias, void* Y, int64_t ldy,
                                         void* workspace, size_t workspace_bytes, void* stream) {
+  NvtxRange nvtx_range("svdq_linear_forward_dynamic");
   if (M < 0) return SVDQ_ERR_INVALID_ARG;
   svdq_status s = check_layer_shape(N, K, r);
   if (s != SVDQ_OK) return s;
@@ -1246,6 +1267,7 @@ svdq_status svdq_awq_sizes(int N, int K, size_t* codes_bytes, size_t* scales_byt
 
 svdq_status svdq_awq_pack(int N, int K, const void* W, const float* act_scale, void* codes, void* scales,
                           void* zeros, float* inv_act, void* stream) {
+  NvtxRange nvtx_range("svdq_awq_pack");
   if (N <= 0 || K <= 0 || !W || !codes || !scales || !zeros) return SVDQ_ERR_INVALID_ARG;
   if ((act_scale == nullptr) != (inv_act == nullptr)) return SVDQ_ERR_INVALID_ARG;
   if (K % kAwqGroup != 0) return SVDQ_ERR_UNSUPPORTED_SHAPE;
@@ -1299,6 +1321,7 @@ extern "C" {
 svdq_status svdq_awq_gemv(int M, int N, int K, const void* X, int64_t ldx, const void* codes, const void* scales,
                           const void* zeros, const float* inv_act, const void* bias, void* Y, int64_t ldy,
                           void* stream) {
+  NvtxRange nvtx_range("svdq_awq_gemv");
   if (M < 0 || N <= 0 || K <= 0) return SVDQ_ERR_INVALID_ARG;
   if (K % kAwqGroup != 0 || ldx < K || ldx % 8 != 0 || ldy < N) return SVDQ_ERR_UNSUPPORTED_SHAPE;
   if (M == 0) return SVDQ_OK;
