@@ -32,11 +32,14 @@ struct QkvPost {
   float eps;
 };
 
-// Epilogue of an MLP pair's up projection: h = bf16(GELU(bf16(alpha acc + b)))
-// quantised in place for the down projection (NVFP4 codes and tiled block
-// scales with the down projection's activation scale g_h) and its fp32 partial
-// products with the down projection's L1 (XL1 partials per 128-column half
-// tile, summed afterwards in tile order).
+// Epilogue of an MLP pair's up projection (blog "Bringing Nunchaku 4-bit
+// Diffusion Inference to Diffusers", section "Quantizing models with
+// structural rewrites": the engine's fused GELU / MLP kernels):
+// h = bf16(GELU(bf16(alpha acc + b))) quantised in place for the down
+// projection (NVFP4 codes and tiled block scales with the down projection's
+// activation scale g_h) and its fp32 partial products with the down
+// projection's L1 (XL1 partials per 128-column half tile, summed afterwards
+// in tile order).
 struct MlpPost {
   const float* g_h;           // device float: the down projection's activation decode scale
   const __nv_bfloat16* l1d;   // [N][r_down] row-major: the down projection's L1 (its K = this layer's N)
