@@ -62,6 +62,16 @@ def _quant_bytes(M, K, r):
     return 2 * M * K + M * K / 2 + M * K / 16 + 2 * M * r + 2 * K * r
 
 
+def gpu_uuid(device: int) -> str | None:
+    """nvidia-smi's identifier ("GPU-xxxxxxxx-...") of the CUDA device `device`,
+    or None if it cannot be read."""
+    try:
+        u = str(torch.cuda.get_device_properties(device).uuid)
+    except (RuntimeError, AssertionError, AttributeError):
+        return None
+    return u if u.startswith("GPU-") else "GPU-" + u
+
+
 class ClockSampler:
     """nvidia-smi clocks / throttle reasons sampled every 50 ms while running."""
 
@@ -69,15 +79,22 @@ class ClockSampler:
               "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
               "clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, index: int):
-        self.index = index
+    def __init__(self, uuid: str | None):
+        # nvidia-smi numbers GPUs physically and ignores CUDA_VISIBLE_DEVICES, so
+        # a CUDA ordinal may name another (possibly another user's) GPU: the
+        # device is selected by its UUID (gpu_uuid), and without one nothing is
+        # sampled.
+        self.uuid = uuid
         self.proc = None
 
     def __enter__(self):
+        if self.uuid is None:
+            time.sleep(0.3)
+            return self
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "50",
-                 "-i", str(self.index)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-i", self.uuid], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
         time.sleep(0.3)
@@ -97,13 +114,13 @@ class ClockSampler:
     def summary(self):
         rows = [l.split(",") for l in (self.out or "").strip().splitlines() if l.count(",") >= 6]
         if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "gpu_uuid": self.uuid}
         sm = [float(r[0]) for r in rows if r[0].strip().replace(".", "").isdigit()]
         mx = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = sorted({names[i] for r in rows for i in range(4) if "Active" == r[3 + i].strip()})
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(rows)}
+                "reasons": reasons, "samples": len(rows), "gpu_uuid": self.uuid}
 
 
 def _dist_init():
@@ -215,6 +232,136 @@ def _gemm_kernel_name(M, N):
     return "w4a4_gemm_2sm_kernel" if N % 256 == 0 and M >= 512 else "w4a4_gemm_kernel"
 
 
+def _gemm_pass_bytes(M, N, K, r):
+    return (M * K + N * K) * (0.5 + 1.0 / 16) + 2 * M * r + 2 * r * N + 2 * N + 2 * M * N
+
+
+def _pct(v, q):
+    v = sorted(v)
+    return v[min(len(v) - 1, max(0, int(round(q * (len(v) - 1)))))]
+
+
+def _oracle_layer_rate(spec, X, W, b, budget_s):
+    """The CPU oracle's forward (activation quantisation, down projection,
+    4-bit product, up projection, bias; float64) on a bounded slice of one
+    layer: the first S rows against the first Ns output features (rows and
+    features are independent, so the slice is exact work of the layer). The
+    low-rank factors are stand-ins of the right shapes (bf16 slices of W): the
+    forward's cost does not depend on their values, and the LAPACK SVD of the
+    large weights would dominate the bench's time. Returns (TFLOP/s, sample)."""
+    from oracle import svdq as osv
+    r = spec.r
+    L1 = W[:r].T.contiguous()
+    L2 = W[:, :r].T.contiguous()
+    S = min(spec.M, 64)
+    g_x = osv.act_global_scale(X[:S])
+
+    def run(ns):
+        pw = osv.pack_weight(W[:ns], L1, L2[:, :ns])
+        t0 = time.perf_counter()
+        osv.forward(X[:S], pw, b[:ns], g_x)
+        return time.perf_counter() - t0
+
+    unit = min(spec.N, 128)
+    t_unit = max(run(unit), 1e-4)
+    ns = int(max(1, min(spec.N // unit, budget_s / t_unit))) * unit
+    dt = run(ns) if ns != unit else t_unit
+    return _flops(S, ns, spec.K, r) / dt / 1e12, f"first {S} of {spec.M} rows x first {ns} of {spec.N} features"
+
+
+def _bench_layer(svdq, spec, dev, stream, reps, peaks, oracle_budget_s):
+    """One layer of a workload: cold-input steps (quantiser + GEMM, rotating
+    input copies totalling at least twice the L2 size), a hot-L2 pass (the same
+    inputs every step), per-kernel times, and the oracle's rate beside it."""
+    M, K, N, r = spec.M, spec.K, spec.N, spec.r
+    X, W, b = workloads.make_layer(spec)
+    Xd, bd, Wd = X.to(dev), b.to(dev), W.to(dev)
+    g_x = svdq.svdq_act_global_scale(Xd)
+    L1, L2, _ = svdq.svdq_lowrank_init(Wd, r)
+    pw = svdq.svdq_pack_weight(Wd, L1, L2, g_x)
+    del Wd, L1, L2
+    l2_bytes = torch.cuda.get_device_properties(dev).L2_cache_size
+    set_bytes = Xd.numel() * 2 + sum(getattr(pw, n).numel() * getattr(pw, n).element_size()
+                                     for n in ("codes", "scales", "gscale", "l1t", "l2s"))
+    n_sets = max(2, -(-2 * l2_bytes // set_bytes))
+    Xs = [Xd] + [Xd.clone() for _ in range(n_sets - 1)]
+    pws = [pw] + [_clone_packed(svdq, pw, dev) for _ in range(n_sets - 1)]
+    qa = svdq.QuantAct(M, K, r, dev)
+    Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+
+    def step(j):
+        svdq.svdq_quantize_act(Xs[j], pws[j], out=qa)
+        svdq.svdq_w4a4_gemm(qa, pws[j], bd, out=Y)
+
+    for i in range(max(10, n_sets)):
+        step(i % n_sets)
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(reps)]
+    for i in range(reps):          # steps as the headline times them (no event between the kernels)
+        ev[i][0].record(stream)
+        step(i % n_sets)
+        ev[i][2].record(stream)
+    torch.cuda.synchronize()
+    t_step = [e[0].elapsed_time(e[2]) for e in ev]
+    for i in range(reps):          # hot L2: the same inputs every step
+        ev[i][0].record(stream)
+        step(0)
+        ev[i][2].record(stream)
+    torch.cuda.synchronize()
+    t_hot = [e[0].elapsed_time(e[2]) for e in ev]
+    for i in range(reps):          # per kernel (an event between them)
+        j = i % n_sets
+        ev[i][0].record(stream)
+        svdq.svdq_quantize_act(Xs[j], pws[j], out=qa)
+        ev[i][1].record(stream)
+        svdq.svdq_w4a4_gemm(qa, pws[j], bd, out=Y)
+        ev[i][2].record(stream)
+    torch.cuda.synchronize()
+    t_q = [e[0].elapsed_time(e[1]) for e in ev]
+    t_g = [e[1].elapsed_time(e[2]) for e in ev]
+    if svdq.svdq_read_device_error() != 0:
+        raise RuntimeError(f"device error while timing {spec.name}")
+    med, q_ms, g_ms = statistics.median(t_step), statistics.median(t_q), statistics.median(t_g)
+    fp4_peak = peaks["bf16_tflops"] * FP4_PER_BF16
+    o_rate, o_sample = _oracle_layer_rate(spec, X, W, b, oracle_budget_s)
+    del Xs, pws, qa, Y
+    return {
+        "layer": spec.name, "M": M, "K": K, "N": N, "r": r, "gemm_kernel": _gemm_kernel_name(M, N),
+        "input_sets": n_sets,
+        "step_ms": {"median": med, "p10": _pct(t_step, 0.1), "p90": _pct(t_step, 0.9)},
+        "hot_l2_step_ms": statistics.median(t_hot),
+        "tflops": _flops(M, N, K, r) / (med * 1e-3) / 1e12,
+        "tokens_per_s": M / (med * 1e-3),
+        "gemm_ms": g_ms,
+        "gemm_frac_of_fp4_peak": 2.0 * M * N * K / (g_ms * 1e-3) / 1e12 / fp4_peak,
+        "gemm_frac_of_hbm": _gemm_pass_bytes(M, N, K, r) / (g_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+        "quant_ms": q_ms,
+        "quant_frac_of_hbm": _quant_bytes(M, K, r) / (q_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+        "oracle": {"tflops": o_rate, "cores": _cores(), "sample": o_sample},
+    }
+
+
+def bench_configs(svdq, dev, stream, reps=100, oracle_budget_s=1.0):
+    """Every benchmark workload (1-5), each layer timed separately; a workload's
+    time is the sum of its layers' median step times."""
+    peaks, kind = _peaks()
+    out = {"note": ("per layer: step = quantiser + GEMM with cold inputs (rotating copies >= 2x L2), median / "
+                    "p10 / p90 over the steps; hot_l2_step_ms with the same inputs every step; gemm_* and "
+                    "quant_* from a pass with an event between the kernels; fractions of "
+                    f"{kind} peaks (fp4 = bf16 burst x {FP4_PER_BF16:g}); oracle = float64 CPU oracle on a "
+                    "bounded slice"), "reps": reps}
+    for wid, wl in workloads.WORKLOADS.items():
+        layers = [_bench_layer(svdq, spec, dev, stream, reps, peaks, oracle_budget_s) for spec in wl.layers]
+        t = sum(L["step_ms"]["median"] for L in layers)
+        fl = sum(_flops(L["M"], L["N"], L["K"], L["r"]) for L in layers)
+        entry = {"workload": wl.name, "layers": layers}
+        if wid in (3, 4):   # one block's layers in sequence: their times summed
+            entry.update({"ms_sum": t, "tflops": fl / (t * 1e-3) / 1e12,
+                          "tokens_per_s": wl.layers[0].M / (t * 1e-3)})
+        out[str(wid)] = entry
+    return out
+
+
 def run_ours(args, spec):
     world, rank, local = _dist_init()
     torch.cuda.set_device(local)
@@ -259,7 +406,7 @@ def run_ours(args, spec):
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
     _barrier(world)
     torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
+    with ClockSampler(gpu_uuid(local)) as clk:
         for i in range(args.steps):
             j = (args.warmup + i) % n_sets
             ev[i][0].record(stream)
@@ -464,6 +611,10 @@ def run_ours(args, spec):
     except Exception as exc:  # reported, not fatal: the headline line above is complete without it
         variants["mlp_pair_4608x3072x12288_r32"] = {"error": f"{type(exc).__name__}: {str(exc)[:160]}"}
 
+    configs = None
+    if not args.no_configs:
+        configs = bench_configs(svdq, dev, stream, reps=100 if args.steps >= 100 else max(args.steps, 10))
+
     peaks, kind = _peaks()
     gemm_name = _gemm_kernel_name(M, N)
     fp4_peak = peaks["bf16_tflops"] * FP4_PER_BF16
@@ -496,6 +647,7 @@ def run_ours(args, spec):
                 "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2, "ms_per_step": e2e_ms},
         "qkv_norm_rope": qkv,
         "variants": variants,
+        "configs": configs,
         "gpu_launches": 2 * args.steps,
         "clocks": clk.summary(),
     }
@@ -520,6 +672,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true", help="skip the per-workload table (configs 1-5)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

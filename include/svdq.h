@@ -309,8 +309,8 @@ svdq_status svdq_linear_forward_noalloc(int M, int N, int K, int r, const void* 
 /* ------------------------------------------------------------ MLP pair */
 /* The up projection of a transformer block's feed-forward pair with GELU and
  * the down projection's activation quantisation fused into its GEMM epilogue
- * (blog section "Quantizing models with structural rewrites": the engine's
- * fused GELU / MLP kernels). For the layer X [M][K] -> N (arguments as
+ * (blog section "Introducing Nunchaku Lite": part of the full engine's speed
+ * comes from fused GELU / MLP kernels). For the layer X [M][K] -> N (arguments as
  * svdq_linear_forward):
  *   y = bf16(layer output), h = bf16(GELU(y)) (GELU = x Phi(x), or with
  *   approximate != 0 its tanh form; fp32, evaluated without cancellation in
@@ -373,6 +373,19 @@ svdq_status svdq_awq_gemv(int M, int N, int K, const void* X, int64_t ldx, const
  * device: 0 or an svdq_status recorded by a kernel (e.g. SVDQ_ERR_TIMEOUT).
  * Synchronises the device first. */
 svdq_status svdq_read_device_error(int* code, int clear);
+
+/* Self-test of the bounded waits (blog section "Hardware support": a failure
+ * must surface as a clear error, not as wrong outputs or a hung process).
+ * Every kernel of this library waits on mbarriers with a time limit; when a
+ * limit runs out the kernel records SVDQ_ERR_TIMEOUT in the per-device error
+ * word and returns. This call launches one small kernel, asynchronously on
+ * `stream`, whose single wait is on an mbarrier that nothing ever arrives on,
+ * with a limit of limit_us microseconds (1 .. 1000000; otherwise
+ * SVDQ_ERR_INVALID_ARG and no launch). After the caller synchronises,
+ * svdq_read_device_error returns SVDQ_ERR_TIMEOUT, and the CUDA context stays
+ * usable: the kernel ends normally, with no trap and no fault. Nothing else
+ * is read or written. */
+svdq_status svdq_selftest_bounded_wait(int limit_us, void* stream);
 
 #ifdef __cplusplus
 }

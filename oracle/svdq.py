@@ -35,8 +35,9 @@ Functions, in the order the method applies them:
                     structural rewrites": the fused operator consumes the QKV
                     projection, the Q/K normalisation and the rotary embedding
                     together)
-  mlp_pair          up projection, GELU, down projection (the same section
-                    names fused GELU / MLP kernels)
+  mlp_pair          up projection, GELU, down projection (section
+                    "Introducing Nunchaku Lite" names the full engine's fused
+                    GELU / MLP kernels)
 """
 from __future__ import annotations
 
@@ -266,8 +267,8 @@ class MlpPair:
 def mlp_pair(X, pw_up: PackedWeight, b_up, g_up, pw_down: PackedWeight, b_down, g_h,
              approximate: bool = False) -> MlpPair:
     """The feed-forward pair of a transformer block as two W4A4 layers with GELU
-    between them (blog section "Quantizing models with structural rewrites":
-    the engine fuses GELU / MLP kernels): h = bf16(GELU(bf16(up(X)))), what the
+    between them (blog section "Introducing Nunchaku Lite": part of the full
+    engine's speed comes from fused GELU / MLP kernels): h = bf16(GELU(bf16(up(X)))), what the
     unfused sequence hands the down projection, which quantises h with its own
     activation scale g_h."""
     up = forward(X, pw_up, b_up, g_up)

@@ -36,3 +36,23 @@ def bf16_ulp_distance(a: np.ndarray, b: np.ndarray) -> np.ndarray:
         u = (np.asarray(x, dtype=np.float64).astype(np.float32).view(np.uint32) >> 16).astype(np.int64)
         return np.where(u & 0x8000, 0x8000 - u, u)
     return np.abs(ordinal(a) - ordinal(b))
+
+
+def bf16_half_ulp(x: np.ndarray) -> np.ndarray:
+    """Half the bf16 spacing at |x| (8 significant bits): the largest error of
+    rounding a real number to the nearest bf16 value x."""
+    return np.ldexp(1.0, np.frexp(np.abs(np.asarray(x, dtype=np.float64)))[1] - 9)
+
+
+def sum_error_bound(n_roundings: int, abs_sum, unit_roundoff: float) -> np.ndarray:
+    """Higham's bound on the error of a sum evaluated with n_roundings rounded
+    additions in any order (Accuracy and Stability of Numerical Algorithms,
+    2nd ed., eq. 4.4): gamma_n * sum|terms| with gamma_n = n u / (1 - n u).
+    Each term must be exact in the working precision (a product of two bf16
+    values is exact in fp32). u = 2^-24 for round-to-nearest fp32; u = 2^-23
+    covers any faithful rounding (round-toward-zero included), the guarantee
+    used for the tensor cores' internal accumulation, whose rounding is not
+    specified."""
+    nu = n_roundings * unit_roundoff
+    assert nu < 0.5
+    return nu / (1.0 - nu) * np.asarray(abs_sum, dtype=np.float64)

@@ -3,9 +3,9 @@
 Bars (from the layer's acceptance criteria):
   * activation codes and scales, packed weight codes / scales / g_w: bit-exact;
   * XL1: within half a bf16 ulp of its own value plus the fp32 summation error
-    bound 2 K 2^-24 sum|x l1| of the exact float64 product (the blog's fused
-    down projection accumulates in fp32 in an order it does not fix), and at
-    most 0.1 % of elements more than 1 bf16 ulp from the oracle;
+    bound of the exact float64 product (the blog's fused down projection
+    accumulates in fp32 in an order it does not fix; see _check_xl1), and within
+    1 bf16 ulp of the oracle wherever that bound is below a quarter ulp;
   * Y: relative Frobenius error <= 1e-3 against the oracle output rounded to
     bf16, and max |Y - y64| <= 2e-2 * RMS of the y64 row.
 Inputs come from the seeded generators in workloads.py; the oracle computes
@@ -69,20 +69,27 @@ def _check_act(lib, X, L1, r, g_x, qa, M, K):
 
 
 def _check_xl1(xl1_gpu, X, L1):
-    """XL1 = bf16(X . L1) accumulated in fp32: |gpu - exact| <= 1/2 ulp_bf16(gpu)
-    (the final rounding) + 2 K 2^-24 sum_k |x_k L1_kj| (fp32 summation in any
-    order, Higham's bound with a factor 2 of slack for tensor-core accumulation).
-    Where the sum does not cancel this is within one bf16 ulp of the oracle."""
+    """XL1 = bf16(X . L1): K exact products (bf16 x bf16 fits fp32) summed in
+    fp32 by the tensor cores and the K-split's partial additions, K - 1
+    roundings in an order the pages leave open, then one rounding to bf16.
+      * bound: |gpu - exact| <= 1/2 ulp_bf16(gpu) + gamma_{K-1} sum_k |x_k L1_kj|
+        with u = 2^-23 (any faithful rounding; the tensor cores' internal
+        rounding is not specified), plus the oracle's own float64 error;
+      * where that summation bound is below a quarter of a bf16 ulp of the
+        oracle's value, the fp32 sum and the exact sum round to bf16 values at
+        most one step apart, so those elements must be within 1 ulp."""
     X64, L164 = osv.to_f64(X), osv.to_f64(L1)
     exact = X64 @ L164
     absum = np.abs(X64) @ np.abs(L164)
     K = X64.shape[1]
-    half_ulp = np.ldexp(1.0, np.frexp(np.abs(xl1_gpu))[1] - 9)
-    bound = half_ulp + 2.0 * K * 2.0 ** -24 * absum
+    summ = layouts.sum_error_bound(K - 1, absum, 2.0 ** -23) + layouts.sum_error_bound(K, absum, 2.0 ** -53)
+    bound = layouts.bf16_half_ulp(xl1_gpu) + summ
     err = np.abs(xl1_gpu - exact)
     assert np.all(err <= bound), f"XL1 error {np.max(err / bound):.2f} x bound"
-    ulps = layouts.bf16_ulp_distance(xl1_gpu, osv.down_proj(X, L1))
-    assert np.mean(ulps > 1) < 1e-3, f"XL1: {np.mean(ulps > 1):.2e} of elements beyond 1 ulp"
+    oracle = osv.down_proj(X, L1)
+    tight = summ < 0.5 * layouts.bf16_half_ulp(oracle)
+    ulps = layouts.bf16_ulp_distance(xl1_gpu, oracle)
+    assert np.all(ulps[tight] <= 1), f"XL1: {np.sum(ulps[tight] > 1)} elements beyond 1 ulp where the bound allows 1"
 
 
 def _check_y(Y, fwd, rows=None):

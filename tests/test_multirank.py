@@ -98,7 +98,8 @@ def test_clock_sampler_summary_parses_nvidia_smi_lines():
     largest max clock, and every throttle reason seen Active in any sample."""
     sys.path.insert(0, ROOT)
     import bench
-    cs = bench.ClockSampler(0)
+    cs = bench.ClockSampler("GPU-00000000-0000-0000-0000-000000000000")
+    assert cs.uuid.startswith("GPU-")
     cs.out = "\n".join([
         "1965, 1965, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active",
         "1800, 1965, 0x0000000000000004, Not Active, Not Active, Not Active, Active",

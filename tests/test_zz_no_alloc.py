@@ -2,8 +2,9 @@
 provide a workspace (runtime plugin interfaces that pass only a layer's inputs
 and outputs; code that must not call an allocator once its memory budget is
 fixed). It is called through the C ABI and compared with svdq_linear_forward,
-which takes a caller-provided workspace, on two calls in a row. This file is
-collected last so that a run stopping at its first failure has already run
+which takes a caller-provided workspace, on two calls in a row after a larger
+call has dirtied the shared scratch; the outputs must be bit-identical. This
+file is collected last so that a run stopping at its first failure has already run
 every other test."""
 import ctypes
 
@@ -39,27 +40,45 @@ def _noalloc(L, X, pw, bias, Y):
                                          Y.stride(0), stream)
 
 
+def _layer(lib, M, K, N, r, seed):
+    _, (X, W, b) = workloads.small_layer(M, K, N, r, seed=seed)
+    L1, L2, _ = osv.lowrank_factors(W, r)
+    to_dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(torch.bfloat16).cuda()  # noqa: E731
+    g_x = osv.act_global_scale(X)
+    pw = lib.svdq_pack_weight(W.cuda(), to_dev(L1), to_dev(L2), float(g_x))
+    return X, W, b, L1, L2, g_x, pw
+
+
 @pytest.mark.parametrize("M,K,N,r", [(256, 1024, 1024, 32), (333, 768, 384, 64)])
 def test_noalloc_forward_matches_workspace_forward(lib, M, K, N, r):
     L = lib.lib()
-    _, (X, W, b) = workloads.small_layer(M, K, N, r, seed=21)
-    L1, L2, _ = osv.lowrank_factors(W, r)
-    to_dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(torch.bfloat16).cuda()  # noqa: E731
-    g_x = float(osv.act_global_scale(X))
-    pw = lib.svdq_pack_weight(W.cuda(), to_dev(L1), to_dev(L2), g_x)
+    # Leave non-zero bytes in the shared scratch first (a larger call with
+    # another K and rank), so nothing below can rely on it starting at zero.
+    Xp, _, bp, _, _, _, pwp = _layer(lib, 640, 2048, 256, 128, seed=5)
+    Yp = torch.empty((640, 256), dtype=torch.bfloat16, device="cuda")
+    assert _noalloc(L, Xp.cuda(), pwp, bp.cuda(), Yp) == 0
+    torch.cuda.synchronize()
+
+    X, W, b, L1, L2, g_x, pw = _layer(lib, M, K, N, r, seed=21)
     Xd, bd = X.cuda(), b.cuda()
-    ref = lib.svdq_linear_forward(Xd, pw, bd).double().cpu().numpy()
+    # the workspace forward, its workspace filled with 0xFF bytes (NaN patterns)
+    ws = torch.full((lib.svdq_forward_workspace_size(M, K, r),), 0xFF, dtype=torch.uint8, device="cuda")
+    ref = lib.svdq_linear_forward(Xd, pw, bd, workspace=ws)
     outs = []
     for _ in range(2):                       # two calls in a row share the scratch
         Y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
         assert _noalloc(L, Xd, pw, bd, Y) == 0
         torch.cuda.synchronize()
-        outs.append(Y.double().cpu().numpy())
+        outs.append(Y)
     assert lib.svdq_read_device_error() == 0
+    # the same kernels on the same inputs: bit-identical to the workspace forward
     for y in outs:
-        assert np.isfinite(y).all()
-        assert osv.rel_fro(y, ref) <= REL_FRO
-        assert osv.max_abs_over_row_rms(y, ref) <= MAX_ROWRMS
+        assert torch.equal(y, ref)
+    # and within the layer's bars of the CPU oracle
+    o = osv.forward(X, osv.pack_weight(W, L1, L2), b, g_x)
+    y = outs[-1].double().cpu().numpy()
+    assert osv.rel_fro(y, o.y_ref) <= REL_FRO
+    assert osv.max_abs_over_row_rms(y, o.y64) <= MAX_ROWRMS
 
 
 def test_noalloc_rejects_shapes_beyond_the_scratch_limit(lib):

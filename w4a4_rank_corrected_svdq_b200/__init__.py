@@ -38,6 +38,7 @@ from ._lib import (  # noqa: F401
     svdq_quantize_act,
     svdq_read_device_error,
     svdq_scale_offset,
+    svdq_selftest_bounded_wait,
     svdq_smooth_factors,
     svdq_w4a4_gemm,
     svdq_weight_sizes,

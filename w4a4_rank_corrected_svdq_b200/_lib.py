@@ -39,6 +39,7 @@ SIGNATURES = {
     "svdq_w4a4_gemm": (_i, [_i, _i, _i, _i, _p, _p, _p, _p, _p, _p, _p, _p, _p, _i64, _p]),
     "svdq_linear_forward": (_i, [_i, _i, _i, _i, _p, _i64, _p, _p, _p, _p, _p, _p, _p, _p, _i64, _p, _sz, _p]),
     "svdq_read_device_error": (_i, [_pi, _i]),
+    "svdq_selftest_bounded_wait": (_i, [_i, _p]),
     "svdq_linear_forward_noalloc": (_i, [_i, _i, _i, _i, _p, _i64, _p, _p, _p, _p, _p, _p, _p, _p, _i64, _p]),
     "svdq_linear_forward_qkv": (_i, [_i, _i, _i, _i, _p, _i64, _p, _p, _p, _p, _p, _p, _p, _i, _p, _p, _f, _p,
                                      _p, _i64, _p, _i64, _p, _sz, _p]),
@@ -455,6 +456,12 @@ def svdq_awq_gemv(X: torch.Tensor, aw: AwqWeight, bias: torch.Tensor | None = No
                                                 _ptr(aw.zeros), _ptr(aw.inv_act), _ptr(bias), _ptr(Y), ldy,
                                                 _stream(X)))
     return Y
+
+
+def svdq_selftest_bounded_wait(limit_us: int = 1000) -> None:
+    """Launch the bounded-wait self-test on the current stream (its wait gives up
+    after limit_us and records SVDQ_ERR_TIMEOUT in the device error word)."""
+    _check("svdq_selftest_bounded_wait", lib().svdq_selftest_bounded_wait(int(limit_us), _stream()))
 
 
 def svdq_read_device_error(clear: bool = True) -> int:

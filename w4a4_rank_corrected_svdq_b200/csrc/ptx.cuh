@@ -61,9 +61,11 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Waits until the phase with the given parity of `bar` has completed.
-// Returns false (and records SVDQ_ERR_TIMEOUT = 6) if it did not within the limit
-// or if another role of the CTA has already given up (*abort != 0).
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+// Returns false (and records SVDQ_ERR_TIMEOUT = 6) if it did not within
+// limit_ns nanoseconds or if another role of the CTA has already given up
+// (*abort != 0); on a timeout it sets *abort so the CTA's other roles stop too.
+__device__ __forceinline__ bool mbar_wait_for(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                              uint64_t limit_ns) {
   const uint32_t a = smem_u32(bar);
   if (mbar_try_wait(a, parity)) return true;
   const uint64_t t0 = globaltimer();
@@ -72,12 +74,16 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     for (int i = 0; i < 32; ++i)
       if (mbar_try_wait(a, parity)) return true;
     if (*abort) return false;
-    if (globaltimer() - t0 > kWaitLimitNs) {
+    if (globaltimer() - t0 > limit_ns) {
       record_error(6);
       *abort = 1;
       return false;
     }
   }
+}
+// The wait every kernel uses: mbar_wait_for with the library-wide limit.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  return mbar_wait_for(bar, parity, abort, kWaitLimitNs);
 }
 
 // ------------------------------------------------------------------ clusters

@@ -33,8 +33,8 @@ struct QkvPost {
 };
 
 // Epilogue of an MLP pair's up projection (blog "Bringing Nunchaku 4-bit
-// Diffusion Inference to Diffusers", section "Quantizing models with
-// structural rewrites": the engine's fused GELU / MLP kernels):
+// Diffusion Inference to Diffusers", section "Introducing Nunchaku Lite":
+// the full engine's speed comes partly from fused GELU / MLP kernels):
 // h = bf16(GELU(bf16(alpha acc + b))) quantised in place for the down
 // projection (NVFP4 codes and tiled block scales with the down projection's
 // activation scale g_h) and its fp32 partial products with the down

@@ -1353,6 +1353,40 @@ svdq_status svdq_awq_gemv(int M, int N, int K, const void* X, int64_t ldx, const
   }
 }
 
+}  // extern "C"
+
+namespace svdq {
+namespace {
+// The bounded wait of every kernel, exercised on purpose: one thread waits on
+// an mbarrier that nothing arrives on, with a short limit, so the wait gives
+// up, records SVDQ_ERR_TIMEOUT and the kernel returns normally.
+__global__ void bounded_wait_selftest_kernel(uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait_for(&bar, 0, &abort_flag, limit_ns);
+  __syncthreads();
+}
+}  // namespace
+}  // namespace svdq
+
+extern "C" {
+
+svdq_status svdq_selftest_bounded_wait(int limit_us, void* stream) {
+  NvtxRange nvtx_range("svdq_selftest_bounded_wait");
+  if (limit_us < 1 || limit_us > 1000000) return SVDQ_ERR_INVALID_ARG;
+  svdq_status s;
+  if ((s = current_device(nullptr, nullptr)) != SVDQ_OK) return s;
+  bounded_wait_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<uint64_t>(limit_us) * 1000ull);
+  return launch_status();
+}
+
 svdq_status svdq_read_device_error(int* code, int clear) {
   if (!code) return SVDQ_ERR_INVALID_ARG;
   svdq_status s;
