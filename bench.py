@@ -296,29 +296,50 @@ def _bench_layer(svdq, spec, dev, stream, reps, peaks, oracle_budget_s):
     for i in range(max(10, n_sets)):
         step(i % n_sets)
     torch.cuda.synchronize()
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(reps)]
-    for i in range(reps):          # steps as the headline times them (no event between the kernels)
-        ev[i][0].record(stream)
+    # A step of a small layer is shorter than the host needs to issue its two
+    # calls, so the steps are replayed from CUDA graphs (device time; the
+    # library's launches are stream-ordered and capture as they are): one graph
+    # of G steps over the rotating sets (cold inputs), one of G steps on the
+    # same set (hot L2), one per kernel; `reps` replays each, per-step times =
+    # replay time / G.
+    G = max(n_sets, 8)
+
+    def graph_of(fn):
+        g = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            with torch.cuda.graph(g, stream=side, capture_error_mode="relaxed"):
+                for i in range(G):
+                    fn(i)
+        stream.wait_stream(side)
+        return g
+
+    def replay_times(g):
+        g.replay()
+        torch.cuda.synchronize()
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(reps)]
+        for e in ev:
+            e[0].record(stream)
+            g.replay()
+            e[1].record(stream)
+        torch.cuda.synchronize()
+        return [e[0].elapsed_time(e[1]) / G for e in ev]
+
+    g_cold = graph_of(lambda i: step(i % n_sets))
+    g_hot = graph_of(lambda i: step(0))
+    g_q = graph_of(lambda i: svdq.svdq_quantize_act(Xs[i % n_sets], pws[i % n_sets], out=qa))
+    g_g = graph_of(lambda i: svdq.svdq_w4a4_gemm(qa, pws[i % n_sets], bd, out=Y))
+    t_step, t_hot, t_q, t_g = (replay_times(g) for g in (g_cold, g_hot, g_q, g_g))
+    # the same steps issued from the host one call at a time (includes any host gap)
+    a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for i in range(reps):
         step(i % n_sets)
-        ev[i][2].record(stream)
+    z.record(stream)
     torch.cuda.synchronize()
-    t_step = [e[0].elapsed_time(e[2]) for e in ev]
-    for i in range(reps):          # hot L2: the same inputs every step
-        ev[i][0].record(stream)
-        step(0)
-        ev[i][2].record(stream)
-    torch.cuda.synchronize()
-    t_hot = [e[0].elapsed_time(e[2]) for e in ev]
-    for i in range(reps):          # per kernel (an event between them)
-        j = i % n_sets
-        ev[i][0].record(stream)
-        svdq.svdq_quantize_act(Xs[j], pws[j], out=qa)
-        ev[i][1].record(stream)
-        svdq.svdq_w4a4_gemm(qa, pws[j], bd, out=Y)
-        ev[i][2].record(stream)
-    torch.cuda.synchronize()
-    t_q = [e[0].elapsed_time(e[1]) for e in ev]
-    t_g = [e[1].elapsed_time(e[2]) for e in ev]
+    t_api = a.elapsed_time(z) / reps
+    del g_cold, g_hot, g_q, g_g
     if svdq.svdq_read_device_error() != 0:
         raise RuntimeError(f"device error while timing {spec.name}")
     med, q_ms, g_ms = statistics.median(t_step), statistics.median(t_q), statistics.median(t_g)
@@ -330,6 +351,7 @@ def _bench_layer(svdq, spec, dev, stream, reps, peaks, oracle_budget_s):
         "input_sets": n_sets,
         "step_ms": {"median": med, "p10": _pct(t_step, 0.1), "p90": _pct(t_step, 0.9)},
         "hot_l2_step_ms": statistics.median(t_hot),
+        "api_loop_step_ms": t_api,
         "tflops": _flops(M, N, K, r) / (med * 1e-3) / 1e12,
         "tokens_per_s": M / (med * 1e-3),
         "gemm_ms": g_ms,
@@ -345,9 +367,10 @@ def bench_configs(svdq, dev, stream, reps=100, oracle_budget_s=1.0):
     """Every benchmark workload (1-5), each layer timed separately; a workload's
     time is the sum of its layers' median step times."""
     peaks, kind = _peaks()
-    out = {"note": ("per layer: step = quantiser + GEMM with cold inputs (rotating copies >= 2x L2), median / "
-                    "p10 / p90 over the steps; hot_l2_step_ms with the same inputs every step; gemm_* and "
-                    "quant_* from a pass with an event between the kernels; fractions of "
+    out = {"note": ("per layer: step = quantiser + GEMM with cold inputs (rotating copies >= 2x L2), device "
+                    "time from CUDA-graph replays of the steps (median / p10 / p90 over replays); "
+                    "hot_l2_step_ms with the same inputs every step; gemm_* and quant_* from graphs of one "
+                    "kernel; api_loop_step_ms = the same steps issued call by call from the host; fractions of "
                     f"{kind} peaks (fp4 = bf16 burst x {FP4_PER_BF16:g}); oracle = float64 CPU oracle on a "
                     "bounded slice"), "reps": reps}
     for wid, wl in workloads.WORKLOADS.items():

@@ -57,7 +57,12 @@ struct MlpPost {
 __device__ __forceinline__ float gelu_f32(float x, bool approximate) {
   if (approximate) {
     const float u = __fmul_rn(0.7978845608028654f, __fmaf_rn(__fmul_rn(0.044715f, x), __fmul_rn(x, x), x));
-    return __fdiv_rn(x, __fadd_rn(1.0f, expf(__fmul_rn(-2.0f, u))));
+    if (u >= 0.0f) return __fdiv_rn(x, __fadd_rn(1.0f, expf(__fmul_rn(-2.0f, u))));
+    // the same function for u < 0 as x e^{2u} / (1 + e^{2u}): e^{2u} <= 1 never
+    // overflows, so the far negative tail keeps its tiny (possibly subnormal)
+    // values instead of collapsing to x / inf = -0
+    const float e = expf(__fmul_rn(2.0f, u));
+    return __fdiv_rn(__fmul_rn(x, e), __fadd_rn(1.0f, e));
   }
   return __fmul_rn(__fmul_rn(0.5f, x), erfcf(__fmul_rn(x, -0.7071067811865476f)));
 }

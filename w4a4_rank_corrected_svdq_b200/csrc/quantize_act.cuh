@@ -355,7 +355,15 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quantize_act_kernel(
     tmem_dealloc(tmem, C::kTmemCols);
   }
   // ---- this CTA's output rows: add the KS slots in rank order
-  if (!mbar_wait_cluster(&bars->xl1_in, 0, abort)) return;
+  if (!mbar_wait_cluster(&bars->xl1_in, 0, abort)) {
+    // Error path: the reduction is skipped, but partial rows that cluster peers
+    // have already sent may still be landing in this CTA's shared memory; give
+    // them a bounded time to arrive before the CTA exits.
+    const uint64_t t0 = globaltimer();
+    while (!mbar_try_wait_cluster(smem_u32(&bars->xl1_in), 0) && globaltimer() - t0 < 1000000ull) {
+    }
+    return;
+  }
   constexpr int kChunks = R / 4;
   for (int i = threadIdx.x; i < rpc * kChunks; i += kQuantThreads) {
     const int orow = i / kChunks;
