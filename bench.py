@@ -11,7 +11,10 @@ step reads its own copy of X and of the packed weight, cycling through enough
 copies that their total is at least twice the L2 size, so each step starts
 with its inputs out of cache (no flush kernel runs between steps: a 256 MiB
 write flush leaves DRAM busy with its write-back and is charged to the next
-kernel). Each step is timed with CUDA events on the launching stream. Multi-GPU: independent replicas (the layer shards by tokens with no
+kernel). The timed steps are captured once into a CUDA graph and replayed
+between two CUDA events on the launching stream (device time, not the host's
+issue rate; ms_per_step_loop reports the same steps issued call by call).
+Multi-GPU: independent replicas (the layer shards by tokens with no
 exchange), max time over ranks. Rank 0 prints one JSON line.
 
 --impl reference times the CPU oracle (float64 restatement of the layer) on
@@ -424,24 +427,48 @@ def run_ours(args, spec):
     if svdq.svdq_read_device_error() != 0:
         raise RuntimeError("device error during warm-up")
 
-    # Timed steps: one event pair per step around both kernels (no event between
-    # them, so the GEMM's programmatic launch overlaps the quantiser's end).
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    # Timed steps: the K steps (quantiser then GEMM, the GEMM a programmatic
+    # dependent of the quantiser) captured once into a CUDA graph and replayed
+    # inside the timed region, so the device time is not stretched by the
+    # host's issue rate; one event pair on the launching stream around the
+    # replay.
+    def steps_graph():
+        g = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            with torch.cuda.graph(g, stream=side, capture_error_mode="relaxed"):
+                for i in range(args.steps):
+                    j = (args.warmup + i) % n_sets
+                    svdq.svdq_quantize_act(Xs[j], pws[j], out=qa)
+                    svdq.svdq_w4a4_gemm(qa, pws[j], bd, out=Y)
+        stream.wait_stream(side)
+        return g
+
+    graph = steps_graph()
+    graph.replay()                   # upload, then one untimed replay
+    torch.cuda.synchronize()
+    e_a, e_b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     _barrier(world)
     torch.cuda.synchronize()
     with ClockSampler(gpu_uuid(local)) as clk:
-        for i in range(args.steps):
-            j = (args.warmup + i) % n_sets
-            ev[i][0].record(stream)
-            svdq.svdq_quantize_act(Xs[j], pws[j], out=qa)
-            svdq.svdq_w4a4_gemm(qa, pws[j], bd, out=Y)
-            ev[i][1].record(stream)
+        e_a.record(stream)
+        graph.replay()
+        e_b.record(stream)
         torch.cuda.synchronize()
     _barrier(world)
-    t_step = [e[0].elapsed_time(e[1]) for e in ev]
-    total_ms = _max_over_ranks(sum(t_step), world)
+    total_ms = _max_over_ranks(e_a.elapsed_time(e_b), world)
     ms_per_step = total_ms / args.steps
-    loop_ms = _max_over_ranks(ev[0][0].elapsed_time(ev[-1][1]), world) / args.steps
+    del graph
+    # the same steps issued call by call from the host (adds any host gap)
+    e_a.record(stream)
+    for i in range(args.steps):
+        j = (args.warmup + i) % n_sets
+        svdq.svdq_quantize_act(Xs[j], pws[j], out=qa)
+        svdq.svdq_w4a4_gemm(qa, pws[j], bd, out=Y)
+    e_b.record(stream)
+    torch.cuda.synchronize()
+    loop_ms = _max_over_ranks(e_a.elapsed_time(e_b), world) / args.steps
 
     # Per-kernel breakdown (separate pass, an event between the kernels).
     nb = min(args.steps, 200)
@@ -603,7 +630,8 @@ def run_ours(args, spec):
         Mu, Fu = up_s.M, up_s.N
         Hd = torch.empty((Mu, Fu), dtype=torch.bfloat16, device=dev)
         one = torch.ones(1, dtype=torch.float32, device=dev)
-        svdq.svdq_mlp_up_forward(Xud, pw_u, bud, one, Ld1, h_out=Hd)   # calibration pass for h's scale
+        l1t_d = Ld1.t().contiguous()     # the down projection's L1^T (the layout its packed l1t holds)
+        svdq.svdq_mlp_up_forward(Xud, pw_u, bud, one, l1t_d, h_out=Hd)   # calibration pass for h's scale
         g_h = svdq.svdq_act_global_scale(Hd)
         pw_d = svdq.svdq_pack_weight(Wdd, Ld1, Ld2, g_h)
         del Wdd
@@ -615,7 +643,7 @@ def run_ours(args, spec):
         Yd = torch.empty((Mu, dn_s.N), dtype=torch.bfloat16, device=dev)
 
         def fused(i):
-            svdq.svdq_mlp_up_forward(Xud, pw_u, bud, g_h, Ld1, out=qa_h, workspace=ws_m)
+            svdq.svdq_mlp_up_forward(Xud, pw_u, bud, g_h, pw_d.l1t, out=qa_h, workspace=ws_m)
             svdq.svdq_w4a4_gemm(qa_h, pw_d, bdd, out=Yd)
 
         def unfused(i):

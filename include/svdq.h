@@ -318,9 +318,11 @@ svdq_status svdq_linear_forward_noalloc(int M, int N, int K, int r, const void* 
  * and h is written directly as the down projection's quantised activation:
  *   h_codes  [M][N/2], h_scales (tiled, rows padded to 128, padding zero):
  *            the NVFP4 rule of svdq_quantize_act with g = *g_h;
- *   h_xl1    [M][r_down] = bf16(h . L1_down), L1_down bf16 [N][r_down]
- *            row-major; fp32 partial sums per 128-column half tile, summed in
- *            tile order (deterministic).
+ *   h_xl1    [M][r_down] = bf16(h . L1_down), given l1t_down = L1_down^T,
+ *            bf16 [r_down][N] row-major (the l1t that svdq_pack_weight writes
+ *            for the down projection); accumulated in fp32 on the tensor cores
+ *            over each CTA pair's run of tiles sharing their rows, one partial
+ *            per run, the partials summed in tile order (deterministic).
  * These are the buffers svdq_w4a4_gemm takes as a_codes, a_scales and xl1 for
  * the down projection (a QuantAct of M rows, K = N, rank r_down). h itself is
  * stored only when h_out (bf16 [M][ldh]) is given. Requires N % 256 == 0 (the
@@ -330,7 +332,7 @@ svdq_status svdq_mlp_workspace_size(int M, int N, int K, int r, int r_down, size
 svdq_status svdq_mlp_up_forward(int M, int N, int K, int r, const void* X, int64_t ldx, const void* w_codes,
                                 const void* w_scales, const float* gscale, const void* l1t, const void* l2s,
                                 const float* inv_smooth, const void* bias, int r_down, const float* g_h,
-                                const void* l1_down, int approximate, void* h_codes, void* h_scales, void* h_xl1,
+                                const void* l1t_down, int approximate, void* h_codes, void* h_scales, void* h_xl1,
                                 void* h_out, int64_t ldh, void* workspace, size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------------------ AWQ W4A16 */

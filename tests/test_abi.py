@@ -165,7 +165,8 @@ def test_mlp_up_sizes_and_validation(L):
     p = ctypes.c_void_p(0x10000)
     odd = ctypes.c_void_p(0x10008)
     base = _lib.svdq_forward_workspace_size(300, 512, 32)
-    assert _lib.svdq_mlp_workspace_size(300, 1024, 512, 32, 32) == base + 2 * 4 * 300 * 32 * 4
+    # one 256-row fp32 partial slot of r_down = 32 per 256 x 256 tile: 2 x 4 tiles
+    assert _lib.svdq_mlp_workspace_size(300, 1024, 512, 32, 32) == base + 2 * 4 * 256 * 32 * 4
     with pytest.raises(_lib.SvdqError):
         _lib.svdq_mlp_workspace_size(300, 1024, 512, 32, 16)          # r_down must be 32
     with pytest.raises(_lib.SvdqError):

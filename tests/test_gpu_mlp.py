@@ -78,7 +78,7 @@ def test_mlp_up_staged(lib, monkeypatch, M, D, F, r, approximate):
         b.fill_(0xA5)
     H = torch.empty((M, F), dtype=torch.bfloat16, device="cuda")
     ghd = torch.tensor([float(gh)], dtype=torch.float32, device="cuda")
-    lib.svdq_mlp_up_forward(X.cuda(), pu, bu.cuda(), ghd, _dev(Ld1), approximate, out=qa, h_out=H)
+    lib.svdq_mlp_up_forward(X.cuda(), pu, bu.cuda(), ghd, _dev(Ld1.T), approximate, out=qa, h_out=H)
     pd = lib.svdq_pack_weight(Wd.cuda(), _dev(Ld1), _dev(Ld2), float(gh))
     Yd = lib.svdq_w4a4_gemm(qa, pd, bd.cuda())
     torch.cuda.synchronize()
@@ -105,8 +105,8 @@ def test_mlp_up_without_storing_h(lib):
     X, Wd, bu, bd, Ld1, Ld2, pu, h_st, gh = _case(lib, M, D, F, r, False, seed=5)
     ghd = torch.tensor([float(gh)], dtype=torch.float32, device="cuda")
     H = torch.empty((M, F), dtype=torch.bfloat16, device="cuda")
-    a = lib.svdq_mlp_up_forward(X.cuda(), pu, bu.cuda(), ghd, _dev(Ld1), out=None, h_out=H)
-    b = lib.svdq_mlp_up_forward(X.cuda(), pu, bu.cuda(), ghd, _dev(Ld1))
+    a = lib.svdq_mlp_up_forward(X.cuda(), pu, bu.cuda(), ghd, _dev(Ld1.T), out=None, h_out=H)
+    b = lib.svdq_mlp_up_forward(X.cuda(), pu, bu.cuda(), ghd, _dev(Ld1.T))
     torch.cuda.synchronize()
     assert lib.svdq_read_device_error() == 0
     assert torch.equal(a.codes[: M * F // 2], b.codes[: M * F // 2])
@@ -167,7 +167,7 @@ def test_mlp_pair_config3_full_size(lib, monkeypatch, config3, approximate):
         b.fill_(0xA5)
     H = torch.empty((M, F), dtype=torch.bfloat16, device="cuda")
     ghd = torch.tensor([float(c["g_h"])], dtype=torch.float32, device="cuda")
-    lib.svdq_mlp_up_forward(Xd, c["pu"], c["bu"].cuda(), ghd, _dev(c["Ld1"]), approximate, out=qa, h_out=H)
+    lib.svdq_mlp_up_forward(Xd, c["pu"], c["bu"].cuda(), ghd, _dev(c["Ld1"].T), approximate, out=qa, h_out=H)
     Yd = lib.svdq_w4a4_gemm(qa, c["pd"], c["bd"].cuda())
     Yup = lib.svdq_linear_forward(Xd, c["pu"], c["bu"].cuda())
     torch.cuda.synchronize()

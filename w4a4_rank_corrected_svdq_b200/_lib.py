@@ -375,21 +375,22 @@ def svdq_mlp_workspace_size(M: int, N: int, K: int, r: int, r_down: int = 32) ->
 
 
 def svdq_mlp_up_forward(X: torch.Tensor, pw: PackedWeight, bias: torch.Tensor | None, g_h: torch.Tensor,
-                        l1_down: torch.Tensor, approximate: bool = False, out: QuantAct | None = None,
+                        l1t_down: torch.Tensor, approximate: bool = False, out: QuantAct | None = None,
                         h_out: torch.Tensor | None = None, workspace: torch.Tensor | None = None) -> QuantAct:
     """The up projection with GELU, writing h quantised for the down projection:
     returns the down projection's QuantAct (codes, scales, xl1 of h). g_h: the
-    down projection's activation scale (CUDA float32, one element); l1_down:
-    its L1, bf16 [N, r_down]; h_out: optional bf16 [M, N] copy of h."""
+    down projection's activation scale (CUDA float32, one element); l1t_down:
+    its L1 transposed, bf16 [r_down, N] (the down projection's packed
+    PackedWeight.l1t); h_out: optional bf16 [M, N] copy of h."""
     _dev(X, "X", torch.bfloat16)
     M, K = X.shape
     N, r = pw.N, pw.r
     ldx = _rows(X, "X", K)
     _dev(g_h, "g_h", torch.float32)
-    _dev(l1_down, "l1_down", torch.bfloat16)
-    if l1_down.dim() != 2 or l1_down.shape[0] != N or not l1_down.is_contiguous():
-        raise ValueError("l1_down must be a contiguous [N, r_down] tensor")
-    rd = l1_down.shape[1]
+    _dev(l1t_down, "l1t_down", torch.bfloat16)
+    if l1t_down.dim() != 2 or l1t_down.shape[1] != N or not l1t_down.is_contiguous():
+        raise ValueError("l1t_down must be a contiguous [r_down, N] tensor")
+    rd = l1t_down.shape[0]
     if bias is not None:
         _dev(bias, "bias", torch.bfloat16, (N,))
     ldh = 0
@@ -401,7 +402,7 @@ def svdq_mlp_up_forward(X: torch.Tensor, pw: PackedWeight, bias: torch.Tensor | 
     ws = workspace if workspace is not None else torch.empty(need, dtype=torch.uint8, device=X.device)
     _check("svdq_mlp_up_forward", lib().svdq_mlp_up_forward(
         M, N, K, r, _ptr(X), ldx, _ptr(pw.codes), _ptr(pw.scales), _ptr(pw.gscale), _ptr(pw.l1t), _ptr(pw.l2s),
-        _ptr(pw.inv_smooth), _ptr(bias), rd, _ptr(g_h), _ptr(l1_down), int(approximate), _ptr(qa.codes),
+        _ptr(pw.inv_smooth), _ptr(bias), rd, _ptr(g_h), _ptr(l1t_down), int(approximate), _ptr(qa.codes),
         _ptr(qa.scales), _ptr(qa.xl1), _ptr(h_out), ldh, _ptr(ws), ws.numel(), _stream(X)))
     return qa
 

@@ -12,32 +12,38 @@
 // A cluster of two CTAs on two SMs owns a 256 x 256 tile. Each CTA loads its
 // own 128 rows of A and its own 128 rows of B; one thread of the even CTA issues
 // 256x256xK MMAs that read both CTAs' shared memory and write each CTA's
-// 128 x 256 half of the accumulator into that CTA's TMEM. Per 256-wide K block
-// and SM this moves 38 KB for 8.4 MFLOP (half the bytes per FLOP of a 128 x 128
-// single-CTA tile), which keeps the L2 -> SM traffic within what L2 delivers.
-// No load uses cluster multicast: each CTA fetches every byte it stores.
+// 128 x 256 half of the accumulator into that CTA's TMEM. No load uses cluster
+// multicast: each CTA fetches every byte it stores.
+//
+// Tile order: the tiles are numbered M-block-major (N fastest) and each CTA
+// pair takes one contiguous run of them, so consecutive tiles of a pair mostly
+// share their 128-row A block. The A block's scale factors are then copied
+// into TMEM once per run of tiles with the same A block (when all of K fits:
+// K <= 14 x 256) and stay there: per 256-deep K block only the weight scales
+// (SFB) are copied, four tcgen05.cp of 128x256b instead of six.
 //
 // Roles (320 threads per CTA):
 //  * warp 0     TMA producer (both CTAs): per tile first r/c low-rank stages
 //               (XL1 columns, hi and lo columns of l2s; c = min(r, 32)), then
 //               K/256 stages of E2M1 codes (128-byte swizzle) and UE4M3 scale
-//               atoms. Completion bytes of both CTAs land on the even CTA's
-//               barrier (cp.async.bulk.tensor .cta_group::2).
+//               atoms (SFA only when the tile starts a new A block).
+//               Completion bytes of both CTAs land on the even CTA's barrier
+//               (cp.async.bulk.tensor .cta_group::2).
 //  * warp 1     TMEM owner (both CTAs, 512 columns); in the even CTA lane 0
 //               issues the MMAs and the scale copies smem -> TMEM.
-//  * warps 2-9  epilogue (both CTAs): TMEM -> registers, y = alpha acc + b,
-//               bf16 stores; two warps per 32-lane TMEM quadrant, one per
-//               128-column half. The epilogue mode EPI selects the plain
-//               layer (0), the fused QKV post-processing (1: per-head RMSNorm
-//               of Q/K and the rotary embedding; the two warps of a quadrant
-//               then split a tile by chunks) or the MLP up projection (2:
-//               GELU and the down projection's NVFP4 codes, scales and XL1
-//               partials instead of y).
-// TMEM: accumulator 0 = columns [0,256), accumulator 1 = [208,464): the two
-// share [208,256), which the epilogue reads first and releases early, so the
-// next tile's MMAs start long before the previous tile is fully stored; scale
-// factors at [464,480) (A) and [480,512) (B, 256 rows).
-// Every wait is bounded; see mbar_wait.
+//  * warps 2-9  epilogue (both CTAs): two warps per 32-lane TMEM quadrant, one
+//               per 128-column half. Each warp first drains its whole
+//               32 x 128 share of the accumulator into registers and releases
+//               it, so the next tile's MMAs start at once; then y = alpha acc + b
+//               (bias staged in shared memory per tile), bf16, TMA stores. The
+//               epilogue mode EPI selects the plain layer (0), the fused QKV
+//               post-processing (1: per-head RMSNorm of Q/K and the rotary
+//               embedding; the two warps of a quadrant then split a tile by
+//               chunks) or the MLP up projection (2: GELU and the down
+//               projection's NVFP4 codes, scales and XL1 partials instead of y).
+// TMEM (512 columns): accumulator [0, 256), weight scales of the current K
+// block [256, 288), A scales [288, 512) in 14 slots of 16 columns, one per K
+// block. Every wait is bounded; see mbar_wait.
 #pragma once
 
 #include "ptx.cuh"
@@ -122,15 +128,19 @@ __device__ __forceinline__ void tc_commit_cg2_mc(uint64_t* bar, uint16_t mask) {
 
 // ------------------------------------------------------------------ configuration
 constexpr int k2Threads = 320;
-constexpr int k2TileM = 256;  // per CTA pair; 128 rows per CTA
-constexpr int k2TileN = 256;  // per CTA pair; each CTA loads 128 rows of B
-constexpr int k2Acc1Col = 208;
-constexpr int k2SfaCol = 464;
-constexpr int k2SfbCol = 480;
+constexpr int k2TileM = 256;   // per CTA pair; 128 rows per CTA
+constexpr int k2TileN = 256;   // per CTA pair; each CTA loads 128 rows of B
+constexpr int k2SfbCol = 256;  // weight scales of one K block: 4 K-steps x 8 columns
+constexpr int k2SfaCol = 288;  // A scales: kSfaSlots slots of 16 columns (4 K-steps x 4)
+
+constexpr int k2Xl1Col = 480;  // MLP up projection: h . L1_down accumulator (32 columns)
 
 template <int R, int EPI = 0>
 struct Gemm2Cfg {
   static constexpr bool QKV = EPI == 1;
+  static constexpr bool MLP = EPI == 2;
+  // the MLP up projection adds one warp that loads L1_down and issues h . L1_down
+  static constexpr int kThreads = MLP ? 352 : 320;
   static constexpr int kABytes = 128 * 128;     // 128 rows x 256 E2M1
   static constexpr int kBBytes = 128 * 128;
   // Scale factors are staged in smem already replicated four times (the
@@ -140,36 +150,65 @@ struct Gemm2Cfg {
   static constexpr int kSfbBytes = 2 * 4 * 2048;  // 2 row blocks x 4 K-steps x 4 replicas x 512 B
   static constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;  // 56 KB
   static constexpr int kStages = 3;
+  // K blocks of A scales held in TMEM (MLP: the last 32 columns hold h . L1_down)
+  static constexpr int kSfaSlots = ((MLP ? k2Xl1Col : 512) - k2SfaCol) / 16;
   static constexpr int kLrCols = R < 32 ? R : 32;           // low-rank columns per stage
   static constexpr int kLrSteps = R / kLrCols;              // low-rank stages per tile
   static constexpr int kLrRowBytes = kLrCols * 2;
   static constexpr int kLrTileBytes = 128 * kLrRowBytes;    // per operand per CTA
   static constexpr SwizzleMode kLrSwizzle = kLrRowBytes == 64 ? kSwizzle64B : kSwizzle32B;
   static constexpr uint32_t kMainTx = 2u * kStageBytes;     // both CTAs
+  static constexpr uint32_t kSfaTx = 2u * kSfaBytes;
   static constexpr uint32_t kLrTx = 2u * 3u * kLrTileBytes;
-  // Epilogue staging per warp: two 2 KB bf16 TMA-store buffers.
+  // Epilogue staging per warp (4 KB): the plain layer stages 32 rows x 64
+  // columns (128-byte swizzle, one TMA store); the fused modes two 32 x 32
+  // buffers (64-byte swizzle).
   static constexpr int kOutPerWarp = 4096;
   static constexpr int kOutOff = kStages * kStageBytes;
   static constexpr int kOutBytes = 8 * kOutPerWarp;
+  // The tile's 256 bias values, double-buffered by tile parity.
+  static constexpr int kBiasOff = kOutOff + kOutBytes;
+  static constexpr int kBiasBytes = 2 * k2TileN * 2;
   // Fused QKV: per warp, partial sums of squares of its rows for the two heads
   // of a tile, double-buffered (2 x 2 x 32 floats).
-  static constexpr int kXchgOff = kOutOff + kOutBytes;
+  static constexpr int kXchgOff = kBiasOff + kBiasBytes;
   static constexpr int kXchgBytes = QKV ? 8 * 512 : 0;
-  static constexpr int kBarOff = kXchgOff + kXchgBytes;
-  static constexpr int kSmemBytes = kBarOff + 256 + 1024;
+  // MLP: L1_down^T for a tile's 256 columns, each CTA its 16 of the 32 rows
+  // (4 chunks of 16 rows x 64 columns, 128-byte swizzle), double-buffered.
+  static constexpr int kL1dOff = kXchgOff + kXchgBytes;
+  static constexpr int kL1dChunk = 16 * 128;
+  static constexpr int kL1dBytes = MLP ? 2 * 4 * kL1dChunk : 0;
+  static constexpr int kBarOff = kL1dOff + kL1dBytes;
+  static constexpr int kSmemBytes = kBarOff + 512 + 1024;
 };
 
 struct Gemm2Barriers {
   uint64_t full[8];
   uint64_t empty[8];
-  uint64_t acc_full[2];
-  uint64_t acc_empty[2];
-  uint64_t ovl_free;
+  uint64_t acc_full;       // the tile's MMAs have completed (one commit, both CTAs)
+  uint64_t acc_empty;      // the accumulator has been drained (8 epilogue warps x 2 CTAs)
+  uint64_t bias_ready[2];  // the tile's bias is in shared memory (256 epilogue threads)
   uint64_t teardown;
-  uint64_t xchg[4];  // fused QKV: the two epilogue warps of a TMEM lane quadrant (64 arrivals)
+  uint64_t xchg[4];        // fused QKV: the two epilogue warps of a TMEM lane quadrant (64 arrivals)
+  // MLP up projection
+  uint64_t chunk_ready[2];  // per column half: a 64-column chunk of h is staged (4 warps x 2 CTAs)
+  uint64_t chunk_free[2];   // per column half: the h . L1_down MMAs of the staged chunk completed
+  uint64_t l1d_full[2];     // L1_down^T of a tile is in shared memory (both CTAs' halves)
+  uint64_t l1d_free[2];     // its MMAs completed
+  uint64_t xl1_done;        // the run's h . L1_down accumulator is complete
+  uint64_t xl1_free;        // and has been read out (4 warps x 2 CTAs)
+  uint64_t xl1_teardown;    // every h . L1_down MMA has completed
   uint32_t tmem_base;
   int abort;
 };
+
+// The contiguous run of tiles [t0, t1) of CTA pair `pair` (balanced: runs
+// differ by at most one tile).
+__device__ __forceinline__ void pair_tile_range(int pair, int num_pairs, int num_tiles, int& t0, int& t1) {
+  const int base = num_tiles / num_pairs, rem = num_tiles % num_pairs;
+  t0 = pair * base + (pair < rem ? pair : rem);
+  t1 = t0 + base + (pair < rem ? 1 : 0);
+}
 
 // bf16 tile store from shared memory (TMA, async bulk group).
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap* m, const void* src, int x, int y) {
@@ -186,73 +225,53 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-// y = alpha * acc + b for one 32-column chunk of this lane's row, packed to
-// bf16 and written into a 32-row x 64-byte staging buffer in the 64-byte
-// swizzled order the Y tensor map expects; then lane 0 issues the TMA store.
-__device__ __forceinline__ void store_chunk(const uint32_t (&v)[32], const uint4 (&bv)[16], int c, float alpha,
-                                            uint8_t* stage, const CUtensorMap* tm_y, int x, int y, int lane) {
-  uint32_t packed[16];
-#pragma unroll
-  for (int p = 0; p < 16; ++p) {
-    const uint4 bq = bv[4 * c + p / 4];
-    const uint32_t bw = (p % 4 == 0) ? bq.x : (p % 4 == 1) ? bq.y : (p % 4 == 2) ? bq.z : bq.w;
-    const float y0 = __fmaf_rn(__uint_as_float(v[2 * p]), alpha, __uint_as_float(bw << 16));
-    const float y1 = __fmaf_rn(__uint_as_float(v[2 * p + 1]), alpha, __uint_as_float(bw & 0xFFFF0000u));
-    const __nv_bfloat162 hv = __floats2bfloat162_rn(y0, y1);
-    packed[p] = *reinterpret_cast<const uint32_t*>(&hv);
-  }
-  if (lane == 0) bulk_wait_read1();  // the previous store from this buffer has read it
+// 64 columns of this lane's row (two 32-column chunks of packed bf16 pairs)
+// written into a 32-row x 128-byte staging buffer in the 128-byte swizzle of
+// the Y store map, then stored with one TMA store by lane 0.
+__device__ __forceinline__ void store_row64(uint8_t* buf, const uint32_t (&pa)[16], const uint32_t (&pb)[16],
+                                            const CUtensorMap* tm_y, int x, int y, int lane) {
+  if (lane == 0) bulk_wait_read0();  // the previous store from this buffer has read it
   __syncwarp();
-  const int sw = (lane >> 1) & 3;
+  uint8_t* row = buf + lane * 128;
+  const int sw = lane & 7;
 #pragma unroll
-  for (int j = 0; j < 4; ++j)
-    *reinterpret_cast<uint4*>(stage + lane * 64 + ((j ^ sw) << 4)) =
-        make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
+  for (int j = 0; j < 4; ++j) {
+    *reinterpret_cast<uint4*>(row + ((j ^ sw) << 4)) = make_uint4(pa[4 * j], pa[4 * j + 1], pa[4 * j + 2], pa[4 * j + 3]);
+    *reinterpret_cast<uint4*>(row + (((j + 4) ^ sw) << 4)) =
+        make_uint4(pb[4 * j], pb[4 * j + 1], pb[4 * j + 2], pb[4 * j + 3]);
+  }
   fence_proxy_async_smem();
   __syncwarp();
   if (lane == 0) {
-    tma_store_2d(tm_y, stage, x, y);
+    tma_store_2d(tm_y, buf, x, y);
     bulk_commit();
   }
 }
 
-// One epilogue warp's 128-column half of a tile, in four 32-column chunks.
-// If the warp holds the columns shared by the two accumulators (chunks 2,3 of
-// accumulator 0's upper half; chunks 0,1 of accumulator 1's lower half), it
-// reads those first and releases them before doing any other work.
-template <int FIRST>
-__device__ __forceinline__ void epilogue_half(uint32_t taddr, const uint4 (&bv)[16], float alpha, uint8_t* stage,
-                                              int& nbuf, const CUtensorMap* tm_y, int x0, int y0, bool holds_overlap,
-                                              uint32_t ovl_bar, int lane) {
-  uint32_t va[32], vb[32];
-  tmem_ld_32x32b_x32(taddr + 32 * ((FIRST + 0) & 3), va);
-  tmem_ld_32x32b_x32(taddr + 32 * ((FIRST + 1) & 3), vb);
+// Drains this warp's four 32-column chunks of the accumulator (TMEM columns
+// c0, c1, c2, c3 of its lane quadrant at tq) into registers and releases the
+// accumulator to the MMA issuer (a relaxed arrive: the loads have completed,
+// nothing is published).
+__device__ __forceinline__ void drain4(uint32_t tq, int c0, int c1, int c2, int c3, uint32_t (&v0)[32],
+                                       uint32_t (&v1)[32], uint32_t (&v2)[32], uint32_t (&v3)[32],
+                                       uint32_t acc_empty_remote, int lane) {
+  tmem_ld_32x32b_x32(tq + c0, v0);
+  tmem_ld_32x32b_x32(tq + c1, v1);
+  tmem_ld_32x32b_x32(tq + c2, v2);
+  tmem_ld_32x32b_x32(tq + c3, v3);
   tmem_ld_wait();
-  if (holds_overlap) {  // the loads above have completed (tcgen05.wait::ld): nothing else to publish
-    tc_fence_before();
-    __syncwarp();
-    if (lane == 0) mbar_arrive_cluster_relaxed(ovl_bar);
-  }
-  store_chunk(va, bv, (FIRST + 0) & 3, alpha, stage + 2048 * (nbuf & 1), tm_y, x0 + 32 * ((FIRST + 0) & 3), y0, lane);
-  ++nbuf;
-  store_chunk(vb, bv, (FIRST + 1) & 3, alpha, stage + 2048 * (nbuf & 1), tm_y, x0 + 32 * ((FIRST + 1) & 3), y0, lane);
-  ++nbuf;
-  tmem_ld_32x32b_x32(taddr + 32 * ((FIRST + 2) & 3), va);
-  tmem_ld_32x32b_x32(taddr + 32 * ((FIRST + 3) & 3), vb);
-  tmem_ld_wait();
-  store_chunk(va, bv, (FIRST + 2) & 3, alpha, stage + 2048 * (nbuf & 1), tm_y, x0 + 32 * ((FIRST + 2) & 3), y0, lane);
-  ++nbuf;
-  store_chunk(vb, bv, (FIRST + 3) & 3, alpha, stage + 2048 * (nbuf & 1), tm_y, x0 + 32 * ((FIRST + 3) & 3), y0, lane);
-  ++nbuf;
+  tc_fence_before();
+  __syncwarp();
+  if (lane == 0) mbar_arrive_cluster_relaxed(acc_empty_remote);
 }
 
 // ------------------------------------------------------------------ fused QKV epilogue
-// For the fused QKV variant the two epilogue warps of a TMEM lane quadrant
-// split a 256-column tile (two 128-column heads) by chunks rather than by
-// heads: warp h takes chunks 2h, 2h+1 of both heads, so the rotary angles it
-// needs (pairs 32h..32h+31 of its rows) are the same for both heads and are
-// fetched once, before the accumulator is ready. The per-row sums of squares
-// of the two warps are combined through shared memory.
+// The two epilogue warps of a TMEM lane quadrant split a 256-column tile (two
+// 128-column heads) by chunks rather than by heads: warp h takes chunks 2h,
+// 2h+1 of both heads, so the rotary angles it needs (pairs 32h..32h+31 of its
+// rows) are the same for both heads; those of its first chunk are fetched
+// before the accumulator is ready. The per-row sums of squares of the two
+// warps are combined through shared memory.
 
 // Writes / reads this lane's row of 16 packed bf16 pairs in a 2 KB staging
 // buffer (32 rows x 64 bytes, the 64-byte swizzle of the store map).
@@ -338,148 +357,92 @@ __device__ __forceinline__ void qk_rot16(uint32_t (&pk)[16], float rstd, const _
   }
 }
 
-// One fused-QKV tile for one epilogue warp: chunks c0 = 2h, c0 + 1 of head F
-// (read first: it holds the columns shared by the two accumulators when
-// holds_overlap) and of head 1 - F. tacc: the accumulator's TMEM address for
-// this lane quadrant. For a Q/K tile (w_f, w_s the norm weights of heads F
-// and 1 - F)
-// tc0/ts0 hold the angles of chunk c0's pairs (fetched before the
-// accumulator was ready), cr/sr point at those of chunk c0 + 1 (fetched once
-// the first head is read) and xs_* are the exchange slots; a V tile
-// (w_f == nullptr) is stored as computed. Returns false on abort.
-__device__ __forceinline__ bool epilogue_qkv_tile(uint32_t tacc, int F, int h, const __nv_bfloat16* btile, float alpha,
-                                                  uint8_t* stage, const CUtensorMap* tm_y, int xt, int y0,
-                                                  bool holds_overlap, uint32_t ovl_bar, int lane,
-                                                  const __nv_bfloat16* w_f, const __nv_bfloat16* w_s,
-                                                  const float (&tc0)[16],
-                                                  const float (&ts0)[16], const float* cr, const float* sr,
-                                                  float* xs_mine, const float* xs_peer,
+
+// One fused-QKV tile for one epilogue warp, y already packed (bf16 pairs):
+// y0c, y0d = head 0's chunks c0 = 2h, c0 + 1; y1c, y1d = head 1's. For a Q/K
+// tile (w0, w1: the norm weights of heads 0 and 1; cr/sr: this lane's row of
+// rotary angles from chunk c0's first pair on; xs_*: the exchange slots) the
+// rows are normalised and rotated, chunk c0 of both heads first so that only
+// one chunk's angles are held at a time; a V tile (w0 == nullptr) is stored as
+// computed. Returns false on abort.
+__device__ __forceinline__ bool epilogue_qkv_tile(uint32_t (&y0c)[16], uint32_t (&y0d)[16], uint32_t (&y1c)[16],
+                                                  uint32_t (&y1d)[16], int h, uint8_t* stage,
+                                                  const CUtensorMap* tm_y, int xt, int y0, int lane,
+                                                  const __nv_bfloat16* w0, const __nv_bfloat16* w1, const float* cr,
+                                                  const float* sr, float* xs_mine, const float* xs_peer,
                                                   uint64_t* xbar, uint32_t xpar, float eps, volatile int* abort) {
-  const int S = 1 - F;
-  const bool qk = w_f != nullptr;
   const int c0 = 2 * h;
-  const auto bcol = [&](int head, int c) { return btile != nullptr ? btile + 128 * head + 32 * c : nullptr; };
-  float ssf = 0.0f, sss = 0.0f;  // this warp's part of the rows' sums of squares
   if (lane == 0) bulk_wait_read0();  // both staging buffers are free
   __syncwarp();
-  {
-    uint32_t va[32], vb[32];
-    tmem_ld_32x32b_x32(tacc + 128 * F + 32 * c0, va);
-    tmem_ld_32x32b_x32(tacc + 128 * F + 32 * (c0 + 1), vb);
-    tmem_ld_wait();
-    if (holds_overlap) {  // the loads above have completed (tcgen05.wait::ld): nothing else to publish
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cluster_relaxed(ovl_bar);
-    }
-    uint32_t pk[16];
-    pack32(va, bcol(F, c0), alpha, pk);
-    ssf = sumsq16(pk, ssf);
-    stage_row16(stage, pk, lane);
-    if (!qk) store_staged(stage, tm_y, xt + 128 * F + 32 * c0, y0, lane);
-    pack32(vb, bcol(F, c0 + 1), alpha, pk);
-    ssf = sumsq16(pk, ssf);
-    stage_row16(stage + 2048, pk, lane);
-    if (!qk) store_staged(stage + 2048, tm_y, xt + 128 * F + 32 * (c0 + 1), y0, lane);
-  }
-  float tc1[16], ts1[16];
-  if (qk) {
-    load_angles16(cr, sr, tc1, ts1);
-    // head 1 - F never holds shared columns: read it for its sums now and
-    // again, to store it, after the exchange
-#pragma unroll 1
-    for (int k = 0; k < 2; ++k) {
-      uint32_t va[32], pk[16];
-      tmem_ld_32x32b_x32(tacc + 128 * S + 32 * (c0 + k), va);
-      tmem_ld_wait();
-      pack32(va, bcol(S, c0 + k), alpha, pk);
-      sss = sumsq16(pk, sss);
-    }
-    // this warp's partial sums for heads 0 / 1, then the partner's
-    xs_mine[32 * F + lane] = ssf;
-    xs_mine[32 * S + lane] = sss;
-    mbar_arrive(xbar);
-    if (!mbar_wait(xbar, xpar, abort)) return false;
-    const float pf = xs_peer[32 * F + lane], pss = xs_peer[32 * S + lane];
-    // rows' sums in chunk order: warp 0's chunks 0, 1 then warp 1's chunks 2, 3
-    const float tf = h == 0 ? ssf + pf : pf + ssf;
-    const float tsum = h == 0 ? sss + pss : pss + sss;
-    const float rs_f = 1.0f / sqrtf(__fmaf_rn(tf, 1.0f / kHeadDim, eps));
-    const float rs_s = 1.0f / sqrtf(__fmaf_rn(tsum, 1.0f / kHeadDim, eps));
-    uint32_t pk[16];
-    load_row16(stage, pk, lane);
-    qk_rot16(pk, rs_f, w_f + 32 * c0, tc0, ts0);
-    stage_row16(stage, pk, lane);
-    store_staged(stage, tm_y, xt + 128 * F + 32 * c0, y0, lane);
-    load_row16(stage + 2048, pk, lane);
-    qk_rot16(pk, rs_f, w_f + 32 * (c0 + 1), tc1, ts1);
-    stage_row16(stage + 2048, pk, lane);
-    store_staged(stage + 2048, tm_y, xt + 128 * F + 32 * (c0 + 1), y0, lane);
-    {
-      uint32_t va[32];
-      tmem_ld_32x32b_x32(tacc + 128 * S + 32 * c0, va);
-      tmem_ld_wait();
-      pack32(va, bcol(S, c0), alpha, pk);
-    }
-    qk_rot16(pk, rs_s, w_s + 32 * c0, tc0, ts0);
+  if (w0 == nullptr) {
+    stage_row16(stage, y0c, lane);
+    store_staged(stage, tm_y, xt + 32 * c0, y0, lane);
+    stage_row16(stage + 2048, y0d, lane);
+    store_staged(stage + 2048, tm_y, xt + 32 * (c0 + 1), y0, lane);
     if (lane == 0) bulk_wait_read1();  // the store from buffer 0 has read it
     __syncwarp();
-    stage_row16(stage, pk, lane);
-    store_staged(stage, tm_y, xt + 128 * S + 32 * c0, y0, lane);
-    {
-      uint32_t va[32];
-      tmem_ld_32x32b_x32(tacc + 128 * S + 32 * (c0 + 1), va);
-      tmem_ld_wait();
-      pack32(va, bcol(S, c0 + 1), alpha, pk);
-    }
-    qk_rot16(pk, rs_s, w_s + 32 * (c0 + 1), tc1, ts1);
+    stage_row16(stage, y1c, lane);
+    store_staged(stage, tm_y, xt + 128 + 32 * c0, y0, lane);
     if (lane == 0) bulk_wait_read1();
     __syncwarp();
-    stage_row16(stage + 2048, pk, lane);
-    store_staged(stage + 2048, tm_y, xt + 128 * S + 32 * (c0 + 1), y0, lane);
+    stage_row16(stage + 2048, y1d, lane);
+    store_staged(stage + 2048, tm_y, xt + 128 + 32 * (c0 + 1), y0, lane);
     return true;
   }
-#pragma unroll 1
-  for (int k = 0; k < 2; ++k) {  // V: head 1 - F as computed
-    uint32_t va[32], pk[16];
-    tmem_ld_32x32b_x32(tacc + 128 * S + 32 * (c0 + k), va);
-    tmem_ld_wait();
-    pack32(va, bcol(S, c0 + k), alpha, pk);
-    if (lane == 0) bulk_wait_read1();
-    __syncwarp();
-    stage_row16(stage + 2048 * k, pk, lane);
-    store_staged(stage + 2048 * k, tm_y, xt + 128 * S + 32 * (c0 + k), y0, lane);
-  }
+  // this warp's part of each row's sum of squares, chunk c0 then c0 + 1
+  const float s0 = sumsq16(y0d, sumsq16(y0c, 0.0f));
+  const float s1 = sumsq16(y1d, sumsq16(y1c, 0.0f));
+  xs_mine[lane] = s0;
+  xs_mine[32 + lane] = s1;
+  mbar_arrive(xbar);
+  float tc[16], ts[16];
+  load_angles16(cr, sr, tc, ts);  // chunk c0's pairs
+  if (!mbar_wait(xbar, xpar, abort)) return false;
+  const float p0 = xs_peer[lane], p1 = xs_peer[32 + lane];
+  // rows' sums in chunk order: warp 0's chunks 0, 1 then warp 1's chunks 2, 3
+  const float t0 = h == 0 ? s0 + p0 : p0 + s0;
+  const float t1 = h == 0 ? s1 + p1 : p1 + s1;
+  const float r0 = 1.0f / sqrtf(__fmaf_rn(t0, 1.0f / kHeadDim, eps));
+  const float r1 = 1.0f / sqrtf(__fmaf_rn(t1, 1.0f / kHeadDim, eps));
+  qk_rot16(y0c, r0, w0 + 32 * c0, tc, ts);
+  stage_row16(stage, y0c, lane);
+  store_staged(stage, tm_y, xt + 32 * c0, y0, lane);
+  qk_rot16(y1c, r1, w1 + 32 * c0, tc, ts);
+  stage_row16(stage + 2048, y1c, lane);
+  store_staged(stage + 2048, tm_y, xt + 128 + 32 * c0, y0, lane);
+  load_angles16(cr + 16, sr + 16, tc, ts);  // chunk c0 + 1's pairs
+  qk_rot16(y0d, r0, w0 + 32 * (c0 + 1), tc, ts);
+  if (lane == 0) bulk_wait_read1();  // the store from buffer 0 has read it
+  __syncwarp();
+  stage_row16(stage, y0d, lane);
+  store_staged(stage, tm_y, xt + 32 * (c0 + 1), y0, lane);
+  qk_rot16(y1d, r1, w1 + 32 * (c0 + 1), tc, ts);
+  if (lane == 0) bulk_wait_read1();
+  __syncwarp();
+  stage_row16(stage + 2048, y1d, lane);
+  store_staged(stage + 2048, tm_y, xt + 128 + 32 * (c0 + 1), y0, lane);
   return true;
 }
 
 // ------------------------------------------------------------------ MLP up-projection epilogue
 constexpr int kMlpRank = 32;  // the down projection's rank the fused epilogue supports
-// One 32-column chunk c (columns x0 + 32 c ..) of this lane's row: y, h =
-// bf16(GELU(y)), the two NVFP4 blocks of h (the activation quantiser's rule:
-// S = e4m3(amax / fp32(6 g)), q = h * fp32(1 / fp32(dec(S) g))), their codes
-// and scales stored for the down projection, h added into the XL1 partial
-// (part[j] += h_i L1d[x0 + 32 c + i][j]), and h optionally staged for a TMA
-// store.
-template <int RD>
-__device__ __forceinline__ void mlp_chunk(const uint32_t (&v)[32], const __nv_bfloat16* bcol, float alpha, int c,
-                                          int x0, int row, int M, int N, const MlpPost& mp, float g, float d,
-                                          float (&part)[RD], uint8_t* stage, int& nbuf, const CUtensorMap* tm_y,
-                                          int y0, int lane) {
-  uint32_t pk[16];
-  pack_chunk(v, bcol != nullptr ? bcol + 32 * c : nullptr, alpha, pk);  // y, exactly as the plain epilogue
+
+// 32 columns of this lane's row given y as 16 packed bf16 pairs (overwritten
+// with h): h = bf16(GELU(y)) and its two NVFP4 blocks by the activation
+// quantiser's rule (S = e4m3(amax / fp32(6 g)), q = h * fp32(1 / fp32(dec(S) g)),
+// zero reciprocal for a zero or saturated scale): the 32 codes as four words
+// in w (two per block) and the two scale bytes in sc.
+__device__ __forceinline__ void mlp_gelu_quant32(uint32_t (&pk)[16], bool approximate, float g, float d,
+                                                 uint32_t (&w)[4], uint32_t& sc) {
   float hf[32];
 #pragma unroll
   for (int p = 0; p < 16; ++p) {
-    const uint32_t hp = pack_bf16(gelu_f32(bf16_lo(pk[p]), mp.approximate != 0),
-                                  gelu_f32(bf16_hi(pk[p]), mp.approximate != 0));
+    const uint32_t hp = pack_bf16(gelu_f32(bf16_lo(pk[p]), approximate), gelu_f32(bf16_hi(pk[p]), approximate));
     pk[p] = hp;
     hf[2 * p] = bf16_lo(hp);
     hf[2 * p + 1] = bf16_hi(hp);
   }
-  const int col = x0 + 32 * c;
-  uint32_t words[4];
-  uint32_t sc = 0;
+  sc = 0;
 #pragma unroll
   for (int blk = 0; blk < 2; ++blk) {
     float am = 0.0f;
@@ -494,100 +457,91 @@ __device__ __forceinline__ void mlp_chunk(const uint32_t (&v)[32], const __nv_bf
       q0[i] = __fmul_rn(hf[16 * blk + i], inv);
       q1[i] = __fmul_rn(hf[16 * blk + 8 + i], inv);
     }
-    words[2 * blk] = f32x8_to_e2m1(q0);
-    words[2 * blk + 1] = f32x8_to_e2m1(q1);
+    w[2 * blk] = f32x8_to_e2m1(q0);
+    w[2 * blk + 1] = f32x8_to_e2m1(q1);
     sc |= S << (8 * blk);
   }
+}
+
+// 64 columns x0 .. x0 + 63 of this lane's row (y in pa, pb; replaced by h):
+// GELU, NVFP4 codes (32 bytes) and the scale word (4 blocks) stored for the
+// down projection; padding rows (M <= row < m_pad) get zero scales.
+__device__ __forceinline__ void mlp_quantize64(uint32_t (&pa)[16], uint32_t (&pb)[16], int x0, int row, int M, int N,
+                                               const MlpPost& mp, float g, float d) {
+  uint32_t wa[4], wb[4], sa, sb;
+  mlp_gelu_quant32(pa, mp.approximate != 0, g, d, wa, sa);
+  mlp_gelu_quant32(pb, mp.approximate != 0, g, d, wb, sb);
   if (row < M) {
-    *reinterpret_cast<uint4*>(mp.codes + static_cast<int64_t>(row) * (N / 2) + col / 2) =
-        make_uint4(words[0], words[1], words[2], words[3]);
+    uint4* c = reinterpret_cast<uint4*>(mp.codes + static_cast<int64_t>(row) * (N / 2) + x0 / 2);
+    c[0] = make_uint4(wa[0], wa[1], wa[2], wa[3]);
+    c[1] = make_uint4(wb[0], wb[1], wb[2], wb[3]);
   }
-  if (row < mp.m_pad)
-    *reinterpret_cast<uint16_t*>(mp.scales + scale_offset(N, row, col / 16)) =
-        static_cast<uint16_t>(row < M ? sc : 0u);
-  // XL1 partial: the L1 rows of these 32 columns are the same for every lane (broadcast loads);
-  // fully unrolled so that hf stays in registers
+  if (row < mp.m_pad)  // the four scale bytes of a row's 64 columns are one aligned word of the tiled layout
+    *reinterpret_cast<uint32_t*>(mp.scales + scale_offset(N, row, x0 / 16)) = row < M ? (sa | (sb << 16)) : 0u;
+}
+
+// 64 columns of packed bf16 pairs (pa, pb) of this lane's row into a 32-row x
+// 128-byte buffer in the 128-byte swizzle (the K-major layout the MMA reads,
+// and the box layout of the 64-column store map).
+__device__ __forceinline__ void stage_row64(uint8_t* buf, const uint32_t (&pa)[16], const uint32_t (&pb)[16],
+                                            int lane) {
+  uint8_t* row = buf + lane * 128;
+  const int sw = lane & 7;
 #pragma unroll
-  for (int i = 0; i < 32; ++i) {
-    const uint4* lrow = reinterpret_cast<const uint4*>(mp.l1d + static_cast<int64_t>(col + i) * RD);
-#pragma unroll
-    for (int j8 = 0; j8 < RD / 8; ++j8) {
-      float l[8];
-      bf16x8_to_f32(__ldg(lrow + j8), l);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) part[8 * j8 + e] = __fmaf_rn(hf[i], l[e], part[8 * j8 + e]);
-    }
-  }
-  if (mp.store_h) {
-    uint8_t* out = stage + 2048 * (nbuf & 1);
-    ++nbuf;
-    if (lane == 0) bulk_wait_read1();
-    __syncwarp();
-    stage_row16(out, pk, lane);
-    store_staged(out, tm_y, col, y0, lane);
+  for (int j = 0; j < 4; ++j) {
+    *reinterpret_cast<uint4*>(row + ((j ^ sw) << 4)) = make_uint4(pa[4 * j], pa[4 * j + 1], pa[4 * j + 2], pa[4 * j + 3]);
+    *reinterpret_cast<uint4*>(row + (((j + 4) ^ sw) << 4)) =
+        make_uint4(pb[4 * j], pb[4 * j + 1], pb[4 * j + 2], pb[4 * j + 3]);
   }
 }
 
-// The MLP variant of epilogue_half: the warp's 128-column half in four chunks
-// (the shared accumulator columns first, released at once), then its XL1
-// partial for rows y0 .. y0 + 31 written to partial slot 2 nt + h.
-template <int RD, int FIRST>
-__device__ __forceinline__ void epilogue_half_mlp(uint32_t taddr, const __nv_bfloat16* bcol, float alpha,
-                                                  uint8_t* stage, int& nbuf, const CUtensorMap* tm_y, int x0, int y0,
-                                                  bool holds_overlap, uint32_t ovl_bar, int lane, const MlpPost& mp,
-                                                  int M, int N, int slot) {
-  const int row = y0 + lane;
-  const float g = *mp.g_h;
-  const float d = __fmul_rn(6.0f, g);
-  float part[RD];
-#pragma unroll
-  for (int j = 0; j < RD; ++j) part[j] = 0.0f;
-  {
-    uint32_t va[32], vb[32];
-    tmem_ld_32x32b_x32(taddr + 32 * ((FIRST + 0) & 3), va);
-    tmem_ld_32x32b_x32(taddr + 32 * ((FIRST + 1) & 3), vb);
-    tmem_ld_wait();
-    if (holds_overlap) {  // the loads above have completed (tcgen05.wait::ld): nothing else to publish
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cluster_relaxed(ovl_bar);
-    }
-    mlp_chunk<RD>(va, bcol, alpha, (FIRST + 0) & 3, x0, row, M, N, mp, g, d, part, stage, nbuf, tm_y, y0, lane);
-    mlp_chunk<RD>(vb, bcol, alpha, (FIRST + 1) & 3, x0, row, M, N, mp, g, d, part, stage, nbuf, tm_y, y0, lane);
-  }
-#pragma unroll 1
-  for (int k = 2; k < 4; ++k) {
-    uint32_t va[32];
-    tmem_ld_32x32b_x32(taddr + 32 * ((FIRST + k) & 3), va);
-    tmem_ld_wait();
-    mlp_chunk<RD>(va, bcol, alpha, (FIRST + k) & 3, x0, row, M, N, mp, g, d, part, stage, nbuf, tm_y, y0, lane);
-  }
-  if (row < M) {
-    float4* dst = reinterpret_cast<float4*>(mp.partial + (static_cast<int64_t>(slot) * M + row) * RD);
-#pragma unroll
-    for (int j = 0; j < RD / 4; ++j) dst[j] = make_float4(part[4 * j], part[4 * j + 1], part[4 * j + 2], part[4 * j + 3]);
-  }
+// Arrival that publishes this thread's earlier writes to a cluster CTA's observer.
+__device__ __forceinline__ void mbar_arrive_cluster_release(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
-// Sums the XL1 partials of an MLP up projection in slot order:
-// xl1[m][j] = bf16(sum_p partial[p][m][j]) (fp32, p ascending: deterministic).
-__global__ void mlp_xl1_reduce_kernel(const float* __restrict__ partial, int slots, int M, int rd,
-                                      __nv_bfloat16* __restrict__ xl1) {
-  const int64_t total = static_cast<int64_t>(M) * rd;
+// The first tile of CTA pair p's run (the pair_tile_range split) and the pair
+// that owns tile t.
+__host__ __device__ __forceinline__ int pair_first_tile(int p, int num_pairs, int num_tiles) {
+  const int base = num_tiles / num_pairs, rem = num_tiles % num_pairs;
+  return p * base + (p < rem ? p : rem);
+}
+__host__ __device__ __forceinline__ int pair_of_tile(int t, int num_pairs, int num_tiles) {
+  const int base = num_tiles / num_pairs, rem = num_tiles % num_pairs;
+  const int big = rem * (base + 1);
+  return t < big ? t / (base + 1) : rem + (t - big) / base;
+}
+
+// Sums the XL1 partials of an MLP up projection: the partial of a run of tiles
+// sits in the slot of the run's first tile; the runs covering row block
+// m / 256 start at that block's first tile and at every CTA pair's first tile
+// inside it. xl1[m][j] = bf16(sum over those runs in tile order) (fp32,
+// deterministic).
+__global__ void mlp_xl1_reduce_kernel(const float* __restrict__ partial, int num_tiles, int num_pairs, int num_nt,
+                                      int M, __nv_bfloat16* __restrict__ xl1) {
+  const int64_t total = static_cast<int64_t>(M) * kMlpRank;
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int m = static_cast<int>(i / kMlpRank), j = static_cast<int>(i % kMlpRank);
+    const int mt = m / k2TileM, lr = m % k2TileM;
+    const int t_lo = mt * num_nt, t_hi = t_lo + num_nt;
     float s = 0.0f;
-    for (int p = 0; p < slots; ++p) s = __fadd_rn(s, partial[p * total + i]);
+    for (int p = pair_of_tile(t_lo, num_pairs, num_tiles); p < num_pairs; ++p) {
+      const int f = pair_first_tile(p, num_pairs, num_tiles);
+      if (f >= t_hi) break;
+      const int t = f > t_lo ? f : t_lo;
+      s = __fadd_rn(s, partial[(static_cast<int64_t>(t) * k2TileM + lr) * kMlpRank + j]);
+    }
     xl1[i] = __float2bfloat16_rn(s);
   }
 }
 
 template <int R, int EPI>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(k2Threads, 1) w4a4_gemm_2sm_kernel(
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<R, EPI>::kThreads, 1) w4a4_gemm_2sm_kernel(
     const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
     const __grid_constant__ CUtensorMap tm_sfa, const __grid_constant__ CUtensorMap tm_sfb,
     const __grid_constant__ CUtensorMap tm_xl1, const __grid_constant__ CUtensorMap tm_l2s,
-    const __grid_constant__ CUtensorMap tm_y, const float* __restrict__ gscale,
+    const __grid_constant__ CUtensorMap tm_y, const __grid_constant__ CUtensorMap tm_l1d, const float* __restrict__ gscale,
     const __nv_bfloat16* __restrict__ bias, int M, int N, int K, const QkvPost post, const MlpPost mlp) {
   using C = Gemm2Cfg<R, EPI>;
   constexpr bool QKV = EPI == 1;
@@ -607,19 +561,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(k2Threads, 1) w4a4_g
   const int nk = K / 256;
   const int steps = C::kLrSteps + nk;
   const int sf_row_stride = K / 64;  // scale atoms per 128-row block
+  // A scales stay in TMEM across the tiles of one A block when every K block has a slot
+  const bool sfa_resident = nk <= C::kSfaSlots;
+  int t_begin, t_end;
+  pair_tile_range(pair, num_pairs, num_tiles, t_begin, t_end);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(&bars->full[s], 1);
       mbar_init(&bars->empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&bars->acc_full[b], 1);
-      mbar_init(&bars->acc_empty[b], 16);  // 8 epilogue warps x 2 CTAs
-    }
-    mbar_init(&bars->ovl_free, 8);         // 4 warps (the half holding the shared columns) x 2 CTAs
+    mbar_init(&bars->acc_full, 1);
+    mbar_init(&bars->acc_empty, 16);  // 8 epilogue warps x 2 CTAs
+    mbar_init(&bars->bias_ready[0], 256);
+    mbar_init(&bars->bias_ready[1], 256);
     mbar_init(&bars->teardown, 1);
     for (int i = 0; i < 4; ++i) mbar_init(&bars->xchg[i], 64);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bars->chunk_ready[i], 8);  // 4 warps x 2 CTAs
+      mbar_init(&bars->chunk_free[i], 1);
+      mbar_init(&bars->l1d_full[i], 1);
+      mbar_init(&bars->l1d_free[i], 1);
+    }
+    mbar_init(&bars->xl1_done, 1);
+    mbar_init(&bars->xl1_free, 8);
+    mbar_init(&bars->xl1_teardown, 1);
     bars->abort = 0;
     fence_barrier_init();
   }
@@ -631,6 +597,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(k2Threads, 1) w4a4_g
     prefetch_tmap(&tm_xl1);
     prefetch_tmap(&tm_l2s);
     prefetch_tmap(&tm_y);
+    if (C::MLP) prefetch_tmap(&tm_l1d);
   }
   if (warp == 1) {
     tmem_alloc_cg2(&bars->tmem_base, 512);
@@ -651,8 +618,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(k2Threads, 1) w4a4_g
       int s = 0;
       uint32_t ph = 0;
       bool ok = true;
-      for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
-        const int mt = tile % num_mt, nt = tile / num_mt;
+      int prev_mt = -1;
+      for (int tile = t_begin; tile < t_end && ok; ++tile) {
+        const int mt = tile / num_nt, nt = tile % num_nt;
+        const bool sfa_load = !sfa_resident || mt != prev_mt;
+        prev_mt = mt;
         const int m_own = mt * k2TileM + static_cast<int>(rank) * 128;
         const int n_own = nt * k2TileN + static_cast<int>(rank) * 128;
         const int nblk = nt * 2;  // first 128-row block of B in this tile
@@ -668,11 +638,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(k2Threads, 1) w4a4_g
             tma_load_2d_cg2(st + C::kABytes + C::kLrTileBytes, &tm_l2s, x, N + n_own, bar);
           } else {
             const int kb = step - C::kLrSteps;
-            if (rank == 0) mbar_arrive_expect_tx(&bars->full[s], C::kMainTx);
+            if (rank == 0) mbar_arrive_expect_tx(&bars->full[s], sfa_load ? C::kMainTx : C::kMainTx - C::kSfaTx);
             tma_load_2d_cg2(st, &tm_a, kb * 128, m_own, bar);
             tma_load_2d_cg2(st + C::kABytes, &tm_b, kb * 128, n_own, bar);
             uint8_t* sf = st + C::kABytes + C::kBBytes;
-            tma_load_4d_cg2(sf, &tm_sfa, 0, 0, 0, (m_own / 128) * sf_row_stride + 4 * kb, bar);
+            if (sfa_load) tma_load_4d_cg2(sf, &tm_sfa, 0, 0, 0, (m_own / 128) * sf_row_stride + 4 * kb, bar);
             tma_load_5d_cg2(sf + C::kSfaBytes, &tm_sfb, 0, 0, 0, 4 * kb, nblk, bar);
           }
           if (++s == S) { s = 0; ph ^= 1; }
@@ -691,17 +661,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(k2Threads, 1) w4a4_g
       const uint32_t idesc_fp4 = (1u << 7) | (1u << 10) | (uint32_t(k2TileN >> 3) << 17) | (uint32_t(k2TileM >> 4) << 24);
       const uint32_t idesc_bf16 =
           (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(k2TileN >> 3) << 17) | (uint32_t(k2TileM >> 4) << 24);
-      const uint32_t t_sfa = tmem + k2SfaCol;
       const uint32_t t_sfb = tmem + k2SfbCol;
       int s = 0;
       uint32_t ph = 0;
       int it = 0;
       bool ok = true;
-      for (int tile = pair; tile < num_tiles && ok; tile += num_pairs, ++it) {
-        const int b = it & 1;
-        const uint32_t t_acc = tmem + (b ? k2Acc1Col : 0);
-        if (!mbar_wait_cluster(&bars->acc_empty[b], ((it >> 1) & 1) ^ 1, abort)) { ok = false; break; }
-        if (it > 0 && !mbar_wait_cluster(&bars->ovl_free, (it - 1) & 1, abort)) { ok = false; break; }
+      int prev_mt = -1;
+      for (int tile = t_begin; tile < t_end && ok; ++tile, ++it) {
+        const int mt = tile / num_nt;
+        const bool sfa_load = !sfa_resident || mt != prev_mt;
+        prev_mt = mt;
+        // the epilogue has drained the previous tile's accumulator
+        if (!mbar_wait_cluster(&bars->acc_empty, (it & 1) ^ 1, abort)) { ok = false; break; }
         tc_fence_after();
         for (int step = 0; step < steps; ++step) {
           if (!mbar_wait(&bars->full[s], ph, abort)) { ok = false; break; }
@@ -714,15 +685,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(k2Threads, 1) w4a4_g
               const uint64_t bh = smem_desc(st + C::kABytes + 32 * k16, 16, 8 * C::kLrRowBytes, C::kLrSwizzle);
               const uint64_t bl =
                   smem_desc(st + C::kABytes + C::kLrTileBytes + 32 * k16, 16, 8 * C::kLrRowBytes, C::kLrSwizzle);
-              mma_bf16_cg2(t_acc, a, bh, idesc_bf16, (step | k16) != 0 ? 1u : 0u);
-              mma_bf16_cg2(t_acc, a, bl, idesc_bf16, 1u);
+              mma_bf16_cg2(tmem, a, bh, idesc_bf16, (step | k16) != 0 ? 1u : 0u);
+              mma_bf16_cg2(tmem, a, bl, idesc_bf16, 1u);
             }
           } else {
+            const int kb = step - C::kLrSteps;
+            const uint32_t t_sfa = tmem + k2SfaCol + 16 * (kb % C::kSfaSlots);
             const uint32_t sfa = st + C::kABytes + C::kBBytes;
             const uint32_t sfb = sfa + C::kSfaBytes;
-            // A: K-steps (0,1) and (2,3), 2 KB apart; B: K-step j, row blocks 8 KB apart
-            tmem_cp_128x256b_cg2(t_sfa, smem_desc(sfa, 2048, 128, kSwizzleNone));
-            tmem_cp_128x256b_cg2(t_sfa + 8, smem_desc(sfa + 4096, 2048, 128, kSwizzleNone));
+            // A: K-steps (0,1) and (2,3), 2 KB apart (only when the tile starts a new A block);
+            // B: K-step j, row blocks 8 KB apart
+            if (sfa_load) {
+              tmem_cp_128x256b_cg2(t_sfa, smem_desc(sfa, 2048, 128, kSwizzleNone));
+              tmem_cp_128x256b_cg2(t_sfa + 8, smem_desc(sfa + 4096, 2048, 128, kSwizzleNone));
+            }
 #pragma unroll
             for (int j = 0; j < 4; ++j)
               tmem_cp_128x256b_cg2(t_sfb + 8 * j, smem_desc(sfb + 2048 * j, 8192, 128, kSwizzleNone));
@@ -730,109 +706,218 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(k2Threads, 1) w4a4_g
             const uint64_t bdesc = smem_desc(st + C::kABytes, 16, 1024, kSwizzle128B);
 #pragma unroll
             for (int j = 0; j < 4; ++j)
-              mma_nvf4_cg2(t_acc, adesc + 2 * j, bdesc + 2 * j, idesc_fp4, t_sfa + 4 * j, t_sfb + 8 * j, 1u);
+              mma_nvf4_cg2(tmem, adesc + 2 * j, bdesc + 2 * j, idesc_fp4, t_sfa + 4 * j, t_sfb + 8 * j, 1u);
           }
           tc_commit_cg2_mc(&bars->empty[s], 0x3);
           if (++s == S) { s = 0; ph ^= 1; }
         }
         if (!ok) break;
-        tc_commit_cg2_mc(&bars->acc_full[b], 0x3);
+        tc_commit_cg2_mc(&bars->acc_full, 0x3);
       }
       // every MMA this thread issued completes before TMEM is released
       tc_commit(&bars->teardown);
       volatile int never = 0;
       mbar_wait(&bars->teardown, 0, &never);
     }
-  } else {
+  } else if (C::MLP && warp == 10) {
+    // ------------------------------------------------------------ MLP: h . L1_down (both CTAs load, even CTA issues)
+    // Per tile: L1_down^T for the tile's 256 columns (each CTA its 16 of the 32
+    // rows; completion bytes on the even CTA's barrier), then for each staged
+    // 64-column chunk of h four bf16 MMAs (M = 256, N = 32, K = 16) into the
+    // h . L1_down accumulator, which runs over the pair's tiles that share
+    // their rows and is read out at the end of each such run.
+    if (lane == 0) {
+      const uint32_t idesc =
+          (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(kMlpRank >> 3) << 17) | (uint32_t(k2TileM >> 4) << 24);
+      uint8_t* l1d = smem + C::kL1dOff;
+      const uint32_t t_xl1 = tmem + k2Xl1Col;
+      // L1_down^T of the pair's it-th tile into buffer it & 1 (once the MMAs of
+      // tile it - 2 have read that buffer)
+      auto load_l1d = [&](int it, int tile) -> bool {
+        const int b = it & 1;
+        if (!mbar_wait(&bars->l1d_free[b], ((it >> 1) & 1) ^ 1, abort)) return false;
+        if (rank == 0) mbar_arrive_expect_tx(&bars->l1d_full[b], 2u * 4u * C::kL1dChunk);
+        const uint32_t lbar = mapa_shared(smem_u32(&bars->l1d_full[b]), 0);
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          tma_load_2d_cg2(l1d + (4 * b + k) * C::kL1dChunk, &tm_l1d, (tile % num_nt) * k2TileN + 64 * k,
+                          16 * static_cast<int>(rank), lbar);
+        return true;
+      };
+      int it = 0, run = 0, prev_mt = -1;
+      bool ok = t_begin >= t_end || load_l1d(0, t_begin);
+      for (int tile = t_begin; tile < t_end && ok; ++tile, ++it) {
+        const int mt = tile / num_nt;
+        const bool first = mt != prev_mt;
+        prev_mt = mt;
+        const bool last = tile + 1 == t_end || (tile + 1) / num_nt != mt;
+        const int b = it & 1;
+        if (tile + 1 < t_end && !load_l1d(it + 1, tile + 1)) { ok = false; break; }  // the next tile's, early
+        if (rank != 0) continue;
+        // a new run starts once the previous run's accumulator has been read out
+        if (first && it > 0 && !mbar_wait_cluster(&bars->xl1_free, (run - 1) & 1, abort)) { ok = false; break; }
+        if (!mbar_wait(&bars->l1d_full[b], (it >> 1) & 1, abort)) { ok = false; break; }
+        // chunks alternate between the column halves' warps: (half 0, chunk 0),
+        // (half 1, chunk 0), (half 0, chunk 1), (half 1, chunk 1), so each half
+        // stages its next chunk while the other half's is multiplied
+        for (int k = 0; k < 4; ++k) {
+          const int hh = k & 1, cc = k >> 1;
+          if (!mbar_wait_cluster(&bars->chunk_ready[hh], cc, abort)) { ok = false; break; }
+          tc_fence_after();
+          const uint64_t a = smem_desc(smem_u32(smem + C::kOutOff + hh * 16384), 16, 1024, kSwizzle128B);
+          const uint64_t bd =
+              smem_desc(smem_u32(l1d + (4 * b + 2 * hh + cc) * C::kL1dChunk), 16, 1024, kSwizzle128B);
+#pragma unroll
+          for (int k16 = 0; k16 < 4; ++k16)
+            mma_bf16_cg2(t_xl1, a + 2 * k16, bd + 2 * k16, idesc, (first && k == 0 && k16 == 0) ? 0u : 1u);
+          tc_commit_cg2_mc(&bars->chunk_free[hh], 0x3);
+        }
+        if (!ok) break;
+        tc_commit_cg2_mc(&bars->l1d_free[b], 0x3);
+        if (last) {
+          tc_commit_cg2_mc(&bars->xl1_done, 0x3);
+          ++run;
+        }
+      }
+      if (rank == 0) {  // every MMA this thread issued completes before TMEM is released
+        tc_commit(&bars->xl1_teardown);
+        volatile int never = 0;
+        mbar_wait(&bars->xl1_teardown, 0, &never);
+      }
+      if (!ok) {
+        const uint64_t t0 = globaltimer();
+        while (globaltimer() - t0 < 2000000ull) {
+        }
+      }
+    }
+  } else if (warp < 10) {
     // ------------------------------------------------------------ epilogue (both CTAs)
     const int e = warp - 2;
     const int q = warp & 3;  // TMEM lane quadrant this warp may access
-    const int h = e >> 2;    // 128-column half of the tile
+    const int h = e >> 2;    // 128-column half of the tile (fused QKV: chunk pair)
     const float alpha = gscale[2];
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(32 * q) << 16);
-    const uint32_t ovl_bar = mapa_shared(smem_u32(&bars->ovl_free), 0);
-    uint8_t* stage = smem + C::kOutOff + e * C::kOutPerWarp;
-    int nbuf = 0;
+    const uint32_t acc_empty_remote = mapa_shared(smem_u32(&bars->acc_empty), 0);
+    // staging buffer of warp (h, q): the MLP epilogue's chunk buffer of half h
+    // holds the four quadrants' rows in order (rows 32 q .. 32 q + 31 at q x 4 KB)
+    uint8_t* stage = smem + C::kOutOff + (4 * h + q) * C::kOutPerWarp;
+    __nv_bfloat16* bias_s = reinterpret_cast<__nv_bfloat16*>(smem + C::kBiasOff);
     uint32_t nx = 0;  // fused QKV: exchanges of row sums done by this warp
+    int mlp_prev_mt = -1, run_first = 0, nrun = 0;  // MLP: runs of tiles sharing their rows
     int it = 0;
-    for (int tile = pair; tile < num_tiles; tile += num_pairs, ++it) {
-      const int mt = tile % num_mt, nt = tile / num_mt;
-      const int b = it & 1;
+    for (int tile = t_begin; tile < t_end; ++tile, ++it) {
+      const int mt = tile / num_nt, nt = tile % num_nt;
       const int y0 = mt * k2TileM + static_cast<int>(rank) * 128 + 32 * q;
       const int col0 = nt * k2TileN + 128 * h;
+      // the tile's bias into shared memory (thread 32 e + lane loads one value)
+      __nv_bfloat16* bb = bias_s + (it & 1) * k2TileN;
+      if (bias != nullptr) bb[32 * e + lane] = bias[nt * k2TileN + 32 * e + lane];
+      mbar_arrive(&bars->bias_ready[it & 1]);
       if constexpr (QKV) {
-        // Q / K tiles: this lane's rotary angles for the warp's first chunk,
-        // fetched before the accumulator is ready. A tile is all Q/K or all V (the
-        // V block starts at 2 * hd, a multiple of 256).
+        // A tile is all Q/K or all V (the V block starts at 2 * hd, a multiple of 256).
+        if (!mbar_wait(&bars->acc_full, it & 1, abort)) break;
+        tc_fence_after();
+        uint32_t y0c[16], y0d[16], y1c[16], y1d[16];
+        {
+          uint32_t va[32], vb[32], vc[32], vd[32];
+          const int c0 = 2 * h;
+          drain4(lane_base, 32 * c0, 32 * (c0 + 1), 128 + 32 * c0, 128 + 32 * (c0 + 1), va, vb, vc, vd,
+                 acc_empty_remote, lane);
+          if (!mbar_wait(&bars->bias_ready[it & 1], (it >> 1) & 1, abort)) break;
+          const __nv_bfloat16* bt = bias != nullptr ? bb : nullptr;
+          pack_chunk(va, bt ? bt + 32 * c0 : nullptr, alpha, y0c);
+          pack_chunk(vb, bt ? bt + 32 * (c0 + 1) : nullptr, alpha, y0d);
+          pack_chunk(vc, bt ? bt + 128 + 32 * c0 : nullptr, alpha, y1c);
+          pack_chunk(vd, bt ? bt + 128 + 32 * (c0 + 1) : nullptr, alpha, y1d);
+        }
+
         const int xt = nt * k2TileN;
         const bool qk = xt < 2 * post.hd;
-        float tc0[16], ts0[16];
         const int64_t row = (y0 + lane < M) ? y0 + lane : M - 1;
         const float* cr = post.cos + row * post.ld_rope + 32 * h;
         const float* sr = post.sin + row * post.ld_rope + 32 * h;
-        if (qk) {
-          load_angles16(cr, sr, tc0, ts0);
-        } else {
-#pragma unroll
-          for (int i = 0; i < 16; ++i) tc0[i] = ts0[i] = 0.0f;
-        }
         const __nv_bfloat16* w0 = qk ? (xt < post.hd ? post.w_q : post.w_k) : nullptr;
         const __nv_bfloat16* w1 = qk ? (xt + 128 < post.hd ? post.w_q : post.w_k) : nullptr;
-        if (!mbar_wait(&bars->acc_full[b], (it >> 1) & 1, abort)) break;
-        tc_fence_after();
-        const uint32_t tacc = lane_base + (b ? k2Acc1Col : 0);
-        const __nv_bfloat16* btile = bias != nullptr ? bias + xt : nullptr;
         float* xs = reinterpret_cast<float*>(smem + C::kXchgOff) + 128 * (2 * q + h) + 64 * (nx & 1);
         const float* xp = reinterpret_cast<const float*>(smem + C::kXchgOff) + 128 * (2 * q + (h ^ 1)) + 64 * (nx & 1);
-        // accumulator 0's shared columns lie in head 1 (warp 1's chunks),
-        // accumulator 1's in head 0 (warp 0's chunks)
-        const bool ok = epilogue_qkv_tile(tacc, b == 0 ? 1 : 0, h, btile, alpha, stage, &tm_y, xt, y0, h == (b == 0),
-                                          ovl_bar, lane, b == 0 ? w1 : w0, b == 0 ? w0 : w1, tc0, ts0, cr + 16, sr + 16, xs, xp, &bars->xchg[q], nx & 1,
-                                          post.eps, abort);
+        // (the accumulator is already released: the angles' latency no longer holds the MMAs up)
+        const bool ok = epilogue_qkv_tile(y0c, y0d, y1c, y1d, h, stage, &tm_y, xt, y0, lane, w0, w1, cr, sr, xs,
+                                          xp, &bars->xchg[q], nx & 1, post.eps, abort);
         if (!ok) break;
         if (qk) ++nx;
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive_cluster_relaxed(mapa_shared(smem_u32(&bars->acc_empty[b]), 0));
         continue;
       }
-      if constexpr (EPI == 2) {
-        if (!mbar_wait(&bars->acc_full[b], (it >> 1) & 1, abort)) break;
-        tc_fence_after();
-        const uint32_t acc = lane_base + (b ? k2Acc1Col : 0) + 128 * h;
-        const __nv_bfloat16* bcol = bias != nullptr ? bias + col0 : nullptr;
-        const int slot = 2 * nt + h;
-        if (b == 0 && h == 1)
-          epilogue_half_mlp<kMlpRank, 2>(acc, bcol, alpha, stage, nbuf, &tm_y, col0, y0, true, ovl_bar, lane, mlp, M,
-                                         N, slot);
-        else
-          epilogue_half_mlp<kMlpRank, 0>(acc, bcol, alpha, stage, nbuf, &tm_y, col0, y0, b == 1 && h == 0, ovl_bar,
-                                         lane, mlp, M, N, slot);
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive_cluster_relaxed(mapa_shared(smem_u32(&bars->acc_empty[b]), 0));
-        continue;
-      }
-      // bias of this warp's 128 columns, fetched before the accumulator is ready
-      uint4 bv[16];
-      if (bias != nullptr) {
-#pragma unroll
-        for (int i = 0; i < 16; ++i) bv[i] = ldg_v4(bias + col0 + 8 * i);
-      } else {
-#pragma unroll
-        for (int i = 0; i < 16; ++i) bv[i] = make_uint4(0u, 0u, 0u, 0u);
-      }
-      if (!mbar_wait(&bars->acc_full[b], (it >> 1) & 1, abort)) break;
+      if (!mbar_wait(&bars->acc_full, it & 1, abort)) break;
       tc_fence_after();
-      const uint32_t acc = lane_base + (b ? k2Acc1Col : 0) + 128 * h;
-      if (b == 0 && h == 1)
-        epilogue_half<2>(acc, bv, alpha, stage, nbuf, &tm_y, col0, y0, true, ovl_bar, lane);
-      else
-        epilogue_half<0>(acc, bv, alpha, stage, nbuf, &tm_y, col0, y0, b == 1 && h == 0, ovl_bar, lane);
-      tc_fence_before();
-      __syncwarp();
-      // every TMEM load of this accumulator has completed; the MMAs read nothing this warp wrote
-      if (lane == 0) mbar_arrive_cluster_relaxed(mapa_shared(smem_u32(&bars->acc_empty[b]), 0));
+      uint32_t va[32], vb[32], vc[32], vd[32];
+      drain4(lane_base + 128 * h, 0, 32, 64, 96, va, vb, vc, vd, acc_empty_remote, lane);
+      if (!mbar_wait(&bars->bias_ready[it & 1], (it >> 1) & 1, abort)) break;
+      const __nv_bfloat16* bcol = bias != nullptr ? bb + 128 * h : nullptr;
+      if constexpr (EPI == 2) {
+        const int row = y0 + lane;
+        const float g = *mlp.g_h;
+        const float d = __fmul_rn(6.0f, g);
+        uint32_t pk0[16], pk1[16], pk2[16], pk3[16];
+        pack_chunk(va, bcol, alpha, pk0);
+        pack_chunk(vb, bcol ? bcol + 32 : nullptr, alpha, pk1);
+        pack_chunk(vc, bcol ? bcol + 64 : nullptr, alpha, pk2);
+        pack_chunk(vd, bcol ? bcol + 96 : nullptr, alpha, pk3);
+        const bool first = mt != mlp_prev_mt;
+        mlp_prev_mt = mt;
+        if (first) run_first = tile;
+        const bool last = tile + 1 == t_end || (tile + 1) / num_nt != mt;
+        const uint32_t ready = mapa_shared(smem_u32(&bars->chunk_ready[h]), 0);
+        bool ok = true;
+#pragma unroll
+        for (int cc = 0; cc < 2 && ok; ++cc) {
+          uint32_t(&pa)[16] = cc == 0 ? pk0 : pk2;
+          uint32_t(&pb)[16] = cc == 0 ? pk1 : pk3;
+          mlp_quantize64(pa, pb, col0 + 64 * cc, row, M, N, mlp, g, d);
+          // this half's chunk buffer: its previous chunk's MMAs have read it
+          if (!mbar_wait(&bars->chunk_free[h], cc ^ 1, abort)) { ok = false; break; }
+          if (mlp.store_h && lane == 0) bulk_wait_read0();  // and so has the previous store of h
+          __syncwarp();
+          stage_row64(stage, pa, pb, lane);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive_cluster_release(ready);
+            if (mlp.store_h) {
+              tma_store_2d(&tm_y, stage, col0 + 64 * cc, y0);
+              bulk_commit();
+            }
+          }
+        }
+        if (!ok) break;
+        if (last) {
+          if (h == 0) {  // the first half's warps read the run's accumulator out (their lane quadrant)
+            if (!mbar_wait(&bars->xl1_done, nrun & 1, abort)) break;
+            tc_fence_after();
+            uint32_t xv[32];
+            tmem_ld_32x32b_x32(lane_base + k2Xl1Col, xv);
+            tmem_ld_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster_relaxed(mapa_shared(smem_u32(&bars->xl1_free), 0));
+            float4* dst = reinterpret_cast<float4*>(
+                mlp.partial + (static_cast<int64_t>(run_first) * k2TileM + static_cast<int>(rank) * 128 + 32 * q + lane) *
+                                  kMlpRank);
+#pragma unroll
+            for (int j = 0; j < kMlpRank / 4; ++j)
+              dst[j] = make_float4(__uint_as_float(xv[4 * j]), __uint_as_float(xv[4 * j + 1]),
+                                   __uint_as_float(xv[4 * j + 2]), __uint_as_float(xv[4 * j + 3]));
+          }
+          ++nrun;
+        }
+        continue;
+      }
+      uint32_t pa[16], pb[16];
+      pack_chunk(va, bcol, alpha, pa);
+      pack_chunk(vb, bcol ? bcol + 32 : nullptr, alpha, pb);
+      store_row64(stage, pa, pb, &tm_y, col0, y0, lane);
+      pack_chunk(vc, bcol ? bcol + 64 : nullptr, alpha, pa);
+      pack_chunk(vd, bcol ? bcol + 96 : nullptr, alpha, pb);
+      store_row64(stage, pa, pb, &tm_y, col0 + 64, y0, lane);
     }
     if (lane == 0) bulk_wait_all();
     __syncwarp();

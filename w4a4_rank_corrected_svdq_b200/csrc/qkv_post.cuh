@@ -37,15 +37,14 @@ struct QkvPost {
 // the full engine's speed comes partly from fused GELU / MLP kernels):
 // h = bf16(GELU(bf16(alpha acc + b))) quantised in place for the down
 // projection (NVFP4 codes and tiled block scales with the down projection's
-// activation scale g_h) and its fp32 partial products with the down
-// projection's L1 (XL1 partials per 128-column half tile, summed afterwards
-// in tile order).
+// activation scale g_h), and h . L1_down accumulated on the tensor cores over
+// each CTA pair's run of tiles that share their rows (one fp32 XL1 partial per
+// run, summed afterwards in tile order).
 struct MlpPost {
   const float* g_h;           // device float: the down projection's activation decode scale
-  const __nv_bfloat16* l1d;   // [N][r_down] row-major: the down projection's L1 (its K = this layer's N)
   uint8_t* codes;             // [M][N/2]
   uint8_t* scales;            // tiled, rows padded to 128 (padding rows get zero scales)
-  float* partial;             // [2 N / 256][M][r_down] fp32
+  float* partial;             // [tiles][256][r_down] fp32: XL1 partial of each run of tiles (slot = first tile)
   int m_pad;                  // M rounded up to 128
   int store_h;                // also store h (bf16) through the output map
   int approximate;            // tanh form of GELU
@@ -54,17 +53,53 @@ struct MlpPost {
 // GELU in fp32: x Phi(x) = x erfc(-x / sqrt 2) / 2, or the tanh form
 // x (1 + tanh u) / 2 = x / (1 + exp(-2u)), u = sqrt(2/pi) (x + 0.044715 x^3);
 // both written without the cancellation of 1 + erf / 1 + tanh for negative x.
+//
+// h is rounded to bf16 (8 significant bits), so a relative error far below
+// 2^-10 is enough for the result to lie within one bf16 step of the correctly
+// rounded value. The fast paths below stay far inside that:
+//  * erfc(z), z >= 0, by the Chebyshev fit of Press, Teukolsky, Vetterling and
+//    Flannery (Numerical Recipes in C, 2nd ed., section 6.2, erfcc): with
+//    t = 1 / (1 + z/2), erfc(z) = t exp(-z^2 + P(t)), P of degree 9, fractional
+//    error below 1.2e-7 for every z >= 0; erfc(-z) = 2 - erfc(z);
+//  * exponentials by the hardware exp2 (__expf, relative error ~2^-21),
+//    reciprocals by __fdividef.
+// Where a result would fall below the normal fp32 range (|z| > 9 for erfc,
+// 2u < -80 in the tanh form) the accurate library functions take over, so the
+// far negative tail keeps its tiny values (subnormals included) instead of
+// flushing them to zero.
+__device__ __forceinline__ float erfc_fast_nonneg(float z) {
+  const float t = __fdividef(1.0f, __fmaf_rn(0.5f, z, 1.0f));
+  float p = 0.17087277f;
+  p = __fmaf_rn(p, t, -0.82215223f);
+  p = __fmaf_rn(p, t, 1.48851587f);
+  p = __fmaf_rn(p, t, -1.13520398f);
+  p = __fmaf_rn(p, t, 0.27886807f);
+  p = __fmaf_rn(p, t, -0.18628806f);
+  p = __fmaf_rn(p, t, 0.09678418f);
+  p = __fmaf_rn(p, t, 0.37409196f);
+  p = __fmaf_rn(p, t, 1.00002368f);
+  p = __fmaf_rn(p, t, -1.26551223f);
+  return t * __expf(__fmaf_rn(-z, z, p));
+}
+
 __device__ __forceinline__ float gelu_f32(float x, bool approximate) {
   if (approximate) {
     const float u = __fmul_rn(0.7978845608028654f, __fmaf_rn(__fmul_rn(0.044715f, x), __fmul_rn(x, x), x));
-    if (u >= 0.0f) return __fdiv_rn(x, __fadd_rn(1.0f, expf(__fmul_rn(-2.0f, u))));
+    if (u >= 0.0f) return __fdividef(x, 1.0f + __expf(-2.0f * u));
     // the same function for u < 0 as x e^{2u} / (1 + e^{2u}): e^{2u} <= 1 never
-    // overflows, so the far negative tail keeps its tiny (possibly subnormal)
-    // values instead of collapsing to x / inf = -0
+    // overflows
+    if (u > -40.0f) {
+      const float e = __expf(2.0f * u);
+      return __fdividef(x * e, 1.0f + e);
+    }
     const float e = expf(__fmul_rn(2.0f, u));
     return __fdiv_rn(__fmul_rn(x, e), __fadd_rn(1.0f, e));
   }
-  return __fmul_rn(__fmul_rn(0.5f, x), erfcf(__fmul_rn(x, -0.7071067811865476f)));
+  const float z = x * -0.7071067811865476f;
+  const float az = fabsf(z);
+  if (az > 9.0f) return __fmul_rn(__fmul_rn(0.5f, x), erfcf(z));
+  const float e = erfc_fast_nonneg(az);
+  return 0.5f * x * (z >= 0.0f ? e : 2.0f - e);
 }
 
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }

@@ -426,13 +426,20 @@ svdq_status launch_gemm(int M, int N, int K, const void* a_codes, const void* a_
   return launch_status();
 }
 
+// CTA pairs the 2-SM GEMM launches: one per tile, at most one per two SMs.
+int gemm2_pairs(int M, int N, int sm_count) {
+  const int tiles = ((M + k2TileM - 1) / k2TileM) * (N / k2TileN);
+  const int max_pairs = sm_count / 2;
+  return tiles < max_pairs ? tiles : max_pairs;
+}
+
 template <int R, int EPI>
 svdq_status launch_gemm_2sm(int M, int N, int K, const void* a_codes, const void* a_scales, const void* xl1,
                             const void* w_codes, const void* w_scales, const float* gscale, const void* l2s,
                             const void* bias, void* Y, int64_t ldy, cudaStream_t stream, int sm_count,
-                            const QkvPost& post, const MlpPost& mlp) {
+                            const QkvPost& post, const MlpPost& mlp, const void* l1t_down) {
   using C = Gemm2Cfg<R, EPI>;
-  CUtensorMap tm_a, tm_b, tm_sfa, tm_sfb, tm_x, tm_l, tm_y;
+  CUtensorMap tm_a, tm_b, tm_sfa, tm_sfb, tm_x, tm_l, tm_y, tm_l1d;
   const uint64_t kb = static_cast<uint64_t>(K / 2);
   const uint64_t mpad = round_up(static_cast<size_t>(M), 128);
   const CUtensorMapSwizzle lr_sw = C::kLrRowBytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B;
@@ -444,17 +451,24 @@ svdq_status launch_gemm_2sm(int M, int N, int K, const void* a_codes, const void
       !make_tmap_2d(&tm_x, xl1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, R, M, R * 2, C::kLrCols, 128, lr_sw) ||
       !make_tmap_2d(&tm_l, l2s, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, R, 2 * static_cast<uint64_t>(N), R * 2,
                     C::kLrCols, 128, lr_sw) ||
-      !make_tmap_2d(&tm_y, Y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, M, static_cast<uint64_t>(ldy) * 2, 32, 32,
-                    CU_TENSOR_MAP_SWIZZLE_64B))
+      // the fused QKV epilogue stores 32 rows x 32 columns (64-byte swizzle), the others 32 x 64 (128-byte)
+      !make_tmap_2d(&tm_y, Y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, M, static_cast<uint64_t>(ldy) * 2,
+                    EPI == 1 ? 32 : 64, 32, EPI == 1 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B))
     return SVDQ_ERR_CUDA;
+  // MLP: L1_down^T [32][N] (bf16, row pitch 2N), boxes of 16 rows x 64 columns; otherwise unused
+  if (EPI == 2) {
+    if (!make_tmap_2d(&tm_l1d, l1t_down, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, kMlpRank,
+                      static_cast<uint64_t>(N) * 2, 64, 16, CU_TENSOR_MAP_SWIZZLE_128B))
+      return SVDQ_ERR_CUDA;
+  } else {
+    tm_l1d = tm_y;
+  }
   auto kern = w4a4_gemm_2sm_kernel<R, EPI>;
   static std::atomic<uint64_t> attr_done{0};
   ensure_smem_attr(kern, C::kSmemBytes, attr_done);
-  const int tiles = ((M + k2TileM - 1) / k2TileM) * (N / k2TileN);
-  const int max_pairs = sm_count / 2;
-  const int pairs = tiles < max_pairs ? tiles : max_pairs;
-  PdlLaunch pl(dim3(2 * pairs), dim3(k2Threads), C::kSmemBytes, stream);
-  cudaLaunchKernelEx(&pl.cfg, kern, tm_a, tm_b, tm_sfa, tm_sfb, tm_x, tm_l, tm_y, gscale,
+  const int pairs = gemm2_pairs(M, N, sm_count);
+  PdlLaunch pl(dim3(2 * pairs), dim3(C::kThreads), C::kSmemBytes, stream);
+  cudaLaunchKernelEx(&pl.cfg, kern, tm_a, tm_b, tm_sfa, tm_sfb, tm_x, tm_l, tm_y, tm_l1d, gscale,
                      static_cast<const __nv_bfloat16*>(bias), M, N, K, post, mlp);
   return launch_status();
 }
@@ -477,14 +491,16 @@ bool use_2sm(int M, int N) {
 svdq_status gemm_dispatch(int M, int N, int K, int r, const void* a_codes, const void* a_scales, const void* xl1,
                           const void* w_codes, const void* w_scales, const float* gscale, const void* l2s,
                           const void* bias, void* Y, int64_t ldy, cudaStream_t st, int sms,
-                          const QkvPost* post = nullptr, const MlpPost* mlp = nullptr) {
+                          const QkvPost* post = nullptr, const MlpPost* mlp = nullptr,
+                          const void* l1t_down = nullptr) {
   const QkvPost none{};
   const QkvPost& pp = post != nullptr ? *post : none;
   const MlpPost mnone{};
   const MlpPost& mp = mlp != nullptr ? *mlp : mnone;
   if (mlp != nullptr) {  // the MLP up-projection epilogue exists for the CTA-pair GEMM only
     if (N % 256 != 0) return SVDQ_ERR_UNSUPPORTED_SHAPE;
-#define SVDQ_GEMM2_ARGS M, N, K, a_codes, a_scales, xl1, w_codes, w_scales, gscale, l2s, bias, Y, ldy, st, sms, pp, mp
+#define SVDQ_GEMM2_ARGS M, N, K, a_codes, a_scales, xl1, w_codes, w_scales, gscale, l2s, bias, Y, ldy, st, sms, pp, mp, \
+                        l1t_down
     switch (r) {
       case 16: return launch_gemm_2sm<16, 2>(SVDQ_GEMM2_ARGS);
       case 32: return launch_gemm_2sm<32, 2>(SVDQ_GEMM2_ARGS);
@@ -1075,14 +1091,16 @@ svdq_status svdq_mlp_workspace_size(int M, int N, int K, int r, int r_down, size
   if (r_down != kMlpRank || N % 256 != 0) return SVDQ_ERR_UNSUPPORTED_SHAPE;
   if ((s = svdq_forward_workspace_size(M, K, r, &base)) != SVDQ_OK) return s;
   if (!bytes) return SVDQ_ERR_INVALID_ARG;
-  *bytes = base + round_up(static_cast<size_t>(2 * (N / 256)) * M * r_down * 4, 256);
+  // one fp32 XL1 partial slot of 256 rows per 256 x 256 tile (used by the tiles that start a run)
+  const size_t tiles = static_cast<size_t>((M + 255) / 256) * (N / 256);
+  *bytes = base + round_up(tiles * 256 * r_down * 4, 256);
   return SVDQ_OK;
 }
 
 svdq_status svdq_mlp_up_forward(int M, int N, int K, int r, const void* X, int64_t ldx, const void* w_codes,
                                 const void* w_scales, const float* gscale, const void* l1t, const void* l2s,
                                 const float* inv_smooth, const void* bias, int r_down, const float* g_h,
-                                const void* l1_down, int approximate, void* h_codes, void* h_scales, void* h_xl1,
+                                const void* l1t_down, int approximate, void* h_codes, void* h_scales, void* h_xl1,
                                 void* h_out, int64_t ldh, void* workspace, size_t workspace_bytes, void* stream) {
   NvtxRange nvtx_range("svdq_mlp_up_forward");
   if (M < 0) return SVDQ_ERR_INVALID_ARG;
@@ -1091,10 +1109,10 @@ svdq_status svdq_mlp_up_forward(int M, int N, int K, int r, const void* X, int64
   if (r_down != kMlpRank || N % 256 != 0 || ldx < K || ldx % 8 != 0 || (h_out && (ldh < N || ldh % 8 != 0)))
     return SVDQ_ERR_UNSUPPORTED_SHAPE;
   if (M == 0) return SVDQ_OK;
-  if (!X || !gscale || !l1t || !g_h || !l1_down || !h_codes || !h_scales || !h_xl1 || !workspace || !w_codes ||
+  if (!X || !gscale || !l1t || !g_h || !l1t_down || !h_codes || !h_scales || !h_xl1 || !workspace || !w_codes ||
       !w_scales || !l2s)
     return SVDQ_ERR_INVALID_ARG;
-  if (!aligned16(l1_down) || !aligned16(h_codes) || !aligned16(h_scales) || !aligned16(h_xl1) ||
+  if (!aligned16(l1t_down) || !aligned16(h_codes) || !aligned16(h_scales) || !aligned16(h_xl1) ||
       !aligned16(workspace) || (h_out && !aligned16(h_out)) || (reinterpret_cast<uintptr_t>(g_h) & 3u) ||
       !aligned16(w_codes) || !aligned16(w_scales) || !aligned16(l2s) || !aligned16(gscale) ||
       (bias && !aligned16(bias)))
@@ -1115,7 +1133,6 @@ svdq_status svdq_mlp_up_forward(int M, int N, int K, int r, const void* X, int64
   if ((s = current_device(nullptr, &di)) != SVDQ_OK) return s;
   MlpPost mp{};
   mp.g_h = g_h;
-  mp.l1d = static_cast<const __nv_bfloat16*>(l1_down);
   mp.codes = static_cast<uint8_t*>(h_codes);
   mp.scales = static_cast<uint8_t*>(h_scales);
   mp.partial = partial;
@@ -1125,13 +1142,15 @@ svdq_status svdq_mlp_up_forward(int M, int N, int K, int r, const void* X, int64
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   // without h_out nothing is stored through the output map; it is built on h_codes only to be valid
   s = gemm_dispatch(M, N, K, r, a_codes, a_scales, xl1, w_codes, w_scales, gscale, l2s, bias,
-                    h_out ? h_out : h_codes, h_out ? ldh : N, st, di.sm_count, nullptr, &mp);
+                    h_out ? h_out : h_codes, h_out ? ldh : N, st, di.sm_count, nullptr, &mp, l1t_down);
   if (s != SVDQ_OK) return s;
   const int64_t tot = static_cast<int64_t>(M) * r_down;
   int64_t blocks = (tot + 255) / 256;
   if (blocks > 4 * di.sm_count) blocks = 4 * di.sm_count;
-  mlp_xl1_reduce_kernel<<<static_cast<int>(blocks), 256, 0, st>>>(partial, 2 * (N / 256), M, r_down,
-                                                                    static_cast<__nv_bfloat16*>(h_xl1));
+  const int num_nt = N / k2TileN;
+  const int num_tiles = ((M + k2TileM - 1) / k2TileM) * num_nt;
+  mlp_xl1_reduce_kernel<<<static_cast<int>(blocks), 256, 0, st>>>(partial, num_tiles, gemm2_pairs(M, N, di.sm_count),
+                                                                    num_nt, M, static_cast<__nv_bfloat16*>(h_xl1));
   return launch_status();
 }
 
