@@ -207,4 +207,185 @@ __global__ void __launch_bounds__(kAwqThreads) awq_gemv_kernel(int M, int N, int
   }
 }
 
+// ------------------------------------------------------------------ bulk-copy ring variant
+// The same layer with the weight rows streamed by one producer thread through a
+// ring of shared-memory stages (cp.async.bulk, completion counted on an
+// mbarrier), so each SM keeps a whole stage ring of weight bytes in flight
+// instead of the 16 bytes per lane and row of direct loads. A stage holds
+// kAwqRingRows consecutive weight rows: their codes (rows x K/2 bytes), bf16
+// scales and zero points (rows x K/64 each) as three contiguous bulk copies,
+// which needs K % 1024 == 0 (16-byte multiples for every row count). Each CTA
+// owns one contiguous run of rows; its 8 consumer warps take kAwqRows rows of
+// every stage each, with the activations staged as in awq_gemv_kernel. Every
+// wait is bounded (mbar_wait).
+constexpr int kAwqRingRows = 8 * kAwqRows;  // rows per stage (8 consumer warps)
+constexpr int kAwqRingThreads = 288;        // 8 consumer warps + 1 producer warp
+constexpr int kAwqRingMaxStages = 8;
+
+__host__ __device__ constexpr int awq_ring_stage_bytes(int K) {
+  return kAwqRingRows * (K / 2 + (K / kAwqGroup) * 3);
+}
+
+template <int MT>
+__global__ void __launch_bounds__(kAwqRingThreads, 1) awq_gemv_ring_kernel(
+    int M, int N, int K, const __nv_bfloat16* __restrict__ X, int64_t ldx, const uint8_t* __restrict__ codes,
+    const __nv_bfloat16* __restrict__ scales, const uint8_t* __restrict__ zeros, const float* __restrict__ inv_act,
+    const __nv_bfloat16* __restrict__ bias, __nv_bfloat16* __restrict__ Y, int64_t ldy, int stages) {
+  extern __shared__ __align__(16) uint8_t ring_smem[];
+  const int rows = M < MT ? M : MT;
+  const int C = K / 32;
+  const int G = K / kAwqGroup;
+  float4* xs4 = reinterpret_cast<float4*>(ring_smem);  // [MT][K/32][8], swizzled
+  uint8_t* ring = ring_smem + MT * K * 4;
+  const int stage_bytes = awq_ring_stage_bytes(K);
+  uint64_t* full = reinterpret_cast<uint64_t*>(ring + stages * stage_bytes);
+  uint64_t* empty = full + kAwqRingMaxStages;
+  int* abort_flag = reinterpret_cast<int*>(empty + kAwqRingMaxStages);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // this CTA's rows [r0, r1) (balanced split) and their stages
+  const int base = N / static_cast<int>(gridDim.x), rem = N % static_cast<int>(gridDim.x);
+  const int r0 = static_cast<int>(blockIdx.x) * base + (static_cast<int>(blockIdx.x) < rem ? blockIdx.x : rem);
+  const int r1 = r0 + base + (static_cast<int>(blockIdx.x) < rem ? 1 : 0);
+  const int nst = (r1 - r0 + kAwqRingRows - 1) / kAwqRingRows;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < stages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 8);  // the 8 consumer warps
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  volatile int* abort = abort_flag;
+  if (warp == 8) {
+    // ---------------------------------------------------------------- producer
+    if (lane == 0) {
+      for (int i = 0; i < nst; ++i) {
+        const int s = i % stages;
+        if (!mbar_wait(&empty[s], ((i / stages) & 1) ^ 1, abort)) break;
+        const int n0 = r0 + i * kAwqRingRows;
+        const int nr = r1 - n0 < kAwqRingRows ? r1 - n0 : kAwqRingRows;
+        uint8_t* st = ring + s * stage_bytes;
+        const uint32_t cb = static_cast<uint32_t>(nr) * (K / 2), sb = static_cast<uint32_t>(nr) * G * 2,
+                       zb = static_cast<uint32_t>(nr) * G;
+        mbar_arrive_expect_tx(&full[s], cb + sb + zb);
+        bulk_load(st, codes + static_cast<int64_t>(n0) * (K / 2), cb, &full[s]);
+        bulk_load(st + kAwqRingRows * (K / 2), scales + static_cast<int64_t>(n0) * G, sb, &full[s]);
+        bulk_load(st + kAwqRingRows * (K / 2 + 2 * G), zeros + static_cast<int64_t>(n0) * G, zb, &full[s]);
+      }
+      if (*abort) {  // error path: give copies that may still be in flight time to land
+        const uint64_t t0 = globaltimer();
+        while (globaltimer() - t0 < 2000000ull) {
+        }
+      }
+    }
+    return;
+  }
+  // ------------------------------------------------------------------ consumers: stage the activations
+  for (int i = threadIdx.x; i < MT * (K / 4); i += 256) {
+    const int m = i / (K / 4), q4 = i % (K / 4);
+    float4 f = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    if (m < rows) {
+      const __nv_bfloat16* src = X + static_cast<int64_t>(m) * ldx + 4 * q4;
+      const uint2 raw = *reinterpret_cast<const uint2*>(src);
+      f = make_float4(__uint_as_float(raw.x << 16), __uint_as_float(raw.x & 0xFFFF0000u),
+                      __uint_as_float(raw.y << 16), __uint_as_float(raw.y & 0xFFFF0000u));
+      if (inv_act != nullptr) {
+        const float4 iv = *reinterpret_cast<const float4*>(inv_act + 4 * q4);
+        f = make_float4(__fmul_rn(f.x, iv.x), __fmul_rn(f.y, iv.y), __fmul_rn(f.z, iv.z), __fmul_rn(f.w, iv.w));
+      }
+    }
+    const int c = q4 >> 3, fi = q4 & 7;
+    xs4[(m * C + c) * 8 + (fi ^ (c & 7))] = f;
+  }
+  asm volatile("bar.sync 1, 256;" ::: "memory");  // the 8 consumer warps only
+  for (int i = 0; i < nst; ++i) {
+    const int s = i % stages;
+    if (!mbar_wait(&full[s], (i / stages) & 1, abort)) break;
+    const uint8_t* st = ring + s * stage_bytes;
+    const __nv_bfloat16* st_sc = reinterpret_cast<const __nv_bfloat16*>(st + kAwqRingRows * (K / 2));
+    const uint8_t* st_z = st + kAwqRingRows * (K / 2 + 2 * G);
+    const int lr0 = warp * kAwqRows;                 // this warp's first row of the stage
+    const int n0 = r0 + i * kAwqRingRows + lr0;
+    float2 acc[kAwqRows][MT];
+#pragma unroll
+    for (int r = 0; r < kAwqRows; ++r)
+#pragma unroll
+      for (int m = 0; m < MT; ++m) acc[r][m] = make_float2(0.0f, 0.0f);
+    for (int c = lane; c < C; c += 32) {
+      uint4 v[kAwqRows];
+      float sv[kAwqRows], zf[kAwqRows];
+#pragma unroll
+      for (int r = 0; r < kAwqRows; ++r) {
+        // rows past the CTA's run read the stage's stale bytes and are not stored
+        v[r] = *reinterpret_cast<const uint4*>(st + (lr0 + r) * (K / 2) + 16 * c);
+        sv[r] = __bfloat162float(st_sc[(lr0 + r) * G + (c >> 1)]);
+        zf[r] = __fadd_rn(8388608.0f, static_cast<float>(st_z[(lr0 + r) * G + (c >> 1)]));
+      }
+      const int sw = c & 7;
+      float2 t[kAwqRows][MT];
+#pragma unroll
+      for (int r = 0; r < kAwqRows; ++r)
+#pragma unroll
+        for (int m = 0; m < MT; ++m) t[r][m] = make_float2(0.0f, 0.0f);
+#pragma unroll
+      for (int wd = 0; wd < 4; ++wd) {
+        float2 d[kAwqRows][4];
+#pragma unroll
+        for (int r = 0; r < kAwqRows; ++r) {
+          const uint32_t word = wd == 0 ? v[r].x : (wd == 1 ? v[r].y : (wd == 2 ? v[r].z : v[r].w));
+          const uint32_t lo = word & 0x0F0F0F0Fu, hi = (word >> 4) & 0x0F0F0F0Fu;
+          const float2 nz2 = make_float2(-zf[r], -zf[r]);
+#pragma unroll
+          for (int b = 0; b < 4; ++b) {
+            const float2 q = make_float2(__uint_as_float(__byte_perm(lo, 0x4B000000u, 0x7650u + b)),
+                                         __uint_as_float(__byte_perm(hi, 0x4B000000u, 0x7650u + b)));
+            d[r][b] = __fadd2_rn(q, nz2);
+          }
+        }
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
+          const float4* xc = xs4 + (m * C + c) * 8;
+          const float4 a = xc[(2 * wd) ^ sw];
+          const float4 e = xc[(2 * wd + 1) ^ sw];
+          const float2 x01 = make_float2(a.x, a.y), x23 = make_float2(a.z, a.w);
+          const float2 x45 = make_float2(e.x, e.y), x67 = make_float2(e.z, e.w);
+#pragma unroll
+          for (int r = 0; r < kAwqRows; ++r) {
+            t[r][m] = __ffma2_rn(x01, d[r][0], t[r][m]);
+            t[r][m] = __ffma2_rn(x23, d[r][1], t[r][m]);
+            t[r][m] = __ffma2_rn(x45, d[r][2], t[r][m]);
+            t[r][m] = __ffma2_rn(x67, d[r][3], t[r][m]);
+          }
+        }
+      }
+#pragma unroll
+      for (int r = 0; r < kAwqRows; ++r) {
+        const float2 s2 = make_float2(sv[r], sv[r]);
+#pragma unroll
+        for (int m = 0; m < MT; ++m) acc[r][m] = __ffma2_rn(t[r][m], s2, acc[r][m]);
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[s]);  // this warp is done with the stage
+#pragma unroll
+    for (int r = 0; r < kAwqRows; ++r) {
+      const int n = n0 + r;
+      float res[MT];
+#pragma unroll
+      for (int m = 0; m < MT; ++m) {
+        res[m] = __fadd_rn(acc[r][m].x, acc[r][m].y);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) res[m] += __shfl_xor_sync(0xffffffffu, res[m], o);
+      }
+      if (lane == 0 && n < r1) {
+        const float bn = bias != nullptr ? __bfloat162float(bias[n]) : 0.0f;
+#pragma unroll
+        for (int m = 0; m < MT; ++m)
+          if (m < rows) Y[static_cast<int64_t>(m) * ldy + n] = __float2bfloat16_rn(__fadd_rn(res[m], bn));
+      }
+    }
+  }
+}
+
 }  // namespace svdq

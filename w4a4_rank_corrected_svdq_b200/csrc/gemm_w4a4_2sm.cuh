@@ -427,57 +427,53 @@ __device__ __forceinline__ bool epilogue_qkv_tile(uint32_t (&y0c)[16], uint32_t 
 // ------------------------------------------------------------------ MLP up-projection epilogue
 constexpr int kMlpRank = 32;  // the down projection's rank the fused epilogue supports
 
-// 32 columns of this lane's row given y as 16 packed bf16 pairs (overwritten
-// with h): h = bf16(GELU(y)) and its two NVFP4 blocks by the activation
-// quantiser's rule (S = e4m3(amax / fp32(6 g)), q = h * fp32(1 / fp32(dec(S) g)),
-// zero reciprocal for a zero or saturated scale): the 32 codes as four words
-// in w (two per block) and the two scale bytes in sc.
-__device__ __forceinline__ void mlp_gelu_quant32(uint32_t (&pk)[16], bool approximate, float g, float d,
-                                                 uint32_t (&w)[4], uint32_t& sc) {
-  float hf[32];
+// In place on this lane's staged row of 64 columns (rowp: its 128 bytes in the
+// 128-byte swizzle, sw = row % 8), holding y as bf16: h = bf16(GELU(y)),
+// written back, and its four NVFP4 blocks by the activation quantiser's rule
+// (S = e4m3(amax / fp32(6 g)), q = h * fp32(1 / fp32(dec(S) g)), zero
+// reciprocal for a zero or saturated scale): 32 code bytes stored for the down
+// projection and the row's scale word of the tiled layout (zero for padding
+// rows M <= row < m_pad). One block per iteration keeps the code compact.
+__device__ __forceinline__ void mlp_gelu_quant_row64(uint8_t* rowp, int sw, int x0, int row, int M, int N,
+                                                     const MlpPost& mp, float g, float d) {
+  uint32_t sc = 0;
+  const bool approximate = mp.approximate != 0;
+#pragma unroll 1
+  for (int blk = 0; blk < 4; ++blk) {
+    uint4* p0 = reinterpret_cast<uint4*>(rowp + (((2 * blk) ^ sw) << 4));
+    uint4* p1 = reinterpret_cast<uint4*>(rowp + (((2 * blk + 1) ^ sw) << 4));
+    const uint4 v0 = *p0, v1 = *p1;
+    uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+    if (approximate) {
 #pragma unroll
-  for (int p = 0; p < 16; ++p) {
-    const uint32_t hp = pack_bf16(gelu_f32(bf16_lo(pk[p]), approximate), gelu_f32(bf16_hi(pk[p]), approximate));
-    pk[p] = hp;
-    hf[2 * p] = bf16_lo(hp);
-    hf[2 * p + 1] = bf16_hi(hp);
-  }
-  sc = 0;
+      for (int i = 0; i < 8; ++i) w[i] = pack_bf16(gelu_tanh_f32(bf16_lo(w[i])), gelu_tanh_f32(bf16_hi(w[i])));
+    } else {
 #pragma unroll
-  for (int blk = 0; blk < 2; ++blk) {
+      for (int i = 0; i < 8; ++i) w[i] = pack_bf16(gelu_erf_f32(bf16_lo(w[i])), gelu_erf_f32(bf16_hi(w[i])));
+    }
+    *p0 = make_uint4(w[0], w[1], w[2], w[3]);
+    *p1 = make_uint4(w[4], w[5], w[6], w[7]);
     float am = 0.0f;
 #pragma unroll
-    for (int i = 0; i < 16; ++i) am = fmaxf(am, fabsf(hf[16 * blk + i]));
+    for (int i = 0; i < 8; ++i) am = fmaxf(am, fmaxf(fabsf(bf16_lo(w[i])), fabsf(bf16_hi(w[i]))));
     const uint32_t S = f32_to_e4m3(__fdiv_rn(am, d));
     const float sd = __fmul_rn(e4m3_to_f32(S), g);
     const float inv = (sd == 0.0f || S >= 0x7Fu) ? 0.0f : __frcp_rn(sd);
     float q0[8], q1[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      q0[i] = __fmul_rn(hf[16 * blk + i], inv);
-      q1[i] = __fmul_rn(hf[16 * blk + 8 + i], inv);
+    for (int i = 0; i < 4; ++i) {
+      q0[2 * i] = __fmul_rn(bf16_lo(w[i]), inv);
+      q0[2 * i + 1] = __fmul_rn(bf16_hi(w[i]), inv);
+      q1[2 * i] = __fmul_rn(bf16_lo(w[4 + i]), inv);
+      q1[2 * i + 1] = __fmul_rn(bf16_hi(w[4 + i]), inv);
     }
-    w[2 * blk] = f32x8_to_e2m1(q0);
-    w[2 * blk + 1] = f32x8_to_e2m1(q1);
+    if (row < M)
+      *reinterpret_cast<uint2*>(mp.codes + static_cast<int64_t>(row) * (N / 2) + x0 / 2 + 8 * blk) =
+          make_uint2(f32x8_to_e2m1(q0), f32x8_to_e2m1(q1));
     sc |= S << (8 * blk);
   }
-}
-
-// 64 columns x0 .. x0 + 63 of this lane's row (y in pa, pb; replaced by h):
-// GELU, NVFP4 codes (32 bytes) and the scale word (4 blocks) stored for the
-// down projection; padding rows (M <= row < m_pad) get zero scales.
-__device__ __forceinline__ void mlp_quantize64(uint32_t (&pa)[16], uint32_t (&pb)[16], int x0, int row, int M, int N,
-                                               const MlpPost& mp, float g, float d) {
-  uint32_t wa[4], wb[4], sa, sb;
-  mlp_gelu_quant32(pa, mp.approximate != 0, g, d, wa, sa);
-  mlp_gelu_quant32(pb, mp.approximate != 0, g, d, wb, sb);
-  if (row < M) {
-    uint4* c = reinterpret_cast<uint4*>(mp.codes + static_cast<int64_t>(row) * (N / 2) + x0 / 2);
-    c[0] = make_uint4(wa[0], wa[1], wa[2], wa[3]);
-    c[1] = make_uint4(wb[0], wb[1], wb[2], wb[3]);
-  }
   if (row < mp.m_pad)  // the four scale bytes of a row's 64 columns are one aligned word of the tiled layout
-    *reinterpret_cast<uint32_t*>(mp.scales + scale_offset(N, row, x0 / 16)) = row < M ? (sa | (sb << 16)) : 0u;
+    *reinterpret_cast<uint32_t*>(mp.scales + scale_offset(N, row, x0 / 16)) = row < M ? sc : 0u;
 }
 
 // 64 columns of packed bf16 pairs (pa, pb) of this lane's row into a 32-row x
@@ -868,16 +864,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<R, EPI>::kT
         const bool last = tile + 1 == t_end || (tile + 1) / num_nt != mt;
         const uint32_t ready = mapa_shared(smem_u32(&bars->chunk_ready[h]), 0);
         bool ok = true;
-#pragma unroll
-        for (int cc = 0; cc < 2 && ok; ++cc) {
-          uint32_t(&pa)[16] = cc == 0 ? pk0 : pk2;
-          uint32_t(&pb)[16] = cc == 0 ? pk1 : pk3;
-          mlp_quantize64(pa, pb, col0 + 64 * cc, row, M, N, mlp, g, d);
+#pragma unroll 1
+        for (int cc = 0; cc < 2; ++cc) {
           // this half's chunk buffer: its previous chunk's MMAs have read it
           if (!mbar_wait(&bars->chunk_free[h], cc ^ 1, abort)) { ok = false; break; }
           if (mlp.store_h && lane == 0) bulk_wait_read0();  // and so has the previous store of h
           __syncwarp();
-          stage_row64(stage, pa, pb, lane);
+          uint32_t ta[16], tb[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            ta[i] = cc == 0 ? pk0[i] : pk2[i];
+            tb[i] = cc == 0 ? pk1[i] : pk3[i];
+          }
+          stage_row64(stage, ta, tb, lane);  // y, then GELU and the quantisation in place
+          mlp_gelu_quant_row64(stage + lane * 128, lane & 7, col0 + 64 * cc, row, M, N, mlp, g, d);
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {

@@ -82,24 +82,37 @@ __device__ __forceinline__ float erfc_fast_nonneg(float z) {
   return t * __expf(__fmaf_rn(-z, z, p));
 }
 
-__device__ __forceinline__ float gelu_f32(float x, bool approximate) {
+// The far negative tail with the accurate library functions (rarely reached,
+// kept out of line so the fast paths stay compact).
+__device__ __noinline__ float gelu_tail(float x, bool approximate) {
   if (approximate) {
     const float u = __fmul_rn(0.7978845608028654f, __fmaf_rn(__fmul_rn(0.044715f, x), __fmul_rn(x, x), x));
-    if (u >= 0.0f) return __fdividef(x, 1.0f + __expf(-2.0f * u));
-    // the same function for u < 0 as x e^{2u} / (1 + e^{2u}): e^{2u} <= 1 never
-    // overflows
-    if (u > -40.0f) {
-      const float e = __expf(2.0f * u);
-      return __fdividef(x * e, 1.0f + e);
-    }
     const float e = expf(__fmul_rn(2.0f, u));
     return __fdiv_rn(__fmul_rn(x, e), __fadd_rn(1.0f, e));
   }
+  return __fmul_rn(__fmul_rn(0.5f, x), erfcf(__fmul_rn(x, -0.7071067811865476f)));
+}
+
+// tanh form; for u < 0 as x e^{2u} / (1 + e^{2u}) (e^{2u} <= 1 never overflows)
+__device__ __forceinline__ float gelu_tanh_f32(float x) {
+  const float u = __fmul_rn(0.7978845608028654f, __fmaf_rn(__fmul_rn(0.044715f, x), __fmul_rn(x, x), x));
+  if (u >= 0.0f) return __fdividef(x, 1.0f + __expf(-2.0f * u));
+  if (u <= -40.0f) return gelu_tail(x, true);
+  const float e = __expf(2.0f * u);
+  return __fdividef(x * e, 1.0f + e);
+}
+
+// erf form
+__device__ __forceinline__ float gelu_erf_f32(float x) {
   const float z = x * -0.7071067811865476f;
   const float az = fabsf(z);
-  if (az > 9.0f) return __fmul_rn(__fmul_rn(0.5f, x), erfcf(z));
+  if (az > 9.0f) return gelu_tail(x, false);
   const float e = erfc_fast_nonneg(az);
   return 0.5f * x * (z >= 0.0f ? e : 2.0f - e);
+}
+
+__device__ __forceinline__ float gelu_f32(float x, bool approximate) {
+  return approximate ? gelu_tanh_f32(x) : gelu_erf_f32(x);
 }
 
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }

@@ -13,6 +13,7 @@
 #include "../../include/svdq.h"
 #include "gemm_w4a4.cuh"
 #include "gemm_w4a4_2sm.cuh"
+#include "gemm_w4a4_splitk.cuh"
 #include "lowrank_svd.cuh"
 #include "pack_weight.cuh"
 #include "smooth.cuh"
@@ -426,6 +427,59 @@ svdq_status launch_gemm(int M, int N, int K, const void* a_codes, const void* a_
   return launch_status();
 }
 
+// K split of the few-row GEMM: the largest KS in {8, 4, 2} that divides the
+// K blocks and keeps one CTA per SM for every tile's cluster; 1 = no split.
+// SVDQ_GEMM_SPLITK=0 turns the split off (tests, benchmarks).
+int gemm_split(int M, int N, int K, int sm_count) {
+  const char* env = std::getenv("SVDQ_GEMM_SPLITK");
+  if (env != nullptr && std::strcmp(env, "0") == 0) return 1;
+  const int tiles = ((M + kBM - 1) / kBM) * (N / kBN);
+  const int nk = K / 256;
+  for (int ks = kSplitMaxKS; ks >= 2; ks /= 2)
+    if (nk % ks == 0 && tiles * ks <= sm_count) return ks;
+  return 1;
+}
+
+template <int R>
+svdq_status launch_gemm_splitk(int M, int N, int K, int ks, const void* a_codes, const void* a_scales,
+                               const void* xl1, const void* w_codes, const void* w_scales, const float* gscale,
+                               const void* l2s, const void* bias, void* Y, int64_t ldy, cudaStream_t stream) {
+  using C = SplitCfg<R>;
+  CUtensorMap tm_a, tm_b, tm_x, tm_l;
+  const uint64_t kb = static_cast<uint64_t>(K / 2);
+  if (!make_tmap_2d(&tm_a, a_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, kb, M, kb, kBKBytes, kBM,
+                    CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_tmap_2d(&tm_b, w_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, kb, N, kb, kBKBytes, kBN,
+                    CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_tmap_2d(&tm_x, xl1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, R, M, R * 2, C::kLrAtomCols, kBM,
+                    lr_swizzle(R)) ||
+      !make_tmap_2d(&tm_l, l2s, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, R, 2 * static_cast<uint64_t>(N), R * 2,
+                    C::kLrAtomCols, kBN, lr_swizzle(R)))
+    return SVDQ_ERR_CUDA;
+  auto kern = w4a4_gemm_splitk_kernel<R>;
+  static std::atomic<uint64_t> attr_done{0};
+  ensure_smem_attr(kern, C::kSmemBytes, attr_done);
+  const int tiles = ((M + kBM - 1) / kBM) * (N / kBN);
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = ks;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  cfg.blockDim = dim3(kSplitThreads, 1, 1);
+  cfg.gridDim = dim3(ks, tiles, 1);
+  cfg.dynamicSmemBytes = C::kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchKernelEx(&cfg, kern, tm_a, tm_b, tm_x, tm_l, static_cast<const uint8_t*>(a_scales),
+                     static_cast<const uint8_t*>(w_scales), gscale, static_cast<const __nv_bfloat16*>(bias),
+                     static_cast<__nv_bfloat16*>(Y), ldy, M, N, K);
+  return launch_status();
+}
+
 // CTA pairs the 2-SM GEMM launches: one per tile, at most one per two SMs.
 int gemm2_pairs(int M, int N, int sm_count) {
   const int tiles = ((M + k2TileM - 1) / k2TileM) * (N / k2TileN);
@@ -533,6 +587,18 @@ svdq_status gemm_dispatch(int M, int N, int K, int r, const void* a_codes, const
     }
   }
   if (post != nullptr) SVDQ_GEMM_CASES(launch_gemm, true)
+  // few rows: K split across a cluster when that fills more SMs (16-byte aligned bias)
+  const int ks = gemm_split(M, N, K, sms);
+  if (ks > 1 && (bias == nullptr || (reinterpret_cast<uintptr_t>(bias) & 15u) == 0)) {
+#define SVDQ_SPLIT_ARGS M, N, K, ks, a_codes, a_scales, xl1, w_codes, w_scales, gscale, l2s, bias, Y, ldy, st
+    switch (r) {
+      case 16: return launch_gemm_splitk<16>(SVDQ_SPLIT_ARGS);
+      case 32: return launch_gemm_splitk<32>(SVDQ_SPLIT_ARGS);
+      case 64: return launch_gemm_splitk<64>(SVDQ_SPLIT_ARGS);
+      default: return launch_gemm_splitk<128>(SVDQ_SPLIT_ARGS);
+    }
+#undef SVDQ_SPLIT_ARGS
+  }
   SVDQ_GEMM_CASES(launch_gemm, false)
 #undef SVDQ_GEMM_CASES
 #undef SVDQ_GEMM_ARGS
@@ -662,18 +728,34 @@ __global__ void __launch_bounds__(256) dynamic_scale_kernel(const float* __restr
   }
   const bool same = alpha_d == alpha;
   const float ratio = __fdiv_rn(alpha, alpha_d);
-  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+  // eight elements per step: total is a multiple of 16 (N r with r % 16 == 0)
+  const uint4* hi8 = reinterpret_cast<const uint4*>(l2s);
+  const uint4* lo8 = reinterpret_cast<const uint4*>(l2s + total);
+  uint4* ohi8 = reinterpret_cast<uint4*>(l2s_out);
+  uint4* olo8 = reinterpret_cast<uint4*>(l2s_out + total);
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total / 8;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const __nv_bfloat16 hi = l2s[i], lo = l2s[total + i];
+    const uint4 h = ldg_v4(hi8 + i), l = ldg_v4(lo8 + i);
     if (same) {
-      l2s_out[i] = hi;
-      l2s_out[total + i] = lo;
+      ohi8[i] = h;
+      olo8[i] = l;
       continue;
     }
-    const float v = __fmul_rn(__fadd_rn(__bfloat162float(hi), __bfloat162float(lo)), ratio);
-    const __nv_bfloat16 h2 = __float2bfloat16_rn(v);
-    l2s_out[i] = h2;
-    l2s_out[total + i] = __float2bfloat16_rn(__fsub_rn(v, __bfloat162float(h2)));
+    const uint32_t hw[4] = {h.x, h.y, h.z, h.w}, lw[4] = {l.x, l.y, l.z, l.w};
+    uint32_t oh[4], ol[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float v0 = __fmul_rn(__fadd_rn(__uint_as_float(hw[j] << 16), __uint_as_float(lw[j] << 16)), ratio);
+      const float v1 =
+          __fmul_rn(__fadd_rn(__uint_as_float(hw[j] & 0xFFFF0000u), __uint_as_float(lw[j] & 0xFFFF0000u)), ratio);
+      const __nv_bfloat162 hh = __floats2bfloat162_rn(v0, v1);
+      const float h0 = __low2float(hh), h1 = __high2float(hh);
+      const __nv_bfloat162 ll = __floats2bfloat162_rn(__fsub_rn(v0, h0), __fsub_rn(v1, h1));
+      oh[j] = *reinterpret_cast<const uint32_t*>(&hh);
+      ol[j] = *reinterpret_cast<const uint32_t*>(&ll);
+    }
+    ohi8[i] = make_uint4(oh[0], oh[1], oh[2], oh[3]);
+    olo8[i] = make_uint4(ol[0], ol[1], ol[2], ol[3]);
   }
 }
 
@@ -1257,7 +1339,7 @@ svdq_status svdq_linear_forward_dynamic(int M, int N, int K, int r, const void* 
   const int nparts = launch_act_amax(static_cast<const __nv_bfloat16*>(X), ldx, M, K, inv_smooth, nullptr, partial,
                                      di.sm_count, st);
   const int64_t total = static_cast<int64_t>(N) * r;
-  const int64_t sblocks = (total + 255) / 256 < 2 * di.sm_count ? (total + 255) / 256 : 2 * di.sm_count;
+  const int64_t sblocks = (total / 8 + 255) / 256 < 2 * di.sm_count ? (total / 8 + 255) / 256 : 2 * di.sm_count;
   {
     PdlLaunch pl(static_cast<int>(sblocks), 256, 0, st);
     cudaLaunchKernelEx(&pl.cfg, dynamic_scale_kernel, static_cast<const float*>(gscale),
@@ -1309,12 +1391,40 @@ svdq_status svdq_awq_pack(int N, int K, const void* W, const float* act_scale, v
 namespace svdq {
 namespace {
 constexpr int kAwqSmemCap = 96 * 1024;  // activation rows staged per CTA: at most 96 KB
+constexpr int kAwqRingSmemCap = 226 * 1024;  // the ring variant: staged activations + stage ring
 
 template <int MT>
 svdq_status launch_awq_gemv(int M, int N, int K, const __nv_bfloat16* X, int64_t ldx, const uint8_t* codes,
                             const __nv_bfloat16* scales, const uint8_t* zeros, const float* inv_act,
                             const __nv_bfloat16* bias, __nv_bfloat16* Y, int64_t ldy, int sm_count,
                             cudaStream_t st) {
+  // The bulk-copy ring variant: K % 1024 == 0 (every row count's codes, scales
+  // and zero points are 16-byte multiples), 16-byte aligned scales and zero
+  // points, and room for at least two stages next to the staged activations.
+  // SVDQ_AWQ_KERNEL=direct|ring overrides the choice where both apply (tests).
+  {
+    const char* env = std::getenv("SVDQ_AWQ_KERNEL");
+    const bool want_ring = env == nullptr || std::strcmp(env, "direct") != 0;
+    const int stage = awq_ring_stage_bytes(K);
+    const int room = kAwqRingSmemCap - MT * K * 4 - 2 * kAwqRingMaxStages * 8 - 16;
+    int stages = room > 0 ? room / stage : 0;
+    if (stages > kAwqRingMaxStages) stages = kAwqRingMaxStages;
+    if (want_ring && K % 1024 == 0 && aligned16(scales) && aligned16(zeros) && stages >= 2) {
+      const int smem_r = MT * K * 4 + stages * stage + 2 * kAwqRingMaxStages * 8 + 16;
+      static std::atomic<uint64_t> attr_r{0};
+      ensure_smem_attr(awq_gemv_ring_kernel<MT>, kAwqRingSmemCap, attr_r);
+      int blocks = (N + kAwqRingRows - 1) / kAwqRingRows;
+      if (blocks > sm_count) blocks = sm_count;  // one CTA per SM, each a contiguous run of rows
+      for (int m0 = 0; m0 < M; m0 += MT) {
+        awq_gemv_ring_kernel<MT><<<blocks, kAwqRingThreads, smem_r, st>>>(
+            M - m0, N, K, X + static_cast<int64_t>(m0) * ldx, ldx, codes, scales, zeros, inv_act, bias,
+            Y + static_cast<int64_t>(m0) * ldy, ldy, stages);
+        const svdq_status s = launch_status();
+        if (s != SVDQ_OK) return s;
+      }
+      return SVDQ_OK;
+    }
+  }
   const int smem = MT * K * 4;
   static std::atomic<uint64_t> attr_done{0};  // set once to the cap, which covers every K accepted
   ensure_smem_attr(awq_gemv_kernel<MT>, kAwqSmemCap, attr_done);
