@@ -184,16 +184,15 @@ def test_pack_weight_bitexact(lib, N, K, r):
 
 
 # ------------------------------------------------------------------ full layer
-@pytest.mark.parametrize("splitk", ["auto", "0"])
+@pytest.mark.parametrize("splitk", ["0", "1"])
 @pytest.mark.parametrize("M,K,N,r,bias", [(256, 1024, 1024, 32, True), (1, 256, 128, 16, True),
                                           (129, 512, 384, 64, False), (300, 768, 256, 128, True),
                                           (517, 1280, 640, 32, True), (128, 4096, 1024, 16, True),
                                           (200, 2048, 768, 128, True), (64, 512, 2048, 32, False)])
 def test_linear_forward_parity(lib, monkeypatch, splitk, M, K, N, r, bias):
-    """The layer through the library's own kernel choice; with few rows the GEMM
-    splits K across a thread-block cluster (SVDQ_GEMM_SPLITK=0: one CTA per tile)."""
-    if splitk == "0":
-        monkeypatch.setenv("SVDQ_GEMM_SPLITK", "0")
+    """The layer through the library's own kernel choice, and with few rows also
+    with K split across a thread-block cluster (SVDQ_GEMM_SPLITK=1)."""
+    monkeypatch.setenv("SVDQ_GEMM_SPLITK", splitk)
     X, W, b, L1, L2 = _layer(M, K, N, r, bias=bias)
     g_x = osv.act_global_scale(X)
     pw = lib.svdq_pack_weight(W.cuda(), _to_dev(L1), _to_dev(L2), float(g_x))

@@ -133,16 +133,31 @@ __global__ void __launch_bounds__(kAwqThreads) awq_gemv_kernel(int M, int N, int
     for (int r = 0; r < kAwqRows; ++r)
 #pragma unroll
       for (int m = 0; m < MT; ++m) acc[r][m] = make_float2(0.0f, 0.0f);
+    // chunk loads are software-pipelined: the next chunk's codes, scales and zero
+    // points are requested before the current chunk's arithmetic
+    uint4 vn[kAwqRows];
+    __nv_bfloat16 sn[kAwqRows];
+    uint8_t zn[kAwqRows];
+    auto fetch = [&](int c) {
+#pragma unroll
+      for (int r = 0; r < kAwqRows; ++r) {
+        const int n = n0 + r < N ? n0 + r : N - 1;  // rows past N repeat the last one and are not stored
+        vn[r] = ldg_nc_v4(codes + static_cast<int64_t>(n) * (K / 2) + 16 * c);
+        sn[r] = scales[static_cast<int64_t>(n) * G + (c >> 1)];
+        zn[r] = zeros[static_cast<int64_t>(n) * G + (c >> 1)];
+      }
+    };
+    if (lane < C) fetch(lane);
     for (int c = lane; c < C; c += 32) {
       uint4 v[kAwqRows];
       float sv[kAwqRows], zf[kAwqRows];
 #pragma unroll
       for (int r = 0; r < kAwqRows; ++r) {
-        const int n = n0 + r < N ? n0 + r : N - 1;  // rows past N repeat the last one and are not stored
-        v[r] = ldg_nc_v4(codes + static_cast<int64_t>(n) * (K / 2) + 16 * c);
-        sv[r] = __bfloat162float(scales[static_cast<int64_t>(n) * G + (c >> 1)]);
-        zf[r] = __fadd_rn(8388608.0f, static_cast<float>(zeros[static_cast<int64_t>(n) * G + (c >> 1)]));
+        v[r] = vn[r];
+        sv[r] = __bfloat162float(sn[r]);
+        zf[r] = __fadd_rn(8388608.0f, static_cast<float>(zn[r]));
       }
+      if (c + 32 < C) fetch(c + 32);
       const int sw = c & 7;
       float2 t[kAwqRows][MT];
 #pragma unroll

@@ -444,13 +444,24 @@ __device__ __forceinline__ void mlp_gelu_quant_row64(uint8_t* rowp, int sw, int 
     uint4* p1 = reinterpret_cast<uint4*>(rowp + (((2 * blk + 1) ^ sw) << 4));
     const uint4 v0 = *p0, v1 = *p1;
     uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-    if (approximate) {
+    // branch-free fast paths for all 16 values (independent: full ILP), then the
+    // rare far-tail values recomputed exactly
+    float hv[16];
+    bool tail[16];
+    bool any_tail = false;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) w[i] = pack_bf16(gelu_tanh_f32(bf16_lo(w[i])), gelu_tanh_f32(bf16_hi(w[i])));
-    } else {
-#pragma unroll
-      for (int i = 0; i < 8; ++i) w[i] = pack_bf16(gelu_erf_f32(bf16_lo(w[i])), gelu_erf_f32(bf16_hi(w[i])));
+    for (int i = 0; i < 16; ++i) {
+      const float y = (i & 1) ? bf16_hi(w[i >> 1]) : bf16_lo(w[i >> 1]);
+      hv[i] = approximate ? gelu_tanh_fast(y, tail[i]) : gelu_erf_fast(y, tail[i]);
+      any_tail |= tail[i];
     }
+    if (any_tail) {
+#pragma unroll
+      for (int i = 0; i < 16; ++i)
+        if (tail[i]) hv[i] = gelu_tail((i & 1) ? bf16_hi(w[i >> 1]) : bf16_lo(w[i >> 1]), approximate);
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) w[i] = pack_bf16(hv[2 * i], hv[2 * i + 1]);
     *p0 = make_uint4(w[0], w[1], w[2], w[3]);
     *p1 = make_uint4(w[4], w[5], w[6], w[7]);
     float am = 0.0f;

@@ -93,22 +93,35 @@ __device__ __noinline__ float gelu_tail(float x, bool approximate) {
   return __fmul_rn(__fmul_rn(0.5f, x), erfcf(__fmul_rn(x, -0.7071067811865476f)));
 }
 
-// tanh form; for u < 0 as x e^{2u} / (1 + e^{2u}) (e^{2u} <= 1 never overflows)
-__device__ __forceinline__ float gelu_tanh_f32(float x) {
+// tanh form, x sigma(2u) with the logistic sigma evaluated as 1 / (1 + e^{-t})
+// for t >= 0 and e^{t} / (1 + e^{t}) for t < 0 (e^{-|t|} <= 1 never
+// overflows), branch-free; *tail is set where the result may fall below the
+// normal fp32 range (u <= -40), for which gelu_tail recomputes it.
+__device__ __forceinline__ float gelu_tanh_fast(float x, bool& tail) {
   const float u = __fmul_rn(0.7978845608028654f, __fmaf_rn(__fmul_rn(0.044715f, x), __fmul_rn(x, x), x));
-  if (u >= 0.0f) return __fdividef(x, 1.0f + __expf(-2.0f * u));
-  if (u <= -40.0f) return gelu_tail(x, true);
-  const float e = __expf(2.0f * u);
-  return __fdividef(x * e, 1.0f + e);
+  const float e = __expf(-2.0f * fabsf(u));
+  tail = u <= -40.0f;
+  return __fdividef(u >= 0.0f ? x : x * e, 1.0f + e);
 }
 
-// erf form
-__device__ __forceinline__ float gelu_erf_f32(float x) {
+// erf form, x erfc(-x / sqrt 2) / 2, branch-free; *tail where |z| > 9.
+__device__ __forceinline__ float gelu_erf_fast(float x, bool& tail) {
   const float z = x * -0.7071067811865476f;
   const float az = fabsf(z);
-  if (az > 9.0f) return gelu_tail(x, false);
-  const float e = erfc_fast_nonneg(az);
+  const float e = erfc_fast_nonneg(fminf(az, 9.0f));
+  tail = az > 9.0f;
   return 0.5f * x * (z >= 0.0f ? e : 2.0f - e);
+}
+
+__device__ __forceinline__ float gelu_tanh_f32(float x) {
+  bool tail;
+  const float h = gelu_tanh_fast(x, tail);
+  return tail ? gelu_tail(x, true) : h;
+}
+__device__ __forceinline__ float gelu_erf_f32(float x) {
+  bool tail;
+  const float h = gelu_erf_fast(x, tail);
+  return tail ? gelu_tail(x, false) : h;
 }
 
 __device__ __forceinline__ float gelu_f32(float x, bool approximate) {

@@ -429,10 +429,12 @@ svdq_status launch_gemm(int M, int N, int K, const void* a_codes, const void* a_
 
 // K split of the few-row GEMM: the largest KS in {8, 4, 2} that divides the
 // K blocks and keeps one CTA per SM for every tile's cluster; 1 = no split.
-// SVDQ_GEMM_SPLITK=0 turns the split off (tests, benchmarks).
+// Opt-in (SVDQ_GEMM_SPLITK=1): on B200 it measured slower than one CTA per
+// tile for the few-row layers (the cluster exchange costs more than the split
+// saves at these sizes).
 int gemm_split(int M, int N, int K, int sm_count) {
   const char* env = std::getenv("SVDQ_GEMM_SPLITK");
-  if (env != nullptr && std::strcmp(env, "0") == 0) return 1;
+  if (env == nullptr || std::strcmp(env, "1") != 0) return 1;
   const int tiles = ((M + kBM - 1) / kBM) * (N / kBN);
   const int nk = K / 256;
   for (int ks = kSplitMaxKS; ks >= 2; ks /= 2)
@@ -1404,12 +1406,15 @@ svdq_status launch_awq_gemv(int M, int N, int K, const __nv_bfloat16* X, int64_t
   // SVDQ_AWQ_KERNEL=direct|ring overrides the choice where both apply (tests).
   {
     const char* env = std::getenv("SVDQ_AWQ_KERNEL");
-    const bool want_ring = env == nullptr || std::strcmp(env, "direct") != 0;
     const int stage = awq_ring_stage_bytes(K);
     const int room = kAwqRingSmemCap - MT * K * 4 - 2 * kAwqRingMaxStages * 8 - 16;
     int stages = room > 0 ? room / stage : 0;
     if (stages > kAwqRingMaxStages) stages = kAwqRingMaxStages;
-    if (want_ring && K % 1024 == 0 && aligned16(scales) && aligned16(zeros) && stages >= 2) {
+    // by default from four activation rows on: with one or two rows the direct
+    // kernel (two CTAs per SM) measured faster on B200
+    const bool ring_default = MT >= 4;
+    const bool use_ring = env == nullptr ? ring_default : std::strcmp(env, "ring") == 0;
+    if (use_ring && K % 1024 == 0 && aligned16(scales) && aligned16(zeros) && stages >= 2) {
       const int smem_r = MT * K * 4 + stages * stage + 2 * kAwqRingMaxStages * 8 + 16;
       static std::atomic<uint64_t> attr_r{0};
       ensure_smem_attr(awq_gemv_ring_kernel<MT>, kAwqRingSmemCap, attr_r);
