@@ -178,7 +178,10 @@ struct Gemm2Cfg {
   static constexpr int kL1dOff = kXchgOff + kXchgBytes;
   static constexpr int kL1dChunk = 16 * 128;
   static constexpr int kL1dBytes = MLP ? 2 * 4 * kL1dChunk : 0;
-  static constexpr int kBarOff = kL1dOff + kL1dBytes;
+  // MLP: the 128 reciprocals 1 / fp32(dec(S) g_h) of every E4M3 scale code
+  static constexpr int kInvOff = kL1dOff + kL1dBytes;
+  static constexpr int kInvBytes = MLP ? 512 : 0;
+  static constexpr int kBarOff = kInvOff + kInvBytes;
   static constexpr int kSmemBytes = kBarOff + 512 + 1024;
 };
 
@@ -430,12 +433,13 @@ constexpr int kMlpRank = 32;  // the down projection's rank the fused epilogue s
 // In place on this lane's staged row of 64 columns (rowp: its 128 bytes in the
 // 128-byte swizzle, sw = row % 8), holding y as bf16: h = bf16(GELU(y)),
 // written back, and its four NVFP4 blocks by the activation quantiser's rule
-// (S = e4m3(amax / fp32(6 g)), q = h * fp32(1 / fp32(dec(S) g)), zero
-// reciprocal for a zero or saturated scale): 32 code bytes stored for the down
-// projection and the row's scale word of the tiled layout (zero for padding
-// rows M <= row < m_pad). One block per iteration keeps the code compact.
+// (S = e4m3(amax / fp32(6 g)), q = h * fp32(1 / fp32(dec(S) g)), with the
+// reciprocal from inv_tab, zero for a zero or saturated scale): 32 code bytes
+// stored for the down projection and the row's scale word of the tiled layout
+// (zero for padding rows M <= row < m_pad). One block per iteration keeps the
+// code compact; within a block the values are processed as pairs.
 __device__ __forceinline__ void mlp_gelu_quant_row64(uint8_t* rowp, int sw, int x0, int row, int M, int N,
-                                                     const MlpPost& mp, float g, float d) {
+                                                     const MlpPost& mp, float d, const float* inv_tab) {
   uint32_t sc = 0;
   const bool approximate = mp.approximate != 0;
 #pragma unroll 1
@@ -444,39 +448,34 @@ __device__ __forceinline__ void mlp_gelu_quant_row64(uint8_t* rowp, int sw, int 
     uint4* p1 = reinterpret_cast<uint4*>(rowp + (((2 * blk + 1) ^ sw) << 4));
     const uint4 v0 = *p0, v1 = *p1;
     uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-    // branch-free fast paths for all 16 values (independent: full ILP), then the
-    // rare far-tail values recomputed exactly
-    float hv[16];
-    bool tail[16];
-    bool any_tail = false;
+    // branch-free GELU of all 16 values (8 independent pairs)
+    float2 hv[8];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const float y = (i & 1) ? bf16_hi(w[i >> 1]) : bf16_lo(w[i >> 1]);
-      hv[i] = approximate ? gelu_tanh_fast(y, tail[i]) : gelu_erf_fast(y, tail[i]);
-      any_tail |= tail[i];
+    for (int i = 0; i < 8; ++i) {
+      const float2 y = make_float2(bf16_lo(w[i]), bf16_hi(w[i]));
+      hv[i] = approximate ? gelu_tanh_pair(y) : gelu_erf_pair(y);
     }
-    if (any_tail) {
+    __nv_bfloat162 am2 = __float2bfloat162_rn(0.0f);
 #pragma unroll
-      for (int i = 0; i < 16; ++i)
-        if (tail[i]) hv[i] = gelu_tail((i & 1) ? bf16_hi(w[i >> 1]) : bf16_lo(w[i >> 1]), approximate);
+    for (int i = 0; i < 8; ++i) {
+      w[i] = pack_bf16(hv[i].x, hv[i].y);
+      const uint32_t ab = w[i] & 0x7FFF7FFFu;  // |h| of both halves, exact
+      am2 = __hmax2(am2, *reinterpret_cast<const __nv_bfloat162*>(&ab));
     }
-#pragma unroll
-    for (int i = 0; i < 8; ++i) w[i] = pack_bf16(hv[2 * i], hv[2 * i + 1]);
     *p0 = make_uint4(w[0], w[1], w[2], w[3]);
     *p1 = make_uint4(w[4], w[5], w[6], w[7]);
-    float am = 0.0f;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) am = fmaxf(am, fmaxf(fabsf(bf16_lo(w[i])), fabsf(bf16_hi(w[i]))));
+    const float am = fmaxf(__low2float(am2), __high2float(am2));
     const uint32_t S = f32_to_e4m3(__fdiv_rn(am, d));
-    const float sd = __fmul_rn(e4m3_to_f32(S), g);
-    const float inv = (sd == 0.0f || S >= 0x7Fu) ? 0.0f : __frcp_rn(sd);
+    const float2 inv = f2(inv_tab[S]);
     float q0[8], q1[8];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      q0[2 * i] = __fmul_rn(bf16_lo(w[i]), inv);
-      q0[2 * i + 1] = __fmul_rn(bf16_hi(w[i]), inv);
-      q1[2 * i] = __fmul_rn(bf16_lo(w[4 + i]), inv);
-      q1[2 * i + 1] = __fmul_rn(bf16_hi(w[4 + i]), inv);
+      const float2 a = __fmul2_rn(make_float2(bf16_lo(w[i]), bf16_hi(w[i])), inv);
+      const float2 c = __fmul2_rn(make_float2(bf16_lo(w[4 + i]), bf16_hi(w[4 + i])), inv);
+      q0[2 * i] = a.x;
+      q0[2 * i + 1] = a.y;
+      q1[2 * i] = c.x;
+      q1[2 * i + 1] = c.y;
     }
     if (row < M)
       *reinterpret_cast<uint2*>(mp.codes + static_cast<int64_t>(row) * (N / 2) + x0 / 2 + 8 * blk) =
@@ -618,6 +617,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<R, EPI>::kT
   // Everything above overlaps the previous kernel of the stream (programmatic
   // dependent launch); nothing global is read or written before this wait.
   pdl_wait();
+  if constexpr (C::MLP) {
+    // reciprocal of every possible block decode scale of h (dec(S) g_h takes at
+    // most 127 finite values); the epilogue warps read it after their first
+    // acc_full wait, which follows this CTA-wide barrier
+    float* inv_tab = reinterpret_cast<float*>(smem + C::kInvOff);
+    if (threadIdx.x < 128) {
+      const float sd = __fmul_rn(e4m3_to_f32(threadIdx.x), *mlp.g_h);
+      inv_tab[threadIdx.x] = (sd == 0.0f || threadIdx.x >= 0x7Fu) ? 0.0f : __frcp_rn(sd);
+    }
+    __syncthreads();
+  }
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer (both CTAs)
@@ -888,7 +898,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<R, EPI>::kT
             tb[i] = cc == 0 ? pk1[i] : pk3[i];
           }
           stage_row64(stage, ta, tb, lane);  // y, then GELU and the quantisation in place
-          mlp_gelu_quant_row64(stage + lane * 128, lane & 7, col0 + 64 * cc, row, M, N, mlp, g, d);
+          mlp_gelu_quant_row64(stage + lane * 128, lane & 7, col0 + 64 * cc, row, M, N, mlp, d,
+                               reinterpret_cast<const float*>(smem + C::kInvOff));
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {

@@ -56,76 +56,79 @@ struct MlpPost {
 //
 // h is rounded to bf16 (8 significant bits), so a relative error far below
 // 2^-10 is enough for the result to lie within one bf16 step of the correctly
-// rounded value. The fast paths below stay far inside that:
+// rounded value. The paths below stay far inside that:
 //  * erfc(z), z >= 0, by the Chebyshev fit of Press, Teukolsky, Vetterling and
 //    Flannery (Numerical Recipes in C, 2nd ed., section 6.2, erfcc): with
 //    t = 1 / (1 + z/2), erfc(z) = t exp(-z^2 + P(t)), P of degree 9, fractional
 //    error below 1.2e-7 for every z >= 0; erfc(-z) = 2 - erfc(z);
-//  * exponentials by the hardware exp2 (__expf, relative error ~2^-21),
-//    reciprocals by __fdividef.
-// Where a result would fall below the normal fp32 range (|z| > 9 for erfc,
-// 2u < -80 in the tanh form) the accurate library functions take over, so the
-// far negative tail keeps its tiny values (subnormals included) instead of
-// flushing them to zero.
-__device__ __forceinline__ float erfc_fast_nonneg(float z) {
-  const float t = __fdividef(1.0f, __fmaf_rn(0.5f, z, 1.0f));
-  float p = 0.17087277f;
-  p = __fmaf_rn(p, t, -0.82215223f);
-  p = __fmaf_rn(p, t, 1.48851587f);
-  p = __fmaf_rn(p, t, -1.13520398f);
-  p = __fmaf_rn(p, t, 0.27886807f);
-  p = __fmaf_rn(p, t, -0.18628806f);
-  p = __fmaf_rn(p, t, 0.09678418f);
-  p = __fmaf_rn(p, t, 0.37409196f);
-  p = __fmaf_rn(p, t, 1.00002368f);
-  p = __fmaf_rn(p, t, -1.26551223f);
-  return t * __expf(__fmaf_rn(-z, z, p));
+//  * exponentials by the hardware exp2 (ex2.approx, relative error ~2^-22),
+//    reciprocals by rcp.approx.
+// The far negative tail keeps its tiny values (subnormals included): the
+// exponential is taken as 2^(e + 64), which stays a normal number for every
+// exponent e >= -190, and the product is scaled by 2^-64 (and 1/2) last, so
+// a result below the normal range is rounded once, by that multiplication.
+// Where e < -190 the true result is below 2^-180 in magnitude, rounds to zero
+// in fp32, and the flushed exponential gives that zero. Both forms are
+// branch-free and work on a pair of values (packed f32x2 arithmetic for the
+// polynomial and products; the hardware exp2 and reciprocal per lane).
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float rcp_approx(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float2 f2(float a) { return make_float2(a, a); }
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kTwoPowM64 = 0x1p-64f;
+constexpr float kTwoPowM65 = 0x1p-65f;
+
+// erf form: z = -x / sqrt 2, a = |z|, E = 2^64 erfc(a); x <= 0 (z >= 0):
+// (x E) 2^-65; x > 0: (x/2) (2 - E 2^-64). a is capped at 16, where erfc is
+// below 2^-370 (the product rounds to zero either way); the cap keeps a huge
+// |x| from turning a^2 into inf.
+__device__ __forceinline__ float2 gelu_erf_pair(float2 x) {
+  const float2 z = __fmul2_rn(x, f2(-0.7071067811865476f));
+  const float2 a = make_float2(fminf(fabsf(z.x), 16.0f), fminf(fabsf(z.y), 16.0f));
+  const float2 d = __ffma2_rn(a, f2(0.5f), f2(1.0f));
+  const float2 t = make_float2(rcp_approx(d.x), rcp_approx(d.y));
+  float2 p = f2(0.17087277f);
+  p = __ffma2_rn(p, t, f2(-0.82215223f));
+  p = __ffma2_rn(p, t, f2(1.48851587f));
+  p = __ffma2_rn(p, t, f2(-1.13520398f));
+  p = __ffma2_rn(p, t, f2(0.27886807f));
+  p = __ffma2_rn(p, t, f2(-0.18628806f));
+  p = __ffma2_rn(p, t, f2(0.09678418f));
+  p = __ffma2_rn(p, t, f2(0.37409196f));
+  p = __ffma2_rn(p, t, f2(1.00002368f));
+  p = __ffma2_rn(p, t, f2(-1.26551223f));
+  // log2 of erfc(a) 2^64
+  const float2 arg = __ffma2_rn(__ffma2_rn(make_float2(-a.x, -a.y), a, p), f2(kLog2e), f2(64.0f));
+  const float2 E = __fmul2_rn(t, make_float2(ex2_approx(arg.x), ex2_approx(arg.y)));
+  const float2 c = __ffma2_rn(E, f2(-kTwoPowM64), f2(2.0f));
+  const float2 phi = make_float2(z.x >= 0.0f ? E.x : c.x, z.y >= 0.0f ? E.y : c.y);
+  const float2 sc = make_float2(z.x >= 0.0f ? kTwoPowM65 : 0.5f, z.y >= 0.0f ? kTwoPowM65 : 0.5f);
+  return __fmul2_rn(__fmul2_rn(x, phi), sc);
 }
 
-// The far negative tail with the accurate library functions (rarely reached,
-// kept out of line so the fast paths stay compact).
-__device__ __noinline__ float gelu_tail(float x, bool approximate) {
-  if (approximate) {
-    const float u = __fmul_rn(0.7978845608028654f, __fmaf_rn(__fmul_rn(0.044715f, x), __fmul_rn(x, x), x));
-    const float e = expf(__fmul_rn(2.0f, u));
-    return __fdiv_rn(__fmul_rn(x, e), __fadd_rn(1.0f, e));
-  }
-  return __fmul_rn(__fmul_rn(0.5f, x), erfcf(__fmul_rn(x, -0.7071067811865476f)));
-}
-
-// tanh form, x sigma(2u) with the logistic sigma evaluated as 1 / (1 + e^{-t})
-// for t >= 0 and e^{t} / (1 + e^{t}) for t < 0 (e^{-|t|} <= 1 never
-// overflows), branch-free; *tail is set where the result may fall below the
-// normal fp32 range (u <= -40), for which gelu_tail recomputes it.
-__device__ __forceinline__ float gelu_tanh_fast(float x, bool& tail) {
-  const float u = __fmul_rn(0.7978845608028654f, __fmaf_rn(__fmul_rn(0.044715f, x), __fmul_rn(x, x), x));
-  const float e = __expf(-2.0f * fabsf(u));
-  tail = u <= -40.0f;
-  return __fdividef(u >= 0.0f ? x : x * e, 1.0f + e);
-}
-
-// erf form, x erfc(-x / sqrt 2) / 2, branch-free; *tail where |z| > 9.
-__device__ __forceinline__ float gelu_erf_fast(float x, bool& tail) {
-  const float z = x * -0.7071067811865476f;
-  const float az = fabsf(z);
-  const float e = erfc_fast_nonneg(fminf(az, 9.0f));
-  tail = az > 9.0f;
-  return 0.5f * x * (z >= 0.0f ? e : 2.0f - e);
-}
-
-__device__ __forceinline__ float gelu_tanh_f32(float x) {
-  bool tail;
-  const float h = gelu_tanh_fast(x, tail);
-  return tail ? gelu_tail(x, true) : h;
-}
-__device__ __forceinline__ float gelu_erf_f32(float x) {
-  bool tail;
-  const float h = gelu_erf_fast(x, tail);
-  return tail ? gelu_tail(x, false) : h;
-}
-
-__device__ __forceinline__ float gelu_f32(float x, bool approximate) {
-  return approximate ? gelu_tanh_f32(x) : gelu_erf_f32(x);
+// tanh form: x sigma(2u) with sigma(s) = 1 / (1 + e^{-s}) for s >= 0 and
+// e^{s} / (1 + e^{s}) for s < 0 (e^{-|s|} <= 1 never overflows). With
+// E = 2^64 e^{-2|u|}: u >= 0: x / (1 + E 2^-64); u < 0: (x E / (1 + E 2^-64)) 2^-64.
+// |u| is capped at 128, beyond which e^{-2|u|} < 2^-369.
+__device__ __forceinline__ float2 gelu_tanh_pair(float2 x) {
+  const float2 x2 = __fmul2_rn(x, x);
+  const float2 u = __fmul2_rn(f2(0.7978845608028654f), __ffma2_rn(__fmul2_rn(f2(0.044715f), x), x2, x));
+  const float2 au = make_float2(fminf(fabsf(u.x), 128.0f), fminf(fabsf(u.y), 128.0f));
+  const float2 arg = __ffma2_rn(au, f2(-2.0f * kLog2e), f2(64.0f));
+  const float2 E = make_float2(ex2_approx(arg.x), ex2_approx(arg.y));
+  const float2 den = __ffma2_rn(E, f2(kTwoPowM64), f2(1.0f));
+  const float2 num = make_float2(u.x >= 0.0f ? x.x : x.x * E.x, u.y >= 0.0f ? x.y : x.y * E.y);
+  const float2 sc = make_float2(u.x >= 0.0f ? 1.0f : kTwoPowM64, u.y >= 0.0f ? 1.0f : kTwoPowM64);
+  return __fmul2_rn(__fmul2_rn(num, make_float2(rcp_approx(den.x), rcp_approx(den.y))), sc);
 }
 
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
