@@ -612,10 +612,11 @@ def run_ours(args, spec):
     variants["awq_w4a16_modulation_3072x18432"] = awq_out
 
     # MLP pair (the DiT feed-forward shapes, 3072 -> 12288 -> 3072, M = 4608):
-    # the fused up projection (GELU and the down projection's activation
-    # quantisation in its GEMM epilogue) plus the down GEMM, against the
-    # unfused pair without a GELU pass (the up projection writing y in bf16,
-    # the down projection reading it back), a lower bound of the unfused cost.
+    # the fused up projection (GELU, erf form and tanh form, and the down
+    # projection's activation quantisation in its GEMM epilogue) plus the down
+    # GEMM, against the unfused pair without a GELU pass (the up projection
+    # writing y in bf16, the down projection reading it back), a lower bound
+    # of the unfused cost.
     try:
         up_s, dn_s = workloads.WORKLOADS[3].layers[:2]
         Xu, Wu, bu = workloads.make_layer(up_s)
@@ -642,8 +643,8 @@ def run_ours(args, spec):
         ws_d = torch.empty(svdq.svdq_forward_workspace_size(Mu, Fu, dn_s.r), dtype=torch.uint8, device=dev)
         Yd = torch.empty((Mu, dn_s.N), dtype=torch.bfloat16, device=dev)
 
-        def fused(i):
-            svdq.svdq_mlp_up_forward(Xud, pw_u, bud, g_h, pw_d.l1t, out=qa_h, workspace=ws_m)
+        def fused(i, approximate=False):
+            svdq.svdq_mlp_up_forward(Xud, pw_u, bud, g_h, pw_d.l1t, approximate, out=qa_h, workspace=ws_m)
             svdq.svdq_w4a4_gemm(qa_h, pw_d, bdd, out=Yd)
 
         def unfused(i):
@@ -651,11 +652,13 @@ def run_ours(args, spec):
             svdq.svdq_linear_forward(Hd, pw_d, bdd, out=Yd, workspace=ws_d)
 
         fused_ms, unfused_ms = timed(fused), timed(unfused)
+        fused_tanh_ms = timed(lambda i: fused(i, True))
         if svdq.svdq_read_device_error() != 0:
             raise RuntimeError("device error during the MLP pair timing")
         pair_flops = _flops(Mu, Fu, up_s.K, up_s.r) + _flops(Mu, dn_s.N, Fu, dn_s.r)
         variants["mlp_pair_4608x3072x12288_r32"] = {
-            "fused_ms_per_step": fused_ms, "unfused_without_gelu_ms_per_step": unfused_ms,
+            "fused_ms_per_step": fused_ms, "fused_tanh_gelu_ms_per_step": fused_tanh_ms,
+            "unfused_without_gelu_ms_per_step": unfused_ms,
             "fused_tflops": pair_flops / (fused_ms * 1e-3) / 1e12,
             "note": "one input set; the per-step working set (about 150 MB) exceeds L2"}
         del pw_u, pw_d, qa_h, ws_m, ws_u, ws_d, Hd, Yd
