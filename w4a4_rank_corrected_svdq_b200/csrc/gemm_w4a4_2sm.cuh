@@ -434,14 +434,17 @@ constexpr int kMlpRank = 32;  // the down projection's rank the fused epilogue s
 // 128-byte swizzle, sw = row % 8), holding y as bf16: h = bf16(GELU(y)),
 // written back, and its four NVFP4 blocks by the activation quantiser's rule
 // (S = e4m3(amax / fp32(6 g)), q = h * fp32(1 / fp32(dec(S) g)), with the
-// reciprocal from inv_tab, zero for a zero or saturated scale): 32 code bytes
-// stored for the down projection and the row's scale word of the tiled layout
-// (zero for padding rows M <= row < m_pad). One block per iteration keeps the
-// code compact; within a block the values are processed as pairs.
-__device__ __forceinline__ void mlp_gelu_quant_row64(uint8_t* rowp, int sw, int x0, int row, int M, int N,
-                                                     const MlpPost& mp, float d, const float* inv_tab) {
-  uint32_t sc = 0;
-  const bool approximate = mp.approximate != 0;
+// reciprocal from inv_tab, zero for a zero or saturated scale): the 32 code
+// bytes into cw (block b in bytes 8b .. 8b + 7) and the four scale bytes into
+// sc (block b in byte b), for mlp_store_row64 to write once the staged chunk
+// has been handed to the MMA (a release arrive waits for this thread's earlier
+// global stores). One block per iteration keeps the code compact (the codes
+// shift through cw so it stays in registers); within a block the values are
+// processed as pairs.
+__device__ __forceinline__ void mlp_gelu_quant_row64(uint8_t* rowp, int sw, bool approximate, float d,
+                                                     const float* inv_tab, uint4 (&cw)[2], uint32_t& sc) {
+  uint2 c0 = make_uint2(0u, 0u), c1 = c0, c2 = c0, c3 = c0;
+  sc = 0;
 #pragma unroll 1
   for (int blk = 0; blk < 4; ++blk) {
     uint4* p0 = reinterpret_cast<uint4*>(rowp + (((2 * blk) ^ sw) << 4));
@@ -477,10 +480,25 @@ __device__ __forceinline__ void mlp_gelu_quant_row64(uint8_t* rowp, int sw, int 
       q1[2 * i] = c.x;
       q1[2 * i + 1] = c.y;
     }
-    if (row < M)
-      *reinterpret_cast<uint2*>(mp.codes + static_cast<int64_t>(row) * (N / 2) + x0 / 2 + 8 * blk) =
-          make_uint2(f32x8_to_e2m1(q0), f32x8_to_e2m1(q1));
+    c0 = c1;
+    c1 = c2;
+    c2 = c3;
+    c3 = make_uint2(f32x8_to_e2m1(q0), f32x8_to_e2m1(q1));
     sc |= S << (8 * blk);
+  }
+  cw[0] = make_uint4(c0.x, c0.y, c1.x, c1.y);
+  cw[1] = make_uint4(c2.x, c2.y, c3.x, c3.y);
+}
+
+// The codes and scale word of mlp_gelu_quant_row64 for this lane's row of
+// columns x0 .. x0 + 63: 32 code bytes for the down projection and the row's
+// scale word of the tiled layout (zero for padding rows M <= row < m_pad).
+__device__ __forceinline__ void mlp_store_row64(const uint4 (&cw)[2], uint32_t sc, int x0, int row, int M, int N,
+                                                const MlpPost& mp) {
+  if (row < M) {
+    uint4* dst = reinterpret_cast<uint4*>(mp.codes + static_cast<int64_t>(row) * (N / 2) + x0 / 2);
+    dst[0] = cw[0];
+    dst[1] = cw[1];
   }
   if (row < mp.m_pad)  // the four scale bytes of a row's 64 columns are one aligned word of the tiled layout
     *reinterpret_cast<uint32_t*>(mp.scales + scale_offset(N, row, x0 / 16)) = row < M ? sc : 0u;
@@ -898,8 +916,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<R, EPI>::kT
             tb[i] = cc == 0 ? pk1[i] : pk3[i];
           }
           stage_row64(stage, ta, tb, lane);  // y, then GELU and the quantisation in place
-          mlp_gelu_quant_row64(stage + lane * 128, lane & 7, col0 + 64 * cc, row, M, N, mlp, d,
-                               reinterpret_cast<const float*>(smem + C::kInvOff));
+          uint4 cw[2];
+          uint32_t scw;
+          mlp_gelu_quant_row64(stage + lane * 128, lane & 7, mlp.approximate != 0, d,
+                               reinterpret_cast<const float*>(smem + C::kInvOff), cw, scw);
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
@@ -909,6 +929,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<R, EPI>::kT
               bulk_commit();
             }
           }
+          mlp_store_row64(cw, scw, col0 + 64 * cc, row, M, N, mlp);
         }
         if (!ok) break;
         if (last) {
