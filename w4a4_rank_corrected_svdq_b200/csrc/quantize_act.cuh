@@ -84,7 +84,59 @@ struct QuantBarriers {
   uint64_t xl1_in;   // every partial row for this CTA's output rows has arrived
   uint32_t tmem_base;
   int abort;
+  float red[kQuantThreads / 32];  // per-warp maxima of the per-call activation scale
 };
+static_assert(sizeof(QuantBarriers) <= 256, "the barrier block of quantize_smem_bytes");
+
+// Per-call (dynamic) activation scale, computed by every CTA of the quantiser
+// from the amax pass's per-block maxima instead of read from g_x:
+// g = fp32(amax / 2688) (1 for amax = 0), alpha' = fp32(g g_w). CTA 0 writes
+// {g, g_w, alpha', amax} to gs_out, and the CTAs together re-express the
+// packed hi/lo planes of L2^T / alpha for alpha' (reexpress_planes) while their
+// first stages are in flight. partial == nullptr: the calibrated scale *g_x.
+struct DynScale {
+  const float* partial;         // [nparts] block maxima of |X^|
+  int nparts;
+  const float* gscale;          // the layer's {g_x, g_w, alpha, 0}
+  float* gs_out;                // this call's {g, g_w, alpha', amax}
+  const __nv_bfloat16* l2s;     // [2][total]: hi, lo planes for alpha
+  __nv_bfloat16* l2s_out;       // [2][total]: for alpha'
+  int64_t total;                // N r (a multiple of 16)
+};
+
+// Elements [8 i0, 8 i1) of the planes: v = hi + lo (exact in fp32),
+// v' = fp32(v * ratio), hi' = bf16(v'), lo' = bf16(v' - hi'); copied
+// unchanged when alpha' == alpha (same).
+__device__ __forceinline__ void reexpress_planes(const DynScale& dyn, int64_t i0, int64_t i1, int64_t stride,
+                                                 bool same, float ratio) {
+  const uint4* hi8 = reinterpret_cast<const uint4*>(dyn.l2s);
+  const uint4* lo8 = reinterpret_cast<const uint4*>(dyn.l2s + dyn.total);
+  uint4* ohi8 = reinterpret_cast<uint4*>(dyn.l2s_out);
+  uint4* olo8 = reinterpret_cast<uint4*>(dyn.l2s_out + dyn.total);
+  for (int64_t i = i0; i < i1; i += stride) {
+    const uint4 h = ldg_v4(hi8 + i), l = ldg_v4(lo8 + i);
+    if (same) {
+      ohi8[i] = h;
+      olo8[i] = l;
+      continue;
+    }
+    const uint32_t hw[4] = {h.x, h.y, h.z, h.w}, lw[4] = {l.x, l.y, l.z, l.w};
+    uint32_t oh[4], ol[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float v0 = __fmul_rn(__fadd_rn(__uint_as_float(hw[j] << 16), __uint_as_float(lw[j] << 16)), ratio);
+      const float v1 =
+          __fmul_rn(__fadd_rn(__uint_as_float(hw[j] & 0xFFFF0000u), __uint_as_float(lw[j] & 0xFFFF0000u)), ratio);
+      const __nv_bfloat162 hh = __floats2bfloat162_rn(v0, v1);
+      const float h0 = __low2float(hh), h1 = __high2float(hh);
+      const __nv_bfloat162 ll = __floats2bfloat162_rn(__fsub_rn(v0, h0), __fsub_rn(v1, h1));
+      oh[j] = *reinterpret_cast<const uint32_t*>(&hh);
+      ol[j] = *reinterpret_cast<const uint32_t*>(&ll);
+    }
+    ohi8[i] = make_uint4(oh[0], oh[1], oh[2], oh[3]);
+    olo8[i] = make_uint4(ol[0], ol[1], ol[2], ol[3]);
+  }
+}
 
 // Dynamic shared memory: stage ring (later XL1 partial slots), smoothing-factor
 // ring, scale staging for the CTA's K-range, reciprocal table, barriers,
@@ -144,7 +196,7 @@ template <int R, int ROWS, bool SMOOTH>
 __global__ void __launch_bounds__(kQuantThreads, 2) quantize_act_kernel(
     const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_l1t, int M, int K,
     const float* __restrict__ g_x, const float* __restrict__ inv_smooth, uint8_t* __restrict__ codes,
-    uint8_t* __restrict__ scales, __nv_bfloat16* __restrict__ xl1, int kchunk) {
+    uint8_t* __restrict__ scales, __nv_bfloat16* __restrict__ xl1, int kchunk, const DynScale dyn) {
   using C = QuantCfg<R, ROWS>;
   constexpr int S = C::kStages;
   constexpr int BPT = C::kBpt;
@@ -193,7 +245,39 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quantize_act_kernel(
     }
   }
   pdl_wait();
-  const float g = *g_x;
+  float g;
+  if (dyn.partial != nullptr) {
+    // this call's scale from the amax pass's block maxima (the same maximum,
+    // hence the same g, in every CTA)
+    float am = 0.0f;
+    for (int i = threadIdx.x; i < dyn.nparts; i += kQuantThreads) am = fmaxf(am, dyn.partial[i]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
+    if (lane == 0) bars->red[warp] = am;
+    __syncthreads();
+    am = bars->red[0];
+#pragma unroll
+    for (int w = 1; w < kQuantThreads / 32; ++w) am = fmaxf(am, bars->red[w]);
+    g = (am == 0.0f) ? 1.0f : __fdiv_rn(am, kGlobalDivisor);
+    const float gw = dyn.gscale[1], alpha = dyn.gscale[2];
+    const float alpha_d = __fmul_rn(g, gw);
+    const int cta = blockIdx.y * gridDim.x + blockIdx.x;
+    if (cta == 0 && threadIdx.x == 0) {
+      dyn.gs_out[0] = g;
+      dyn.gs_out[1] = gw;
+      dyn.gs_out[2] = alpha_d;
+      dyn.gs_out[3] = am;
+    }
+    if (warp > 0) {  // the quantiser warps, while the first stages are in flight
+      const int64_t vecs = dyn.total / 8, ncta = static_cast<int64_t>(gridDim.x) * gridDim.y;
+      const int64_t per = (vecs + ncta - 1) / ncta;
+      const int64_t i0 = cta * per, i1 = i0 + per < vecs ? i0 + per : vecs;
+      reexpress_planes(dyn, i0 + threadIdx.x - 32, i1, kQuantThreads - 32, alpha_d == alpha,
+                       __fdiv_rn(alpha, alpha_d));
+    }
+  } else {
+    g = *g_x;
+  }
   // The GEMM that consumes this kernel's output may be scheduled now: it
   // prepares its shared memory and TMEM, then waits for this grid to finish.
   pdl_launch_dependents();

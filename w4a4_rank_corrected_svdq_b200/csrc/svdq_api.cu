@@ -340,7 +340,7 @@ QuantPlan plan_quantize(int M, int K, int sm_count) {
 template <int R, int ROWS>
 svdq_status launch_quantize(int M, int K, int ks, const void* X, int64_t ldx, const float* g_x, const void* l1t,
                             const float* inv_smooth, void* codes, void* scales, void* xl1, cudaStream_t stream,
-                            bool pdl) {
+                            bool pdl, const DynScale& dyn) {
   const int row_tiles = (M + ROWS - 1) / ROWS;
   const int kchunk = K / ks;
   const size_t smem = quantize_smem_bytes<R, ROWS>(kchunk);
@@ -371,24 +371,25 @@ svdq_status launch_quantize(int M, int K, int ks, const void* X, int64_t ldx, co
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 2 : 1;
   cudaLaunchKernelEx(&cfg, kern, tm_x, tm_l, M, K, g_x, inv_smooth, static_cast<uint8_t*>(codes),
-                     static_cast<uint8_t*>(scales), static_cast<__nv_bfloat16*>(xl1), kchunk);
+                     static_cast<uint8_t*>(scales), static_cast<__nv_bfloat16*>(xl1), kchunk, dyn);
   return launch_status();
 }
 
 template <int R>
 svdq_status launch_quantize_planned(int M, int K, const void* X, int64_t ldx, const float* g_x, const void* l1t,
                                     const float* inv_smooth, void* codes, void* scales, void* xl1, cudaStream_t st,
-                                    int sms, bool pdl) {
+                                    int sms, bool pdl, const DynScale& dyn) {
   const QuantPlan plan = plan_quantize<R>(M, K, sms);
   if (plan.rows == 64)
-    return launch_quantize<R, 64>(M, K, plan.ks, X, ldx, g_x, l1t, inv_smooth, codes, scales, xl1, st, pdl);
-  return launch_quantize<R, 128>(M, K, plan.ks, X, ldx, g_x, l1t, inv_smooth, codes, scales, xl1, st, pdl);
+    return launch_quantize<R, 64>(M, K, plan.ks, X, ldx, g_x, l1t, inv_smooth, codes, scales, xl1, st, pdl, dyn);
+  return launch_quantize<R, 128>(M, K, plan.ks, X, ldx, g_x, l1t, inv_smooth, codes, scales, xl1, st, pdl, dyn);
 }
 
+// dyn: the per-call scale (svdq_linear_forward_dynamic), or none (g from g_x).
 svdq_status quantize_dispatch(int M, int K, int r, const void* X, int64_t ldx, const float* g_x, const void* l1t,
                               const float* inv_smooth, void* codes, void* scales, void* xl1, cudaStream_t st,
-                              int sms, bool pdl = false) {
-#define SVDQ_Q_ARGS M, K, X, ldx, g_x, l1t, inv_smooth, codes, scales, xl1, st, sms, pdl
+                              int sms, bool pdl = false, const DynScale& dyn = DynScale{}) {
+#define SVDQ_Q_ARGS M, K, X, ldx, g_x, l1t, inv_smooth, codes, scales, xl1, st, sms, pdl, dyn
   switch (r) {
     case 16: return launch_quantize_planned<16>(SVDQ_Q_ARGS);
     case 32: return launch_quantize_planned<32>(SVDQ_Q_ARGS);
@@ -693,72 +694,6 @@ int launch_act_amax(const __nv_bfloat16* X, int64_t ldx, int M, int K, const flo
   else
     act_amax_kernel<uint64_t><<<static_cast<int>(blocks), 256, 0, st>>>(X, ldx, M, K, inv, bits, partial);
   return static_cast<int>(blocks);
-}
-
-// Dynamic activation scale: partial[0..nparts) hold the per-block maxima of
-// amax|X^| of this call. Writes gs_out[0..3] = {g = fp32(amax / 2688) (1 if 0),
-// g_w, alpha' = fp32(g g_w), amax} and re-expresses the packed hi/lo planes of
-// L2^T / alpha for alpha': v = hi + lo (exact in fp32), v' = fp32(v *
-// fp32(alpha / alpha')), hi' = bf16(v'), lo' = bf16(v' - hi'); when alpha' ==
-// alpha the planes are copied unchanged. Launched as a programmatic dependent
-// of the amax pass (it waits for that grid here).
-__global__ void __launch_bounds__(256) dynamic_scale_kernel(const float* __restrict__ gscale,
-                                                            const float* __restrict__ partial, int nparts,
-                                                            float* __restrict__ gs_out,
-                                                            const __nv_bfloat16* __restrict__ l2s,
-                                                            __nv_bfloat16* __restrict__ l2s_out, int64_t total) {
-  pdl_wait();
-  pdl_launch_dependents();
-  __shared__ float red[8];
-  float am = 0.0f;
-  for (int i = threadIdx.x; i < nparts; i += blockDim.x) am = fmaxf(am, partial[i]);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = am;
-  __syncthreads();
-  am = red[0];
-  for (int w = 1; w < static_cast<int>(blockDim.x >> 5); ++w) am = fmaxf(am, red[w]);
-  const float g = (am == 0.0f) ? 1.0f : __fdiv_rn(am, kGlobalDivisor);
-  const float gw = gscale[1];
-  const float alpha = gscale[2];
-  const float alpha_d = __fmul_rn(g, gw);
-  if (blockIdx.x == 0 && threadIdx.x == 0) {
-    gs_out[0] = g;
-    gs_out[1] = gw;
-    gs_out[2] = alpha_d;
-    gs_out[3] = am;
-  }
-  const bool same = alpha_d == alpha;
-  const float ratio = __fdiv_rn(alpha, alpha_d);
-  // eight elements per step: total is a multiple of 16 (N r with r % 16 == 0)
-  const uint4* hi8 = reinterpret_cast<const uint4*>(l2s);
-  const uint4* lo8 = reinterpret_cast<const uint4*>(l2s + total);
-  uint4* ohi8 = reinterpret_cast<uint4*>(l2s_out);
-  uint4* olo8 = reinterpret_cast<uint4*>(l2s_out + total);
-  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total / 8;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const uint4 h = ldg_v4(hi8 + i), l = ldg_v4(lo8 + i);
-    if (same) {
-      ohi8[i] = h;
-      olo8[i] = l;
-      continue;
-    }
-    const uint32_t hw[4] = {h.x, h.y, h.z, h.w}, lw[4] = {l.x, l.y, l.z, l.w};
-    uint32_t oh[4], ol[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const float v0 = __fmul_rn(__fadd_rn(__uint_as_float(hw[j] << 16), __uint_as_float(lw[j] << 16)), ratio);
-      const float v1 =
-          __fmul_rn(__fadd_rn(__uint_as_float(hw[j] & 0xFFFF0000u), __uint_as_float(lw[j] & 0xFFFF0000u)), ratio);
-      const __nv_bfloat162 hh = __floats2bfloat162_rn(v0, v1);
-      const float h0 = __low2float(hh), h1 = __high2float(hh);
-      const __nv_bfloat162 ll = __floats2bfloat162_rn(__fsub_rn(v0, h0), __fsub_rn(v1, h1));
-      oh[j] = *reinterpret_cast<const uint32_t*>(&hh);
-      ol[j] = *reinterpret_cast<const uint32_t*>(&ll);
-    }
-    ohi8[i] = make_uint4(oh[0], oh[1], oh[2], oh[3]);
-    olo8[i] = make_uint4(ol[0], ol[1], ol[2], ol[3]);
-  }
 }
 
 template <int R>
@@ -1335,26 +1270,26 @@ svdq_status svdq_linear_forward_dynamic(int M, int N, int K, int r, const void* 
   float* gs = reinterpret_cast<float*>(ws + base);
   float* partial = reinterpret_cast<float*>(ws + base + 256);
   __nv_bfloat16* l2s_d = reinterpret_cast<__nv_bfloat16*>(ws + base + kDynScaleBytes);
-  // amax|X^| of this call as per-block maxima, then the per-call scales and
-  // l2 planes, then the layer; each kernel after the first is a programmatic
-  // dependent of the one before (it waits for it before reading its output).
+  // amax|X^| of this call as per-block maxima; the quantiser (a programmatic
+  // dependent of the amax pass) reduces them to this call's scale, writes
+  // {g, g_w, alpha', amax} and re-expresses the l2 planes; then the GEMM.
   const int nparts = launch_act_amax(static_cast<const __nv_bfloat16*>(X), ldx, M, K, inv_smooth, nullptr, partial,
                                      di.sm_count, st);
-  const int64_t total = static_cast<int64_t>(N) * r;
-  const int64_t sblocks = (total / 8 + 255) / 256 < 2 * di.sm_count ? (total / 8 + 255) / 256 : 2 * di.sm_count;
-  {
-    PdlLaunch pl(static_cast<int>(sblocks), 256, 0, st);
-    cudaLaunchKernelEx(&pl.cfg, dynamic_scale_kernel, static_cast<const float*>(gscale),
-                       static_cast<const float*>(partial), nparts, gs, static_cast<const __nv_bfloat16*>(l2s), l2s_d,
-                       total);
-  }
   if ((s = launch_status()) != SVDQ_OK) return s;
   size_t c = 0, sc = 0, x = 0;
   svdq_act_sizes(M, K, r, &c, &sc, &x);
   uint8_t* a_codes = ws;
   uint8_t* a_scales = ws + round_up(c, 256);
   uint8_t* xl1 = a_scales + round_up(sc, 256);
-  s = quantize_dispatch(M, K, r, X, ldx, gs, l1t, inv_smooth, a_codes, a_scales, xl1, st, di.sm_count, true);
+  DynScale dyn{};
+  dyn.partial = partial;
+  dyn.nparts = nparts;
+  dyn.gscale = gscale;
+  dyn.gs_out = gs;
+  dyn.l2s = static_cast<const __nv_bfloat16*>(l2s);
+  dyn.l2s_out = l2s_d;
+  dyn.total = static_cast<int64_t>(N) * r;
+  s = quantize_dispatch(M, K, r, X, ldx, gs, l1t, inv_smooth, a_codes, a_scales, xl1, st, di.sm_count, true, dyn);
   if (s != SVDQ_OK) return s;
   return svdq_w4a4_gemm(M, N, K, r, a_codes, a_scales, xl1, w_codes, w_scales, gs, l2s_d, bias, Y, ldy, stream);
 }
