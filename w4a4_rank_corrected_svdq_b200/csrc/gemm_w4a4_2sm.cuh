@@ -23,10 +23,13 @@
 // (SFB) are copied, four tcgen05.cp of 128x256b instead of six.
 //
 // Roles (320 threads per CTA):
-//  * warp 0     TMA producer (both CTAs): per tile first r/c low-rank stages
-//               (XL1 columns, hi and lo columns of l2s; c = min(r, 32)), then
-//               K/256 stages of E2M1 codes (128-byte swizzle) and UE4M3 scale
-//               atoms (SFA only when the tile starts a new A block).
+//  * warp 0     TMA producer (both CTAs): per tile K/256 stages of E2M1
+//               codes (128-byte swizzle) and UE4M3 scale atoms (SFA only when
+//               the tile starts a new A block), then r/c low-rank stages (XL1
+//               columns, hi and lo columns of l2s; c = min(r, 32)). The small
+//               low-rank stages come last: when the ring refills at a tile
+//               boundary its first stages are then full K blocks, whose MMAs
+//               cover the load latency of the next ones.
 //               Completion bytes of both CTAs land on the even CTA's barrier
 //               (cp.async.bulk.tensor .cta_group::2).
 //  * warp 1     TMEM owner (both CTAs, 512 columns); in the even CTA lane 0
@@ -665,14 +668,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<R, EPI>::kT
           if (!mbar_wait(&bars->empty[s], ph ^ 1, abort)) { ok = false; break; }
           uint8_t* st = smem + s * C::kStageBytes;
           const uint32_t bar = mapa_shared(smem_u32(&bars->full[s]), 0);
-          if (step < C::kLrSteps) {
+          if (step >= nk) {  // the low-rank stages come last, after the K blocks
             if (rank == 0) mbar_arrive_expect_tx(&bars->full[s], C::kLrTx);
-            const int x = step * C::kLrCols;
+            const int x = (step - nk) * C::kLrCols;
             tma_load_2d_cg2(st, &tm_xl1, x, m_own, bar);
             tma_load_2d_cg2(st + C::kABytes, &tm_l2s, x, n_own, bar);
             tma_load_2d_cg2(st + C::kABytes + C::kLrTileBytes, &tm_l2s, x, N + n_own, bar);
           } else {
-            const int kb = step - C::kLrSteps;
+            const int kb = step;
             if (rank == 0) mbar_arrive_expect_tx(&bars->full[s], sfa_load ? C::kMainTx : C::kMainTx - C::kSfaTx);
             tma_load_2d_cg2(st, &tm_a, kb * 128, m_own, bar);
             tma_load_2d_cg2(st + C::kABytes, &tm_b, kb * 128, n_own, bar);
@@ -713,18 +716,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<R, EPI>::kT
           if (!mbar_wait(&bars->full[s], ph, abort)) { ok = false; break; }
           tc_fence_after();
           const uint32_t st = smem_u32(smem + s * C::kStageBytes);
-          if (step < C::kLrSteps) {
+          if (step >= nk) {  // low-rank stages, after the K blocks: XL1 . (hi, lo) into the same accumulator
 #pragma unroll
             for (int k16 = 0; k16 < C::kLrCols / 16; ++k16) {
               const uint64_t a = smem_desc(st + 32 * k16, 16, 8 * C::kLrRowBytes, C::kLrSwizzle);
               const uint64_t bh = smem_desc(st + C::kABytes + 32 * k16, 16, 8 * C::kLrRowBytes, C::kLrSwizzle);
               const uint64_t bl =
                   smem_desc(st + C::kABytes + C::kLrTileBytes + 32 * k16, 16, 8 * C::kLrRowBytes, C::kLrSwizzle);
-              mma_bf16_cg2(tmem, a, bh, idesc_bf16, (step | k16) != 0 ? 1u : 0u);
+              mma_bf16_cg2(tmem, a, bh, idesc_bf16, 1u);
               mma_bf16_cg2(tmem, a, bl, idesc_bf16, 1u);
             }
           } else {
-            const int kb = step - C::kLrSteps;
+            const int kb = step;
             const uint32_t t_sfa = tmem + k2SfaCol + 16 * (kb % C::kSfaSlots);
             const uint32_t sfa = st + C::kABytes + C::kBBytes;
             const uint32_t sfb = sfa + C::kSfaBytes;
@@ -740,8 +743,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<R, EPI>::kT
             const uint64_t adesc = smem_desc(st, 16, 1024, kSwizzle128B);
             const uint64_t bdesc = smem_desc(st + C::kABytes, 16, 1024, kSwizzle128B);
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
-              mma_nvf4_cg2(tmem, adesc + 2 * j, bdesc + 2 * j, idesc_fp4, t_sfa + 4 * j, t_sfb + 8 * j, 1u);
+            for (int j = 0; j < 4; ++j)  // the tile's first MMA overwrites the accumulator
+              mma_nvf4_cg2(tmem, adesc + 2 * j, bdesc + 2 * j, idesc_fp4, t_sfa + 4 * j, t_sfb + 8 * j,
+                           (kb | j) != 0 ? 1u : 0u);
           }
           tc_commit_cg2_mc(&bars->empty[s], 0x3);
           if (++s == S) { s = 0; ph ^= 1; }
