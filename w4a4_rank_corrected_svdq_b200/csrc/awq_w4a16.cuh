@@ -89,8 +89,9 @@ __global__ void __launch_bounds__(kAwqThreads) awq_pack_kernel(const __nv_bfloat
 // of warps); lane l takes the rows' chunks l, l + 32, ... (32 codes = 16 bytes,
 // half a 64-group, so one scale and zero point each). Per
 // 8-code word the integers q - z are formed exactly (2^23 + q from one byte
-// permute, minus the exact 2^23 + z), the products x (q - z) are summed as
-// fp32 pairs over the chunk and scaled by s once. Packed f32x2 arithmetic.
+// permute, plus -(2^23 + z) built from its bit pattern), the products
+// x (q - z) are summed as fp32 pairs over the chunk and scaled by s once.
+// Packed f32x2 arithmetic.
 template <int MT>
 __global__ void __launch_bounds__(kAwqThreads) awq_gemv_kernel(int M, int N, int K,
                                                                const __nv_bfloat16* __restrict__ X, int64_t ldx,
@@ -138,24 +139,34 @@ __global__ void __launch_bounds__(kAwqThreads) awq_gemv_kernel(int M, int N, int
     uint4 vn[kAwqRows];
     __nv_bfloat16 sn[kAwqRows];
     uint8_t zn[kAwqRows];
+    // the pass's row bases (rows past N repeat the last one and are not stored)
+    const uint8_t* rc[kAwqRows];
+    const __nv_bfloat16* rs[kAwqRows];
+    const uint8_t* rz[kAwqRows];
+#pragma unroll
+    for (int r = 0; r < kAwqRows; ++r) {
+      const int64_t n = n0 + r < N ? n0 + r : N - 1;
+      rc[r] = codes + n * (K / 2);
+      rs[r] = scales + n * G;
+      rz[r] = zeros + n * G;
+    }
     auto fetch = [&](int c) {
 #pragma unroll
       for (int r = 0; r < kAwqRows; ++r) {
-        const int n = n0 + r < N ? n0 + r : N - 1;  // rows past N repeat the last one and are not stored
-        vn[r] = ldg_nc_v4(codes + static_cast<int64_t>(n) * (K / 2) + 16 * c);
-        sn[r] = scales[static_cast<int64_t>(n) * G + (c >> 1)];
-        zn[r] = zeros[static_cast<int64_t>(n) * G + (c >> 1)];
+        vn[r] = ldg_nc_v4(rc[r] + 16 * c);
+        sn[r] = rs[r][c >> 1];
+        zn[r] = rz[r][c >> 1];
       }
     };
     if (lane < C) fetch(lane);
     for (int c = lane; c < C; c += 32) {
       uint4 v[kAwqRows];
-      float sv[kAwqRows], zf[kAwqRows];
+      float sv[kAwqRows], nz[kAwqRows];
 #pragma unroll
       for (int r = 0; r < kAwqRows; ++r) {
         v[r] = vn[r];
         sv[r] = __bfloat162float(sn[r]);
-        zf[r] = __fadd_rn(8388608.0f, static_cast<float>(zn[r]));
+        nz[r] = __uint_as_float(0xCB000000u | zn[r]);  // -(2^23 + z), exact
       }
       if (c + 32 < C) fetch(c + 32);
       const int sw = c & 7;
@@ -171,7 +182,7 @@ __global__ void __launch_bounds__(kAwqThreads) awq_gemv_kernel(int M, int N, int
         for (int r = 0; r < kAwqRows; ++r) {
           const uint32_t word = wd == 0 ? v[r].x : (wd == 1 ? v[r].y : (wd == 2 ? v[r].z : v[r].w));
           const uint32_t lo = word & 0x0F0F0F0Fu, hi = (word >> 4) & 0x0F0F0F0Fu;
-          const float2 nz2 = make_float2(-zf[r], -zf[r]);
+          const float2 nz2 = make_float2(nz[r], nz[r]);
 #pragma unroll
           for (int b = 0; b < 4; ++b) {
             const float2 q = make_float2(__uint_as_float(__byte_perm(lo, 0x4B000000u, 0x7650u + b)),
@@ -329,13 +340,13 @@ __global__ void __launch_bounds__(kAwqRingThreads, 1) awq_gemv_ring_kernel(
       for (int m = 0; m < MT; ++m) acc[r][m] = make_float2(0.0f, 0.0f);
     for (int c = lane; c < C; c += 32) {
       uint4 v[kAwqRows];
-      float sv[kAwqRows], zf[kAwqRows];
+      float sv[kAwqRows], nz[kAwqRows];
 #pragma unroll
       for (int r = 0; r < kAwqRows; ++r) {
         // rows past the CTA's run read the stage's stale bytes and are not stored
         v[r] = *reinterpret_cast<const uint4*>(st + (lr0 + r) * (K / 2) + 16 * c);
         sv[r] = __bfloat162float(st_sc[(lr0 + r) * G + (c >> 1)]);
-        zf[r] = __fadd_rn(8388608.0f, static_cast<float>(st_z[(lr0 + r) * G + (c >> 1)]));
+        nz[r] = __uint_as_float(0xCB000000u | st_z[(lr0 + r) * G + (c >> 1)]);  // -(2^23 + z), exact
       }
       const int sw = c & 7;
       float2 t[kAwqRows][MT];
@@ -350,7 +361,7 @@ __global__ void __launch_bounds__(kAwqRingThreads, 1) awq_gemv_ring_kernel(
         for (int r = 0; r < kAwqRows; ++r) {
           const uint32_t word = wd == 0 ? v[r].x : (wd == 1 ? v[r].y : (wd == 2 ? v[r].z : v[r].w));
           const uint32_t lo = word & 0x0F0F0F0Fu, hi = (word >> 4) & 0x0F0F0F0Fu;
-          const float2 nz2 = make_float2(-zf[r], -zf[r]);
+          const float2 nz2 = make_float2(nz[r], nz[r]);
 #pragma unroll
           for (int b = 0; b < 4; ++b) {
             const float2 q = make_float2(__uint_as_float(__byte_perm(lo, 0x4B000000u, 0x7650u + b)),
