@@ -32,6 +32,7 @@ namespace svdq {
 constexpr int kAwqGroup = 64;
 constexpr int kAwqThreads = 256;
 constexpr int kAwqRows = 4;  // weight rows per warp pass of the GEMV
+static_assert(kAwqGroup / 2 == 32, "a row's code bytes are 32 per group (the GEMV's scale offset is n K/2 >> 5)");
 
 // One thread per (row, group): codes (element 2j in the low nibble of byte j),
 // bf16 scale, u8 zero point.
@@ -104,6 +105,38 @@ __global__ void __launch_bounds__(kAwqThreads) awq_gemv_kernel(int M, int N, int
   extern __shared__ float4 xs4[];  // [MT][K/32][8], swizzled
   const int rows = M < MT ? M : MT;
   const int C = K / 32;
+  const int lane = threadIdx.x & 31;
+  const int warps = static_cast<int>(gridDim.x) * (kAwqThreads / 32);
+  const int G = K / kAwqGroup;
+  const int nstep = warps * kAwqRows;
+  int n0 = (blockIdx.x * (kAwqThreads / 32) + (threadIdx.x >> 5)) * kAwqRows;
+  // chunk loads are software-pipelined: the next chunk's codes, scales and zero
+  // points (after a pass's last chunk: the next pass's first) are requested
+  // before the current chunk's arithmetic, and the first pass's first chunk
+  // before the activations are staged
+  uint4 vn[kAwqRows];
+  __nv_bfloat16 sn[kAwqRows];
+  uint8_t zn[kAwqRows];
+  // the code-row offsets n K/2 of the pass being fetched (rows past N repeat
+  // the last one and are not stored); a row's scales and zero points start at
+  // n G = n K/2 / 32
+  int64_t ro[kAwqRows];
+  auto bases = [&](int nb) {
+#pragma unroll
+    for (int r = 0; r < kAwqRows; ++r) ro[r] = static_cast<int64_t>(nb + r < N ? nb + r : N - 1) * (K / 2);
+  };
+  auto fetch = [&](int c) {
+#pragma unroll
+    for (int r = 0; r < kAwqRows; ++r) {
+      vn[r] = ldg_nc_v4(codes + ro[r] + 16 * c);
+      sn[r] = scales[(ro[r] >> 5) + (c >> 1)];
+      zn[r] = zeros[(ro[r] >> 5) + (c >> 1)];
+    }
+  };
+  if (n0 < N) {
+    bases(n0);
+    if (lane < C) fetch(lane);
+  }
   for (int i = threadIdx.x; i < MT * (K / 4); i += blockDim.x) {
     const int m = i / (K / 4), q4 = i % (K / 4);  // float4 q4 of row m: elements 4 q4 .. 4 q4 + 3
     float4 f = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
@@ -121,44 +154,15 @@ __global__ void __launch_bounds__(kAwqThreads) awq_gemv_kernel(int M, int N, int
     xs4[(m * C + c) * 8 + (fi ^ (c & 7))] = f;
   }
   __syncthreads();
-  const int lane = threadIdx.x & 31;
-  const int warps = static_cast<int>(gridDim.x) * (kAwqThreads / 32);
-  const int G = K / kAwqGroup;
   // kAwqRows weight rows per warp pass: each X^ value read from shared memory
   // serves all of them (shared-memory bandwidth, not HBM, bounds a pass over
   // one row at a time).
-  for (int n0 = (blockIdx.x * (kAwqThreads / 32) + (threadIdx.x >> 5)) * kAwqRows; n0 < N;
-       n0 += warps * kAwqRows) {
+  for (; n0 < N; n0 += nstep) {
     float2 acc[kAwqRows][MT];
 #pragma unroll
     for (int r = 0; r < kAwqRows; ++r)
 #pragma unroll
       for (int m = 0; m < MT; ++m) acc[r][m] = make_float2(0.0f, 0.0f);
-    // chunk loads are software-pipelined: the next chunk's codes, scales and zero
-    // points are requested before the current chunk's arithmetic
-    uint4 vn[kAwqRows];
-    __nv_bfloat16 sn[kAwqRows];
-    uint8_t zn[kAwqRows];
-    // the pass's row bases (rows past N repeat the last one and are not stored)
-    const uint8_t* rc[kAwqRows];
-    const __nv_bfloat16* rs[kAwqRows];
-    const uint8_t* rz[kAwqRows];
-#pragma unroll
-    for (int r = 0; r < kAwqRows; ++r) {
-      const int64_t n = n0 + r < N ? n0 + r : N - 1;
-      rc[r] = codes + n * (K / 2);
-      rs[r] = scales + n * G;
-      rz[r] = zeros + n * G;
-    }
-    auto fetch = [&](int c) {
-#pragma unroll
-      for (int r = 0; r < kAwqRows; ++r) {
-        vn[r] = ldg_nc_v4(rc[r] + 16 * c);
-        sn[r] = rs[r][c >> 1];
-        zn[r] = rz[r][c >> 1];
-      }
-    };
-    if (lane < C) fetch(lane);
     for (int c = lane; c < C; c += 32) {
       uint4 v[kAwqRows];
       float sv[kAwqRows], nz[kAwqRows];
@@ -168,7 +172,12 @@ __global__ void __launch_bounds__(kAwqThreads) awq_gemv_kernel(int M, int N, int
         sv[r] = __bfloat162float(sn[r]);
         nz[r] = __uint_as_float(0xCB000000u | zn[r]);  // -(2^23 + z), exact
       }
-      if (c + 32 < C) fetch(c + 32);
+      if (c + 32 < C) {
+        fetch(c + 32);
+      } else if (n0 + nstep < N) {
+        bases(n0 + nstep);
+        fetch(lane);
+      }
       const int sw = c & 7;
       float2 t[kAwqRows][MT];
 #pragma unroll
