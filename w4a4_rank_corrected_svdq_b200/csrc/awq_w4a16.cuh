@@ -107,7 +107,6 @@ __global__ void __launch_bounds__(kAwqThreads) awq_gemv_kernel(int M, int N, int
   const int C = K / 32;
   const int lane = threadIdx.x & 31;
   const int warps = static_cast<int>(gridDim.x) * (kAwqThreads / 32);
-  const int G = K / kAwqGroup;
   const int nstep = warps * kAwqRows;
   int n0 = (blockIdx.x * (kAwqThreads / 32) + (threadIdx.x >> 5)) * kAwqRows;
   // chunk loads are software-pipelined: the next chunk's codes, scales and zero
