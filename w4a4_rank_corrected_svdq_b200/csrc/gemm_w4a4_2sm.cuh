@@ -117,9 +117,6 @@ __device__ __forceinline__ void mma_bf16_cg2(uint32_t d_tmem, uint64_t a_desc, u
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
-__device__ __forceinline__ void tmem_cp_cg2(uint32_t taddr, uint64_t s_desc) {
-  asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(s_desc) : "memory");
-}
 // Arrives on the barrier at this shared-memory offset in every CTA of `mask`
 // once all prior tcgen05 operations of this thread have completed.
 __device__ __forceinline__ void tc_commit_cg2_mc(uint64_t* bar, uint16_t mask) {
@@ -288,17 +285,6 @@ __device__ __forceinline__ void stage_row16(uint8_t* buf, const uint32_t (&pk)[1
     *reinterpret_cast<uint4*>(buf + lane * 64 + ((j ^ sw) << 4)) =
         make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
 }
-__device__ __forceinline__ void load_row16(const uint8_t* buf, uint32_t (&pk)[16], int lane) {
-  const int sw = (lane >> 1) & 3;
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const uint4 v = *reinterpret_cast<const uint4*>(buf + lane * 64 + ((j ^ sw) << 4));
-    pk[4 * j] = v.x;
-    pk[4 * j + 1] = v.y;
-    pk[4 * j + 2] = v.z;
-    pk[4 * j + 3] = v.w;
-  }
-}
 // This lane's row of 16 rotary angles (cos at cr, sin at sr; 16-byte aligned).
 __device__ __forceinline__ void load_angles16(const float* cr, const float* sr, float (&tc)[16], float (&ts)[16]) {
 #pragma unroll
@@ -324,12 +310,6 @@ __device__ __forceinline__ void store_staged(const uint8_t* buf, const CUtensorM
     tma_store_2d(tm_y, buf, x, y);
     bulk_commit();
   }
-}
-
-// bf16 pairs of alpha * acc + b for one 32-column chunk (bias at bcol, or none).
-__device__ __forceinline__ void pack32(const uint32_t (&v)[32], const __nv_bfloat16* bcol, float alpha,
-                                       uint32_t (&pk)[16]) {
-  pack_chunk(v, bcol, alpha, pk);
 }
 
 // Sum of squares of 16 packed bf16 pairs, added to ss in element order.
