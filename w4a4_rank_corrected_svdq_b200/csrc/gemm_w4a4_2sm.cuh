@@ -148,8 +148,14 @@ struct Gemm2Cfg {
   // lane: two K-steps of A scales, or one K-step of both 128-row halves of B.
   static constexpr int kSfaBytes = 4 * 2048;    // 4 K-steps x 4 replicas x 512 B (128 rows)
   static constexpr int kSfbBytes = 2 * 4 * 2048;  // 2 row blocks x 4 K-steps x 4 replicas x 512 B
-  static constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;  // 56 KB
-  static constexpr int kStages = 3;
+  // The plain layer (EPI 0) runs four stages: its A scales, needed only when a
+  // tile starts a new A block, move to a two-slot ring of their own, and its
+  // epilogue stages 32 x 32 (2 KB) per warp. The fused modes keep three stages
+  // with the A scales in every stage.
+  static constexpr bool kLean = EPI == 0;
+  static constexpr int kSfbOff = kABytes + kBBytes + (kLean ? 0 : kSfaBytes);  // within a stage
+  static constexpr int kStageBytes = kSfbOff + kSfbBytes;  // 48 or 56 KB
+  static constexpr int kStages = kLean ? 4 : 3;
   // K blocks of A scales held in TMEM (MLP: the last 32 columns hold h . L1_down)
   static constexpr int kSfaSlots = ((MLP ? k2Xl1Col : 512) - k2SfaCol) / 16;
   static constexpr int kLrCols = R < 32 ? R : 32;           // low-rank columns per stage
@@ -160,14 +166,17 @@ struct Gemm2Cfg {
   static constexpr uint32_t kMainTx = 2u * kStageBytes;     // both CTAs
   static constexpr uint32_t kSfaTx = 2u * kSfaBytes;
   static constexpr uint32_t kLrTx = 2u * 3u * kLrTileBytes;
-  // Epilogue staging per warp (4 KB): the plain layer stages 32 rows x 64
-  // columns (128-byte swizzle, one TMA store); the fused modes two 32 x 32
-  // buffers (64-byte swizzle).
-  static constexpr int kOutPerWarp = 4096;
+  // Epilogue staging per warp: the plain layer one 32 x 32 buffer (2 KB,
+  // 64-byte swizzle, four TMA stores per tile); the fused QKV mode two such
+  // buffers; the MLP mode one 32-row x 64-column chunk (4 KB, 128-byte swizzle).
+  static constexpr int kOutPerWarp = kLean ? 2048 : 4096;
   static constexpr int kOutOff = kStages * kStageBytes;
   static constexpr int kOutBytes = 8 * kOutPerWarp;
+  // Plain layer: the A-scale ring (two slots of one K block's A scales).
+  static constexpr int kSfaRingOff = kOutOff + kOutBytes;
+  static constexpr int kSfaRingBytes = kLean ? 2 * kSfaBytes : 0;
   // The tile's 256 bias values, double-buffered by tile parity.
-  static constexpr int kBiasOff = kOutOff + kOutBytes;
+  static constexpr int kBiasOff = kSfaRingOff + kSfaRingBytes;
   static constexpr int kBiasBytes = 2 * k2TileN * 2;
   // Fused QKV: per warp, partial sums of squares of its rows for the two heads
   // of a tile, double-buffered (2 x 2 x 32 floats).
@@ -183,6 +192,7 @@ struct Gemm2Cfg {
   static constexpr int kInvBytes = MLP ? 512 : 0;
   static constexpr int kBarOff = kInvOff + kInvBytes;
   static constexpr int kSmemBytes = kBarOff + 512 + 1024;
+  static_assert(kSmemBytes <= 227 * 1024, "dynamic shared memory per CTA");
 };
 
 struct Gemm2Barriers {
@@ -201,9 +211,13 @@ struct Gemm2Barriers {
   uint64_t xl1_done;        // the run's h . L1_down accumulator is complete
   uint64_t xl1_free;        // and has been read out (4 warps x 2 CTAs)
   uint64_t xl1_teardown;    // every h . L1_down MMA has completed
+  // plain layer: the A-scale ring
+  uint64_t sfa_full[2];     // a K block's A scales are in the slot (both CTAs' halves)
+  uint64_t sfa_empty[2];    // and have been copied into TMEM
   uint32_t tmem_base;
   int abort;
 };
+static_assert(sizeof(Gemm2Barriers) <= 512, "the barrier block of Gemm2Cfg::kSmemBytes");
 
 // The contiguous run of tiles [t0, t1) of CTA pair `pair` (balanced: runs
 // differ by at most one tile).
@@ -226,29 +240,6 @@ __device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
-// 64 columns of this lane's row (two 32-column chunks of packed bf16 pairs)
-// written into a 32-row x 128-byte staging buffer in the 128-byte swizzle of
-// the Y store map, then stored with one TMA store by lane 0.
-__device__ __forceinline__ void store_row64(uint8_t* buf, const uint32_t (&pa)[16], const uint32_t (&pb)[16],
-                                            const CUtensorMap* tm_y, int x, int y, int lane) {
-  if (lane == 0) bulk_wait_read0();  // the previous store from this buffer has read it
-  __syncwarp();
-  uint8_t* row = buf + lane * 128;
-  const int sw = lane & 7;
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    *reinterpret_cast<uint4*>(row + ((j ^ sw) << 4)) = make_uint4(pa[4 * j], pa[4 * j + 1], pa[4 * j + 2], pa[4 * j + 3]);
-    *reinterpret_cast<uint4*>(row + (((j + 4) ^ sw) << 4)) =
-        make_uint4(pb[4 * j], pb[4 * j + 1], pb[4 * j + 2], pb[4 * j + 3]);
-  }
-  fence_proxy_async_smem();
-  __syncwarp();
-  if (lane == 0) {
-    tma_store_2d(tm_y, buf, x, y);
-    bulk_commit();
-  }
 }
 
 // Drains this warp's four 32-column chunks of the accumulator (TMEM columns
@@ -310,6 +301,17 @@ __device__ __forceinline__ void store_staged(const uint8_t* buf, const CUtensorM
     tma_store_2d(tm_y, buf, x, y);
     bulk_commit();
   }
+}
+
+// 32 columns of this lane's row (16 packed bf16 pairs) into the warp's
+// 32 x 64-byte staging buffer (64-byte swizzle) and one TMA store, once the
+// previous store from the buffer has read it.
+__device__ __forceinline__ void store_row32(uint8_t* buf, const uint32_t (&pk)[16], const CUtensorMap* tm_y, int x,
+                                            int y, int lane) {
+  if (lane == 0) bulk_wait_read0();
+  __syncwarp();
+  stage_row16(buf, pk, lane);
+  store_staged(buf, tm_y, x, y, lane);
 }
 
 // Sum of squares of 16 packed bf16 pairs, added to ss in element order.
@@ -593,6 +595,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<R, EPI>::kT
     mbar_init(&bars->xl1_done, 1);
     mbar_init(&bars->xl1_free, 8);
     mbar_init(&bars->xl1_teardown, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bars->sfa_full[i], 1);
+      mbar_init(&bars->sfa_empty[i], 1);
+    }
     bars->abort = 0;
     fence_barrier_init();
   }
@@ -637,6 +643,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<R, EPI>::kT
       uint32_t ph = 0;
       bool ok = true;
       int prev_mt = -1;
+      int nsfa = 0;  // plain layer: A-scale loads so far (ring slot nsfa & 1)
       for (int tile = t_begin; tile < t_end && ok; ++tile) {
         const int mt = tile / num_nt, nt = tile % num_nt;
         const bool sfa_load = !sfa_resident || mt != prev_mt;
@@ -656,12 +663,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<R, EPI>::kT
             tma_load_2d_cg2(st + C::kABytes + C::kLrTileBytes, &tm_l2s, x, N + n_own, bar);
           } else {
             const int kb = step;
-            if (rank == 0) mbar_arrive_expect_tx(&bars->full[s], sfa_load ? C::kMainTx : C::kMainTx - C::kSfaTx);
+            if (rank == 0)
+              mbar_arrive_expect_tx(&bars->full[s], (C::kLean || sfa_load) ? C::kMainTx : C::kMainTx - C::kSfaTx);
             tma_load_2d_cg2(st, &tm_a, kb * 128, m_own, bar);
             tma_load_2d_cg2(st + C::kABytes, &tm_b, kb * 128, n_own, bar);
-            uint8_t* sf = st + C::kABytes + C::kBBytes;
-            if (sfa_load) tma_load_4d_cg2(sf, &tm_sfa, 0, 0, 0, (m_own / 128) * sf_row_stride + 4 * kb, bar);
-            tma_load_5d_cg2(sf + C::kSfaBytes, &tm_sfb, 0, 0, 0, 4 * kb, nblk, bar);
+            if (sfa_load) {
+              const int sfa_c = (m_own / 128) * sf_row_stride + 4 * kb;
+              if constexpr (C::kLean) {
+                const int slot = nsfa & 1;
+                if (!mbar_wait(&bars->sfa_empty[slot], ((nsfa >> 1) & 1) ^ 1, abort)) { ok = false; break; }
+                if (rank == 0) mbar_arrive_expect_tx(&bars->sfa_full[slot], C::kSfaTx);
+                tma_load_4d_cg2(smem + C::kSfaRingOff + slot * C::kSfaBytes, &tm_sfa, 0, 0, 0, sfa_c,
+                                mapa_shared(smem_u32(&bars->sfa_full[slot]), 0));
+                ++nsfa;
+              } else {
+                tma_load_4d_cg2(st + C::kABytes + C::kBBytes, &tm_sfa, 0, 0, 0, sfa_c, bar);
+              }
+            }
+            tma_load_5d_cg2(st + C::kSfbOff, &tm_sfb, 0, 0, 0, 4 * kb, nblk, bar);
           }
           if (++s == S) { s = 0; ph ^= 1; }
         }
@@ -685,6 +704,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<R, EPI>::kT
       int it = 0;
       bool ok = true;
       int prev_mt = -1;
+      int nsfa = 0;  // plain layer: A-scale slots consumed so far
       for (int tile = t_begin; tile < t_end && ok; ++tile, ++it) {
         const int mt = tile / num_nt;
         const bool sfa_load = !sfa_resident || mt != prev_mt;
@@ -709,13 +729,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<R, EPI>::kT
           } else {
             const int kb = step;
             const uint32_t t_sfa = tmem + k2SfaCol + 16 * (kb % C::kSfaSlots);
-            const uint32_t sfa = st + C::kABytes + C::kBBytes;
-            const uint32_t sfb = sfa + C::kSfaBytes;
+            const uint32_t sfb = st + C::kSfbOff;
             // A: K-steps (0,1) and (2,3), 2 KB apart (only when the tile starts a new A block);
             // B: K-step j, row blocks 8 KB apart
             if (sfa_load) {
+              uint32_t sfa = st + C::kABytes + C::kBBytes;
+              if constexpr (C::kLean) {
+                const int slot = nsfa & 1;
+                if (!mbar_wait(&bars->sfa_full[slot], (nsfa >> 1) & 1, abort)) { ok = false; break; }
+                tc_fence_after();
+                sfa = smem_u32(smem + C::kSfaRingOff + slot * C::kSfaBytes);
+              }
               tmem_cp_128x256b_cg2(t_sfa, smem_desc(sfa, 2048, 128, kSwizzleNone));
               tmem_cp_128x256b_cg2(t_sfa + 8, smem_desc(sfa + 4096, 2048, 128, kSwizzleNone));
+              if constexpr (C::kLean) tc_commit_cg2_mc(&bars->sfa_empty[nsfa++ & 1], 0x3);  // the slot may be refilled
             }
 #pragma unroll
             for (int j = 0; j < 4; ++j)
@@ -938,13 +965,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<R, EPI>::kT
         }
         continue;
       }
-      uint32_t pa[16], pb[16];
-      pack_chunk(va, bcol, alpha, pa);
-      pack_chunk(vb, bcol ? bcol + 32 : nullptr, alpha, pb);
-      store_row64(stage, pa, pb, &tm_y, col0, y0, lane);
-      pack_chunk(vc, bcol ? bcol + 64 : nullptr, alpha, pa);
-      pack_chunk(vd, bcol ? bcol + 96 : nullptr, alpha, pb);
-      store_row64(stage, pa, pb, &tm_y, col0 + 64, y0, lane);
+      uint32_t pk[16];
+      pack_chunk(va, bcol, alpha, pk);
+      store_row32(stage, pk, &tm_y, col0, y0, lane);
+      pack_chunk(vb, bcol ? bcol + 32 : nullptr, alpha, pk);
+      store_row32(stage, pk, &tm_y, col0 + 32, y0, lane);
+      pack_chunk(vc, bcol ? bcol + 64 : nullptr, alpha, pk);
+      store_row32(stage, pk, &tm_y, col0 + 64, y0, lane);
+      pack_chunk(vd, bcol ? bcol + 96 : nullptr, alpha, pk);
+      store_row32(stage, pk, &tm_y, col0 + 96, y0, lane);
     }
     if (lane == 0) bulk_wait_all();
     __syncwarp();

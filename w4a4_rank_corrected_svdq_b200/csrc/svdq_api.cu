@@ -508,9 +508,9 @@ svdq_status launch_gemm_2sm(int M, int N, int K, const void* a_codes, const void
       !make_tmap_2d(&tm_x, xl1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, R, M, R * 2, C::kLrCols, 128, lr_sw) ||
       !make_tmap_2d(&tm_l, l2s, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, R, 2 * static_cast<uint64_t>(N), R * 2,
                     C::kLrCols, 128, lr_sw) ||
-      // the fused QKV epilogue stores 32 rows x 32 columns (64-byte swizzle), the others 32 x 64 (128-byte)
+      // the plain and fused QKV epilogues store 32 rows x 32 columns (64-byte swizzle), the MLP one 32 x 64 (128-byte)
       !make_tmap_2d(&tm_y, Y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, M, static_cast<uint64_t>(ldy) * 2,
-                    EPI == 1 ? 32 : 64, 32, EPI == 1 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B))
+                    EPI == 2 ? 64 : 32, 32, EPI == 2 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B))
     return SVDQ_ERR_CUDA;
   // MLP: L1_down^T [32][N] (bf16, row pitch 2N), boxes of 16 rows x 64 columns; otherwise unused
   if (EPI == 2) {
