@@ -135,7 +135,7 @@ constexpr int k2SfaCol = 288;  // A scales: kSfaSlots slots of 16 columns (4 K-s
 
 constexpr int k2Xl1Col = 480;  // MLP up projection: h . L1_down accumulator (32 columns)
 
-template <int R, int EPI = 0>
+template <int R, int EPI = 0, bool LEAN = (EPI == 0)>
 struct Gemm2Cfg {
   static constexpr bool QKV = EPI == 1;
   static constexpr bool MLP = EPI == 2;
@@ -148,11 +148,14 @@ struct Gemm2Cfg {
   // lane: two K-steps of A scales, or one K-step of both 128-row halves of B.
   static constexpr int kSfaBytes = 4 * 2048;    // 4 K-steps x 4 replicas x 512 B (128 rows)
   static constexpr int kSfbBytes = 2 * 4 * 2048;  // 2 row blocks x 4 K-steps x 4 replicas x 512 B
-  // The plain layer (EPI 0) runs four stages: its A scales, needed only when a
-  // tile starts a new A block, move to a two-slot ring of their own, and its
-  // epilogue stages 32 x 32 (2 KB) per warp. The fused modes keep three stages
-  // with the A scales in every stage.
-  static constexpr bool kLean = EPI == 0;
+  // LEAN (plain layer, EPI 0, when its A scales stay resident in TMEM): four
+  // stages; the A scales, needed only when a tile starts a new A block, move to
+  // a two-slot ring of their own, and the epilogue stages 32 x 32 (2 KB) per
+  // warp. Otherwise three stages with the A scales in every stage (the fused
+  // modes need the room; a K too long for resident A scales needs them with
+  // every K block, which a two-slot ring would hold back).
+  static_assert(!LEAN || EPI == 0, "the lean layout is for the plain epilogue");
+  static constexpr bool kLean = LEAN;
   static constexpr int kSfbOff = kABytes + kBBytes + (kLean ? 0 : kSfaBytes);  // within a stage
   static constexpr int kStageBytes = kSfbOff + kSfbBytes;  // 48 or 56 KB
   static constexpr int kStages = kLean ? 4 : 3;
@@ -169,7 +172,7 @@ struct Gemm2Cfg {
   // Epilogue staging per warp: the plain layer one 32 x 32 buffer (2 KB,
   // 64-byte swizzle, four TMA stores per tile); the fused QKV mode two such
   // buffers; the MLP mode one 32-row x 64-column chunk (4 KB, 128-byte swizzle).
-  static constexpr int kOutPerWarp = kLean ? 2048 : 4096;
+  static constexpr int kOutPerWarp = kLean ? 2048 : 4096;  // (the plain layer uses 2 KB either way)
   static constexpr int kOutOff = kStages * kStageBytes;
   static constexpr int kOutBytes = 8 * kOutPerWarp;
   // Plain layer: the A-scale ring (two slots of one K block's A scales).
@@ -545,14 +548,14 @@ __global__ void mlp_xl1_reduce_kernel(const float* __restrict__ partial, int num
   }
 }
 
-template <int R, int EPI>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<R, EPI>::kThreads, 1) w4a4_gemm_2sm_kernel(
+template <int R, int EPI, bool LEAN>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<R, EPI, LEAN>::kThreads, 1) w4a4_gemm_2sm_kernel(
     const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
     const __grid_constant__ CUtensorMap tm_sfa, const __grid_constant__ CUtensorMap tm_sfb,
     const __grid_constant__ CUtensorMap tm_xl1, const __grid_constant__ CUtensorMap tm_l2s,
     const __grid_constant__ CUtensorMap tm_y, const __grid_constant__ CUtensorMap tm_l1d, const float* __restrict__ gscale,
     const __nv_bfloat16* __restrict__ bias, int M, int N, int K, const QkvPost post, const MlpPost mlp) {
-  using C = Gemm2Cfg<R, EPI>;
+  using C = Gemm2Cfg<R, EPI, LEAN>;
   constexpr bool QKV = EPI == 1;
   constexpr int S = C::kStages;
   extern __shared__ uint8_t smem_raw[];

@@ -495,7 +495,7 @@ svdq_status launch_gemm_2sm(int M, int N, int K, const void* a_codes, const void
                             const void* w_codes, const void* w_scales, const float* gscale, const void* l2s,
                             const void* bias, void* Y, int64_t ldy, cudaStream_t stream, int sm_count,
                             const QkvPost& post, const MlpPost& mlp, const void* l1t_down) {
-  using C = Gemm2Cfg<R, EPI>;
+  using C = Gemm2Cfg<R, EPI, false>;
   CUtensorMap tm_a, tm_b, tm_sfa, tm_sfb, tm_x, tm_l, tm_y, tm_l1d;
   const uint64_t kb = static_cast<uint64_t>(K / 2);
   const uint64_t mpad = round_up(static_cast<size_t>(M), 128);
@@ -520,11 +520,15 @@ svdq_status launch_gemm_2sm(int M, int N, int K, const void* a_codes, const void
   } else {
     tm_l1d = tm_y;
   }
-  auto kern = w4a4_gemm_2sm_kernel<R, EPI>;
-  static std::atomic<uint64_t> attr_done{0};
-  ensure_smem_attr(kern, C::kSmemBytes, attr_done);
+  // the plain layer takes the four-stage layout when its A scales stay in TMEM
+  using CL = Gemm2Cfg<R, 0, true>;
+  const bool lean = EPI == 0 && K / 256 <= CL::kSfaSlots;
+  auto kern = lean ? w4a4_gemm_2sm_kernel<R, EPI, EPI == 0> : w4a4_gemm_2sm_kernel<R, EPI, false>;
+  const int smem = lean ? CL::kSmemBytes : C::kSmemBytes;
+  static std::atomic<uint64_t> attr_done[2] = {};
+  ensure_smem_attr(kern, smem, attr_done[lean ? 1 : 0]);
   const int pairs = gemm2_pairs(M, N, sm_count);
-  PdlLaunch pl(dim3(2 * pairs), dim3(C::kThreads), C::kSmemBytes, stream);
+  PdlLaunch pl(dim3(2 * pairs), dim3(C::kThreads), smem, stream);
   cudaLaunchKernelEx(&pl.cfg, kern, tm_a, tm_b, tm_sfa, tm_sfb, tm_x, tm_l, tm_y, tm_l1d, gscale,
                      static_cast<const __nv_bfloat16*>(bias), M, N, K, post, mlp);
   return launch_status();
