@@ -46,7 +46,7 @@ FP4_PER_BF16 = 4.0   # nominal dense fp4 / bf16 tensor throughput ratio (9 / 2.2
 # dominant kernel on this workload, from the ncu capture summarised in
 # profiles/w4a4_gemm_2sm_kernel_qkv_4608x3072x9216_r32.md. Valid only for the
 # kernel as captured: set to None whenever the kernel changes.
-NCU_TRAFFIC_BYTES = {}
+NCU_TRAFFIC_BYTES = {("dit_qkv_4608x3072x9216_r32", "w4a4_gemm_2sm_kernel"): 63436032}
 
 
 def _peaks():
