@@ -22,6 +22,13 @@
 // K <= 14 x 256) and stay there: per 256-deep K block only the weight scales
 // (SFB) are copied, four tcgen05.cp of 128x256b instead of six.
 //
+// Stages (one 256-deep K block each): the plain layer with resident A scales
+// runs four 48 KB stages (A, B, SFB), its A scales loaded through a two-slot
+// ring of their own and its epilogue staged 32 x 32 per warp (2 KB). The
+// fused epilogues, and K too long for resident A scales, run three 56 KB
+// stages that carry the A scales too. The fourth stage covers the load delay
+// the epilogue's burst of Y stores causes at every tile start.
+//
 // Roles (320 threads per CTA):
 //  * warp 0     TMA producer (both CTAs): per tile K/256 stages of E2M1
 //               codes (128-byte swizzle) and UE4M3 scale atoms (SFA only when
